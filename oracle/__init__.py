@@ -1,0 +1,270 @@
+"""Plain CPU oracle for the scaled gated activation + MXFP8 path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product path
+(``moe_gated_activation_b200``) never imports, loads or calls it, and this
+package never imports the product.
+
+The arithmetic lives in ``moeact_oracle.c`` (plain C, IEEE binary32 steps in the
+order the method states, binary128 for the sigmoid, binary64 for sums); this
+module only compiles it with gcc and marshals numpy arrays through ctypes.
+
+Array conventions (all numpy, C-contiguous):
+  bf16 data is passed as ``uint16`` bit patterns; fp32 as ``float32``;
+  E4M3 codes and E8M0 scales as ``uint8``; offsets as ``int64``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+ROWWISE = 1
+COLWISE = 2
+SWIGLU = 0
+SRELU = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moeact_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+           "-Wall", "-Wextra", "-std=gnu11"]
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` with gcc if it is missing or older than the source."""
+    with _lock:
+        stale = (not os.path.exists(_LIB)
+                 or os.path.getmtime(_LIB) < os.path.getmtime(_SRC))
+        if force or stale:
+            tmp = _LIB + f".tmp{os.getpid()}"
+            cmd = ["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lquadmath", "-lm", "-lpthread"]
+            subprocess.run(cmd, check=True)
+            os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    I32 = ctypes.c_int32
+    I = ctypes.c_int
+    lib.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.orc_bf16_to_f32.restype = ctypes.c_float
+    lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+    lib.orc_f32_to_bf16.restype = ctypes.c_uint16
+    lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.orc_e4m3_decode.restype = ctypes.c_double
+    lib.orc_e4m3_encode.argtypes = [ctypes.c_double]
+    lib.orc_e4m3_encode.restype = ctypes.c_uint8
+    lib.orc_e8m0_rceil.argtypes = [ctypes.c_float]
+    lib.orc_e8m0_rceil.restype = I
+    lib.orc_sigma_init.argtypes = []
+    lib.orc_sigma_init.restype = I
+    lib.orc_sigmoid_bf16.argtypes = [ctypes.c_uint16]
+    lib.orc_sigmoid_bf16.restype = ctypes.c_float
+    lib.orc_act_fwd.argtypes = [I, P, I64, P, I64, I64, I, I, P, P, P, P]
+    lib.orc_act_fwd.restype = I
+    lib.orc_act_values.argtypes = [I, P, I64, P, I64, I64, I, P]
+    lib.orc_act_values.restype = I
+    lib.orc_mxfp8_quantize.argtypes = [P, I64, I64, I, P, P, P, P]
+    lib.orc_mxfp8_quantize.restype = I
+    lib.orc_act_bwd.argtypes = [I, P, I64, P, I64, P, I64, I64, I, P, P, P, P, P, P]
+    lib.orc_act_bwd.restype = I
+    lib.orc_splits_to_offsets.argtypes = [P, I32, I64, P, P]
+    lib.orc_splits_to_offsets.restype = I
+    lib.orc_grouped_act_fwd.argtypes = [I, P, I64, P, I64, I64, I, I, P, P, I32, P, P, P, P]
+    lib.orc_grouped_act_fwd.restype = I
+    lib.orc_grouped_act_bwd.argtypes = [I, P, I64, P, I64, P, I64, I64, I, P, P, I32,
+                                        P, P, P, P, P, P]
+    lib.orc_grouped_act_bwd.restype = I
+    if lib.orc_sigma_init() != 0:
+        raise RuntimeError("oracle: sigmoid table has uncertified roundings")
+    _lib = lib
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+# ---------------------------------------------------------------- scalars
+def bf16_to_f32(b: int) -> float:
+    return _load().orc_bf16_to_f32(b)
+
+
+def f32_to_bf16(f: float) -> int:
+    return _load().orc_f32_to_bf16(f)
+
+
+def e4m3_decode(c: int) -> float:
+    return _load().orc_e4m3_decode(c)
+
+
+def e4m3_encode(x: float) -> int:
+    return _load().orc_e4m3_encode(x)
+
+
+def e8m0_rceil(amax: float) -> int:
+    return _load().orc_e8m0_rceil(amax)
+
+
+def sigmoid_bf16(bits: int) -> float:
+    return _load().orc_sigmoid_bf16(bits)
+
+
+def sigmoid_table() -> np.ndarray:
+    """fp32 sigma for every bf16 bit pattern 0..65535."""
+    lib = _load()
+    return np.array([lib.orc_sigmoid_bf16(b) for b in range(65536)], dtype=np.float32)
+
+
+# ---------------------------------------------------------------- helpers
+def mx_widths(M: int, W: int):
+    """Shapes of (row codes, row scales, col codes, col scales) for [M, W]."""
+    return (M, W), (M, W // 32), (M, W), ((M + 31) // 32, W)
+
+
+def _alloc_mx(M, W, dirs, colblk_rows=None):
+    rq, rs, cq, cs = mx_widths(M, W)
+    if colblk_rows is not None:
+        cs = (colblk_rows, W)
+    out = {"row_codes": None, "row_scales": None, "col_codes": None, "col_scales": None}
+    if dirs & ROWWISE:
+        out["row_codes"] = np.zeros(rq, np.uint8)
+        out["row_scales"] = np.zeros(rs, np.uint8)
+    if dirs & COLWISE:
+        out["col_codes"] = np.zeros(cq, np.uint8)
+        out["col_scales"] = np.zeros(cs, np.uint8)
+    return out
+
+
+def _mx_ptrs(out):
+    return (_ptr(out["row_codes"]), _ptr(out["row_scales"]),
+            _ptr(out["col_codes"]), _ptr(out["col_scales"]))
+
+
+# ---------------------------------------------------------------- forward
+def act_fwd(x_bits: np.ndarray, s: np.ndarray, N: int, dirs: int, act: int = SWIGLU,
+            staged: bool = False, ldx: int | None = None) -> dict:
+    """Forward: MXFP8 of y = act(x) * s.  x_bits uint16 [M, ldx]."""
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    M = x_bits.shape[0]
+    ldx = x_bits.shape[1] if ldx is None else ldx
+    out = _alloc_mx(M, N, dirs)
+    rc = _load().orc_act_fwd(act, _ptr(x_bits), ldx, _ptr(s), M, N, dirs, int(staged),
+                             *_mx_ptrs(out))
+    if rc:
+        raise ValueError(f"oracle act_fwd failed ({rc})")
+    return out
+
+
+def act_values(x_bits: np.ndarray, s: np.ndarray, N: int, act: int = SWIGLU,
+               staged: bool = False) -> np.ndarray:
+    """The fp32 activation y = act(x) * s before quantization, [M, N]."""
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    M = x_bits.shape[0]
+    y = np.zeros((M, N), np.float32)
+    _load().orc_act_values(act, _ptr(x_bits), x_bits.shape[1], _ptr(s), M, N, int(staged),
+                           _ptr(y))
+    return y
+
+
+def mxfp8_quantize(y: np.ndarray, dirs: int) -> dict:
+    """Stand-alone MXFP8 quantizer of an fp32 [M, W] matrix."""
+    y = _c(y, np.float32)
+    M, W = y.shape
+    out = _alloc_mx(M, W, dirs)
+    rc = _load().orc_mxfp8_quantize(_ptr(y), M, W, dirs, *_mx_ptrs(out))
+    if rc:
+        raise ValueError(f"oracle mxfp8_quantize failed ({rc})")
+    return out
+
+
+# ---------------------------------------------------------------- backward
+def act_bwd(dy_bits: np.ndarray, x_bits: np.ndarray, s: np.ndarray, N: int, dirs: int,
+            act: int = SWIGLU, want_dx: bool = True, want_dscale: bool = True) -> dict:
+    """Backward: dx (bf16 bits [M, W]), dscale (fp32 [M]) and MXFP8 of dx."""
+    dy_bits = _c(dy_bits, np.uint16)
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    M = x_bits.shape[0]
+    W = 2 * N if act == SWIGLU else N
+    out = _alloc_mx(M, W, dirs)
+    out["dx"] = np.zeros((M, W), np.uint16) if want_dx else None
+    out["dscale"] = np.zeros(M, np.float32) if want_dscale else None
+    rc = _load().orc_act_bwd(act, _ptr(dy_bits), dy_bits.shape[1], _ptr(x_bits),
+                             x_bits.shape[1], _ptr(s), M, N, dirs,
+                             _ptr(out["dx"]), _ptr(out["dscale"]), *_mx_ptrs(out))
+    if rc:
+        raise ValueError(f"oracle act_bwd failed ({rc})")
+    return out
+
+
+# ---------------------------------------------------------------- grouped
+def splits_to_offsets(m_splits: np.ndarray, total_rows: int):
+    """(status, row_offs[E+1], colblk_offs[E+1]); offsets are None on error."""
+    m = _c(m_splits, np.int64)
+    E = m.shape[0]
+    ro = np.zeros(E + 1, np.int64)
+    co = np.zeros(E + 1, np.int64)
+    st = _load().orc_splits_to_offsets(_ptr(m), E, total_rows, _ptr(ro), _ptr(co))
+    if st:
+        return st, None, None
+    return 0, ro, co
+
+
+def grouped_act_fwd(x_bits, s, N, dirs, row_offs, colblk_offs, act=SWIGLU, staged=False):
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    ro = _c(row_offs, np.int64)
+    co = _c(colblk_offs, np.int64)
+    E = ro.shape[0] - 1
+    M = x_bits.shape[0]
+    out = _alloc_mx(M, N, dirs, colblk_rows=int(co[-1]))
+    rc = _load().orc_grouped_act_fwd(act, _ptr(x_bits), x_bits.shape[1], _ptr(s), M, N, dirs,
+                                     int(staged), _ptr(ro), _ptr(co), E, *_mx_ptrs(out))
+    if rc:
+        raise ValueError(f"oracle grouped_act_fwd failed ({rc})")
+    return out
+
+
+def grouped_act_bwd(dy_bits, x_bits, s, N, dirs, row_offs, colblk_offs, act=SWIGLU,
+                    want_dx=True, want_dscale=True):
+    dy_bits = _c(dy_bits, np.uint16)
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    ro = _c(row_offs, np.int64)
+    co = _c(colblk_offs, np.int64)
+    E = ro.shape[0] - 1
+    M = x_bits.shape[0]
+    W = 2 * N if act == SWIGLU else N
+    out = _alloc_mx(M, W, dirs, colblk_rows=int(co[-1]))
+    out["dx"] = np.zeros((M, W), np.uint16) if want_dx else None
+    out["dscale"] = np.zeros(M, np.float32) if want_dscale else None
+    rc = _load().orc_grouped_act_bwd(act, _ptr(dy_bits), dy_bits.shape[1], _ptr(x_bits),
+                                     x_bits.shape[1], _ptr(s), M, N, dirs, _ptr(ro), _ptr(co), E,
+                                     _ptr(out["dx"]), _ptr(out["dscale"]), *_mx_ptrs(out))
+    if rc:
+        raise ValueError(f"oracle grouped_act_bwd failed ({rc})")
+    return out

@@ -1,0 +1,467 @@
+"""Benchmark of the fused scaled gated activation + MXFP8 path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+splits_to_offsets (per-expert offsets) -> grouped forward (scaled SwiGLU, MXFP8
+with the requested scale directions) -> grouped backward (dgate/dup bf16, dscale,
+MXFP8 of the gradient).  A single-group workload runs the same calls with one
+group.  The metric is algorithmic bytes / device time (GB/s), the byte model of
+the pytorch/ao PR #4743 performance table extended with the per-row scale and
+the backward's bf16 dX and dscale.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
+                    [--dirs both|row|col] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank runs its own replica of the workload on
+its GPU (rows are independent; there is no exchange step), and the device time
+is the max over ranks.  L2 is flushed (written then read, 256 MiB) before every
+timed step, outside the timed events.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "fused act+MXFP8 quant GB/s (fwd & bwd) and % of B200 HBM roofline"
+DIRS = {"both": 3, "row": 1, "col": 2}
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ byte model
+def byte_model(M, N, E, dirs, srelu=False, S=None):
+    """Algorithmic bytes of one forward and one backward (dx and dscale on)."""
+    S = (M + 31) // 32 if S is None else S
+    xin = 2 * M * (N if srelu else 2 * N)
+    W = N if srelu else 2 * N
+
+    def mx(width):
+        b = 0
+        if dirs & 1:
+            b += M * width + M * width // 32
+        if dirs & 2:
+            b += M * width + S * width
+        return b
+
+    splits = 8 * E + 2 * 8 * (E + 1) + 4
+    fwd = xin + 4 * M + mx(N)
+    bwd = 2 * M * N + xin + 4 * M + 2 * M * W + 4 * M + mx(W)
+    return {"splits": splits, "fwd": fwd, "bwd": bwd}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device):
+        self.samples = []
+        self.active = False
+        self.stop = threading.Event()
+        self.err = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            try:
+                if self.active:
+                    sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((sm, rs))
+            except Exception as e:  # noqa: BLE001
+                self.err = repr(e)
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.h is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self.stop.set()
+        if self.h is not None:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "error": self.err}
+        mhz = [s for s, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [n for b, n in self.REASONS.items() if bits & b]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz), "sm_mhz_min": min(mhz)}
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_gated_activation_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload, kernel, dirs_name):
+    """Per-launch DRAM bytes from profiles/ncu_traffic.txt, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = kernel_source_hash()
+    with open(p) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if len(line) >= 5 and line[0] == workload and line[1] == kernel and \
+                    line[2] == dirs_name and line[3] == cur:
+                return int(float(line[4]))
+    return None
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import moe_gated_activation_b200 as mg
+    from moe_gated_activation_b200.workloads import WORKLOADS, make_inputs
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    mg.init()
+    wl = WORKLOADS[args.workload]
+    dirs = DIRS[args.dirs]
+    inp = make_inputs(wl, device=dev)
+    x, s, dy = inp["x"], inp["s"], inp["dy"]
+    assert dy is not None, "the benchmark workload needs a backward (dY)"
+    m_host = inp["m_splits"]
+    m_dev = m_host.to(dev)
+    E = int(m_host.numel())
+    S = int(((m_host + 31) // 32).sum())
+    M, N = wl.M, wl.N
+    rw, cw = bool(dirs & 1), bool(dirs & 2)
+    bm = byte_model(M, N, E, dirs, S=S)
+    step_bytes = bm["splits"] + bm["fwd"] + bm["bwd"]
+
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def do_flush(i):
+        flush.fill_(float(i & 7))
+        flush.amax()
+
+    def step():
+        ro, cb, st = mg.splits_to_offsets(m_dev, M)
+        ev[1].record(stream)
+        f, _ = mg.grouped_scaled_swiglu_mxfp8_fwd(x, s, ro, cb, rowwise=rw, colwise=cw,
+                                                  col_scale_rows=S)
+        ev[2].record(stream)
+        b, _ = mg.grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, ro, cb, rowwise=rw, colwise=cw,
+                                                  col_scale_rows=S)
+        return f, b
+
+    # warm-up
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for i in range(args.warmup):
+        do_flush(i)
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev)
+    with sampler:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        sampler.active = True
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            do_flush(i)
+            ev = evs[i]
+            ev[0].record(stream)
+            step()
+            ev[3].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+        sampler.active = False
+        if world > 1:
+            torch.distributed.barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    splits_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public API with host buffers (pinned), H2D of the
+    # step's inputs and D2H of every output inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world)
+
+    peak, peak_kind = measured_peak()
+    mean = lambda v: sum(v) / len(v)
+    fwd_us, bwd_us = 1e3 * mean(fwd_ms), 1e3 * mean(bwd_ms)
+    dom = "bwd" if bwd_us >= fwd_us else "fwd"
+    dom_us = bwd_us if dom == "bwd" else fwd_us
+    achieved = bm[dom] / (dom_us * 1e-6) / 1e9
+    kname = "act_bwd_kernel" if dom == "bwd" else "act_fwd_kernel"
+    traffic = ncu_traffic(args.workload, kname, args.dirs)
+    value = world * step_bytes / (total_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded torch generators; shapes and statistics of the pages' workloads)",
+        "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
+                   "dirs": args.dirs, "activation": "swiglu",
+                   "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
+                   "l2": "flushed before every step (256 MiB written then read), outside the timed events",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes": bm[dom]},
+        "kernels": {
+            "fwd": {"us": round(fwd_us, 2), "bytes": bm["fwd"],
+                    "gbs": round(bm["fwd"] / (fwd_us * 1e-6) / 1e9, 1),
+                    "frac": round(bm["fwd"] / (fwd_us * 1e-6) / 1e9 / peak, 4)},
+            "bwd": {"us": round(bwd_us, 2), "bytes": bm["bwd"],
+                    "gbs": round(bm["bwd"] / (bwd_us * 1e-6) / 1e9, 1),
+                    "frac": round(bm["bwd"] / (bwd_us * 1e-6) / 1e9 / peak, 4)},
+            "splits_to_offsets": {"us": round(1e3 * mean(splits_ms), 2)},
+        },
+        "wall_s_timed_region": round(wall, 4),
+        "gpu_launches": 3 * args.steps,
+        "clocks": sampler.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, dirs, budget_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
+    M, N = wl.M, wl.N
+    rw, cw = bool(dirs & 1), bool(dirs & 2)
+    xh = inp["x"].cpu().pin_memory()
+    sh = inp["s"].cpu().pin_memory()
+    dyh = inp["dy"].cpu().pin_memory()
+    mh = inp["m_splits"].clone().pin_memory()
+    xd, sd, dyd, md = (torch.empty_like(t, device=dev) for t in (xh, sh, dyh, mh))
+    h2d = sum(t.numel() * t.element_size() for t in (xh, sh, dyh, mh))
+    outs_h = None
+
+    def one():
+        nonlocal outs_h
+        xd.copy_(xh, non_blocking=True)
+        sd.copy_(sh, non_blocking=True)
+        dyd.copy_(dyh, non_blocking=True)
+        md.copy_(mh, non_blocking=True)
+        ro, cb, st = mg.splits_to_offsets(md, M)
+        f, fst = mg.grouped_scaled_swiglu_mxfp8_fwd(xd, sd, ro, cb, rowwise=rw, colwise=cw,
+                                                    col_scale_rows=S, status=st)
+        b, bst = mg.grouped_scaled_swiglu_mxfp8_bwd(dyd, xd, sd, ro, cb, rowwise=rw, colwise=cw,
+                                                    col_scale_rows=S, status=st)
+        outs = [t for t in (*f, *b.mx, b.dx, b.dscale, st) if t is not None and t.numel()]
+        if outs_h is None:
+            outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        for h, t in zip(outs_h, outs):
+            h.copy_(t, non_blocking=True)
+        return outs
+
+    outs = one()
+    torch.cuda.synchronize()
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    steps = max(1, min(args.steps, 20))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    E = int(inp["m_splits"].numel())
+    bm = byte_model(M, N, E, dirs, S=S)
+    step_bytes = bm["splits"] + bm["fwd"] + bm["bwd"]
+    return {"value": round(world * step_bytes * steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 4)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def _oracle_sample(wl, dirs, rows):
+    """Inputs of the first `rows` rows of the workload, as numpy bit arrays."""
+    from moe_gated_activation_b200.workloads import bf16_bits, make_inputs
+    inp = make_inputs(wl, device="cpu") if wl.M * wl.N <= (1 << 26) else None
+    if inp is None:
+        # large workloads: draw the same law for a sample of rows only
+        from moe_gated_activation_b200.workloads import random_case
+        c = random_case(rows, wl.N, wl.seed, std=wl.x_std)
+        return bf16_bits(c["x"]), c["s"].numpy(), bf16_bits(c["dy"])
+    return (bf16_bits(inp["x"][:rows]), inp["s"][:rows].numpy().copy(),
+            bf16_bits(inp["dy"][:rows]))
+
+
+def _oracle_step(oracle, xb, s, dyb, N, dirs):
+    oracle.act_fwd(xb, s, N, dirs)
+    oracle.act_bwd(dyb, xb, s, N, dirs)
+
+
+def _calibrate_rows(oracle, wl, dirs, budget_s):
+    xb, s, dyb = _oracle_sample(wl, dirs, 32)
+    t0 = time.perf_counter()
+    _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+    per32 = max(time.perf_counter() - t0, 1e-4)
+    rows = int(budget_s / per32) * 32
+    return max(32, min(wl.M, rows))
+
+
+def cpu_baseline(wl, dirs, budget_s=10.0):
+    import oracle
+    oracle.sigmoid_table()
+    rows = _calibrate_rows(oracle, wl, dirs, budget_s)
+    xb, s, dyb = _oracle_sample(wl, dirs, rows)
+    t0 = time.perf_counter()
+    _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+    dt = time.perf_counter() - t0
+    bm = byte_model(rows, wl.N, 1, dirs)
+    return {"value": round((bm["fwd"] + bm["bwd"]) / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"rows [0, {rows}) of {wl.M} ({wl.key}), forward + backward, "
+                      f"dirs={dirs}, {dt:.1f} s single-threaded"}
+
+
+def run_reference(args):
+    from moe_gated_activation_b200.workloads import WORKLOADS
+    import oracle
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    dirs = DIRS[args.dirs]
+    oracle.sigmoid_table()
+    per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = _calibrate_rows(oracle, wl, dirs, per_step)
+    xb, s, dyb = _oracle_sample(wl, dirs, rows)
+    for _ in range(args.warmup):
+        _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+    dt = time.perf_counter() - t0
+    bm = byte_model(rows, wl.N, 1, dirs)
+    value = args.steps * (bm["fwd"] + bm["bwd"]) / dt / 1e9
+    sample = (f"rows [0, {rows}) of {wl.M} ({wl.key}) per step, forward + backward, "
+              f"single-threaded C oracle")
+    out = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+           "data": "synthetic (seeded torch generators)",
+           "config": {"workload": f"{wl.key}: {wl.title}", "M": wl.M, "N": wl.N,
+                      "dirs": args.dirs, "activation": "swiglu"},
+           "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "c5"])
+    ap.add_argument("--dirs", default="both", choices=list(DIRS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,242 @@
+/*
+ * moeact.h -- C ABI of libmoeact.so: per-row-scaled gated activation
+ * (SwiGLU, SReLU) fused with MXFP8 quantization, forward and backward, dense
+ * and grouped (MoE experts), for NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute is defined by these pages (title, section):
+ *   [AO]   pytorch/ao PR #4743 "[mxfp8 training] Add a fused gated-activation
+ *          (SwiGLU) + MXFP8 quantization kernel" -- Summary (gate and up read
+ *          once, the bf16 activation never materialised, RCEIL MXFP8 with
+ *          rowwise 1x32, colwise 32x1 or both scales in one pass), API
+ *          (gated input packs [gate | up]; backward returns [dGate | dUp];
+ *          disabled directions produce nothing), review reply on the
+ *          backward (dact = fma(silu, 1 - sigma, sigma)).
+ *   [TE]   TransformerEngine PR #3238 "Activation + GroupedLinear Fusion for
+ *          MOE and other MOE optimizations" -- Greptile summary (per-row-scaled
+ *          SReLU / SwiGLU; splits_to_offsets_multi computes every offset array
+ *          once, up front) and sequence diagram (grouped activation ->
+ *          quantized grouped storage; grouped dactivation -> grouped_dy
+ *          quantized, dense_dy, grad_scales).
+ *   [GT]   TransformerEngine PR #2600 "[PyTorch] GroupedTensor integration" --
+ *          Key Changes (several tensors stored contiguously, addressed by
+ *          offsets).
+ *   [VO]   VeOmni PR #1340 -- What does this PR do? (SiLU rounded to the
+ *          activation dtype before the multiply; stride-aware; inputs are not
+ *          mutated).
+ *
+ * Numerics (the same for every entry point; where the pages are silent the
+ * reading is stated):
+ *   sigma(g)  correctly rounded fp32 value of 1/(1+exp(-g)) for bf16 g.
+ *   SwiGLU    y = RN(RN(RN(g*sigma) * u) * s_row)   (fp32, in this order);
+ *             staged: y = RN(bf16(RN(bf16(RN(g*sigma)) * u)) * s_row)   [VO].
+ *   SReLU     y = RN(RN(r*r) * s_row), r = relu(x) (NaN kept)            [TE].
+ *   E8M0      per block, b = 127 + e, e the smallest integer in [-127, 127]
+ *             with amax <= 448 * 2^e (RCEIL); amax = NaN-propagating max |y|;
+ *             +Inf -> 254; NaN -> 255.
+ *   E4M3      code = nearest-even E4M3 of y * 2^(127-b), saturating to
+ *             +-448, sign of zero kept; a block with b = 255 has all codes
+ *             0x7F.
+ *   backward  p = RN(dY*s); dsilu = fma(g*sigma, RN(1-sigma), sigma);
+ *             dgate = bf16(RN(RN(p*u)*dsilu)); dup = bf16(RN(p*silu));
+ *             SReLU dx = bf16(RN(p*2r)); dscale_row = sum_j dY*h (h the
+ *             unscaled activation, fp32 accumulation in a fixed order);
+ *             the MXFP8 of the gradient quantizes the bf16 values.
+ *
+ * Layouts (all row-major, byte offsets from the given pointers):
+ *   x        bf16 [M, ldx]; SwiGLU reads gate = x[:, 0:N], up = x[:, N:2N]
+ *            (ldx >= 2N); SReLU reads x[:, 0:N] (ldx >= N).
+ *   dy       bf16 [M, lddy], first N columns (lddy >= N).
+ *   s        fp32 [M] per-row scale (routing probability).
+ *   W        width of the quantized tensor: N in the forward; 2N (SwiGLU,
+ *            [dgate | dup]) or N (SReLU) in the backward.
+ *   row codes  uint8 E4M3 [M, W];     row scales uint8 E8M0 [M, W/32].
+ *   col codes  uint8 E4M3 [M, W] (same row-major layout as row codes);
+ *   col scales uint8 E8M0 [S, W]; S = ceil(M/32) for dense calls; for grouped
+ *            calls S = colblk_offs[E] = sum_e ceil(m_e/32) and the buffer must
+ *            hold ceil(M/32) + E rows (rows >= S are not written).
+ *   grouped  expert e owns rows [row_offs[e], row_offs[e+1]); its codes start
+ *            at row row_offs[e], its row scales at row row_offs[e], its col
+ *            scales at row colblk_offs[e]; colwise blocks never cross an
+ *            expert boundary (the last block of an expert may be shorter;
+ *            its amax covers the expert's rows only).
+ *   dx       bf16 [M, W] (SwiGLU: [dgate | dup]).   dscale fp32 [M].
+ *
+ * Ownership and execution: the caller allocates every input, output and
+ * workspace on the device; the library allocates nothing per call (it keeps
+ * one 32 KiB sigmoid table per device, built at moeact_init or at the first
+ * call on that device).  Calls are asynchronous on `stream` (a cudaStream_t
+ * passed as void*, NULL = legacy default stream) and never synchronise the
+ * host, except moeact_init.  Inputs are never written.  Outputs must not
+ * overlap inputs or each other.
+ *
+ * Alignment: x, dy, dx, every code and scale array and the workspace must be
+ * 16-byte aligned, ldx and lddy multiples of 8 elements; s and dscale
+ * 4-byte aligned; offsets 8-byte aligned.  Violations return MOEACT_EALIGN
+ * (there is no unaligned fallback).
+ *
+ * Errors: every call validates its arguments on the host and returns a status
+ * without launching anything on failure; moeact_last_error() gives a
+ * thread-local message.  Data errors only visible on the device (bad splits or
+ * offsets) are written to the caller's int32 device status word, and the
+ * kernels then do no work (their outputs are left untouched).
+ */
+#ifndef MOEACT_H
+#define MOEACT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moeact_status {
+  MOEACT_OK = 0,
+  MOEACT_EINVAL = 1,        /* null required pointer, bad size, flag or stride */
+  MOEACT_EALIGN = 2,        /* a pointer or stride breaks the alignment rules */
+  MOEACT_EUNSUPPORTED = 3,  /* not an sm_100 device; first call inside capture */
+  MOEACT_ERANGE = 4,        /* sizes beyond the supported index range */
+  MOEACT_ECUDA = 5,         /* a CUDA runtime call or launch failed */
+  MOEACT_EWORKSPACE = 6     /* dscale requested without a large enough workspace */
+} moeact_status;
+
+/* dirs bitmask: which MXFP8 outputs to produce. */
+#define MOEACT_ROWWISE 1
+#define MOEACT_COLWISE 2
+
+/* Device status word values (grouped calls and splits_to_offsets). */
+#define MOEACT_DEV_OK 0
+#define MOEACT_DEV_NEGATIVE_SPLIT 1   /* a split < 0 */
+#define MOEACT_DEV_SPLIT_SUM 2        /* splits do not sum to M */
+#define MOEACT_DEV_BAD_OFFSETS 3      /* offsets not those of valid splits */
+
+/* Largest number of groups (experts) a grouped call accepts. */
+#define MOEACT_MAX_GROUPS 4096
+/* Largest M accepted (2^36 rows). */
+#define MOEACT_MAX_ROWS (((int64_t)1) << 36)
+
+/* MXFP8 outputs of one call; a disabled direction's two pointers must be NULL. */
+typedef struct moeact_mx_out {
+  uint8_t* row_codes;   /* [M, W]    E4M3, rowwise 1x32 blocks */
+  uint8_t* row_scales;  /* [M, W/32] E8M0 */
+  uint8_t* col_codes;   /* [M, W]    E4M3, colwise 32x1 blocks */
+  uint8_t* col_scales;  /* [S, W]    E8M0 */
+} moeact_mx_out;
+
+/* Build the sigmoid table on the current device and set up its kernels.
+ * Optional: the first call on a device does it, but that first call must not
+ * be inside a stream capture.  Synchronises the current device once. */
+moeact_status moeact_init(void);
+
+/* Static text of a status; thread-local detail of the last failure. */
+const char* moeact_status_string(moeact_status status);
+const char* moeact_last_error(void);
+
+/* ---------------------------------------------------------------------
+ * splits_to_offsets [TE: splits_to_offsets_multi, offsets computed once]
+ *   m_splits     int64 [E] rows per group (device).
+ *   row_offs     int64 [E+1] out: row_offs[e] = sum_{k<e} m_k (device).
+ *   colblk_offs  int64 [E+1] out: sum_{k<e} ceil(m_k/32), the first
+ *                col-scale row of group e (device).
+ *   status       int32 out (device): MOEACT_DEV_OK, or NEGATIVE_SPLIT /
+ *                SPLIT_SUM, in which case no offset is written.
+ * E = 0 is legal (offsets [0], M must be 0).  Element offsets of any array
+ * are row_offs times its row length.
+ * ------------------------------------------------------------------- */
+moeact_status splits_to_offsets(const int64_t* m_splits, int32_t num_groups,
+                                int64_t total_rows, int64_t* row_offs,
+                                int64_t* colblk_offs, int32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Forward, dense [AO: gated_act_mxfp8_forward, plus TE's per-row scale].
+ *   x [M, ldx] bf16, s [M] fp32, N % 32 == 0, dirs != 0; staged_rounding
+ *   0/1 [VO].  M == 0 returns MOEACT_OK without launching.
+ * ------------------------------------------------------------------- */
+moeact_status scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                      int64_t M, int64_t N, int dirs,
+                                      int staged_rounding, moeact_mx_out out,
+                                      void* stream);
+moeact_status scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                     int64_t M, int64_t N, int dirs,
+                                     moeact_mx_out out, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Forward, grouped [TE: _grouped_scaled_activation; GT layout].
+ *   row_offs / colblk_offs int64 [E+1] (device), as splits_to_offsets
+ *   writes them; status int32 (device) receives MOEACT_DEV_OK or
+ *   MOEACT_DEV_BAD_OFFSETS (then nothing is written).  col_scales must hold
+ *   ceil(M/32) + E rows.
+ * ------------------------------------------------------------------- */
+moeact_status grouped_scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                              int64_t M, int64_t N, int dirs,
+                                              int staged_rounding,
+                                              const int64_t* row_offs,
+                                              const int64_t* colblk_offs,
+                                              int32_t num_groups, int32_t* status,
+                                              moeact_mx_out out, void* stream);
+moeact_status grouped_scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                             int64_t M, int64_t N, int dirs,
+                                             const int64_t* row_offs,
+                                             const int64_t* colblk_offs,
+                                             int32_t num_groups, int32_t* status,
+                                             moeact_mx_out out, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Backward [AO: gated_act_mxfp8_backward; TE: _grouped_scaled_dactivation
+ * returning grouped_dy (MXFP8 of dX), dense_dy (bf16 dX) and grad_scales].
+ *   dy [M, lddy] bf16; x, s as in the forward.
+ *   dx     nullable, bf16 [M, W] (W = 2N SwiGLU, N SReLU).
+ *   dscale nullable, fp32 [M].  Needs `workspace` of at least
+ *          scaled_act_mxfp8_bwd_workspace_size(M, N, E) bytes (E = 1 for
+ *          dense calls), zero-filled before its first use.  It holds per-tile
+ *          partial sums and per-slab counters; every call that completes
+ *          returns the counters to zero, so the workspace can be reused
+ *          without clearing.  Calls sharing one workspace must not overlap on
+ *          the GPU.
+ *   dirs   may be 0 (bf16 dx and/or dscale only); at least one output
+ *          must be requested.
+ * ------------------------------------------------------------------- */
+size_t scaled_act_mxfp8_bwd_workspace_size(int64_t M, int64_t N, int32_t num_groups);
+
+moeact_status scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
+                                      int64_t ldx, const float* s, int64_t M, int64_t N,
+                                      int dirs, void* dx, float* dscale,
+                                      moeact_mx_out out, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+moeact_status scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
+                                     int64_t ldx, const float* s, int64_t M, int64_t N,
+                                     int dirs, void* dx, float* dscale,
+                                     moeact_mx_out out, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+moeact_status grouped_scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
+                                              int64_t ldx, const float* s, int64_t M,
+                                              int64_t N, int dirs,
+                                              const int64_t* row_offs,
+                                              const int64_t* colblk_offs,
+                                              int32_t num_groups, int32_t* status,
+                                              void* dx, float* dscale, moeact_mx_out out,
+                                              void* workspace, size_t workspace_bytes,
+                                              void* stream);
+moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
+                                             int64_t ldx, const float* s, int64_t M,
+                                             int64_t N, int dirs,
+                                             const int64_t* row_offs,
+                                             const int64_t* colblk_offs,
+                                             int32_t num_groups, int32_t* status,
+                                             void* dx, float* dscale, moeact_mx_out out,
+                                             void* workspace, size_t workspace_bytes,
+                                             void* stream);
+
+/* ---------------------------------------------------------------------
+ * Test hook: sigma for every bf16 bit pattern (65536 fp32 values written to
+ * `out`, device memory) exactly as the kernels compute it.  No counterpart on
+ * the pages; it exposes the device table so it can be compared with an
+ * independent CPU computation.
+ * ------------------------------------------------------------------- */
+moeact_status moeact_sigmoid_dump(float* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEACT_H */

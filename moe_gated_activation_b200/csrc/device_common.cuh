@@ -1,0 +1,141 @@
+// Device helpers shared by the kernels of libmoeact: bf16 unpacking, the
+// sigmoid table lookup, the RCEIL E8M0 exponent and E4M3 packing.
+//
+// Numerics follow pytorch/ao PR #4743 "[mxfp8 training] Add a fused
+// gated-activation (SwiGLU) + MXFP8 quantization kernel" (Summary: RCEIL
+// MXFP8 cast of the SwiGLU output, 1x32 / 32x1 blocks) with the readings stated
+// in include/moeact.h.  Every fp32 step is an explicit round-to-nearest
+// intrinsic so that no multiply-add contraction can change a rounding.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+namespace moeact {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// ---------------------------------------------------------------- sigmoid
+// The table holds the correctly rounded fp32 sigma(g) for every bf16 g with
+// |g| in [2^-25, 128] (bit patterns 0x3300..0x4300), positive then negative.
+// Outside that range sigma rounds to 0.5 (|g| < 2^-24), 1 (g > 17.33) or +0
+// (g < -103.97), so clamping the magnitude to the range end gives the right
+// value; NaN inputs are caught by silu = g * sigma, which is NaN.
+constexpr uint32_t kSigLo = 0x3300u;
+constexpr uint32_t kSigHi = 0x4300u;
+constexpr uint32_t kSigPerSign = kSigHi - kSigLo + 1;   // 4097
+constexpr int kSigEntries = 2 * kSigPerSign;            // 8194
+constexpr int kSigEntriesPadded = 8196;                 // whole float4s
+constexpr int kSigBytes = kSigEntriesPadded * 4;
+
+__device__ __forceinline__ float sigma_lookup(const float* tab, uint32_t b16) {
+  uint32_t a = b16 & 0x7FFFu;
+  a = min(max(a, kSigLo), kSigHi) - kSigLo;
+  a += (b16 & 0x8000u) ? kSigPerSign : 0u;
+  return tab[a];
+}
+
+// ---------------------------------------------------------------- bf16
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// The same unpacking through a byte permute; used where a second pass over
+// values that an earlier pass already unpacked must not share (and keep
+// alive) the earlier pass's fp32 copies.
+__device__ __forceinline__ float bf16_lo_p(uint32_t v) { return __uint_as_float(__byte_perm(v, 0u, 0x1044)); }
+__device__ __forceinline__ float bf16_hi_p(uint32_t v) { return __uint_as_float(__byte_perm(v, 0u, 0x3244)); }
+
+__device__ __forceinline__ float bf16_round(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// Two fp32 values -> packed bf16x2 (a in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// relu that keeps NaN (NaN in -> NaN out); negative and zero inputs give +0.
+__device__ __forceinline__ float relu_keep_nan(float v) {
+  return v > 0.0f ? v : (v != v ? v : 0.0f);
+}
+
+// ---------------------------------------------------------------- E8M0
+// RCEIL shared exponent from the magnitude bits of the block amax (an fp32
+// bit pattern with the sign cleared; NaN patterns compare above +Inf so an
+// integer max over magnitudes is NaN-propagating).  b = 127 + e with e the
+// smallest integer such that amax <= 448 * 2^e: for a normal amax with biased
+// exponent E and mantissa m that is E - 8, plus one when m > 0x600000
+// (amax above 1.75 * 2^(E-127)); adding 0x1FFFFF carries exactly then.
+// Subnormal and zero amax clamp to 0; +Inf gives 254; NaN 255.
+__device__ __forceinline__ uint32_t e8m0_from_amax(uint32_t amag) {
+  if (amag >= 0x7F800000u) return amag == 0x7F800000u ? 254u : 255u;
+  const int b = (int)((amag + 0x1FFFFFu) >> 23) - 8;
+  return (uint32_t)max(b, 0);
+}
+
+constexpr uint32_t kNanScale = 0x7FC00000u;
+
+// Bit pattern of the quantization multiplier 2^(127-b): 2^127 .. 2^-126 as a
+// normal float, 2^-127 as the subnormal 0x00400000, and a NaN marker for the
+// NaN scale 255 (whose block is all 0x7F codes).
+__device__ __forceinline__ uint32_t scale_multiplier(uint32_t b) {
+  return b < 254u ? (254u - b) << 23 : (b == 254u ? 0x00400000u : kNanScale);
+}
+
+// Two values -> two E4M3 codes (a in the low byte): nearest even of v * 2^(127-b),
+// saturating; a NaN-scale column gives 0x7F.
+__device__ __forceinline__ uint32_t e4m3x2(float a, uint32_t ma, float b, uint32_t mb) {
+  const float2 v = make_float2(__fmul_rn(a, __uint_as_float(ma)),
+                               __fmul_rn(b, __uint_as_float(mb)));
+  uint32_t q = (uint32_t)__nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, __NV_E4M3);
+  if (ma == kNanScale) q = (q & 0xFF00u) | 0x007Fu;
+  if (mb == kNanScale) q = (q & 0x00FFu) | 0x7F00u;
+  return q;
+}
+
+__device__ __forceinline__ uint32_t f32_mag(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+// ---------------------------------------------------------------- warp butterflies
+// "Transposed" butterfly: each lane holds one value per row for 2*HALF rows;
+// after the step it holds HALF partial reductions, over lanes {l, l ^ off},
+// for the rows selected by bit `off` of the lane.  Chaining the steps for
+// off = 8, 4, 2, 1 leaves lane l with rows 2(l & 15) and 2(l & 15) + 1 reduced
+// over its 16-lane half; chaining off = 16 .. 1 leaves lane l with row l
+// reduced over the warp.  The order of every reduction is fixed.
+template <int HALF>
+__device__ __forceinline__ void bfly_max_u32(uint32_t* a, int lane, int off) {
+  const bool up = (lane & off) != 0;
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const uint32_t keep = up ? a[HALF + i] : a[i];
+    const uint32_t send = up ? a[i] : a[HALF + i];
+    a[i] = max(keep, __shfl_xor_sync(kFull, send, off));
+  }
+}
+
+// Same on two packed 16-bit magnitudes per word.
+template <int HALF>
+__device__ __forceinline__ void bfly_max_u16x2(uint32_t* a, int lane, int off) {
+  const bool up = (lane & off) != 0;
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const uint32_t keep = up ? a[HALF + i] : a[i];
+    const uint32_t send = up ? a[i] : a[HALF + i];
+    a[i] = __vmaxu2(keep, __shfl_xor_sync(kFull, send, off));
+  }
+}
+
+template <int HALF>
+__device__ __forceinline__ void bfly_sum_f32(float* a, int lane, int off) {
+  const bool up = (lane & off) != 0;
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const float keep = up ? a[HALF + i] : a[i];
+    const float send = up ? a[i] : a[HALF + i];
+    a[i] = __fadd_rn(keep, __shfl_xor_sync(kFull, send, off));
+  }
+}
+
+}  // namespace moeact

@@ -1,0 +1,279 @@
+"""PyTorch-facing calls of the fused scaled gated activation + MXFP8 path.
+
+These functions only allocate outputs with torch, check dtypes/strides and pass
+pointers and the current CUDA stream to libmoeact (include/moeact.h); every
+step of the computation runs in the library's sm_100a kernels.
+
+Return convention (pytorch/ao PR #4743, section "API"): an ``MXFP8`` tuple
+(row_codes, col_codes, row_scales, col_scales); a disabled direction comes back
+zero-sized.  Codes are ``torch.float8_e4m3fn`` [M, W] (same row-major layout
+for both directions), scales ``torch.uint8`` E8M0 bytes, row scales [M, W/32],
+col scales [S, W].
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+from typing import NamedTuple, Optional
+
+import torch
+
+from . import _capi
+
+ROWWISE = _capi.ROWWISE
+COLWISE = _capi.COLWISE
+
+
+class MXFP8(NamedTuple):
+    row_codes: torch.Tensor
+    col_codes: torch.Tensor
+    row_scales: torch.Tensor
+    col_scales: torch.Tensor
+
+
+class Backward(NamedTuple):
+    mx: MXFP8                     # MXFP8 of dX ("grouped_dy")
+    dx: Optional[torch.Tensor]    # bf16 [M, W] ("dense_dy")
+    dscale: Optional[torch.Tensor]  # fp32 [M] ("grad_scales")
+
+
+def _dirs(rowwise, colwise):
+    return (ROWWISE if rowwise else 0) | (COLWISE if colwise else 0)
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _check_rows(t, name, dtype, width):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit column stride")
+    if t.shape[1] < width:
+        raise ValueError(f"{name} has {t.shape[1]} columns, {width} needed")
+
+
+def _check_s(s, M, device):
+    if s.dtype != torch.float32 or not s.is_cuda or s.dim() != 1 or s.shape[0] != M:
+        raise ValueError(f"s must be a CUDA float32 vector of length {M}")
+    if s.stride(0) != 1:
+        raise ValueError("s must be contiguous")
+
+
+def _alloc_mx(M, W, dirs, device, col_rows):
+    e = torch.empty(0, dtype=torch.uint8, device=device)
+    rq = torch.empty((M, W), dtype=torch.uint8, device=device) if dirs & ROWWISE else e
+    rs = torch.empty((M, W // 32), dtype=torch.uint8, device=device) if dirs & ROWWISE else e
+    cq = torch.empty((M, W), dtype=torch.uint8, device=device) if dirs & COLWISE else e
+    cs = torch.empty((col_rows, W), dtype=torch.uint8, device=device) if dirs & COLWISE else e
+    return rq, rs, cq, cs
+
+
+def _mx_struct(rq, rs, cq, cs, dirs):
+    if dirs & ROWWISE:
+        r = (rq.data_ptr(), rs.data_ptr())
+    else:
+        r = (None, None)
+    if dirs & COLWISE:
+        c = (cq.data_ptr(), cs.data_ptr())
+    else:
+        c = (None, None)
+    return _capi.MxOut(r[0], r[1], c[0], c[1])
+
+
+def _mx_result(rq, rs, cq, cs, col_rows_view=None):
+    if col_rows_view is not None and cs.numel():
+        cs = cs[:col_rows_view]
+    return MXFP8(rq.view(torch.float8_e4m3fn), cq.view(torch.float8_e4m3fn), rs, cs)
+
+
+# ------------------------------------------------------------------ offsets
+def splits_to_offsets(m_splits: torch.Tensor, total_rows: int):
+    """(row_offs, colblk_offs, status) int64/int64/int32 device tensors for the
+    per-expert row counts `m_splits` (int64, on the device)."""
+    if m_splits.dtype != torch.int64 or not m_splits.is_cuda or m_splits.dim() != 1:
+        raise ValueError("m_splits must be a 1-D int64 CUDA tensor")
+    m_splits = m_splits.contiguous()
+    dev = m_splits.device
+    E = m_splits.shape[0]
+    ro = torch.empty(E + 1, dtype=torch.int64, device=dev)
+    cb = torch.empty(E + 1, dtype=torch.int64, device=dev)
+    st = torch.empty(1, dtype=torch.int32, device=dev)
+    _capi.call("splits_to_offsets", _ptr(m_splits), E, int(total_rows), _ptr(ro), _ptr(cb),
+               _ptr(st), _stream(dev))
+    return ro, cb, st
+
+
+# ------------------------------------------------------------------ forward
+def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None):
+    swiglu = act == "swiglu"
+    if N is None:
+        N = x.shape[1] // 2 if swiglu else x.shape[1]
+    _check_rows(x, "x", torch.bfloat16, 2 * N if swiglu else N)
+    M = x.shape[0]
+    _check_s(s, M, x.device)
+    dirs = _dirs(rowwise, colwise)
+    if grouped is None:
+        col_rows, view = (M + 31) // 32, None
+    else:
+        ro, cb, E, st, view = grouped
+        col_rows = (M + 31) // 32 + E
+    rq, rs, cq, cs = _alloc_mx(M, N, dirs, x.device, col_rows)
+    mx = _mx_struct(rq, rs, cq, cs, dirs)
+    stream = _stream(x.device)
+    ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
+    if grouped is None:
+        if swiglu:
+            _capi.call("scaled_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs, int(staged),
+                       mx, stream)
+        else:
+            _capi.call("scaled_srelu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs, mx, stream)
+    else:
+        if swiglu:
+            _capi.call("grouped_scaled_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs,
+                       int(staged), _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
+        else:
+            _capi.call("grouped_scaled_srelu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs,
+                       _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
+    return _mx_result(rq, rs, cq, cs, view)
+
+
+def scaled_swiglu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, staged_rounding=False, N=None):
+    """MXFP8 of SwiGLU(x) * s; x bf16 [M, >=2N] packs [gate | up]."""
+    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding)
+
+
+def scaled_srelu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, N=None):
+    """MXFP8 of relu(x)^2 * s; x bf16 [M, >=N]."""
+    return _fwd("srelu", x, s, N, rowwise, colwise, False)
+
+
+def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
+    E = row_offs.shape[0] - 1
+    if status is None:
+        status = torch.empty(1, dtype=torch.int32, device=device)
+    return (row_offs, colblk_offs, E, status, col_scale_rows), status
+
+
+def grouped_scaled_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
+                                    staged_rounding=False, status=None, col_scale_rows=None,
+                                    N=None):
+    """Grouped forward: experts own the rows given by `row_offs` (from
+    splits_to_offsets).  Returns (MXFP8, status).  Col scales hold
+    ceil(M/32) + E rows unless `col_scale_rows` (sum of ceil(m_e/32), known on
+    the host) is given."""
+    g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
+    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, g), status
+
+
+def grouped_scaled_srelu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
+                                   status=None, col_scale_rows=None, N=None):
+    g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
+    return _fwd("srelu", x, s, N, rowwise, colwise, False, g), status
+
+
+# ------------------------------------------------------------------ backward
+_ws_lock = threading.Lock()
+_ws_cache = {}
+
+
+def bwd_workspace_bytes(M, N, num_groups=1):
+    return int(_capi.lib().scaled_act_mxfp8_bwd_workspace_size(M, N, num_groups))
+
+
+def _workspace(device, nbytes):
+    """A zero-filled workspace per (device, stream); the kernels leave it zeroed."""
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    with _ws_lock:
+        ws = _ws_cache.get(key)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+            _ws_cache[key] = ws
+    return ws
+
+
+def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, grouped=None):
+    swiglu = act == "swiglu"
+    if N is None:
+        N = dy.shape[1]
+    _check_rows(x, "x", torch.bfloat16, 2 * N if swiglu else N)
+    _check_rows(dy, "dy", torch.bfloat16, N)
+    M = x.shape[0]
+    if dy.shape[0] != M:
+        raise ValueError("dy and x must have the same number of rows")
+    _check_s(s, M, x.device)
+    dirs = _dirs(rowwise, colwise)
+    W = 2 * N if swiglu else N
+    dev = x.device
+    if grouped is None:
+        E, col_rows, view = 1, (M + 31) // 32, None
+    else:
+        ro, cb, E, st, view = grouped
+        col_rows = (M + 31) // 32 + E
+    rq, rs, cq, cs = _alloc_mx(M, W, dirs, dev, col_rows)
+    mx = _mx_struct(rq, rs, cq, cs, dirs)
+    dx = torch.empty((M, W), dtype=torch.bfloat16, device=dev) if want_dx else None
+    dscale = torch.empty(M, dtype=torch.float32, device=dev) if want_dscale else None
+    nbytes = bwd_workspace_bytes(M, N, E)
+    ws = None
+    if want_dscale:
+        ws = workspace if workspace is not None else _workspace(dev, nbytes)
+    stream = _stream(dev)
+    ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
+    lddy = dy.stride(0) if M > 1 else max(dy.stride(0), dy.shape[1])
+    common = (_ptr(dy), lddy, _ptr(x), ldx, _ptr(s), M, N, dirs)
+    tail = (mx, _ptr(ws), ws.numel() if ws is not None else 0, stream)
+    if grouped is None:
+        name = "scaled_swiglu_mxfp8_bwd" if swiglu else "scaled_srelu_mxfp8_bwd"
+        _capi.call(name, *common, _ptr(dx), _ptr(dscale), *tail)
+    else:
+        name = "grouped_scaled_swiglu_mxfp8_bwd" if swiglu else "grouped_scaled_srelu_mxfp8_bwd"
+        _capi.call(name, *common, _ptr(ro), _ptr(cb), E, _ptr(st), _ptr(dx), _ptr(dscale), *tail)
+    return Backward(_mx_result(rq, rs, cq, cs, view), dx, dscale)
+
+
+def scaled_swiglu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
+                            want_dscale=True, workspace=None, N=None):
+    """Backward of the scaled SwiGLU: MXFP8 of [dgate | dup], bf16 dx, fp32 dscale."""
+    return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace)
+
+
+def scaled_srelu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
+                           want_dscale=True, workspace=None, N=None):
+    return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace)
+
+
+def grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
+                                    colwise=True, want_dx=True, want_dscale=True,
+                                    workspace=None, status=None, col_scale_rows=None, N=None):
+    g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
+    return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
+                g), status
+
+
+def grouped_scaled_srelu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
+                                   colwise=True, want_dx=True, want_dscale=True,
+                                   workspace=None, status=None, col_scale_rows=None, N=None):
+    g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
+    return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
+                g), status
+
+
+# ------------------------------------------------------------------ misc
+def init():
+    """Set up the current device (sigmoid table); call before any stream capture."""
+    _capi.call("moeact_init")
+
+
+def sigmoid_table(device="cuda"):
+    """fp32 sigma for all 65536 bf16 bit patterns, as the kernels compute it."""
+    out = torch.empty(65536, dtype=torch.float32, device=device)
+    _capi.call("moeact_sigmoid_dump", _ptr(out), _stream(out.device))
+    return out

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/moeact.h declares, and rejects invalid arguments on the
+host before touching CUDA (pytorch/ao PR #4743, Numerics and tests: every
+launcher error path is exercised)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from moe_gated_activation_b200 import _capi
+from moe_gated_activation_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mbuild.build()
+    return _capi.lib()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "moeact.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_expected_entry_points():
+    names = header_functions()
+    for n in ["splits_to_offsets", "scaled_swiglu_mxfp8_fwd", "scaled_swiglu_mxfp8_bwd",
+              "grouped_scaled_swiglu_mxfp8_fwd", "grouped_scaled_swiglu_mxfp8_bwd",
+              "scaled_srelu_mxfp8_fwd", "scaled_srelu_mxfp8_bwd", "moeact_init",
+              "moeact_status_string", "moeact_last_error", "scaled_act_mxfp8_bwd_workspace_size"]:
+        assert n in names, n
+
+
+def test_library_exports_every_declared_function(lib):
+    for n in header_functions():
+        assert hasattr(lib, n), n
+        assert n in _capi._SIGS, f"{n} has no ctypes declaration"
+
+
+def test_status_strings(lib):
+    for st in range(7):
+        assert lib.moeact_status_string(st)
+    assert lib.moeact_status_string(99) == b"unknown status"
+
+
+A16 = 1 << 20          # a fake, 16-byte-aligned device address (never dereferenced)
+MX_ROW = _capi.MxOut(A16, A16, None, None)
+MX_BOTH = _capi.MxOut(A16, A16, A16, A16)
+
+
+def fwd(lib, x=A16, ldx=512, s=A16, M=64, N=256, dirs=1, staged=0, mx=MX_ROW):
+    return lib.scaled_swiglu_mxfp8_fwd(x, ldx, s, M, N, dirs, staged, mx, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), _capi.EINVAL),
+    (dict(s=None), _capi.EINVAL),
+    (dict(M=-1), _capi.EINVAL),
+    (dict(N=0), _capi.EINVAL),
+    (dict(N=48), _capi.EINVAL),                 # not a multiple of 32
+    (dict(ldx=256), _capi.EINVAL),              # narrower than 2N
+    (dict(ldx=516), _capi.EALIGN),              # not a multiple of 8 elements
+    (dict(x=A16 + 8), _capi.EALIGN),
+    (dict(s=A16 + 2), _capi.EALIGN),
+    (dict(dirs=0), _capi.EINVAL),
+    (dict(dirs=4), _capi.EINVAL),
+    (dict(staged=2), _capi.EINVAL),
+    (dict(dirs=3), _capi.EINVAL),               # colwise pointers missing
+    (dict(mx=_capi.MxOut(A16, None, None, None)), _capi.EINVAL),
+    (dict(mx=_capi.MxOut(A16 + 4, A16, None, None)), _capi.EALIGN),
+    (dict(mx=MX_BOTH), _capi.EINVAL),           # colwise pointers given, not requested
+    (dict(M=1 << 37), _capi.ERANGE),
+    (dict(N=1 << 25, ldx=1 << 26), _capi.ERANGE),
+])
+def test_forward_argument_errors(lib, kw, status):
+    assert fwd(lib, **kw) == status
+    assert lib.moeact_last_error()
+
+
+def test_empty_input_is_ok_without_launch(lib):
+    assert fwd(lib, M=0) == _capi.OK
+    assert lib.scaled_srelu_mxfp8_fwd(A16, 256, A16, 0, 256, 1, MX_ROW, None) == _capi.OK
+
+
+def bwd(lib, dy=A16, lddy=256, x=A16, ldx=512, s=A16, M=64, N=256, dirs=1, dx=A16, dscale=A16,
+        mx=MX_ROW, ws=A16, wsb=1 << 30):
+    return lib.scaled_swiglu_mxfp8_bwd(dy, lddy, x, ldx, s, M, N, dirs, dx, dscale, mx, ws, wsb,
+                                       None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dy=None), _capi.EINVAL),
+    (dict(lddy=128), _capi.EINVAL),
+    (dict(lddy=260), _capi.EALIGN),
+    (dict(dy=A16 + 2), _capi.EALIGN),
+    (dict(dx=A16 + 4), _capi.EALIGN),
+    (dict(dscale=A16 + 1), _capi.EALIGN),
+    (dict(ws=None), _capi.EWORKSPACE),
+    (dict(wsb=16), _capi.EWORKSPACE),
+    (dict(ws=A16 + 8), _capi.EALIGN),
+    (dict(dirs=0, dx=None, dscale=None), _capi.EINVAL),
+    (dict(dirs=5), _capi.EINVAL),
+])
+def test_backward_argument_errors(lib, kw, status):
+    assert bwd(lib, **kw) == status
+
+
+def test_backward_workspace_only_needed_for_dscale(lib):
+    assert bwd(lib, M=0, dscale=None, ws=None) == _capi.OK
+    n = lib.scaled_act_mxfp8_bwd_workspace_size(4096, 2048, 1)
+    assert n >= (4096 // 32) * (2048 // 64) * 32 * 4
+    assert n % 16 == 0
+    assert lib.scaled_act_mxfp8_bwd_workspace_size(-1, 2048, 1) == 0
+
+
+def test_grouped_argument_errors(lib):
+    f = lib.grouped_scaled_swiglu_mxfp8_fwd
+    args = lambda ro=A16, cb=A16, E=4, st=A16: (A16, 512, A16, 64, 256, 1, 0, ro, cb, E, st,
+                                                 MX_ROW, None)
+    assert f(*args(ro=None)) == _capi.EINVAL
+    assert f(*args(st=None)) == _capi.EINVAL
+    assert f(*args(E=0)) == _capi.EINVAL
+    assert f(*args(E=_capi.MAX_GROUPS + 1)) == _capi.EINVAL
+    assert f(*args(ro=A16 + 4)) == _capi.EALIGN
+
+
+def test_splits_to_offsets_argument_errors(lib):
+    f = lib.splits_to_offsets
+    assert f(A16, 4, 64, None, A16, A16, None) == _capi.EINVAL
+    assert f(A16, -1, 64, A16, A16, A16, None) == _capi.EINVAL
+    assert f(A16, _capi.MAX_GROUPS + 1, 64, A16, A16, A16, None) == _capi.EINVAL
+    assert f(A16, 4, -1, A16, A16, A16, None) == _capi.EINVAL
+    assert f(A16 + 4, 4, 64, A16, A16, A16, None) == _capi.EALIGN
+    assert f(A16, 4, 1 << 40, A16, A16, A16, None) == _capi.ERANGE

@@ -112,8 +112,8 @@ typedef enum moeact_status {
 
 /* Largest number of groups (experts) a grouped call accepts. */
 #define MOEACT_MAX_GROUPS 4096
-/* Largest M accepted (2^36 rows). */
-#define MOEACT_MAX_ROWS (((int64_t)1) << 36)
+/* Largest M accepted (2^30 rows; TMA coordinates are 32-bit). */
+#define MOEACT_MAX_ROWS (((int64_t)1) << 30)
 
 /* MXFP8 outputs of one call; a disabled direction's two pointers must be NULL. */
 typedef struct moeact_mx_out {
@@ -188,10 +188,10 @@ moeact_status grouped_scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const f
  *   dx     nullable, bf16 [M, W] (W = 2N SwiGLU, N SReLU).
  *   dscale nullable, fp32 [M].  Needs `workspace` of at least
  *          scaled_act_mxfp8_bwd_workspace_size(M, N, E) bytes (E = 1 for
- *          dense calls), zero-filled before its first use.  It holds per-tile
- *          partial sums and per-slab counters; every call that completes
- *          returns the counters to zero, so the workspace can be reused
- *          without clearing.  Calls sharing one workspace must not overlap on
+ *          dense calls; the size does not depend on E): scratch for the
+ *          per-tile partial sums (ceil(N/64) x M fp32), no initial content
+ *          required.  dscale is then summed by a second kernel launched on
+ *          the same stream.  Calls sharing one workspace must not overlap on
  *          the GPU.
  *   dirs   may be 0 (bf16 dx and/or dscale only); at least one output
  *          must be requested.
@@ -226,6 +226,12 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
                                              void* dx, float* dscale, moeact_mx_out out,
                                              void* workspace, size_t workspace_bytes,
                                              void* stream);
+
+/* Reads and clears this device's error word: non-zero if a kernel gave up
+ * waiting for its own input copies (bit 0 forward, bit 1 backward) -- a
+ * defensive bound that ends the kernel instead of letting it hang; never
+ * expected in normal operation.  Synchronous.  No counterpart on the pages. */
+moeact_status moeact_device_error(uint32_t* flags);
 
 /* ---------------------------------------------------------------------
  * Test hook: sigma for every bf16 bit pattern (65536 fp32 values written to

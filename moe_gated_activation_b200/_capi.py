@@ -57,6 +57,7 @@ _SIGS = {
     "grouped_scaled_srelu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, P, P, I32, P, P, P,
                                         MxOut, P, SZ, P], I),
     "moeact_sigmoid_dump": ([P, P], I),
+    "moeact_device_error": ([P], I),
 }
 
 

@@ -7,6 +7,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "../../include/moeact.h"
@@ -36,30 +38,48 @@ int g_sms[kMaxDevices];
 std::mutex g_mu;
 __device__ int g_sigma_uncertain;
 
-using KernelFn = void (*)(const Params);
-struct Variant { KernelFn fn; int threads; };
+using FwdFn = void (*)(const CUtensorMap, const Params);
+using BwdFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
+struct FwdVariant { FwdFn fn; int threads; int smem_fixed; };
+struct BwdVariant { BwdFn fn; int threads; int smem_fixed; };
+
+template <int ACT, int DIRS, bool STAGED, bool GROUPED>
+FwdVariant fwd_variant() {
+  return {act_fwd_kernel<ACT, DIRS, STAGED, GROUPED>, fwd_threads(ACT, DIRS),
+          smem_bytes(fwd_warps(ACT), fwd_operands(ACT), ACT == kSwiGLU, -1)};
+}
+template <int ACT, int DIRS, bool GROUPED>
+BwdVariant bwd_variant() {
+  return {act_bwd_kernel<ACT, DIRS, GROUPED>, bwd_threads(ACT, DIRS),
+          smem_bytes(bwd_warps(ACT), bwd_operands(ACT), ACT == kSwiGLU, -1)};
+}
 
 template <int ACT, bool GROUPED>
-void fwd_kernels(KernelFn* out, int& n) {
-  out[n++] = act_fwd_kernel<ACT, kRow, false, GROUPED>;
-  out[n++] = act_fwd_kernel<ACT, kCol, false, GROUPED>;
-  out[n++] = act_fwd_kernel<ACT, kRow | kCol, false, GROUPED>;
+void fwd_all(FwdVariant* out, int& n) {
+  out[n++] = fwd_variant<ACT, kRow, false, GROUPED>();
+  out[n++] = fwd_variant<ACT, kCol, false, GROUPED>();
+  out[n++] = fwd_variant<ACT, kRow | kCol, false, GROUPED>();
   if (ACT == kSwiGLU) {
-    out[n++] = act_fwd_kernel<ACT, kRow, true, GROUPED>;
-    out[n++] = act_fwd_kernel<ACT, kCol, true, GROUPED>;
-    out[n++] = act_fwd_kernel<ACT, kRow | kCol, true, GROUPED>;
+    out[n++] = fwd_variant<ACT, kRow, true, GROUPED>();
+    out[n++] = fwd_variant<ACT, kCol, true, GROUPED>();
+    out[n++] = fwd_variant<ACT, kRow | kCol, true, GROUPED>();
   }
 }
 
 template <int ACT, bool GROUPED>
-void bwd_kernels(KernelFn* out, int& n) {
-  out[n++] = act_bwd_kernel<ACT, 0, GROUPED>;
-  out[n++] = act_bwd_kernel<ACT, kRow, GROUPED>;
-  out[n++] = act_bwd_kernel<ACT, kCol, GROUPED>;
-  out[n++] = act_bwd_kernel<ACT, kRow | kCol, GROUPED>;
+void bwd_all(BwdVariant* out, int& n) {
+  out[n++] = bwd_variant<ACT, 0, GROUPED>();
+  out[n++] = bwd_variant<ACT, kRow, GROUPED>();
+  out[n++] = bwd_variant<ACT, kCol, GROUPED>();
+  out[n++] = bwd_variant<ACT, kRow | kCol, GROUPED>();
 }
 
-constexpr int kMaxSmem = kSigBytes + (MOEACT_MAX_GROUPS + 1 + 3) * 4;
+// Extra shared memory of a grouped call (its col-block offsets), at most.
+constexpr int kGroupSmem = group_bytes(MOEACT_MAX_GROUPS);
+
+__device__ uint32_t g_err_word;
+uint32_t* g_err_ptr[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 moeact_status init_device(int dev) {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -71,21 +91,41 @@ moeact_status init_device(int dev) {
     return fail(MOEACT_EUNSUPPORTED, "device %d is sm_%d%d; libmoeact is built for sm_100a",
                 dev, prop.major, prop.minor);
   g_sms[dev] = prop.multiProcessorCount;
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
 
-  KernelFn ks[64];
-  int n = 0;
-  fwd_kernels<kSwiGLU, false>(ks, n);
-  fwd_kernels<kSwiGLU, true>(ks, n);
-  fwd_kernels<kSReLU, false>(ks, n);
-  fwd_kernels<kSReLU, true>(ks, n);
-  bwd_kernels<kSwiGLU, false>(ks, n);
-  bwd_kernels<kSwiGLU, true>(ks, n);
-  bwd_kernels<kSReLU, false>(ks, n);
-  bwd_kernels<kSReLU, true>(ks, n);
-  for (int i = 0; i < n; ++i) {
-    e = cudaFuncSetAttribute(ks[i], cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  FwdVariant fv[32];
+  BwdVariant bv[32];
+  int nf = 0, nb = 0;
+  fwd_all<kSwiGLU, false>(fv, nf);
+  fwd_all<kSwiGLU, true>(fv, nf);
+  fwd_all<kSReLU, false>(fv, nf);
+  fwd_all<kSReLU, true>(fv, nf);
+  bwd_all<kSwiGLU, false>(bv, nb);
+  bwd_all<kSwiGLU, true>(bv, nb);
+  bwd_all<kSReLU, false>(bv, nb);
+  bwd_all<kSReLU, true>(bv, nb);
+  for (int i = 0; i < nf; ++i) {
+    e = cudaFuncSetAttribute(fv[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fv[i].smem_fixed + kGroupSmem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
+  for (int i = 0; i < nb; ++i) {
+    e = cudaFuncSetAttribute(bv[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bv[i].smem_fixed + kGroupSmem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  }
+  e = cudaFuncSetAttribute(sigma_table_dump, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSigBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  e = cudaGetSymbolAddress(reinterpret_cast<void**>(&g_err_ptr[dev]), g_err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
 
   cudaStream_t st;
   e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
@@ -151,7 +191,7 @@ moeact_status check_shape(const void* x, int64_t ldx, const float* s, int64_t M,
   if (!x || !s) return fail(MOEACT_EINVAL, "x and s are required");
   if (M < 0) return fail(MOEACT_EINVAL, "M must be >= 0 (got %lld)", (long long)M);
   if (N <= 0 || N % 32 != 0) return fail(MOEACT_EINVAL, "N must be a positive multiple of 32 (got %lld)", (long long)N);
-  if (M > MOEACT_MAX_ROWS) return fail(MOEACT_ERANGE, "M above 2^36");
+  if (M > MOEACT_MAX_ROWS) return fail(MOEACT_ERANGE, "M above 2^30");
   if (N > (1 << 24)) return fail(MOEACT_ERANGE, "N above 2^24");
   const int64_t width = act == kSwiGLU ? 2 * N : N;
   if (ldx < width) return fail(MOEACT_EINVAL, "ldx (%lld) smaller than the input width %lld", (long long)ldx, (long long)width);
@@ -171,23 +211,14 @@ moeact_status check_groups(const int64_t* ro, const int64_t* cb, int32_t E, int3
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-struct WsLayout { size_t tickets_off, part_off, total; };
-WsLayout ws_layout(int64_t M, int64_t N, int32_t E) {
-  const int64_t slabs = ceil_div(M, 32) + (E > 0 ? E : 1);
-  const int64_t tiles = ceil_div(N, kTileCols);
-  WsLayout w;
-  w.tickets_off = 0;
-  w.part_off = (size_t)ceil_div(slabs * 4, 256) * 256;
-  w.total = w.part_off + (size_t)slabs * (size_t)tiles * 32 * 4;
-  return w;
+// Backward workspace: the dscale partials, one fp32 per (64-column tile, row).
+size_t ws_bytes_needed(int64_t M, int64_t N) {
+  return (size_t)ceil_div(N, kTileCols) * (size_t)M * 4;
 }
 
 // ------------------------------------------------------------ launches
-template <int ACT, int DIRS, bool STAGED, bool GROUPED>
-Variant fwd_variant() { return {act_fwd_kernel<ACT, DIRS, STAGED, GROUPED>, fwd_threads(ACT, DIRS)}; }
-
 template <int ACT, bool GROUPED>
-Variant pick_fwd(int dirs, bool staged) {
+FwdVariant pick_fwd(int dirs, bool staged) {
   if (ACT == kSwiGLU && staged) {
     if (dirs == kRow) return fwd_variant<ACT, kRow, true, GROUPED>();
     if (dirs == kCol) return fwd_variant<ACT, kCol, true, GROUPED>();
@@ -198,29 +229,39 @@ Variant pick_fwd(int dirs, bool staged) {
   return fwd_variant<ACT, kRow | kCol, false, GROUPED>();
 }
 
-template <int ACT, int DIRS, bool GROUPED>
-Variant bwd_variant() { return {act_bwd_kernel<ACT, DIRS, GROUPED>, bwd_threads(ACT, DIRS)}; }
-
 template <int ACT, bool GROUPED>
-Variant pick_bwd(int dirs) {
+BwdVariant pick_bwd(int dirs) {
   if (dirs == 0) return bwd_variant<ACT, 0, GROUPED>();
   if (dirs == kRow) return bwd_variant<ACT, kRow, GROUPED>();
   if (dirs == kCol) return bwd_variant<ACT, kCol, GROUPED>();
   return bwd_variant<ACT, kRow | kCol, GROUPED>();
 }
 
-moeact_status launch(Variant v, const Params& p, int dev, int64_t slabs_upper, int act,
-                     bool grouped, cudaStream_t st) {
-  const int64_t items = slabs_upper * p.n_tiles;
-  int64_t blocks = ceil_div(items, v.threads / 32);
-  if (blocks > g_sms[dev]) blocks = g_sms[dev];
-  if (blocks < 1) blocks = 1;
-  size_t smem = (act == kSwiGLU ? kSigBytes : 0) + (grouped ? (size_t)(p.E + 1 + 3) / 4 * 16 : 0);
-  v.fn<<<(unsigned)blocks, v.threads, smem, st>>>(p);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+// Tensor map of a bf16 [rows, width] matrix with a row stride of `ld`
+// elements, read in boxes of 64 columns x 16 rows; out-of-range elements read
+// as zero.  Encoded on the host for every call (no allocation).
+moeact_status make_map(CUtensorMap* map, const void* base, int64_t width, int64_t rows,
+                       int64_t ld) {
+  const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)kTileCols, (cuuint32_t)kHalfRows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MOEACT_OK;
 }
+
+int64_t grid_for(int64_t slabs_upper, int n_tiles, int threads, int dev) {
+  const int64_t items = slabs_upper * n_tiles;
+  int64_t blocks = ceil_div(items, threads / 32);
+  if (blocks > g_sms[dev]) blocks = g_sms[dev];
+  return blocks < 1 ? 1 : blocks;
+}
+
+int group_smem(bool grouped, int E) { return grouped ? group_bytes(E) : 0; }
 
 moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, int64_t M,
                          int64_t N, int dirs, int staged, const int64_t* ro, const int64_t* cb,
@@ -253,11 +294,18 @@ moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, in
   p.status = status;
   p.dense_slabs = ceil_div(M, 32);
   p.n_tiles = (int)ceil_div(N, kTileCols);
+  p.err = g_err_ptr[dev];
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
-  Variant v;
+  FwdVariant v;
   if (act == kSwiGLU) v = grouped ? pick_fwd<kSwiGLU, true>(dirs, staged) : pick_fwd<kSwiGLU, false>(dirs, staged);
   else v = grouped ? pick_fwd<kSReLU, true>(dirs, false) : pick_fwd<kSReLU, false>(dirs, false);
-  return launch(v, p, dev, slabs_upper, act, grouped, cs);
+  CUtensorMap tx;
+  if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
+  const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
+  v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(grouped, p.E), cs>>>(tx, p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return MOEACT_OK;
 }
 
 moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, int64_t ldx,
@@ -278,11 +326,11 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   if (dscale && !aligned(dscale, 4)) return fail(MOEACT_EALIGN, "dscale must be 4-byte aligned");
   if (dirs == 0 && !dx && !dscale) return fail(MOEACT_EINVAL, "nothing requested: dirs == 0 and no dx / dscale");
   if (grouped && (st = check_groups(ro, cb, E, status))) return st;
-  const WsLayout wl = ws_layout(M, N, grouped ? E : 1);
+  const size_t ws_need = ws_bytes_needed(M, N);
   if (dscale) {
     if (!ws) return fail(MOEACT_EWORKSPACE, "dscale needs a workspace");
     if (!aligned(ws, 16)) return fail(MOEACT_EALIGN, "workspace must be 16-byte aligned");
-    if (ws_bytes < wl.total) return fail(MOEACT_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, wl.total);
+    if (ws_bytes < ws_need) return fail(MOEACT_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, ws_need);
   }
   if (M == 0) return MOEACT_OK;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -303,21 +351,31 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   p.cs = out.col_scales;
   p.dx = static_cast<uint16_t*>(dx);
   p.dscale = dscale;
-  if (dscale) {
-    p.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + wl.tickets_off);
-    p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + wl.part_off);
-  }
+  if (dscale) p.part = static_cast<float*>(ws);
   p.row_offs = ro;
   p.cb_offs = cb;
   p.E = grouped ? E : 0;
   p.status = status;
   p.dense_slabs = ceil_div(M, 32);
   p.n_tiles = (int)ceil_div(N, kTileCols);
+  p.err = g_err_ptr[dev];
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
-  Variant v;
+  BwdVariant v;
   if (act == kSwiGLU) v = grouped ? pick_bwd<kSwiGLU, true>(dirs) : pick_bwd<kSwiGLU, false>(dirs);
   else v = grouped ? pick_bwd<kSReLU, true>(dirs) : pick_bwd<kSReLU, false>(dirs);
-  return launch(v, p, dev, slabs_upper, act, grouped, cs);
+  CUtensorMap tx, tdy;
+  if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
+  if ((st = make_map(&tdy, dy, N, M, lddy))) return st;
+  const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
+  v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(grouped, p.E), cs>>>(tx, tdy, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  if (dscale) {
+    dscale_reduce_kernel<<<(unsigned)ceil_div(M, 256), 256, 0, cs>>>(p.part, p.n_tiles, M, dscale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dscale reduction launch");
+  }
+  return MOEACT_OK;
 }
 
 }  // namespace
@@ -360,7 +418,7 @@ moeact_status splits_to_offsets(const int64_t* m_splits, int32_t num_groups, int
   if (num_groups < 0 || num_groups > MOEACT_MAX_GROUPS)
     return fail(MOEACT_EINVAL, "num_groups must be in [0, %d]", MOEACT_MAX_GROUPS);
   if (total_rows < 0) return fail(MOEACT_EINVAL, "total_rows must be >= 0");
-  if (total_rows > MOEACT_MAX_ROWS) return fail(MOEACT_ERANGE, "total_rows above 2^36");
+  if (total_rows > MOEACT_MAX_ROWS) return fail(MOEACT_ERANGE, "total_rows above 2^30");
   if ((m_splits && !aligned(m_splits, 8)) || !aligned(row_offs, 8) ||
       (colblk_offs && !aligned(colblk_offs, 8)) || !aligned(status, 4))
     return fail(MOEACT_EALIGN, "offsets must be 8-byte aligned, status 4-byte aligned");
@@ -407,8 +465,9 @@ moeact_status grouped_scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const f
 }
 
 size_t scaled_act_mxfp8_bwd_workspace_size(int64_t M, int64_t N, int32_t num_groups) {
+  (void)num_groups;
   if (M < 0 || N <= 0) return 0;
-  return ws_layout(M, N, num_groups > 0 ? num_groups : 1).total;
+  return ws_bytes_needed(M, N);
 }
 
 moeact_status scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x, int64_t ldx,
@@ -449,6 +508,23 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
                     status, dx, dscale, out, workspace, workspace_bytes, stream, true);
 }
 
+moeact_status moeact_device_error(uint32_t* flags) {
+  t_err[0] = 0;
+  if (!flags) return fail(MOEACT_EINVAL, "flags is required");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  *flags = 0;
+  if (dev < 0 || dev >= kMaxDevices || !g_ready[dev].load()) return MOEACT_OK;
+  uint32_t v = 0;
+  const uint32_t zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_err_word, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  *flags = v;
+  return MOEACT_OK;
+}
+
 moeact_status moeact_sigmoid_dump(float* out, void* stream) {
   t_err[0] = 0;
   if (!out) return fail(MOEACT_EINVAL, "out is required");
@@ -457,7 +533,7 @@ moeact_status moeact_sigmoid_dump(float* out, void* stream) {
   int dev;
   moeact_status st = ensure_ready(cs, &dev);
   if (st) return st;
-  sigma_table_dump<<<256, 256, 0, cs>>>(out);
+  sigma_table_dump<<<128, 256, kSigBytes, cs>>>(out);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sigmoid dump launch");
   return MOEACT_OK;

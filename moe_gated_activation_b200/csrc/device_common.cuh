@@ -25,15 +25,33 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr uint32_t kSigLo = 0x3300u;
 constexpr uint32_t kSigHi = 0x4300u;
 constexpr uint32_t kSigPerSign = kSigHi - kSigLo + 1;   // 4097
-constexpr int kSigEntries = 2 * kSigPerSign;            // 8194
+constexpr int kSigEntries = 2 * kSigPerSign;            // 8194 (global copy: +, then -)
 constexpr int kSigEntriesPadded = 8196;                 // whole float4s
-constexpr int kSigBytes = kSigEntriesPadded * 4;
+
+// Shared-memory copy: positive gates at float index m, negative gates at
+// 8192 + m (m = clamped magnitude - 0x3300), so that the sign bit of the bf16
+// (0x8000) is itself the byte offset 32768 between the two halves.
+constexpr int kSigNegOffset = 8192;
+constexpr int kSigBytes = (kSigNegOffset + kSigPerSign + 3) / 4 * 16;   // 49168
 
 __device__ __forceinline__ float sigma_lookup(const float* tab, uint32_t b16) {
   uint32_t a = b16 & 0x7FFFu;
   a = min(max(a, kSigLo), kSigHi) - kSigLo;
-  a += (b16 & 0x8000u) ? kSigPerSign : 0u;
+  a += (b16 & 0x8000u) ? kSigNegOffset : 0u;
   return tab[a];
+}
+
+// sigma of both bf16 values of a packed pair: both byte offsets are computed
+// at once in 16-bit lanes (clamp of the magnitude, minus the range start,
+// times 4, plus the sign bit as the 32 KiB offset of the negative half).
+__device__ __forceinline__ void sigma_pair(const float* tab, uint32_t G, float& s_lo,
+                                           float& s_hi) {
+  const uint32_t lo2 = kSigLo * 0x10001u, hi2 = kSigHi * 0x10001u;
+  const uint32_t c = __vimin3_u16x2(__vimax3_u16x2(G & 0x7FFF7FFFu, lo2, lo2), hi2, hi2);
+  const uint32_t off = (c - lo2) * 4u + (G & 0x80008000u);
+  const unsigned char* tb = reinterpret_cast<const unsigned char*>(tab);
+  s_lo = *reinterpret_cast<const float*>(tb + (off & 0xFFFFu));
+  s_hi = *reinterpret_cast<const float*>(tb + (off >> 16));
 }
 
 // ---------------------------------------------------------------- bf16
@@ -85,17 +103,70 @@ __device__ __forceinline__ uint32_t scale_multiplier(uint32_t b) {
 }
 
 // Two values -> two E4M3 codes (a in the low byte): nearest even of v * 2^(127-b),
-// saturating; a NaN-scale column gives 0x7F.
+// saturating.  For the NaN scale (b = 255) the multiplier is a NaN, the
+// product is NaN and the conversion gives the E4M3 NaN code 0x7F.
 __device__ __forceinline__ uint32_t e4m3x2(float a, uint32_t ma, float b, uint32_t mb) {
   const float2 v = make_float2(__fmul_rn(a, __uint_as_float(ma)),
                                __fmul_rn(b, __uint_as_float(mb)));
-  uint32_t q = (uint32_t)__nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, __NV_E4M3);
-  if (ma == kNanScale) q = (q & 0xFF00u) | 0x007Fu;
-  if (mb == kNanScale) q = (q & 0x00FFu) | 0x7F00u;
-  return q;
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+// A copy of v the compiler cannot see through: used so that a later pass
+// recomputes per-row addresses instead of keeping an earlier pass's live.
+__device__ __forceinline__ int opaque(int v) {
+  int r;
+  asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t f32_mag(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+// ---------------------------------------------------------------- TMA / mbarrier
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+               "selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Waits for a phase of `bar` with an iteration limit (each try_wait may itself
+// suspend for a short, hardware-chosen time); false on timeout.
+constexpr uint32_t kSpinLimit = 1u << 22;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// 2-D TMA tile load (no multicast) of box {x .. x+bx, y .. y+by} into shared
+// memory, completing on `bar`; rows and columns outside the tensor read zero.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y),
+        "r"(smem_addr(bar))
+      : "memory");
+}
 
 // ---------------------------------------------------------------- warp butterflies
 // "Transposed" butterfly: each lane holds one value per row for 2*HALF rows;
@@ -109,8 +180,8 @@ __device__ __forceinline__ void bfly_max_u32(uint32_t* a, int lane, int off) {
   const bool up = (lane & off) != 0;
 #pragma unroll
   for (int i = 0; i < HALF; ++i) {
-    const uint32_t keep = up ? a[HALF + i] : a[i];
     const uint32_t send = up ? a[i] : a[HALF + i];
+    const uint32_t keep = a[i] ^ a[HALF + i] ^ send;
     a[i] = max(keep, __shfl_xor_sync(kFull, send, off));
   }
 }
@@ -121,8 +192,8 @@ __device__ __forceinline__ void bfly_max_u16x2(uint32_t* a, int lane, int off) {
   const bool up = (lane & off) != 0;
 #pragma unroll
   for (int i = 0; i < HALF; ++i) {
-    const uint32_t keep = up ? a[HALF + i] : a[i];
     const uint32_t send = up ? a[i] : a[HALF + i];
+    const uint32_t keep = a[i] ^ a[HALF + i] ^ send;
     a[i] = __vmaxu2(keep, __shfl_xor_sync(kFull, send, off));
   }
 }
@@ -132,8 +203,9 @@ __device__ __forceinline__ void bfly_sum_f32(float* a, int lane, int off) {
   const bool up = (lane & off) != 0;
 #pragma unroll
   for (int i = 0; i < HALF; ++i) {
-    const float keep = up ? a[HALF + i] : a[i];
     const float send = up ? a[i] : a[HALF + i];
+    const float keep = __uint_as_float(__float_as_uint(a[i]) ^ __float_as_uint(a[HALF + i]) ^
+                                       __float_as_uint(send));
     a[i] = __fadd_rn(keep, __shfl_xor_sync(kFull, send, off));
   }
 }

@@ -17,14 +17,26 @@
 // 32 rows (one colwise block, never crossing an expert boundary) x 64
 // columns; lane l owns columns 2l and 2l+1 for all 32 rows, so the colwise
 // amax is a per-lane loop over registers and the rowwise 1x32 amax is a
-// 16-lane reduction.  The grid is persistent (one CTA per SM, the
-// sigmoid table staged once per CTA in shared memory); warps walk the items
+// 16-lane reduction.  The grid is persistent (one CTA per SM, the sigmoid
+// table staged once per CTA in shared memory); warps walk the items
 // slab-major so that neighbouring warps read neighbouring columns of the same
-// rows.  All loads and stores are coalesced: a warp moves 128 contiguous bytes
-// of each bf16 input row, and 64 contiguous bytes of each code row.
+// rows.
+//
+// Data movement.  Each warp owns a ring of shared-memory slots, each holding
+// one 16-row half of a warp-tile's inputs ([16 x 64] bf16 per operand), filled
+// by TMA (cp.async.bulk.tensor, no multicast) and signalled through one
+// mbarrier per slot.  Lane 0 keeps two half-tiles in flight ahead of the one
+// being computed, so the warp never waits on global-memory latency and the
+// inputs never occupy registers; rows and columns outside the tensor arrive
+// as zeros.  Lanes read their two columns of each row from shared memory
+// (conflict-free: a warp reads one 128-byte row).  Codes, scales and
+// gradients are stored directly, 64 (codes) or 128 (bf16) contiguous bytes
+// per warp per row; full tiles take a path without bounds predicates.
 #pragma once
 
 #include <cstdint>
+
+#include <cuda.h>
 
 #include "device_common.cuh"
 
@@ -34,14 +46,6 @@ enum Act : int { kSwiGLU = 0, kSReLU = 1 };
 constexpr int kRow = 1;
 constexpr int kCol = 2;
 constexpr int kTileCols = 64;
-
-// CTA size per variant: 512 threads (128 registers each) where the live set
-// fits, 384 (up to 168 registers) for the variants that keep 64 colwise
-// values plus a second half of in-flight loads, so that nothing spills.
-__host__ __device__ constexpr int fwd_threads(int act, int dirs) { return (dirs == 3 && act >= 0) ? 384 : 512; }
-__host__ __device__ constexpr int bwd_threads(int act, int dirs) {
-  return (dirs == 3 || (act == 0 && dirs != 0)) ? 384 : 512;
-}
 
 // The table lives in device global memory of this module: one copy per
 // device, written by sigma_table_init before any activation kernel reads it.
@@ -86,13 +90,21 @@ __global__ void sigma_table_init(int* uncertain) {
   g_sigma_table[i] = f;
 }
 
-// Expands the table to all 65536 bf16 patterns (test hook).
+// Expands the table to all 65536 bf16 patterns (test hook), through the same
+// shared-memory layout and pair lookup the fused kernels use: thread t looks
+// up the packed pair (2t, 2t + 1).
 __global__ void sigma_table_dump(float* out) {
-  __shared__ float tab[kSigEntriesPadded];
-  for (int i = threadIdx.x; i < kSigEntriesPadded; i += blockDim.x) tab[i] = g_sigma_table[i];
+  extern __shared__ __align__(16) float tab[];
+  for (int i = threadIdx.x; i < kSigEntries; i += blockDim.x)
+    tab[i < (int)kSigPerSign ? i : i - (int)kSigPerSign + kSigNegOffset] = g_sigma_table[i];
   __syncthreads();
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < 65536) out[b] = sigma_lookup(tab, (uint32_t)b);
+  const uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < 32768) {
+    float a, b;
+    sigma_pair(tab, (2 * t) | ((2 * t + 1) << 16), a, b);
+    out[2 * t] = a;
+    out[2 * t + 1] = b;
+  }
 }
 
 // ---------------------------------------------------------------- offsets
@@ -156,6 +168,19 @@ __global__ void __launch_bounds__(1024) splits_kernel(const int64_t* __restrict_
   if (t == 0) { ro[E] = total; if (cb) cb[E] = s_c[(blockDim.x >> 5) - 1]; }
 }
 
+// ---------------------------------------------------------------- dscale sum
+// dscale[row] = sum over tiles t = 0, 1, ... of part[t][row], in that order.
+__global__ void __launch_bounds__(256) dscale_reduce_kernel(const float* __restrict__ part,
+                                                            int n_tiles, int64_t M,
+                                                            float* __restrict__ dscale) {
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= M) return;
+  float acc = 0.0f;
+#pragma unroll 8
+  for (int t = 0; t < n_tiles; ++t) acc = __fadd_rn(acc, __ldcg(part + (int64_t)t * M + row));
+  dscale[row] = acc;
+}
+
 // ---------------------------------------------------------------- fused kernels
 struct Params {
   const uint16_t* x;
@@ -172,26 +197,56 @@ struct Params {
   uint8_t* cs;
   uint16_t* dx;
   float* dscale;
-  float* part;        // dscale partials [slabs][tiles][32]
-  uint32_t* tickets;  // [slabs]
+  float* part;        // dscale partials [n_tiles][M] (tile-major)
   const int64_t* row_offs;
   const int64_t* cb_offs;
   int E;
   int32_t* status;
   int64_t dense_slabs;
   int n_tiles;
+  uint32_t* err;      // device error word (timeouts), never expected to be set
 };
 
-// Stages the sigmoid table (and, grouped, the col-block offsets) in shared
-// memory and validates grouped offsets.  Returns the slab count, or -1 if the
-// offsets are not those of valid splits (every CTA reaches the same verdict;
-// CTA 0 writes the status word).
+constexpr int kSlots = 3;            // half-tile slots per warp
+constexpr int kHalfRows = 16;
+constexpr int kOperandHalfBytes = kHalfRows * kTileCols * 2;   // 2 KiB
+
+// Threads per CTA: one CTA per SM; the shared memory of the warps' rings
+// (slots x operands x 2 KiB) plus the sigmoid table bounds the warp count.
+__host__ __device__ constexpr int fwd_warps(int act) { return act == 0 ? 12 : 12; }
+__host__ __device__ constexpr int bwd_warps(int act) { return act == 0 ? 8 : 12; }
+__host__ __device__ constexpr int fwd_threads(int act, int dirs) { return 32 * fwd_warps(act) + 0 * dirs; }
+__host__ __device__ constexpr int bwd_threads(int act, int dirs) { return 32 * bwd_warps(act) + 0 * dirs; }
+__host__ __device__ constexpr int fwd_operands(int act) { return act == 0 ? 2 : 1; }
+__host__ __device__ constexpr int bwd_operands(int act) { return act == 0 ? 3 : 2; }
+__host__ __device__ constexpr int ring_bytes(int warps, int operands) {
+  return warps * kSlots * operands * kOperandHalfBytes;
+}
+
+// Shared-memory layout of a CTA: [rings][sigmoid table][col-block offsets][mbarriers]
+// (E < 0: without the col-block offsets, which the launcher adds for grouped calls)
+// (128 bytes of slack let the kernel align the base for the TMA destinations;
+// a grouped call adds its row and col-block offsets as two int32 arrays)
+__host__ __device__ constexpr int group_bytes(int E) { return 2 * ((E + 1 + 3) / 4) * 16; }
+__host__ __device__ constexpr int smem_bytes(int warps, int operands, bool sig, int E) {
+  return 128 + ring_bytes(warps, operands) + (sig ? kSigBytes : 0) +
+         (E < 0 ? 0 : group_bytes(E)) + warps * kSlots * 8;
+}
+
+__device__ __forceinline__ unsigned char* align_smem(unsigned char* p) {
+  return p + ((128u - (smem_addr(p) & 127u)) & 127u);
+}
+
+// Stages the sigmoid table (and, grouped, the row and col-block offsets as
+// int32) in shared memory and validates grouped offsets.  Returns the slab
+// count, or -1 if the offsets are not those of valid splits (every CTA reaches
+// the same verdict; CTA 0 writes the status word).
 template <bool NEED_SIG, bool GROUPED>
-__device__ __forceinline__ int64_t stage_and_validate(const Params& p, float* sig_s, int* cb_s) {
+__device__ __forceinline__ int64_t stage_and_validate(const Params& p, float* sig_s, int* cb_s,
+                                                      int* ro_s) {
   if (NEED_SIG) {
-    const float4* src = reinterpret_cast<const float4*>(g_sigma_table);
-    float4* dst = reinterpret_cast<float4*>(sig_s);
-    for (int i = threadIdx.x; i < kSigEntriesPadded / 4; i += blockDim.x) dst[i] = src[i];
+    for (int i = threadIdx.x; i < kSigEntries; i += blockDim.x)
+      sig_s[i < (int)kSigPerSign ? i : i - (int)kSigPerSign + kSigNegOffset] = g_sigma_table[i];
   }
   int bad = 0;
   if (GROUPED) {
@@ -208,6 +263,7 @@ __device__ __forceinline__ int64_t stage_and_validate(const Params& p, float* si
       if (e == p.E) ok = ok && (r == p.M);
       if (!ok) bad = 1;
       cb_s[e] = (int)c;
+      ro_s[e] = (int)r;
     }
   }
   bad = __syncthreads_or(bad);
@@ -216,10 +272,11 @@ __device__ __forceinline__ int64_t stage_and_validate(const Params& p, float* si
   return bad ? -1 : (int64_t)cb_s[p.E];
 }
 
-// Rows of slab `slab`: first row and count (<= 32).
+// Rows of slab `slab`: first row and count (<= 32).  Grouped offsets come from
+// shared memory (int32: rows are below 2^30).
 template <bool GROUPED>
-__device__ __forceinline__ void slab_rows(const Params& p, const int* cb_s, int64_t slab,
-                                          int64_t& row0, int& nrows) {
+__device__ __forceinline__ void slab_rows(const Params& p, const int* cb_s, const int* ro_s,
+                                          int64_t slab, int64_t& row0, int& nrows) {
   if (!GROUPED) {
     row0 = slab * 32;
     nrows = (int)min((int64_t)32, p.M - row0);
@@ -231,9 +288,9 @@ __device__ __forceinline__ void slab_rows(const Params& p, const int* cb_s, int6
       const int mid = (lo + hi + 1) >> 1;
       if (cb_s[mid] <= sl) lo = mid; else hi = mid - 1;
     }
-    const int64_t r_e = __ldg(p.row_offs + lo), r_e1 = __ldg(p.row_offs + lo + 1);
-    row0 = r_e + 32 * (int64_t)(sl - cb_s[lo]);
-    nrows = (int)min((int64_t)32, r_e1 - row0);
+    const int r0 = ro_s[lo] + 32 * (sl - cb_s[lo]);
+    row0 = r0;
+    nrows = min(32, ro_s[lo + 1] - r0);
   }
 }
 
@@ -250,43 +307,79 @@ __device__ __forceinline__ void store_row_scales(uint8_t* dst, uint32_t b0, uint
   }
 }
 
+// ------------------------------------------------------------- the warp's ring
+// Half-tile k of a warp is half (k & 1) of its (k >> 1)-th work item; it lives
+// in slot k % kSlots, whose mbarrier completes once per use (parity
+// (k / kSlots) & 1).
+struct Ring {
+  unsigned char* slots;   // kSlots * OPS * 2 KiB
+  uint64_t* bars;         // kSlots
+  int ops;
+};
+
+template <bool GROUPED>
+__device__ __forceinline__ void issue_half(const Params& p, const int* cb_s, const int* ro_s,
+                                           const Ring& r,
+                                           const void* tm_x, const void* tm_dy, int64_t item,
+                                           int k, bool swiglu, bool with_dy) {
+  const int64_t slab = item / p.n_tiles;
+  const int tile = (int)(item - slab * p.n_tiles);
+  int64_t row0;
+  int nrows;
+  slab_rows<GROUPED>(p, cb_s, ro_s, slab, row0, nrows);
+  const int slot = k % kSlots;
+  unsigned char* dst = r.slots + slot * r.ops * kOperandHalfBytes;
+  uint64_t* bar = r.bars + slot;
+  const int x = tile * kTileCols, y = (int)row0 + (k & 1) * kHalfRows;
+  mbar_expect_tx(bar, r.ops * kOperandHalfBytes);
+  int o = 0;
+  if (with_dy) tma_load_2d(dst + (o++) * kOperandHalfBytes, tm_dy, x, y, bar);
+  tma_load_2d(dst + (o++) * kOperandHalfBytes, tm_x, x, y, bar);
+  if (swiglu) tma_load_2d(dst + (o++) * kOperandHalfBytes, tm_x, x + p.N, y, bar);
+}
+
+__device__ __forceinline__ void report_timeout(const Params& p, uint32_t code) {
+  atomicOr(p.err, code);
+}
+
 // ------------------------------------------------------------- forward tile
-// Rowwise work runs in two halves of 16 rows so that only 16 per-row block
-// maxima are live at a time: after the 4-step butterfly (off = 8, 4, 2, 1) lane
-// l holds the amax of row 16h + (l & 15) in block (l >> 4).
-template <int ACT, int DIRS, bool STAGED>
-__device__ __forceinline__ void fwd_tile(const Params& p, const float* sig, int64_t slab,
-                                         int tile, int64_t row0, int nrows, int lane) {
+// Rowwise work runs per 16-row half: after the 4-step butterfly (off = 8, 4,
+// 2, 1) lane l holds the amax of row 16h + (l & 15) in block (l >> 4).
+template <int ACT, int DIRS, bool STAGED, bool GROUPED, bool FULL>
+__device__ __forceinline__ void fwd_tile(const Params& p, const float* sig, const Ring& ring,
+                                         int k0, int64_t slab, int tile, int64_t row0, int nrows,
+                                         int lane, const int* cb_s, const int* ro_s,
+                                         const void* tm_x, int64_t next_item0,
+                                         int64_t next_item1, int K, bool& ok_flag) {
   const int c0 = tile * kTileCols + 2 * lane;
   const bool colok = c0 < p.N;
-  const uint16_t* xb = p.x + row0 * p.ldx + c0;
   const int W = p.W;
-
-  uint32_t G[32], U[32];
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    const bool ok = colok && r < nrows;
-    const unsigned int* px = reinterpret_cast<const unsigned int*>(xb + (int64_t)r * p.ldx);
-    G[r] = ok ? __ldcs(px) : 0u;
-    if (ACT == kSwiGLU) U[r] = ok ? __ldcs(px + (p.N >> 1)) : 0u;
-  }
+  const int Wh = W >> 1;
   const float sv = lane < nrows ? __ldg(p.s + row0 + lane) : 0.0f;
 
   float Y0[32], Y1[32];
   uint32_t bh[2];
-  uint8_t* rqb = p.rq + row0 * (int64_t)W + c0;
+  unsigned short* rqb = reinterpret_cast<unsigned short*>(p.rq + row0 * (int64_t)W + c0);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
+    const int k = k0 + h;
+    const int slot = k % kSlots;
+    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / kSlots) & 1u)) { ok_flag = false; return; }
+    const unsigned char* sm = ring.slots + slot * ring.ops * kOperandHalfBytes + 4 * lane;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int r = 16 * h + i;
+      const uint32_t G = *reinterpret_cast<const uint32_t*>(sm + i * 128);
       const float sr = __shfl_sync(kFull, sv, r);
       float h0, h1;
       if (ACT == kSwiGLU) {
-        const float g0 = bf16_lo(G[r]), g1 = bf16_hi(G[r]);
-        const float u0 = bf16_lo(U[r]), u1 = bf16_hi(U[r]);
-        const float si0 = __fmul_rn(g0, sigma_lookup(sig, G[r] & 0xFFFFu));
-        const float si1 = __fmul_rn(g1, sigma_lookup(sig, G[r] >> 16));
+        const uint32_t U = *reinterpret_cast<const uint32_t*>(sm + kOperandHalfBytes + i * 128);
+        const float g0 = bf16_lo(G), g1 = bf16_hi(G);
+        const float u0 = bf16_lo(U), u1 = bf16_hi(U);
+        float sg0, sg1;
+        sigma_pair(sig, G, sg0, sg1);
+        const float si0 = __fmul_rn(g0, sg0);
+        const float si1 = __fmul_rn(g1, sg1);
         if (STAGED) {
           h0 = bf16_round(__fmul_rn(bf16_round(si0), u0));
           h1 = bf16_round(__fmul_rn(bf16_round(si1), u1));
@@ -295,12 +388,21 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const float* sig, int6
           h1 = __fmul_rn(si1, u1);
         }
       } else {
-        const float r0 = relu_keep_nan(bf16_lo(G[r])), r1 = relu_keep_nan(bf16_hi(G[r]));
+        const float r0 = relu_keep_nan(bf16_lo(G)), r1 = relu_keep_nan(bf16_hi(G));
         h0 = __fmul_rn(r0, r0);
         h1 = __fmul_rn(r1, r1);
       }
       Y0[r] = __fmul_rn(h0, sr);
       Y1[r] = __fmul_rn(h1, sr);
+      if (!FULL && r >= nrows) { Y0[r] = 0.0f; Y1[r] = 0.0f; }
+    }
+    // the slot is consumed: refill it with the half-tile kSlots ahead
+    __syncwarp();
+    if (lane == 0 && k + kSlots < K) {
+      const int kn = k + kSlots;
+      issue_half<GROUPED>(p, cb_s, ro_s, ring, tm_x, nullptr,
+                          (kn >> 1) == (k0 >> 1) + 1 ? next_item0 : next_item1, kn,
+                          ACT == kSwiGLU, false);
     }
     if (DIRS & kRow) {
       uint32_t A[16];
@@ -317,8 +419,7 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const float* sig, int6
         const int r = 16 * h + i;
         const uint32_t m = __shfl_sync(kFull, mh, (lane & 16) | i);
         const uint32_t q = e4m3x2(Y0[r], m, Y1[r], m);
-        if (colok && r < nrows)
-          __stcs(reinterpret_cast<unsigned short*>(rqb + (int64_t)r * W), (unsigned short)q);
+        if (FULL || (colok && r < nrows)) __stcs(rqb + r * Wh, (unsigned short)q);
       }
     }
   }
@@ -336,116 +437,151 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const float* sig, int6
   if (DIRS & kCol) {
     uint32_t a0 = 0u, a1 = 0u;
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      a0 = max(a0, f32_mag(Y0[r]));
-      a1 = max(a1, f32_mag(Y1[r]));
+    for (int r = 0; r < 32; r += 2) {
+      a0 = __vimax3_u32(a0, f32_mag(Y0[r]), f32_mag(Y0[r + 1]));
+      a1 = __vimax3_u32(a1, f32_mag(Y1[r]), f32_mag(Y1[r + 1]));
     }
     const uint32_t b0 = e8m0_from_amax(a0), b1 = e8m0_from_amax(a1);
     const uint32_t m0 = scale_multiplier(b0), m1 = scale_multiplier(b1);
     if (colok)
       __stcs(reinterpret_cast<unsigned short*>(p.cs + slab * (int64_t)W + c0),
              (unsigned short)(b0 | (b1 << 8)));
-    uint8_t* qb = p.cq + row0 * (int64_t)W + c0;
+    unsigned short* qb = reinterpret_cast<unsigned short*>(p.cq + row0 * (int64_t)W + c0);
+    const int Whc = opaque(Wh);
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
       const uint32_t q = e4m3x2(Y0[r], m0, Y1[r], m1);
-      if (colok && r < nrows)
-        __stcs(reinterpret_cast<unsigned short*>(qb + (int64_t)r * W), (unsigned short)q);
+      if (FULL || (colok && r < nrows)) __stcs(qb + r * Whc, (unsigned short)q);
     }
   }
 }
 
+// Sets up the warp's ring (barriers initialised by lane 0) and primes it.
+template <bool GROUPED>
+__device__ __forceinline__ void ring_prime(const Params& p, const int* cb_s, const int* ro_s,
+                                           const Ring& ring,
+                                           const void* tm_x, const void* tm_dy, int64_t first,
+                                           int64_t stride, int K, int lane, bool swiglu,
+                                           bool with_dy) {
+  if (lane == 0) {
+    for (int i = 0; i < kSlots; ++i) mbar_init(ring.bars + i, 1);
+    mbar_init_fence();
+    for (int k = 0; k < kSlots && k < K; ++k)
+      issue_half<GROUPED>(p, cb_s, ro_s, ring, tm_x, tm_dy, first + (k >> 1) * stride, k, swiglu,
+                          with_dy);
+  }
+  __syncwarp();
+}
+
+// After a timeout: bounded waits for the copies still in flight into this
+// warp's slots, so that none lands after the CTA has exited.
+__device__ __forceinline__ void ring_drain(const Ring& ring, int k_next, int K) {
+  for (int k = k_next; k < K && k < k_next + kSlots; ++k)
+    mbar_wait(ring.bars + (k % kSlots), (uint32_t)(k / kSlots) & 1u);
+}
+
 template <int ACT, int DIRS, bool STAGED, bool GROUPED>
-__global__ void __launch_bounds__(fwd_threads(ACT, DIRS), 1) act_fwd_kernel(const Params p) {
-  constexpr int kWarps = fwd_threads(ACT, DIRS) / 32;
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* sig_s = reinterpret_cast<float*>(smem);
-  int* cb_s = reinterpret_cast<int*>(smem + (ACT == kSwiGLU ? kSigBytes : 0));
-  const int64_t n_slabs = stage_and_validate<ACT == kSwiGLU, GROUPED>(p, sig_s, cb_s);
+__global__ void __launch_bounds__(fwd_threads(ACT, DIRS), 1)
+    act_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const Params p) {
+  constexpr int kWarps = fwd_warps(ACT);
+  constexpr int kOps = fwd_operands(ACT);
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char* smem = align_smem(smem_raw);
+  float* sig_s = reinterpret_cast<float*>(smem + ring_bytes(kWarps, kOps));
+  int* cb_s = reinterpret_cast<int*>(smem + ring_bytes(kWarps, kOps) +
+                                     (ACT == kSwiGLU ? kSigBytes : 0));
+  int* ro_s = cb_s + (GROUPED ? ((p.E + 1 + 3) / 4) * 4 : 0);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      smem + ring_bytes(kWarps, kOps) + (ACT == kSwiGLU ? kSigBytes : 0) +
+      (GROUPED ? group_bytes(p.E) : 0));
+  const int64_t n_slabs = stage_and_validate<ACT == kSwiGLU, GROUPED>(p, sig_s, cb_s, ro_s);
   if (n_slabs < 0) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n_items = n_slabs * p.n_tiles;
-  for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < n_items;
-       it += (int64_t)gridDim.x * kWarps) {
+  const int64_t first = (int64_t)blockIdx.x * kWarps + warp;
+  const int64_t stride = (int64_t)gridDim.x * kWarps;
+  const int count = first < n_items ? (int)((n_items - 1 - first) / stride + 1) : 0;
+  const int K = 2 * count;
+  Ring ring{smem + warp * kSlots * kOps * kOperandHalfBytes, bars + warp * kSlots, kOps};
+  ring_prime<GROUPED>(p, cb_s, ro_s, ring, &tm_x, nullptr, first, stride, K, lane, ACT == kSwiGLU,
+                      false);
+  bool ok = true;
+  for (int j = 0; j < count; ++j) {
+    const int64_t it = first + j * stride;
     const int64_t slab = it / p.n_tiles;
     const int tile = (int)(it - slab * p.n_tiles);
     int64_t row0;
     int nrows;
-    slab_rows<GROUPED>(p, cb_s, slab, row0, nrows);
-    fwd_tile<ACT, DIRS, STAGED>(p, sig_s, slab, tile, row0, nrows, lane);
+    slab_rows<GROUPED>(p, cb_s, ro_s, slab, row0, nrows);
+    const bool full = nrows == 32 && (tile + 1) * kTileCols <= p.N;
+    const int64_t n1 = it + stride, n2 = it + 2 * stride;
+    if (full)
+      fwd_tile<ACT, DIRS, STAGED, GROUPED, true>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
+                                        cb_s, ro_s, &tm_x, n1, n2, K, ok);
+    else
+      fwd_tile<ACT, DIRS, STAGED, GROUPED, false>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
+                                         cb_s, ro_s, &tm_x, n1, n2, K, ok);
+    if (!ok) {
+      if (lane == 0) {
+        report_timeout(p, 1u);
+        ring_drain(ring, 2 * j, K);
+      }
+      return;
+    }
   }
 }
 
 // ------------------------------------------------------------- backward tile
-// dscale: each warp reduces its 32 rows x 64 columns to one partial per row,
-// writes it to the workspace (lane = row), and takes a ticket on the slab;
-// the warp that takes the last ticket sums the slab's partials in tile order
-// (a fixed order, so dscale is deterministic) and resets the ticket.  No warp
-// ever waits on another.
-__device__ __forceinline__ void dscale_publish(const Params& p, float v, int64_t slab,
-                                               int tile, int64_t row0, int nrows, int lane) {
-  float* base = p.part + slab * (int64_t)p.n_tiles * 32;
-  __stcg(base + tile * 32 + lane, v);
-  __threadfence();
-  __syncwarp();
-  unsigned int t = 0;
-  if (lane == 0) t = atomicAdd(p.tickets + slab, 1u);
-  t = __shfl_sync(kFull, t, 0);
-  if (t == (unsigned int)p.n_tiles - 1) {
-    __threadfence();
-    float acc = 0.0f;
-#pragma unroll 8
-    for (int k = 0; k < p.n_tiles; ++k) acc = __fadd_rn(acc, __ldcg(base + k * 32 + lane));
-    if (lane < nrows) p.dscale[row0 + lane] = acc;
-    if (lane == 0) p.tickets[slab] = 0u;
-  }
-}
+// dscale: each warp reduces its 32 rows x 64 columns to one partial per row
+// and stores it, lane = row, into the workspace at [tile][row] -- plain
+// stores, no fences or counters.  dscale_reduce_kernel, launched right after
+// on the same stream, sums each row's partials in tile order (a fixed order,
+// so dscale is deterministic).
 
-// Row-direction work (dx stores, dscale partials, rowwise MXFP8) runs in two
-// halves of 16 rows; the packed bf16 gradients of all 32 rows stay in
-// registers for the colwise pass.
-template <int ACT, int DIRS>
-__device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, int64_t slab,
-                                         int tile, int64_t row0, int nrows, int lane) {
+// Row-direction work (dx stores, dscale partials, rowwise MXFP8) runs per
+// 16-row half as the half arrives; the packed bf16 gradients of all 32 rows
+// stay in registers for the colwise pass.
+template <int ACT, int DIRS, bool GROUPED, bool FULL>
+__device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, const Ring& ring,
+                                         int k0, int64_t slab, int tile, int64_t row0, int nrows,
+                                         int lane, const int* cb_s, const int* ro_s,
+                                         const void* tm_x, const void* tm_dy,
+                                         int64_t next_item0, int64_t next_item1, int K,
+                                         bool& ok_flag) {
   const int N = p.N, W = p.W;
+  const int Wh = W >> 1;
   const int c0 = tile * kTileCols + 2 * lane;
   const bool colok = c0 < N;
-  const uint16_t* xb = p.x + row0 * p.ldx + c0;
-  const uint16_t* db = p.dy + row0 * p.lddy + c0;
-
   const float sv = lane < nrows ? __ldg(p.s + row0 + lane) : 0.0f;
+
   uint32_t DG[32], DU[32];
   float ph[2];
   uint32_t bh[2];
-  uint8_t* rqb = p.rq + row0 * (int64_t)W + c0;
+  unsigned short* rqb = reinterpret_cast<unsigned short*>(p.rq + row0 * (int64_t)W + c0);
+  uint32_t* dxb = reinterpret_cast<uint32_t*>(p.dx + row0 * (int64_t)W + c0);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    // The inputs of each 16-row half are loaded when the half starts (a
-    // compiler barrier keeps the second half's loads after the first half's
-    // work), which bounds the live registers without spilling.
-    asm volatile("" ::: "memory");
-    uint32_t D[32], G[32], U[32];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int r = 16 * h + i;
-      const bool ok = colok && r < nrows;
-      const unsigned int* px = reinterpret_cast<const unsigned int*>(xb + (int64_t)r * p.ldx);
-      D[r] = ok ? __ldcs(reinterpret_cast<const unsigned int*>(db + (int64_t)r * p.lddy)) : 0u;
-      G[r] = ok ? __ldcs(px) : 0u;
-      if (ACT == kSwiGLU) U[r] = ok ? __ldcs(px + (N >> 1)) : 0u;
-    }
+    const int k = k0 + h;
+    const int slot = k % kSlots;
+    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / kSlots) & 1u)) { ok_flag = false; return; }
+    const unsigned char* sm = ring.slots + slot * ring.ops * kOperandHalfBytes + 4 * lane;
     float P[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int r = 16 * h + i;
+      const uint32_t D = *reinterpret_cast<const uint32_t*>(sm + i * 128);
+      const uint32_t G = *reinterpret_cast<const uint32_t*>(sm + kOperandHalfBytes + i * 128);
       const float sr = __shfl_sync(kFull, sv, r);
-      const float d0 = bf16_lo(D[r]), d1 = bf16_hi(D[r]);
+      const float d0 = bf16_lo(D), d1 = bf16_hi(D);
       const float p0 = __fmul_rn(d0, sr), p1 = __fmul_rn(d1, sr);
       float h0, h1;
       if (ACT == kSwiGLU) {
-        const float g0 = bf16_lo(G[r]), g1 = bf16_hi(G[r]);
-        const float u0 = bf16_lo(U[r]), u1 = bf16_hi(U[r]);
-        const float s0 = sigma_lookup(sig, G[r] & 0xFFFFu), s1 = sigma_lookup(sig, G[r] >> 16);
+        const uint32_t U =
+            *reinterpret_cast<const uint32_t*>(sm + 2 * kOperandHalfBytes + i * 128);
+        const float g0 = bf16_lo(G), g1 = bf16_hi(G);
+        const float u0 = bf16_lo(U), u1 = bf16_hi(U);
+        float s0, s1;
+        sigma_pair(sig, G, s0, s1);
         const float si0 = __fmul_rn(g0, s0), si1 = __fmul_rn(g1, s1);
         const float ds0 = __fmaf_rn(si0, __fsub_rn(1.0f, s0), s0);
         const float ds1 = __fmaf_rn(si1, __fsub_rn(1.0f, s1), s1);
@@ -454,18 +590,25 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, int6
         h0 = __fmul_rn(si0, u0);
         h1 = __fmul_rn(si1, u1);
       } else {
-        const float r0 = relu_keep_nan(bf16_lo(G[r])), r1 = relu_keep_nan(bf16_hi(G[r]));
+        const float r0 = relu_keep_nan(bf16_lo(G)), r1 = relu_keep_nan(bf16_hi(G));
         DG[r] = pack_bf16x2(__fmul_rn(p0, __fmul_rn(2.0f, r0)), __fmul_rn(p1, __fmul_rn(2.0f, r1)));
         DU[r] = 0u;
         h0 = __fmul_rn(r0, r0);
         h1 = __fmul_rn(r1, r1);
       }
       P[i] = __fmaf_rn(d1, h1, __fmul_rn(d0, h0));
-      if (p.dx != nullptr && colok && r < nrows) {
-        uint16_t* o = p.dx + (row0 + r) * (int64_t)W + c0;
-        __stcs(reinterpret_cast<unsigned int*>(o), DG[r]);
-        if (ACT == kSwiGLU) __stcs(reinterpret_cast<unsigned int*>(o + N), DU[r]);
+      if (!FULL && r >= nrows) { DG[r] = 0u; DU[r] = 0u; P[i] = 0.0f; }
+      if (p.dx != nullptr && (FULL || (colok && r < nrows))) {
+        __stcs(dxb + r * Wh, DG[r]);
+        if (ACT == kSwiGLU) __stcs(dxb + r * Wh + (N >> 1), DU[r]);
       }
+    }
+    __syncwarp();
+    if (lane == 0 && k + kSlots < K) {
+      const int kn = k + kSlots;
+      issue_half<GROUPED>(p, cb_s, ro_s, ring, tm_x, tm_dy,
+                          (kn >> 1) == (k0 >> 1) + 1 ? next_item0 : next_item1, kn,
+                          ACT == kSwiGLU, true);
     }
     if (p.dscale != nullptr) {
       // lane l ends with the warp sum of row 16h + (l >> 1)
@@ -502,10 +645,9 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, int6
           const uint32_t mu = __shfl_sync(kFull, muh, src);
           qu = e4m3x2(bf16_lo(DU[r]), mu, bf16_hi(DU[r]), mu);
         }
-        if (colok && r < nrows) {
-          __stcs(reinterpret_cast<unsigned short*>(rqb + (int64_t)r * W), (unsigned short)qg);
-          if (ACT == kSwiGLU)
-            __stcs(reinterpret_cast<unsigned short*>(rqb + (int64_t)r * W + N), (unsigned short)qu);
+        if (FULL || (colok && r < nrows)) {
+          __stcs(rqb + r * Wh, (unsigned short)qg);
+          if (ACT == kSwiGLU) __stcs(rqb + r * Wh + (N >> 1), (unsigned short)qu);
         }
       }
     }
@@ -513,7 +655,7 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, int6
   if (p.dscale != nullptr) {
     const int src = 2 * (lane & 15);
     const float v0 = __shfl_sync(kFull, ph[0], src), v1 = __shfl_sync(kFull, ph[1], src);
-    dscale_publish(p, lane < 16 ? v0 : v1, slab, tile, row0, nrows, lane);
+    if (lane < nrows) __stcg(p.part + (int64_t)tile * p.M + row0 + lane, lane < 16 ? v0 : v1);
   }
   if (DIRS & kRow) {
     // lane l stores the four blocks (dgate 0/1, dup 0/1) of row l
@@ -546,15 +688,16 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, int6
       if (ACT == kSwiGLU)
         __stcs(reinterpret_cast<unsigned short*>(csr + N), (unsigned short)(bu0 | (bu1 << 8)));
     }
-    uint8_t* qb = p.cq + row0 * (int64_t)W + c0;
+    unsigned short* qb = reinterpret_cast<unsigned short*>(p.cq + row0 * (int64_t)W + c0);
+    const int Whc = opaque(Wh);
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
       const uint32_t qg = e4m3x2(bf16_lo_p(DG[r]), mg0, bf16_hi_p(DG[r]), mg1);
-      if (colok && r < nrows) {
-        __stcs(reinterpret_cast<unsigned short*>(qb + (int64_t)r * W), (unsigned short)qg);
+      if (FULL || (colok && r < nrows)) {
+        __stcs(qb + r * Whc, (unsigned short)qg);
         if (ACT == kSwiGLU) {
           const uint32_t qu = e4m3x2(bf16_lo_p(DU[r]), mu0, bf16_hi_p(DU[r]), mu1);
-          __stcs(reinterpret_cast<unsigned short*>(qb + (int64_t)r * W + N), (unsigned short)qu);
+          __stcs(qb + r * Whc + (N >> 1), (unsigned short)qu);
         }
       }
     }
@@ -562,24 +705,54 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, int6
 }
 
 template <int ACT, int DIRS, bool GROUPED>
-__global__ void __launch_bounds__(bwd_threads(ACT, DIRS), 1) act_bwd_kernel(const Params p) {
-  constexpr int kWarps = bwd_threads(ACT, DIRS) / 32;
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* sig_s = reinterpret_cast<float*>(smem);
-  int* cb_s = reinterpret_cast<int*>(smem + (ACT == kSwiGLU ? kSigBytes : 0));
-  const int64_t n_slabs = stage_and_validate<ACT == kSwiGLU, GROUPED>(p, sig_s, cb_s);
+__global__ void __launch_bounds__(bwd_threads(ACT, DIRS), 1)
+    act_bwd_kernel(const __grid_constant__ CUtensorMap tm_x,
+                   const __grid_constant__ CUtensorMap tm_dy, const Params p) {
+  constexpr int kWarps = bwd_warps(ACT);
+  constexpr int kOps = bwd_operands(ACT);
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char* smem = align_smem(smem_raw);
+  float* sig_s = reinterpret_cast<float*>(smem + ring_bytes(kWarps, kOps));
+  int* cb_s = reinterpret_cast<int*>(smem + ring_bytes(kWarps, kOps) +
+                                     (ACT == kSwiGLU ? kSigBytes : 0));
+  int* ro_s = cb_s + (GROUPED ? ((p.E + 1 + 3) / 4) * 4 : 0);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      smem + ring_bytes(kWarps, kOps) + (ACT == kSwiGLU ? kSigBytes : 0) +
+      (GROUPED ? group_bytes(p.E) : 0));
+  const int64_t n_slabs = stage_and_validate<ACT == kSwiGLU, GROUPED>(p, sig_s, cb_s, ro_s);
   if (n_slabs < 0) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n_items = n_slabs * p.n_tiles;
-  for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < n_items;
-       it += (int64_t)gridDim.x * kWarps) {
+  const int64_t first = (int64_t)blockIdx.x * kWarps + warp;
+  const int64_t stride = (int64_t)gridDim.x * kWarps;
+  const int count = first < n_items ? (int)((n_items - 1 - first) / stride + 1) : 0;
+  const int K = 2 * count;
+  Ring ring{smem + warp * kSlots * kOps * kOperandHalfBytes, bars + warp * kSlots, kOps};
+  ring_prime<GROUPED>(p, cb_s, ro_s, ring, &tm_x, &tm_dy, first, stride, K, lane, ACT == kSwiGLU,
+                      true);
+  bool ok = true;
+  for (int j = 0; j < count; ++j) {
+    const int64_t it = first + j * stride;
     const int64_t slab = it / p.n_tiles;
     const int tile = (int)(it - slab * p.n_tiles);
     int64_t row0;
     int nrows;
-    slab_rows<GROUPED>(p, cb_s, slab, row0, nrows);
-    bwd_tile<ACT, DIRS>(p, sig_s, slab, tile, row0, nrows, lane);
+    slab_rows<GROUPED>(p, cb_s, ro_s, slab, row0, nrows);
+    const bool full = nrows == 32 && (tile + 1) * kTileCols <= p.N;
+    const int64_t n1 = it + stride, n2 = it + 2 * stride;
+    if (full)
+      bwd_tile<ACT, DIRS, GROUPED, true>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
+                                         cb_s, ro_s, &tm_x, &tm_dy, n1, n2, K, ok);
+    else
+      bwd_tile<ACT, DIRS, GROUPED, false>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
+                                          cb_s, ro_s, &tm_x, &tm_dy, n1, n2, K, ok);
+    if (!ok) {
+      if (lane == 0) {
+        report_timeout(p, 2u);
+        ring_drain(ring, 2 * j, K);
+      }
+      return;
+    }
   }
 }
-
 }  // namespace moeact

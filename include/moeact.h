@@ -227,6 +227,30 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
                                              void* workspace, size_t workspace_bytes,
                                              void* stream);
 
+/* ---------------------------------------------------------------------
+ * scaled_swiglu_mxfp8_bwd_noalloc -- the dense SwiGLU backward for callers
+ * that cannot allocate device memory: for example code that runs where a
+ * cudaMalloc (which may synchronise the device, at unbounded latency) is not
+ * acceptable, or a framework that owns all device memory through its own
+ * allocator and cannot pass this library a workspace.  The paper has no
+ * counterpart; this is a convenience of this library.
+ *   Arguments, outputs and results are those of scaled_swiglu_mxfp8_bwd
+ *   without the workspace: the dscale partial sums go to a 16 MiB array built
+ *   into the library (held by every GPU that loads it, until exit), so with
+ *   dscale requested ceil(N/64) * M must not exceed 4194304 (else
+ *   MOEACT_ERANGE, nothing launched).  Allocates nothing.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   All calls share the array and it keeps the last call's contents; nothing
+ *   in it needs to start at zero (every partial is written before it is
+ *   read).  Calls that overlap on the GPU (other streams, other host threads)
+ *   race on it and must be serialised by the caller.
+ * ------------------------------------------------------------------- */
+moeact_status scaled_swiglu_mxfp8_bwd_noalloc(const void* dy, int64_t lddy, const void* x,
+                                              int64_t ldx, const float* s, int64_t M, int64_t N,
+                                              int dirs, void* dx, float* dscale,
+                                              moeact_mx_out out, void* stream);
+
 /* Reads and clears this device's error word: non-zero if a kernel gave up
  * waiting for its own input copies (bit 0 forward, bit 1 backward) -- a
  * defensive bound that ends the kernel instead of letting it hang; never

@@ -58,6 +58,7 @@ _SIGS = {
                                         MxOut, P, SZ, P], I),
     "moeact_sigmoid_dump": ([P, P], I),
     "moeact_device_error": ([P], I),
+    "scaled_swiglu_mxfp8_bwd_noalloc": ([P, I64, P, I64, P, I64, I64, I, P, P, MxOut, P], I),
 }
 
 

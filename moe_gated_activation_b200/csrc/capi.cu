@@ -540,3 +540,61 @@ moeact_status moeact_sigmoid_dump(float* out, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward without any allocation.  Some callers cannot hand the library a
+// workspace: code that runs where a device allocation is not acceptable at the
+// point of the call (cudaMalloc may synchronise the device and its latency is
+// unbounded), or a host framework that owns all device memory through its own
+// allocator and offers the kernel layer no way to request scratch.  For them
+// the dscale partial sums live in a fixed array compiled into this library
+// (every GPU that loads the library holds it until the process exits).
+namespace moeact {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+// Device address of the array, per device.  In host code the array's name is
+// only a host-side stand-in, so the address is taken once per device, with
+// that device current, by cudaGetSymbolAddress.
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+moeact_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOEACT_OK;
+}
+}  // namespace
+}  // namespace moeact
+
+extern "C" moeact_status scaled_swiglu_mxfp8_bwd_noalloc(
+    const void* dy, int64_t lddy, const void* x, int64_t ldx, const float* s, int64_t M,
+    int64_t N, int dirs, void* dx, float* dscale, moeact_mx_out out, void* stream) {
+  t_err[0] = 0;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  if (dscale != nullptr && M > 0 && N > 0) {
+    const size_t need = ws_bytes_needed(M, N);
+    if (need > kNoAllocScratchBytes)
+      return fail(MOEACT_ERANGE,
+                  "dscale for M=%lld, N=%lld needs %zu bytes of scratch; the built-in scratch "
+                  "holds %zu (ceil(N/64) * M <= 4194304); use scaled_swiglu_mxfp8_bwd with a "
+                  "workspace",
+                  (long long)M, (long long)N, need, kNoAllocScratchBytes);
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOEACT_EUNSUPPORTED, "device index %d", dev);
+    const moeact_status st = noalloc_scratch(dev, &ws);
+    if (st != MOEACT_OK) return st;
+    ws_bytes = kNoAllocScratchBytes;
+  }
+  return scaled_swiglu_mxfp8_bwd(dy, lddy, x, ldx, s, M, N, dirs, dx, dscale, out, ws, ws_bytes,
+                                 stream);
+}

@@ -214,60 +214,65 @@ def run_ours(args):
         return mg.grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, ro, cb, rowwise=rw, colwise=cw,
                                                   col_scale_rows=S, workspace=ws, status=st)
 
-    # eager warm-up (also compiles nothing: the kernels are prebuilt)
+    # eager warm-up
     for i in range(3):
         ro, cb, st = splits()
         fwd(ro, cb, st)
         bwd(ro, cb, st)
     torch.cuda.synchronize()
+
     if args.eager:
-        def run_splits():
-            return splits()
-
-        state = {}
-
-        def step_parts():
+        def run_step(ev):
+            ev[0].record(stream)
             ro, cb, st = splits()
-            state.update(ro=ro, cb=cb, st=st)
-            return (lambda: fwd(ro, cb, st)), (lambda: bwd(ro, cb, st))
+            ev[1].record(stream)
+            fwd(ro, cb, st)
+            ev[2].record(stream)
+            bwd(ro, cb, st)
+            ev[3].record(stream)
     else:
-        # the three calls captured once as CUDA graphs and replayed per step
-        graphs = [torch.cuda.CUDAGraph() for _ in range(3)]
+        # the whole step captured once as a CUDA graph, with event-record nodes
+        # between the calls, and replayed once per step
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
         with torch.cuda.stream(side):
-            with torch.cuda.graph(graphs[0], stream=side):
+            with torch.cuda.graph(graph, stream=side):
+                gev[0].record(side)
                 ro, cb, st = splits()
-            with torch.cuda.graph(graphs[1], stream=side):
+                gev[1].record(side)
                 fwd(ro, cb, st)
-            with torch.cuda.graph(graphs[2], stream=side):
+                gev[2].record(side)
                 bwd(ro, cb, st)
+                gev[3].record(side)
         stream.wait_stream(side)
         torch.cuda.synchronize()
 
-    def step(ev):
-        ev[0].record(stream)
+    def timed_steps(n, record):
+        """n steps, each after an L2 flush; returns per-step [splits, fwd, bwd, total] ms."""
+        out = []
+        for i in range(n):
+            do_flush(i)
+            if args.eager:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                run_step(ev)
+                if record:
+                    out.append(ev)
+            else:
+                graph.replay()
+                torch.cuda.synchronize()
+                if record:
+                    out.append([gev[0].elapsed_time(gev[1]), gev[1].elapsed_time(gev[2]),
+                                gev[2].elapsed_time(gev[3]), gev[0].elapsed_time(gev[3])])
         if args.eager:
-            f_call, b_call = step_parts()
-            ev[1].record(stream)
-            f_call()
-            ev[2].record(stream)
-            b_call()
-        else:
-            graphs[0].replay()
-            ev[1].record(stream)
-            graphs[1].replay()
-            ev[2].record(stream)
-            graphs[2].replay()
-        ev[3].record(stream)
+            torch.cuda.synchronize()
+            out = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
+                    e[0].elapsed_time(e[3])] for e in out]
+        return out
 
-    # warm-up
-    for i in range(args.warmup):
-        do_flush(i)
-        step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    timed_steps(args.warmup, False)
     torch.cuda.synchronize()
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     sampler = ClockSampler(dev)
     with sampler:
         if world > 1:
@@ -275,21 +280,18 @@ def run_ours(args):
         torch.cuda.synchronize()
         sampler.active = True
         wall0 = time.perf_counter()
-        for i in range(args.steps):
-            do_flush(i)
-            step(evs[i])
+        times = timed_steps(args.steps, True)
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
         sampler.active = False
         if world > 1:
             torch.distributed.barrier()
     if not args.eager:
-        del graphs
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    splits_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms = sum(step_ms)
+        del graph
+    splits_ms = [t[0] for t in times]
+    fwd_ms = [t[1] for t in times]
+    bwd_ms = [t[2] for t in times]
+    total_ms = sum(t[3] for t in times)
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -309,7 +311,7 @@ def run_ours(args):
     achieved = bm[dom] / (dom_us * 1e-6) / 1e9
     kname = "act_bwd_kernel" if dom == "bwd" else "act_fwd_kernel"
     traffic = ncu_traffic(args.workload, kname, args.dirs)
-    value = world * step_bytes / (total_ms * 1e-3) / 1e9
+    value = world * args.steps * step_bytes / (total_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -326,7 +328,7 @@ def run_ours(args):
         "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
                    "dirs": args.dirs, "activation": "swiglu",
                    "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
-                   "launch": "eager" if args.eager else "CUDA graphs (one per call), replayed per step",
+                   "launch": "eager" if args.eager else "one CUDA graph per step (event nodes between the calls)",
                    "l2": "flushed before every step (256 MiB written then read), outside the timed events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),

@@ -111,7 +111,7 @@ typedef enum moeact_status {
 #define MOEACT_DEV_BAD_OFFSETS 3      /* offsets not those of valid splits */
 
 /* Largest number of groups (experts) a grouped call accepts. */
-#define MOEACT_MAX_GROUPS 4096
+#define MOEACT_MAX_GROUPS 2040
 /* Largest M accepted (2^30 rows; TMA coordinates are 32-bit). */
 #define MOEACT_MAX_ROWS (((int64_t)1) << 30)
 
@@ -189,7 +189,7 @@ moeact_status grouped_scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const f
  *   dscale nullable, fp32 [M].  Needs `workspace` of at least
  *          scaled_act_mxfp8_bwd_workspace_size(M, N, E) bytes (E = 1 for
  *          dense calls; the size does not depend on E): scratch for the
- *          per-tile partial sums (ceil(N/64) x M fp32), no initial content
+ *          per-tile partial sums (ceil(N/128) x M fp32), no initial content
  *          required.  dscale is then summed by a second kernel launched on
  *          the same stream.  Calls sharing one workspace must not overlap on
  *          the GPU.
@@ -237,7 +237,7 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
  *   Arguments, outputs and results are those of scaled_swiglu_mxfp8_bwd
  *   without the workspace: the dscale partial sums go to a 16 MiB array built
  *   into the library (held by every GPU that loads it, until exit), so with
- *   dscale requested ceil(N/64) * M must not exceed 4194304 (else
+ *   dscale requested ceil(N/128) * M must not exceed 4194304 (else
  *   MOEACT_ERANGE, nothing launched).  Allocates nothing.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress); make that first call before any stream capture.

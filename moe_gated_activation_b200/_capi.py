@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libmoeact.so")
 OK, EINVAL, EALIGN, EUNSUPPORTED, ERANGE, ECUDA, EWORKSPACE = range(7)
 ROWWISE, COLWISE = 1, 2
 DEV_OK, DEV_NEGATIVE_SPLIT, DEV_SPLIT_SUM, DEV_BAD_OFFSETS = range(4)
-MAX_GROUPS = 4096
+MAX_GROUPS = 2040
 
 
 class MxOut(ctypes.Structure):

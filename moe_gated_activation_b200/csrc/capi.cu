@@ -40,18 +40,20 @@ __device__ int g_sigma_uncertain;
 
 using FwdFn = void (*)(const CUtensorMap, const Params);
 using BwdFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
-struct FwdVariant { FwdFn fn; int threads; int smem_fixed; };
-struct BwdVariant { BwdFn fn; int threads; int smem_fixed; };
+// smem_fixed: shared memory without group offsets; sig: the kernel carries the
+// sigmoid table, whose gap holds the group offsets (so they add nothing)
+struct FwdVariant { FwdFn fn; int threads; int smem_fixed; bool sig; };
+struct BwdVariant { BwdFn fn; int threads; int smem_fixed; bool sig; };
 
 template <int ACT, int DIRS, bool STAGED, bool GROUPED>
 FwdVariant fwd_variant() {
-  return {act_fwd_kernel<ACT, DIRS, STAGED, GROUPED>, fwd_threads(ACT, DIRS),
-          smem_bytes(fwd_warps(ACT), fwd_operands(ACT), ACT == kSwiGLU, -1)};
+  return {act_fwd_kernel<ACT, DIRS, STAGED, GROUPED>, Cfg<ACT, false>::kThreads,
+          smem_bytes<ACT, false>(false, 0), Cfg<ACT, false>::kSig};
 }
 template <int ACT, int DIRS, bool GROUPED>
 BwdVariant bwd_variant() {
-  return {act_bwd_kernel<ACT, DIRS, GROUPED>, bwd_threads(ACT, DIRS),
-          smem_bytes(bwd_warps(ACT), bwd_operands(ACT), ACT == kSwiGLU, -1)};
+  return {act_bwd_kernel<ACT, DIRS, GROUPED>, Cfg<ACT, true>::kThreads,
+          smem_bytes<ACT, true>(false, 0), Cfg<ACT, true>::kSig};
 }
 
 template <int ACT, bool GROUPED>
@@ -113,12 +115,12 @@ moeact_status init_device(int dev) {
   bwd_all<kSReLU, true>(bv, nb);
   for (int i = 0; i < nf; ++i) {
     e = cudaFuncSetAttribute(fv[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fv[i].smem_fixed + kGroupSmem);
+                             fv[i].smem_fixed + (fv[i].sig ? 0 : kGroupSmem));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
   for (int i = 0; i < nb; ++i) {
     e = cudaFuncSetAttribute(bv[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bv[i].smem_fixed + kGroupSmem);
+                             bv[i].smem_fixed + (bv[i].sig ? 0 : kGroupSmem));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
   e = cudaFuncSetAttribute(sigma_table_dump, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -261,7 +263,7 @@ int64_t grid_for(int64_t slabs_upper, int n_tiles, int threads, int dev) {
   return blocks < 1 ? 1 : blocks;
 }
 
-int group_smem(bool grouped, int E) { return grouped ? group_bytes(E) : 0; }
+int group_smem(bool sig, bool grouped, int E) { return (grouped && !sig) ? group_bytes(E) : 0; }
 
 moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, int64_t M,
                          int64_t N, int dirs, int staged, const int64_t* ro, const int64_t* cb,
@@ -302,7 +304,7 @@ moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, in
   CUtensorMap tx;
   if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
   const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
-  v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(grouped, p.E), cs>>>(tx, p);
+  v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(v.sig, grouped, p.E), cs>>>(tx, p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return MOEACT_OK;
@@ -367,7 +369,7 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
   if ((st = make_map(&tdy, dy, N, M, lddy))) return st;
   const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
-  v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(grouped, p.E), cs>>>(tx, tdy, p);
+  v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(v.sig, grouped, p.E), cs>>>(tx, tdy, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   if (dscale) {
@@ -584,7 +586,7 @@ extern "C" moeact_status scaled_swiglu_mxfp8_bwd_noalloc(
     if (need > kNoAllocScratchBytes)
       return fail(MOEACT_ERANGE,
                   "dscale for M=%lld, N=%lld needs %zu bytes of scratch; the built-in scratch "
-                  "holds %zu (ceil(N/64) * M <= 4194304); use scaled_swiglu_mxfp8_bwd with a "
+                  "holds %zu (ceil(N/128) * M <= 4194304); use scaled_swiglu_mxfp8_bwd with a "
                   "workspace",
                   (long long)M, (long long)N, need, kNoAllocScratchBytes);
     int dev = 0;

@@ -33,6 +33,7 @@ constexpr int kSigEntriesPadded = 8196;                 // whole float4s
 // (0x8000) is itself the byte offset 32768 between the two halves.
 constexpr int kSigNegOffset = 8192;
 constexpr int kSigBytes = (kSigNegOffset + kSigPerSign + 3) / 4 * 16;   // 49168
+constexpr int kSigHalfBytes = (kSigPerSign + 3) / 4 * 16;                 // 16400
 
 __device__ __forceinline__ float sigma_lookup(const float* tab, uint32_t b16) {
   uint32_t a = b16 & 0x7FFFu;
@@ -119,6 +120,43 @@ __device__ __forceinline__ int opaque(int v) {
   return r;
 }
 
+// ---------------------------------------------------------------- packed fp32
+// sm_100 packed fp32 arithmetic: two independent IEEE operations (round to
+// nearest even, subnormals kept) in one instruction.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 r;
+  asm("{ .reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; "
+      "mul.rn.f32x2 rd, ra, rb; mov.b64 {%0, %1}, rd; }"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{ .reg .b64 ra, rb, rc, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; "
+      "mov.b64 rc, {%6, %7}; fma.rn.f32x2 rd, ra, rb, rc; mov.b64 {%0, %1}, rd; }"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 r;
+  asm("{ .reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; "
+      "sub.rn.f32x2 rd, ra, rb; mov.b64 {%0, %1}, rd; }"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t v) { return make_float2(bf16_lo(v), bf16_hi(v)); }
+__device__ __forceinline__ float2 bf16x2_to_f2_p(uint32_t v) { return make_float2(bf16_lo_p(v), bf16_hi_p(v)); }
+
+// E4M3 codes of v * (ma, mb) (low byte: x), as e4m3x2 with a packed multiply.
+__device__ __forceinline__ uint32_t e4m3x2_2(float2 v, uint32_t ma, uint32_t mb) {
+  const float2 q = mul2(v, make_float2(__uint_as_float(ma), __uint_as_float(mb)));
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+}
+
 __device__ __forceinline__ uint32_t f32_mag(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
 
 // ---------------------------------------------------------------- TMA / mbarrier
@@ -154,6 +192,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t i = 0; i < kSpinLimit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
+}
+
+// 1-D bulk copy (no multicast) of `bytes` (a multiple of 16, both addresses
+// 16-byte aligned) from global to shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
 }
 
 // 2-D TMA tile load (no multicast) of box {x .. x+bx, y .. y+by} into shared

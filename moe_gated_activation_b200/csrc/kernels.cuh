@@ -45,11 +45,17 @@ namespace moeact {
 enum Act : int { kSwiGLU = 0, kSReLU = 1 };
 constexpr int kRow = 1;
 constexpr int kCol = 2;
-constexpr int kTileCols = 64;
+constexpr int kTileCols = 128;   // columns of a warp-tile (4 per lane)
 
-// The table lives in device global memory of this module: one copy per
-// device, written by sigma_table_init before any activation kernel reads it.
-__device__ __align__(16) float g_sigma_table[kSigEntriesPadded];
+// The table lives in device global memory of this module, one copy per
+// device, written by sigma_table_init before any activation kernel reads it,
+// already in the shared-memory layout (positive gates at [0, 4097), negative
+// at [8192, 12289)) so that a kernel stages it with one bulk copy.
+__device__ __align__(16) float g_sigma_table[kSigBytes / 4];
+
+__host__ __device__ constexpr int sig_slot(int i) {
+  return i < (int)kSigPerSign ? i : i - (int)kSigPerSign + kSigNegOffset;
+}
 
 // Builds the table.  For |g| < 2^-9, sigma(g) = 1/2 + g/4 - g^3/48 + O(g^5):
 // hi = 1/2 + g/4 is exact in binary64 and the rest is far smaller than any
@@ -62,8 +68,7 @@ __device__ __align__(16) float g_sigma_table[kSigEntriesPadded];
 // 2^-37 away).
 __global__ void sigma_table_init(int* uncertain) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= kSigEntriesPadded) return;
-  if (i >= kSigEntries) { g_sigma_table[i] = 0.0f; return; }
+  if (i >= kSigEntries) return;
   const uint32_t neg = i >= (int)kSigPerSign ? 1u : 0u;
   const uint32_t mag = (uint32_t)i - neg * kSigPerSign + kSigLo;
   const float g = __uint_as_float(((neg << 15) | mag) << 16);
@@ -78,7 +83,7 @@ __global__ void sigma_table_init(int* uncertain) {
     } else {
       f = __double2float_rn(hi);
     }
-    g_sigma_table[i] = f;
+    g_sigma_table[sig_slot(i)] = f;
     return;
   }
   const double sd = 1.0 / (1.0 + exp(-(double)g));
@@ -87,7 +92,7 @@ __global__ void sigma_table_init(int* uncertain) {
   const double dn = 0.5 * ((double)f + (double)nextafterf(f, __int_as_float(0xFF800000)));
   const double tol = fabs(sd) * 0x1p-48;
   if (!(fabs(sd - up) > tol && fabs(sd - dn) > tol)) atomicAdd(uncertain, 1);
-  g_sigma_table[i] = f;
+  g_sigma_table[sig_slot(i)] = f;
 }
 
 // Expands the table to all 65536 bf16 patterns (test hook), through the same
@@ -95,8 +100,7 @@ __global__ void sigma_table_init(int* uncertain) {
 // up the packed pair (2t, 2t + 1).
 __global__ void sigma_table_dump(float* out) {
   extern __shared__ __align__(16) float tab[];
-  for (int i = threadIdx.x; i < kSigEntries; i += blockDim.x)
-    tab[i < (int)kSigPerSign ? i : i - (int)kSigPerSign + kSigNegOffset] = g_sigma_table[i];
+  for (int i = threadIdx.x; i < kSigBytes / 4; i += blockDim.x) tab[i] = g_sigma_table[i];
   __syncthreads();
   const uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t < 32768) {
@@ -207,46 +211,86 @@ struct Params {
   uint32_t* err;      // device error word (timeouts), never expected to be set
 };
 
-constexpr int kSlots = 3;            // half-tile slots per warp
 constexpr int kHalfRows = 16;
-constexpr int kOperandHalfBytes = kHalfRows * kTileCols * 2;   // 2 KiB
+constexpr int kOpHalfBytes = kHalfRows * kTileCols * 2;   // one operand's half-tile: 4 KiB
+constexpr int kRowBytes = kTileCols * 2;                   // 256 B of a bf16 tile row
 
-// Threads per CTA: one CTA per SM; the shared memory of the warps' rings
-// (slots x operands x 2 KiB) plus the sigmoid table bounds the warp count.
-__host__ __device__ constexpr int fwd_warps(int act) { return act == 0 ? 12 : 12; }
-__host__ __device__ constexpr int bwd_warps(int act) { return act == 0 ? 8 : 12; }
-__host__ __device__ constexpr int fwd_threads(int act, int dirs) { return 32 * fwd_warps(act) + 0 * dirs; }
-__host__ __device__ constexpr int bwd_threads(int act, int dirs) { return 32 * bwd_warps(act) + 0 * dirs; }
-__host__ __device__ constexpr int fwd_operands(int act) { return act == 0 ? 2 : 1; }
-__host__ __device__ constexpr int bwd_operands(int act) { return act == 0 ? 3 : 2; }
-__host__ __device__ constexpr int ring_bytes(int warps, int operands) {
-  return warps * kSlots * operands * kOperandHalfBytes;
-}
+// Per-kernel configuration: warps per CTA (one CTA per SM) and ring slots per
+// warp, chosen so that rings + sigmoid table fit the 227 KiB of shared memory.
+template <int ACT, bool BWD>
+struct Cfg {
+  static constexpr bool kSig = ACT == kSwiGLU;
+  static constexpr int kOps = BWD ? (kSig ? 3 : 2) : (kSig ? 2 : 1);
+  static constexpr int kWarps = BWD ? (kSig ? 7 : 8) : 8;
+  static constexpr int kSlots = (!BWD && !kSig) ? 3 : 2;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kRing = kWarps * kSlots * kOps * kOpHalfBytes;
+  static constexpr int kBars = kWarps * kSlots + 1;
+};
 
-// Shared-memory layout of a CTA: [rings][sigmoid table][col-block offsets][mbarriers]
-// (E < 0: without the col-block offsets, which the launcher adds for grouped calls)
-// (128 bytes of slack let the kernel align the base for the TMA destinations;
-// a grouped call adds its row and col-block offsets as two int32 arrays)
+// Grouped offsets (int32 copies of row_offs and colblk_offs): with the
+// sigmoid table they live in its unused gap (float indices 4100.. and 6144..,
+// room for MOEACT_MAX_GROUPS + 1 entries each); without it, after the ring.
+constexpr int kGapCb = 4100;
+constexpr int kGapRo = 6144;
 __host__ __device__ constexpr int group_bytes(int E) { return 2 * ((E + 1 + 3) / 4) * 16; }
-__host__ __device__ constexpr int smem_bytes(int warps, int operands, bool sig, int E) {
-  return 128 + ring_bytes(warps, operands) + (sig ? kSigBytes : 0) +
-         (E < 0 ? 0 : group_bytes(E)) + warps * kSlots * 8;
+
+// Shared memory of a CTA: 128 B of alignment slack, the ring, the table (or
+// the group offsets), the mbarriers.
+template <int ACT, bool BWD>
+__host__ __device__ constexpr int smem_bytes(bool grouped, int E) {
+  using C = Cfg<ACT, BWD>;
+  return 128 + C::kRing + (C::kSig ? kSigBytes : (grouped ? group_bytes(E) : 0)) + C::kBars * 8;
 }
 
 __device__ __forceinline__ unsigned char* align_smem(unsigned char* p) {
   return p + ((128u - (smem_addr(p) & 127u)) & 127u);
 }
 
-// Stages the sigmoid table (and, grouped, the row and col-block offsets as
-// int32) in shared memory and validates grouped offsets.  Returns the slab
-// count, or -1 if the offsets are not those of valid splits (every CTA reaches
-// the same verdict; CTA 0 writes the status word).
-template <bool NEED_SIG, bool GROUPED>
-__device__ __forceinline__ int64_t stage_and_validate(const Params& p, float* sig_s, int* cb_s,
-                                                      int* ro_s) {
-  if (NEED_SIG) {
-    for (int i = threadIdx.x; i < kSigEntries; i += blockDim.x)
-      sig_s[i < (int)kSigPerSign ? i : i - (int)kSigPerSign + kSigNegOffset] = g_sigma_table[i];
+struct Smem {
+  unsigned char* ring;
+  float* sig;
+  int* cb;
+  int* ro;
+  uint64_t* bars;
+};
+
+template <int ACT, bool BWD>
+__device__ __forceinline__ Smem carve(unsigned char* raw, int E) {
+  using C = Cfg<ACT, BWD>;
+  Smem m;
+  unsigned char* base = align_smem(raw);
+  m.ring = base;
+  unsigned char* after = base + C::kRing;
+  if (C::kSig) {
+    m.sig = reinterpret_cast<float*>(after);
+    m.cb = reinterpret_cast<int*>(m.sig + kGapCb);
+    m.ro = reinterpret_cast<int*>(m.sig + kGapRo);
+    after += kSigBytes;
+  } else {
+    m.sig = nullptr;
+    m.cb = reinterpret_cast<int*>(after);
+    m.ro = m.cb + ((E + 1 + 3) / 4) * 4;
+    after += group_bytes(E);
+  }
+  m.bars = reinterpret_cast<uint64_t*>(after);
+  return m;
+}
+
+// Starts the bulk copy of the sigmoid table (thread 0) and validates grouped
+// offsets while staging them as int32.  Returns the slab count, or -1 if the
+// offsets are not those of valid splits (every CTA reaches the same verdict;
+// CTA 0 writes the status word).  The table copy completes on sig_bar.
+template <bool SIG, bool GROUPED>
+__device__ __forceinline__ int64_t stage_and_validate(const Params& p, const Smem& m,
+                                                      uint64_t* sig_bar) {
+  if (SIG && threadIdx.x == 0) {
+    // the two halves of the table; the gap between them is not copied
+    mbar_init(sig_bar, 1);
+    mbar_init_fence();
+    mbar_expect_tx(sig_bar, 2 * kSigHalfBytes);
+    bulk_load(m.sig, g_sigma_table, kSigHalfBytes, sig_bar);
+    bulk_load(m.sig + kSigNegOffset, g_sigma_table + kSigNegOffset, kSigHalfBytes, sig_bar);
   }
   int bad = 0;
   if (GROUPED) {
@@ -257,26 +301,25 @@ __device__ __forceinline__ int64_t stage_and_validate(const Params& p, float* si
         ok = (r == 0) && (c == 0);
       } else {
         const int64_t r0 = p.row_offs[e - 1], c0 = p.cb_offs[e - 1];
-        const int64_t m = r - r0;
-        ok = (m >= 0) && (r <= p.M) && (c - c0 == (m + 31) / 32);
+        const int64_t mm = r - r0;
+        ok = (mm >= 0) && (r <= p.M) && (c - c0 == (mm + 31) / 32);
       }
       if (e == p.E) ok = ok && (r == p.M);
       if (!ok) bad = 1;
-      cb_s[e] = (int)c;
-      ro_s[e] = (int)r;
+      m.cb[e] = (int)c;
+      m.ro[e] = (int)r;
     }
   }
   bad = __syncthreads_or(bad);
   if (!GROUPED) return p.dense_slabs;
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = bad ? 3 : 0;
-  return bad ? -1 : (int64_t)cb_s[p.E];
+  return bad ? -1 : (int64_t)m.cb[p.E];
 }
 
-// Rows of slab `slab`: first row and count (<= 32).  Grouped offsets come from
-// shared memory (int32: rows are below 2^30).
+// Rows of slab `slab`: first row and count (<= 32).
 template <bool GROUPED>
-__device__ __forceinline__ void slab_rows(const Params& p, const int* cb_s, const int* ro_s,
-                                          int64_t slab, int64_t& row0, int& nrows) {
+__device__ __forceinline__ void slab_rows(const Params& p, const Smem& m, int64_t slab,
+                                          int64_t& row0, int& nrows) {
   if (!GROUPED) {
     row0 = slab * 32;
     nrows = (int)min((int64_t)32, p.M - row0);
@@ -286,245 +329,323 @@ __device__ __forceinline__ void slab_rows(const Params& p, const int* cb_s, cons
     const int sl = (int)slab;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (cb_s[mid] <= sl) lo = mid; else hi = mid - 1;
+      if (m.cb[mid] <= sl) lo = mid; else hi = mid - 1;
     }
-    const int r0 = ro_s[lo] + 32 * (sl - cb_s[lo]);
+    const int r0 = m.ro[lo] + 32 * (sl - m.cb[lo]);
     row0 = r0;
-    nrows = min(32, ro_s[lo + 1] - r0);
+    nrows = min(32, m.ro[lo + 1] - r0);
   }
 }
 
-// Stores the two E8M0 bytes (blocks 2*tile, 2*tile+1) of one row.  `blk1`
-// exists only when the tile has a second 32-column block; the 16-bit store is
-// used when the address is even.
-__device__ __forceinline__ void store_row_scales(uint8_t* dst, uint32_t b0, uint32_t b1,
-                                                 bool has1) {
-  if (has1 && ((reinterpret_cast<uintptr_t>(dst) & 1u) == 0)) {
-    __stcs(reinterpret_cast<unsigned short*>(dst), (unsigned short)(b0 | (b1 << 8)));
-  } else {
-    dst[0] = (uint8_t)b0;
-    if (has1) dst[1] = (uint8_t)b1;
+// Walks a warp's work items (item j = first + j * stride) as (slab, tile)
+// without dividing per item.
+struct Cursor {
+  int64_t slab;
+  int tile;
+  int64_t dslab;
+  int dtile;
+  int n_tiles;
+  __device__ __forceinline__ void init(int64_t first, int64_t stride, int nt) {
+    n_tiles = nt;
+    slab = first / nt;
+    tile = (int)(first - slab * nt);
+    dslab = stride / nt;
+    dtile = (int)(stride - dslab * nt);
   }
-}
-
-// ------------------------------------------------------------- the warp's ring
-// Half-tile k of a warp is half (k & 1) of its (k >> 1)-th work item; it lives
-// in slot k % kSlots, whose mbarrier completes once per use (parity
-// (k / kSlots) & 1).
-struct Ring {
-  unsigned char* slots;   // kSlots * OPS * 2 KiB
-  uint64_t* bars;         // kSlots
-  int ops;
+  __device__ __forceinline__ void next() {
+    slab += dslab;
+    tile += dtile;
+    if (tile >= n_tiles) { tile -= n_tiles; ++slab; }
+  }
 };
 
-template <bool GROUPED>
-__device__ __forceinline__ void issue_half(const Params& p, const int* cb_s, const int* ro_s,
-                                           const Ring& r,
-                                           const void* tm_x, const void* tm_dy, int64_t item,
-                                           int k, bool swiglu, bool with_dy) {
-  const int64_t slab = item / p.n_tiles;
-  const int tile = (int)(item - slab * p.n_tiles);
-  int64_t row0;
-  int nrows;
-  slab_rows<GROUPED>(p, cb_s, ro_s, slab, row0, nrows);
-  const int slot = k % kSlots;
-  unsigned char* dst = r.slots + slot * r.ops * kOperandHalfBytes;
+// The warp's ring: half-tile k (half k & 1 of the warp's item k >> 1) lives in
+// slot k % SLOTS, whose mbarrier completes once per use (parity
+// (k / SLOTS) & 1).  Lane 0 issues the loads, walking its own cursor.
+template <int OPS, int SLOTS>
+struct Ring {
+  unsigned char* slots;
+  uint64_t* bars;
+  Cursor cur;        // item of the next half-tile to issue (lane 0)
+  int64_t row0;      // its first row
+  int k_issue;       // next half-tile to issue
+};
+
+template <int OPS, int SLOTS, bool GROUPED>
+__device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
+                                           Ring<OPS, SLOTS>& r, const void* tm_x,
+                                           const void* tm_dy) {
+  const int k = r.k_issue;
+  const int half = k & 1;
+  if (half == 0) {
+    int nrows;
+    slab_rows<GROUPED>(p, m, r.cur.slab, r.row0, nrows);
+  }
+  const int slot = k % SLOTS;
+  unsigned char* dst = r.slots + slot * OPS * kOpHalfBytes;
   uint64_t* bar = r.bars + slot;
-  const int x = tile * kTileCols, y = (int)row0 + (k & 1) * kHalfRows;
-  mbar_expect_tx(bar, r.ops * kOperandHalfBytes);
-  int o = 0;
-  if (with_dy) tma_load_2d(dst + (o++) * kOperandHalfBytes, tm_dy, x, y, bar);
-  tma_load_2d(dst + (o++) * kOperandHalfBytes, tm_x, x, y, bar);
-  if (swiglu) tma_load_2d(dst + (o++) * kOperandHalfBytes, tm_x, x + p.N, y, bar);
+  const int x = r.cur.tile * kTileCols, y = (int)r.row0 + half * kHalfRows;
+  mbar_expect_tx(bar, OPS * kOpHalfBytes);
+  if (OPS == 3 || (OPS == 2 && tm_dy != nullptr)) {
+    // backward: dY, then x (gate), then up (SwiGLU)
+    tma_load_2d(dst, tm_dy, x, y, bar);
+    tma_load_2d(dst + kOpHalfBytes, tm_x, x, y, bar);
+    if (OPS == 3) tma_load_2d(dst + 2 * kOpHalfBytes, tm_x, x + p.N, y, bar);
+  } else {
+    // forward: gate, then up (SwiGLU)
+    tma_load_2d(dst, tm_x, x, y, bar);
+    if (OPS == 2) tma_load_2d(dst + kOpHalfBytes, tm_x, x + p.N, y, bar);
+  }
+  r.k_issue = k + 1;
+  if (half == 1) r.cur.next();
 }
 
 __device__ __forceinline__ void report_timeout(const Params& p, uint32_t code) {
   atomicOr(p.err, code);
 }
 
+// After a timeout: bounded waits for the copies still in flight into the
+// warp's slots, so that none lands after the CTA has exited.
+template <int OPS, int SLOTS>
+__device__ __forceinline__ void ring_drain(const Ring<OPS, SLOTS>& r, int k_next) {
+  for (int k = k_next; k < r.k_issue; ++k)
+    mbar_wait(r.bars + (k % SLOTS), (uint32_t)(k / SLOTS) & 1u);
+}
+
+// Magnitude bits shifted left by one: ordering of |v| with NaN above +Inf
+// (an integer max over them is a NaN-propagating amax); e8m0 takes them >> 1.
+__device__ __forceinline__ uint32_t mag2(float v) { return __float_as_uint(v) << 1; }
+
+// Stores the E8M0 bytes of one row's blocks [4*tile, 4*tile + nb) (packed in
+// v, block 0 in the low byte): one 32-bit store when all four exist and the
+// address is aligned, bytes otherwise.
+__device__ __forceinline__ void store_scales4(uint8_t* dst, uint32_t v, int nb) {
+  if (nb == 4 && ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0)) {
+    __stcs(reinterpret_cast<unsigned int*>(dst), v);
+  } else {
+    for (int b = 0; b < nb; ++b) dst[b] = (uint8_t)(v >> (8 * b));
+  }
+}
+
+// Gathers, for row `lane` of the tile, the four blocks' E8M0 bytes from the
+// lanes that reduced them: bytes `byte_lo` (rows 0-15) / `byte_hi` (rows
+// 16-31) of w[h] in lanes 8k + ((row & 15) >> 1).
+__device__ __forceinline__ uint32_t gather_row_scales(uint32_t w0, uint32_t w1, int lane,
+                                                      int byte_even, int byte_odd) {
+  const int j = lane & 15;
+  const int sh = 8 * ((j & 1) ? byte_odd : byte_even);
+  uint32_t v = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int src = 8 * k + (j >> 1);
+    const uint32_t a = __shfl_sync(kFull, w0, src), b = __shfl_sync(kFull, w1, src);
+    v |= (((lane < 16 ? a : b) >> sh) & 0xFFu) << (8 * k);
+  }
+  return v;
+}
+
 // ------------------------------------------------------------- forward tile
-// Rowwise work runs per 16-row half: after the 4-step butterfly (off = 8, 4,
-// 2, 1) lane l holds the amax of row 16h + (l & 15) in block (l >> 4).
-template <int ACT, int DIRS, bool STAGED, bool GROUPED, bool FULL>
-__device__ __forceinline__ void fwd_tile(const Params& p, const float* sig, const Ring& ring,
-                                         int k0, int64_t slab, int tile, int64_t row0, int nrows,
-                                         int lane, const int* cb_s, const int* ro_s,
-                                         const void* tm_x, int64_t next_item0,
-                                         int64_t next_item1, int K, bool& ok_flag) {
-  const int c0 = tile * kTileCols + 2 * lane;
+// Lane l owns columns 4l .. 4l+3 of a 32 x 128 warp-tile; a rowwise block is
+// 8 lanes.  Rowwise work runs per 16-row half: after the 3-step butterfly
+// (off = 4, 2, 1) lane l holds the amax of rows 16h + 2(l & 7) + {0, 1} of
+// block l >> 3.
+template <int ACT, int DIRS, bool STAGED, bool GROUPED, bool FULL, int OPS, int SLOTS>
+__device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OPS, SLOTS>& ring,
+                                         int k0, int K, int64_t slab, int tile, int64_t row0,
+                                         int nrows, float sv, int lane, const void* tm_x,
+                                         bool& ok_flag) {
+  const int c0 = tile * kTileCols + 4 * lane;
   const bool colok = c0 < p.N;
   const int W = p.W;
-  const int Wh = W >> 1;
-  const float sv = lane < nrows ? __ldg(p.s + row0 + lane) : 0.0f;
+  const int Wq = W >> 2;   // row stride of the code arrays in 32-bit words
 
-  float Y0[32], Y1[32];
+  float Y[32][4];
   uint32_t bh[2];
-  unsigned short* rqb = reinterpret_cast<unsigned short*>(p.rq + row0 * (int64_t)W + c0);
+  unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + c0);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int k = k0 + h;
-    const int slot = k % kSlots;
-    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / kSlots) & 1u)) { ok_flag = false; return; }
-    const unsigned char* sm = ring.slots + slot * ring.ops * kOperandHalfBytes + 4 * lane;
+    const int slot = k % SLOTS;
+    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / SLOTS) & 1u)) { ok_flag = false; return; }
+    const unsigned char* sm = ring.slots + slot * OPS * kOpHalfBytes + 8 * lane;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int r = 16 * h + i;
-      const uint32_t G = *reinterpret_cast<const uint32_t*>(sm + i * 128);
+      const uint2 G = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
       const float sr = __shfl_sync(kFull, sv, r);
-      float h0, h1;
+      const float2 s2 = make_float2(sr, sr);
+      float2 h01, h23;
       if (ACT == kSwiGLU) {
-        const uint32_t U = *reinterpret_cast<const uint32_t*>(sm + kOperandHalfBytes + i * 128);
-        const float g0 = bf16_lo(G), g1 = bf16_hi(G);
-        const float u0 = bf16_lo(U), u1 = bf16_hi(U);
-        float sg0, sg1;
-        sigma_pair(sig, G, sg0, sg1);
-        const float si0 = __fmul_rn(g0, sg0);
-        const float si1 = __fmul_rn(g1, sg1);
+        const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
+        float2 sg01, sg23;
+        sigma_pair(m.sig, G.x, sg01.x, sg01.y);
+        sigma_pair(m.sig, G.y, sg23.x, sg23.y);
+        const float2 si01 = mul2(bf16x2_to_f2(G.x), sg01), si23 = mul2(bf16x2_to_f2(G.y), sg23);
+        const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
         if (STAGED) {
-          h0 = bf16_round(__fmul_rn(bf16_round(si0), u0));
-          h1 = bf16_round(__fmul_rn(bf16_round(si1), u1));
+          h01 = mul2(make_float2(bf16_round(si01.x), bf16_round(si01.y)), u01);
+          h23 = mul2(make_float2(bf16_round(si23.x), bf16_round(si23.y)), u23);
+          h01 = make_float2(bf16_round(h01.x), bf16_round(h01.y));
+          h23 = make_float2(bf16_round(h23.x), bf16_round(h23.y));
         } else {
-          h0 = __fmul_rn(si0, u0);
-          h1 = __fmul_rn(si1, u1);
+          h01 = mul2(si01, u01);
+          h23 = mul2(si23, u23);
         }
       } else {
-        const float r0 = relu_keep_nan(bf16_lo(G)), r1 = relu_keep_nan(bf16_hi(G));
-        h0 = __fmul_rn(r0, r0);
-        h1 = __fmul_rn(r1, r1);
+        const float r0 = relu_keep_nan(bf16_lo(G.x)), r1 = relu_keep_nan(bf16_hi(G.x));
+        const float r2 = relu_keep_nan(bf16_lo(G.y)), r3 = relu_keep_nan(bf16_hi(G.y));
+        h01 = mul2(make_float2(r0, r1), make_float2(r0, r1));
+        h23 = mul2(make_float2(r2, r3), make_float2(r2, r3));
       }
-      Y0[r] = __fmul_rn(h0, sr);
-      Y1[r] = __fmul_rn(h1, sr);
-      if (!FULL && r >= nrows) { Y0[r] = 0.0f; Y1[r] = 0.0f; }
+      const float2 y01 = mul2(h01, s2), y23 = mul2(h23, s2);
+      const bool live = FULL || r < nrows;
+      Y[r][0] = live ? y01.x : 0.0f;
+      Y[r][1] = live ? y01.y : 0.0f;
+      Y[r][2] = live ? y23.x : 0.0f;
+      Y[r][3] = live ? y23.y : 0.0f;
     }
-    // the slot is consumed: refill it with the half-tile kSlots ahead
+    // the slot is consumed: refill it with the half-tile SLOTS ahead
     __syncwarp();
-    if (lane == 0 && k + kSlots < K) {
-      const int kn = k + kSlots;
-      issue_half<GROUPED>(p, cb_s, ro_s, ring, tm_x, nullptr,
-                          (kn >> 1) == (k0 >> 1) + 1 ? next_item0 : next_item1, kn,
-                          ACT == kSwiGLU, false);
-    }
+    if (lane == 0 && ring.k_issue < K) ring_issue<OPS, SLOTS, GROUPED>(p, m, ring, tm_x, nullptr);
     if (DIRS & kRow) {
       uint32_t A[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) A[i] = max(f32_mag(Y0[16 * h + i]), f32_mag(Y1[16 * h + i]));
-      bfly_max_u32<8>(A, lane, 8);
-      bfly_max_u32<4>(A, lane, 4);
-      bfly_max_u32<2>(A, lane, 2);
-      bfly_max_u32<1>(A, lane, 1);
-      bh[h] = e8m0_from_amax(A[0]);
-      const uint32_t mh = scale_multiplier(bh[h]);
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * h + i;
+        A[i] = max(__vimax3_u32(mag2(Y[r][0]), mag2(Y[r][1]), mag2(Y[r][2])), mag2(Y[r][3]));
+      }
+      bfly_max_u32<8>(A, lane, 4);
+      bfly_max_u32<4>(A, lane, 2);
+      bfly_max_u32<2>(A, lane, 1);
+      const uint32_t b0 = e8m0_from_amax(A[0] >> 1), b1 = e8m0_from_amax(A[1] >> 1);
+      bh[h] = b0 | (b1 << 8);
+      const uint32_t m0 = scale_multiplier(b0), m1 = scale_multiplier(b1);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = 16 * h + i;
-        const uint32_t m = __shfl_sync(kFull, mh, (lane & 16) | i);
-        const uint32_t q = e4m3x2(Y0[r], m, Y1[r], m);
-        if (FULL || (colok && r < nrows)) __stcs(rqb + r * Wh, (unsigned short)q);
+        const uint32_t mm = __shfl_sync(kFull, (i & 1) ? m1 : m0, (lane & 24) | (i >> 1));
+        const uint32_t q = e4m3x2_2(make_float2(Y[r][0], Y[r][1]), mm, mm) |
+                           (e4m3x2_2(make_float2(Y[r][2], Y[r][3]), mm, mm) << 16);
+        if (FULL || (colok && r < nrows)) __stcs(rqb + r * Wq, q);
       }
     }
   }
   if (DIRS & kRow) {
-    // lane l stores both blocks of row l
-    const uint32_t mine = bh[0] | (bh[1] << 8);
-    const uint32_t other = __shfl_xor_sync(kFull, mine, 16);
+    // lane l stores the four block scales of row l
+    const uint32_t v = gather_row_scales(bh[0], bh[1], lane, 0, 1);
     if (lane < nrows) {
-      const uint32_t blk0 = lane < 16 ? (mine & 0xFFu) : ((other >> 8) & 0xFFu);
-      const uint32_t blk1 = lane < 16 ? (other & 0xFFu) : ((mine >> 8) & 0xFFu);
-      const bool has1 = tile * kTileCols + 32 < p.N;
-      store_row_scales(p.rs + (row0 + lane) * (int64_t)(W / 32) + 2 * tile, blk0, blk1, has1);
+      const int nb = min(4, (p.N - tile * kTileCols) / 32);
+      store_scales4(p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile, v, nb);
     }
   }
   if (DIRS & kCol) {
-    uint32_t a0 = 0u, a1 = 0u;
+    uint32_t a[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int r = 0; r < 32; r += 2) {
-      a0 = __vimax3_u32(a0, f32_mag(Y0[r]), f32_mag(Y0[r + 1]));
-      a1 = __vimax3_u32(a1, f32_mag(Y1[r]), f32_mag(Y1[r + 1]));
+    for (int r = 0; r < 32; r += 2)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) a[c] = __vimax3_u32(a[c], mag2(Y[r][c]), mag2(Y[r + 1][c]));
+    uint32_t b[4], mu[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      b[c] = e8m0_from_amax(a[c] >> 1);
+      mu[c] = scale_multiplier(b[c]);
     }
-    const uint32_t b0 = e8m0_from_amax(a0), b1 = e8m0_from_amax(a1);
-    const uint32_t m0 = scale_multiplier(b0), m1 = scale_multiplier(b1);
     if (colok)
-      __stcs(reinterpret_cast<unsigned short*>(p.cs + slab * (int64_t)W + c0),
-             (unsigned short)(b0 | (b1 << 8)));
-    unsigned short* qb = reinterpret_cast<unsigned short*>(p.cq + row0 * (int64_t)W + c0);
-    const int Whc = opaque(Wh);
+      __stcs(reinterpret_cast<unsigned int*>(p.cs + slab * (int64_t)W + c0),
+             b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));
+    unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
+    const int Wqc = opaque(Wq);
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
-      const uint32_t q = e4m3x2(Y0[r], m0, Y1[r], m1);
-      if (FULL || (colok && r < nrows)) __stcs(qb + r * Whc, (unsigned short)q);
+      const uint32_t q = e4m3x2_2(make_float2(Y[r][0], Y[r][1]), mu[0], mu[1]) |
+                         (e4m3x2_2(make_float2(Y[r][2], Y[r][3]), mu[2], mu[3]) << 16);
+      if (FULL || (colok && r < nrows)) __stcs(qb + r * Wqc, q);
     }
   }
 }
 
 // Sets up the warp's ring (barriers initialised by lane 0) and primes it.
-template <bool GROUPED>
-__device__ __forceinline__ void ring_prime(const Params& p, const int* cb_s, const int* ro_s,
-                                           const Ring& ring,
-                                           const void* tm_x, const void* tm_dy, int64_t first,
-                                           int64_t stride, int K, int lane, bool swiglu,
-                                           bool with_dy) {
+template <int OPS, int SLOTS, bool GROUPED>
+__device__ __forceinline__ void ring_prime(const Params& p, const Smem& m, Ring<OPS, SLOTS>& r,
+                                           const void* tm_x, const void* tm_dy, int K,
+                                           int lane) {
   if (lane == 0) {
-    for (int i = 0; i < kSlots; ++i) mbar_init(ring.bars + i, 1);
+    for (int i = 0; i < SLOTS; ++i) mbar_init(r.bars + i, 1);
     mbar_init_fence();
-    for (int k = 0; k < kSlots && k < K; ++k)
-      issue_half<GROUPED>(p, cb_s, ro_s, ring, tm_x, tm_dy, first + (k >> 1) * stride, k, swiglu,
-                          with_dy);
+    while (r.k_issue < K && r.k_issue < SLOTS) ring_issue<OPS, SLOTS, GROUPED>(p, m, r, tm_x, tm_dy);
   }
   __syncwarp();
 }
 
-// After a timeout: bounded waits for the copies still in flight into this
-// warp's slots, so that none lands after the CTA has exited.
-__device__ __forceinline__ void ring_drain(const Ring& ring, int k_next, int K) {
-  for (int k = k_next; k < K && k < k_next + kSlots; ++k)
-    mbar_wait(ring.bars + (k % kSlots), (uint32_t)(k / kSlots) & 1u);
-}
-
 template <int ACT, int DIRS, bool STAGED, bool GROUPED>
-__global__ void __launch_bounds__(fwd_threads(ACT, DIRS), 1)
+__global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
     act_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const Params p) {
-  constexpr int kWarps = fwd_warps(ACT);
-  constexpr int kOps = fwd_operands(ACT);
+  using C = Cfg<ACT, false>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  unsigned char* smem = align_smem(smem_raw);
-  float* sig_s = reinterpret_cast<float*>(smem + ring_bytes(kWarps, kOps));
-  int* cb_s = reinterpret_cast<int*>(smem + ring_bytes(kWarps, kOps) +
-                                     (ACT == kSwiGLU ? kSigBytes : 0));
-  int* ro_s = cb_s + (GROUPED ? ((p.E + 1 + 3) / 4) * 4 : 0);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      smem + ring_bytes(kWarps, kOps) + (ACT == kSwiGLU ? kSigBytes : 0) +
-      (GROUPED ? group_bytes(p.E) : 0));
-  const int64_t n_slabs = stage_and_validate<ACT == kSwiGLU, GROUPED>(p, sig_s, cb_s, ro_s);
-  if (n_slabs < 0) return;
+  const Smem m = carve<ACT, false>(smem_raw, GROUPED ? p.E : 0);
+  uint64_t* sig_bar = m.bars + C::kWarps * C::kSlots;
+  const int64_t n_slabs = stage_and_validate<C::kSig, GROUPED>(p, m, sig_bar);
+  if (n_slabs < 0) {
+    // bad offsets: nothing to do, but the table copy must land before exit
+    if (C::kSig && threadIdx.x == 0) mbar_wait(sig_bar, 0u);
+    return;
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n_items = n_slabs * p.n_tiles;
-  const int64_t first = (int64_t)blockIdx.x * kWarps + warp;
-  const int64_t stride = (int64_t)gridDim.x * kWarps;
+  const int64_t first = (int64_t)blockIdx.x * C::kWarps + warp;
+  const int64_t stride = (int64_t)gridDim.x * C::kWarps;
   const int count = first < n_items ? (int)((n_items - 1 - first) / stride + 1) : 0;
   const int K = 2 * count;
-  Ring ring{smem + warp * kSlots * kOps * kOperandHalfBytes, bars + warp * kSlots, kOps};
-  ring_prime<GROUPED>(p, cb_s, ro_s, ring, &tm_x, nullptr, first, stride, K, lane, ACT == kSwiGLU,
-                      false);
+  Ring<C::kOps, C::kSlots> ring;
+  ring.slots = m.ring + warp * C::kSlots * C::kOps * kOpHalfBytes;
+  ring.bars = m.bars + warp * C::kSlots;
+  ring.k_issue = 0;
+  ring.row0 = 0;
+  if (count > 0) ring.cur.init(first, stride, p.n_tiles);
+  ring_prime<C::kOps, C::kSlots, GROUPED>(p, m, ring, &tm_x, nullptr, K, lane);
+  if (C::kSig && !mbar_wait(sig_bar, 0u)) {
+    if (lane == 0) {
+      report_timeout(p, 4u);
+      ring_drain(ring, 0);
+    }
+    return;
+  }
+  // the row scales of each item are loaded one item ahead
+  Cursor cur;
+  int64_t row0 = 0;
+  int nrows = 0;
+  float sv = 0.0f;
+  if (count > 0) {
+    cur.init(first, stride, p.n_tiles);
+    slab_rows<GROUPED>(p, m, cur.slab, row0, nrows);
+    sv = lane < nrows ? __ldg(p.s + row0 + lane) : 0.0f;
+  }
   bool ok = true;
   for (int j = 0; j < count; ++j) {
-    const int64_t it = first + j * stride;
-    const int64_t slab = it / p.n_tiles;
-    const int tile = (int)(it - slab * p.n_tiles);
-    int64_t row0;
-    int nrows;
-    slab_rows<GROUPED>(p, cb_s, ro_s, slab, row0, nrows);
-    const bool full = nrows == 32 && (tile + 1) * kTileCols <= p.N;
-    const int64_t n1 = it + stride, n2 = it + 2 * stride;
+    Cursor nx = cur;
+    nx.next();
+    int64_t row0n = 0;
+    int nrowsn = 0;
+    float svn = 0.0f;
+    if (j + 1 < count) {
+      slab_rows<GROUPED>(p, m, nx.slab, row0n, nrowsn);
+      svn = lane < nrowsn ? __ldg(p.s + row0n + lane) : 0.0f;
+    }
+    const bool full = nrows == 32 && (cur.tile + 1) * kTileCols <= p.N;
     if (full)
-      fwd_tile<ACT, DIRS, STAGED, GROUPED, true>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
-                                        cb_s, ro_s, &tm_x, n1, n2, K, ok);
+      fwd_tile<ACT, DIRS, STAGED, GROUPED, true>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
+                                                 nrows, sv, lane, &tm_x, ok);
     else
-      fwd_tile<ACT, DIRS, STAGED, GROUPED, false>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
-                                         cb_s, ro_s, &tm_x, n1, n2, K, ok);
+      fwd_tile<ACT, DIRS, STAGED, GROUPED, false>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
+                                                  nrows, sv, lane, &tm_x, ok);
+    cur = nx;
+    row0 = row0n;
+    nrows = nrowsn;
+    sv = svn;
     if (!ok) {
       if (lane == 0) {
         report_timeout(p, 1u);
-        ring_drain(ring, 2 * j, K);
+        ring_drain(ring, 2 * j);
       }
       return;
     }
@@ -532,84 +653,88 @@ __global__ void __launch_bounds__(fwd_threads(ACT, DIRS), 1)
 }
 
 // ------------------------------------------------------------- backward tile
-// dscale: each warp reduces its 32 rows x 64 columns to one partial per row
-// and stores it, lane = row, into the workspace at [tile][row] -- plain
-// stores, no fences or counters.  dscale_reduce_kernel, launched right after
-// on the same stream, sums each row's partials in tile order (a fixed order,
-// so dscale is deterministic).
-
-// Row-direction work (dx stores, dscale partials, rowwise MXFP8) runs per
-// 16-row half as the half arrives; the packed bf16 gradients of all 32 rows
-// stay in registers for the colwise pass.
-template <int ACT, int DIRS, bool GROUPED, bool FULL>
-__device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, const Ring& ring,
-                                         int k0, int64_t slab, int tile, int64_t row0, int nrows,
-                                         int lane, const int* cb_s, const int* ro_s,
-                                         const void* tm_x, const void* tm_dy,
-                                         int64_t next_item0, int64_t next_item1, int K,
-                                         bool& ok_flag) {
+// dscale: each warp reduces its 32 rows x 128 columns to one partial per row
+// and stores it, lane = row, into the workspace at [tile][row] (plain stores,
+// no fences or counters); dscale_reduce_kernel, launched next on the same
+// stream, sums each row's partials in tile order (a fixed order, so dscale is
+// deterministic).  Row-direction work runs per 16-row half as the half
+// arrives; the packed bf16 gradients of all 32 rows stay in registers for the
+// colwise pass.
+// (`full`: all 32 rows and 128 columns exist; a runtime flag, so that the
+// large unrolled body exists once)
+template <int ACT, int DIRS, bool GROUPED, int OPS, int SLOTS>
+__device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OPS, SLOTS>& ring,
+                                         int k0, int K, int64_t slab, int tile, int64_t row0,
+                                         int nrows, bool FULL, float sv, int lane,
+                                         const void* tm_x, const void* tm_dy, bool& ok_flag) {
   const int N = p.N, W = p.W;
-  const int Wh = W >> 1;
-  const int c0 = tile * kTileCols + 2 * lane;
+  const int Wq = W >> 2;   // code row stride in 32-bit words
+  const int c0 = tile * kTileCols + 4 * lane;
   const bool colok = c0 < N;
-  const float sv = lane < nrows ? __ldg(p.s + row0 + lane) : 0.0f;
 
-  uint32_t DG[32], DU[32];
+  uint32_t DG[32][2], DU[32][2];
   float ph[2];
   uint32_t bh[2];
-  unsigned short* rqb = reinterpret_cast<unsigned short*>(p.rq + row0 * (int64_t)W + c0);
-  uint32_t* dxb = reinterpret_cast<uint32_t*>(p.dx + row0 * (int64_t)W + c0);
+  unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + c0);
+  uint2* dxb = reinterpret_cast<uint2*>(p.dx + row0 * (int64_t)W + c0);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int k = k0 + h;
-    const int slot = k % kSlots;
-    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / kSlots) & 1u)) { ok_flag = false; return; }
-    const unsigned char* sm = ring.slots + slot * ring.ops * kOperandHalfBytes + 4 * lane;
+    const int slot = k % SLOTS;
+    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / SLOTS) & 1u)) { ok_flag = false; return; }
+    const unsigned char* sm = ring.slots + slot * OPS * kOpHalfBytes + 8 * lane;
     float P[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int r = 16 * h + i;
-      const uint32_t D = *reinterpret_cast<const uint32_t*>(sm + i * 128);
-      const uint32_t G = *reinterpret_cast<const uint32_t*>(sm + kOperandHalfBytes + i * 128);
+      const uint2 D = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
+      const uint2 G = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
       const float sr = __shfl_sync(kFull, sv, r);
-      const float d0 = bf16_lo(D), d1 = bf16_hi(D);
-      const float p0 = __fmul_rn(d0, sr), p1 = __fmul_rn(d1, sr);
-      float h0, h1;
+      const float2 s2 = make_float2(sr, sr);
+      const float2 d01 = bf16x2_to_f2(D.x), d23 = bf16x2_to_f2(D.y);
+      const float2 p01 = mul2(d01, s2), p23 = mul2(d23, s2);
+      float2 dg01, dg23, du01, du23, h01, h23;
       if (ACT == kSwiGLU) {
-        const uint32_t U =
-            *reinterpret_cast<const uint32_t*>(sm + 2 * kOperandHalfBytes + i * 128);
-        const float g0 = bf16_lo(G), g1 = bf16_hi(G);
-        const float u0 = bf16_lo(U), u1 = bf16_hi(U);
-        float s0, s1;
-        sigma_pair(sig, G, s0, s1);
-        const float si0 = __fmul_rn(g0, s0), si1 = __fmul_rn(g1, s1);
-        const float ds0 = __fmaf_rn(si0, __fsub_rn(1.0f, s0), s0);
-        const float ds1 = __fmaf_rn(si1, __fsub_rn(1.0f, s1), s1);
-        DG[r] = pack_bf16x2(__fmul_rn(__fmul_rn(p0, u0), ds0), __fmul_rn(__fmul_rn(p1, u1), ds1));
-        DU[r] = pack_bf16x2(__fmul_rn(p0, si0), __fmul_rn(p1, si1));
-        h0 = __fmul_rn(si0, u0);
-        h1 = __fmul_rn(si1, u1);
+        const uint2 U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
+        const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
+        float2 sg01, sg23;
+        sigma_pair(m.sig, G.x, sg01.x, sg01.y);
+        sigma_pair(m.sig, G.y, sg23.x, sg23.y);
+        const float2 si01 = mul2(bf16x2_to_f2(G.x), sg01), si23 = mul2(bf16x2_to_f2(G.y), sg23);
+        const float2 one = make_float2(1.0f, 1.0f);
+        const float2 ds01 = fma2(si01, sub2(one, sg01), sg01);
+        const float2 ds23 = fma2(si23, sub2(one, sg23), sg23);
+        dg01 = mul2(mul2(p01, u01), ds01);
+        dg23 = mul2(mul2(p23, u23), ds23);
+        du01 = mul2(p01, si01);
+        du23 = mul2(p23, si23);
+        h01 = mul2(si01, u01);
+        h23 = mul2(si23, u23);
       } else {
-        const float r0 = relu_keep_nan(bf16_lo(G)), r1 = relu_keep_nan(bf16_hi(G));
-        DG[r] = pack_bf16x2(__fmul_rn(p0, __fmul_rn(2.0f, r0)), __fmul_rn(p1, __fmul_rn(2.0f, r1)));
-        DU[r] = 0u;
-        h0 = __fmul_rn(r0, r0);
-        h1 = __fmul_rn(r1, r1);
+        const float r0 = relu_keep_nan(bf16_lo(G.x)), r1 = relu_keep_nan(bf16_hi(G.x));
+        const float r2 = relu_keep_nan(bf16_lo(G.y)), r3 = relu_keep_nan(bf16_hi(G.y));
+        const float2 two = make_float2(2.0f, 2.0f);
+        dg01 = mul2(p01, mul2(two, make_float2(r0, r1)));
+        dg23 = mul2(p23, mul2(two, make_float2(r2, r3)));
+        du01 = du23 = make_float2(0.0f, 0.0f);
+        h01 = mul2(make_float2(r0, r1), make_float2(r0, r1));
+        h23 = mul2(make_float2(r2, r3), make_float2(r2, r3));
       }
-      P[i] = __fmaf_rn(d1, h1, __fmul_rn(d0, h0));
-      if (!FULL && r >= nrows) { DG[r] = 0u; DU[r] = 0u; P[i] = 0.0f; }
+      const bool live = FULL || r < nrows;
+      DG[r][0] = live ? pack_bf16x2(dg01.x, dg01.y) : 0u;
+      DG[r][1] = live ? pack_bf16x2(dg23.x, dg23.y) : 0u;
+      DU[r][0] = (live && ACT == kSwiGLU) ? pack_bf16x2(du01.x, du01.y) : 0u;
+      DU[r][1] = (live && ACT == kSwiGLU) ? pack_bf16x2(du23.x, du23.y) : 0u;
+      P[i] = live ? __fmaf_rn(d23.y, h23.y, __fmaf_rn(d23.x, h23.x,
+                              __fmaf_rn(d01.y, h01.y, __fmul_rn(d01.x, h01.x))))
+                  : 0.0f;
       if (p.dx != nullptr && (FULL || (colok && r < nrows))) {
-        __stcs(dxb + r * Wh, DG[r]);
-        if (ACT == kSwiGLU) __stcs(dxb + r * Wh + (N >> 1), DU[r]);
+        __stcs(dxb + r * Wq, make_uint2(DG[r][0], DG[r][1]));
+        if (ACT == kSwiGLU) __stcs(dxb + r * Wq + (N >> 2), make_uint2(DU[r][0], DU[r][1]));
       }
     }
     __syncwarp();
-    if (lane == 0 && k + kSlots < K) {
-      const int kn = k + kSlots;
-      issue_half<GROUPED>(p, cb_s, ro_s, ring, tm_x, tm_dy,
-                          (kn >> 1) == (k0 >> 1) + 1 ? next_item0 : next_item1, kn,
-                          ACT == kSwiGLU, true);
-    }
+    if (lane == 0 && ring.k_issue < K) ring_issue<OPS, SLOTS, GROUPED>(p, m, ring, tm_x, tm_dy);
     if (p.dscale != nullptr) {
       // lane l ends with the warp sum of row 16h + (l >> 1)
       bfly_sum_f32<8>(P, lane, 16);
@@ -619,35 +744,41 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, cons
       ph[h] = __fadd_rn(P[0], __shfl_xor_sync(kFull, P[0], 1));
     }
     if (DIRS & kRow) {
-      // packed per-row block maxima: low half dgate, high half dup
+      // packed per-row block maxima over the lane's 4 columns: low half dgate,
+      // high half dup
       uint32_t A[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const uint32_t ag = DG[16 * h + i] & 0x7FFF7FFFu, au = DU[16 * h + i] & 0x7FFF7FFFu;
-        A[i] = __vmaxu2(__byte_perm(ag, au, 0x5410), __byte_perm(ag, au, 0x7632));
+        const int r = 16 * h + i;
+        const uint32_t mg = __vmaxu2(DG[r][0] & 0x7FFF7FFFu, DG[r][1] & 0x7FFF7FFFu);
+        const uint32_t mu = __vmaxu2(DU[r][0] & 0x7FFF7FFFu, DU[r][1] & 0x7FFF7FFFu);
+        A[i] = __vmaxu2(__byte_perm(mg, mu, 0x5410), __byte_perm(mg, mu, 0x7632));
       }
-      bfly_max_u16x2<8>(A, lane, 8);
-      bfly_max_u16x2<4>(A, lane, 4);
-      bfly_max_u16x2<2>(A, lane, 2);
-      bfly_max_u16x2<1>(A, lane, 1);
-      // lane l: row 16h + (l & 15), block (l >> 4)
-      const uint32_t bg = e8m0_from_amax(A[0] << 16), bu = e8m0_from_amax(A[0] & 0xFFFF0000u);
-      bh[h] = bg | (bu << 8);
-      const uint32_t mgh = scale_multiplier(bg), muh = scale_multiplier(bu);
+      bfly_max_u16x2<8>(A, lane, 4);
+      bfly_max_u16x2<4>(A, lane, 2);
+      bfly_max_u16x2<2>(A, lane, 1);
+      // lane l: rows 16h + 2(l & 7) + {0, 1} of block l >> 3
+      const uint32_t bg0 = e8m0_from_amax(A[0] << 16), bu0 = e8m0_from_amax(A[0] & 0xFFFF0000u);
+      const uint32_t bg1 = e8m0_from_amax(A[1] << 16), bu1 = e8m0_from_amax(A[1] & 0xFFFF0000u);
+      bh[h] = bg0 | (bu0 << 8) | (bg1 << 16) | (bu1 << 24);
+      const uint32_t mg0 = scale_multiplier(bg0), mg1 = scale_multiplier(bg1);
+      const uint32_t mu0 = scale_multiplier(bu0), mu1 = scale_multiplier(bu1);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = 16 * h + i;
-        const int src = (lane & 16) | i;
-        const uint32_t mg = __shfl_sync(kFull, mgh, src);
-        const uint32_t qg = e4m3x2(bf16_lo(DG[r]), mg, bf16_hi(DG[r]), mg);
+        const int src = (lane & 24) | (i >> 1);
+        const uint32_t mg = __shfl_sync(kFull, (i & 1) ? mg1 : mg0, src);
+        const uint32_t qg = e4m3x2_2(bf16x2_to_f2(DG[r][0]), mg, mg) |
+                            (e4m3x2_2(bf16x2_to_f2(DG[r][1]), mg, mg) << 16);
         uint32_t qu = 0;
         if (ACT == kSwiGLU) {
-          const uint32_t mu = __shfl_sync(kFull, muh, src);
-          qu = e4m3x2(bf16_lo(DU[r]), mu, bf16_hi(DU[r]), mu);
+          const uint32_t mu = __shfl_sync(kFull, (i & 1) ? mu1 : mu0, src);
+          qu = e4m3x2_2(bf16x2_to_f2(DU[r][0]), mu, mu) |
+               (e4m3x2_2(bf16x2_to_f2(DU[r][1]), mu, mu) << 16);
         }
         if (FULL || (colok && r < nrows)) {
-          __stcs(rqb + r * Wh, (unsigned short)qg);
-          if (ACT == kSwiGLU) __stcs(rqb + r * Wh + (N >> 1), (unsigned short)qu);
+          __stcs(rqb + r * Wq, qg);
+          if (ACT == kSwiGLU) __stcs(rqb + r * Wq + (N >> 2), qu);
         }
       }
     }
@@ -658,46 +789,57 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, cons
     if (lane < nrows) __stcg(p.part + (int64_t)tile * p.M + row0 + lane, lane < 16 ? v0 : v1);
   }
   if (DIRS & kRow) {
-    // lane l stores the four blocks (dgate 0/1, dup 0/1) of row l
-    const uint32_t mine = bh[0] | (bh[1] << 16);   // bytes: g(h0) u(h0) g(h1) u(h1)
-    const uint32_t other = __shfl_xor_sync(kFull, mine, 16);
+    // lane l stores the block scales of row l (dgate blocks, then dup blocks)
+    const uint32_t vg = gather_row_scales(bh[0], bh[1], lane, 0, 2);
+    const uint32_t vu = gather_row_scales(bh[0], bh[1], lane, 1, 3);
     if (lane < nrows) {
-      const int sh = lane < 16 ? 0 : 16;
-      const uint32_t lo = lane < 16 ? mine : other, hi = lane < 16 ? other : mine;
-      const bool has1 = tile * kTileCols + 32 < N;
-      uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 2 * tile;
-      store_row_scales(rsr, (lo >> sh) & 0xFFu, (hi >> sh) & 0xFFu, has1);
-      if (ACT == kSwiGLU)
-        store_row_scales(rsr + N / 32, (lo >> (sh + 8)) & 0xFFu, (hi >> (sh + 8)) & 0xFFu, has1);
+      const int nb = min(4, (N - tile * kTileCols) / 32);
+      uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
+      store_scales4(rsr, vg, nb);
+      if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
     }
   }
   if (DIRS & kCol) {
-    uint32_t ag = 0u, au = 0u;
+    uint32_t ag[2] = {0u, 0u}, au[2] = {0u, 0u};
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      ag = __vmaxu2(ag, DG[r] & 0x7FFF7FFFu);
-      au = __vmaxu2(au, DU[r] & 0x7FFF7FFFu);
+    for (int r = 0; r < 32; r += 2)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        ag[c] = __vimax3_u16x2(ag[c], DG[r][c] & 0x7FFF7FFFu, DG[r + 1][c] & 0x7FFF7FFFu);
+        au[c] = __vimax3_u16x2(au[c], DU[r][c] & 0x7FFF7FFFu, DU[r + 1][c] & 0x7FFF7FFFu);
+      }
+    uint32_t bg[4], bu[4], mg[4], mu[4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      bg[2 * c] = e8m0_from_amax(ag[c] << 16);
+      bg[2 * c + 1] = e8m0_from_amax(ag[c] & 0xFFFF0000u);
+      bu[2 * c] = e8m0_from_amax(au[c] << 16);
+      bu[2 * c + 1] = e8m0_from_amax(au[c] & 0xFFFF0000u);
     }
-    const uint32_t bg0 = e8m0_from_amax(ag << 16), bg1 = e8m0_from_amax(ag & 0xFFFF0000u);
-    const uint32_t bu0 = e8m0_from_amax(au << 16), bu1 = e8m0_from_amax(au & 0xFFFF0000u);
-    const uint32_t mg0 = scale_multiplier(bg0), mg1 = scale_multiplier(bg1);
-    const uint32_t mu0 = scale_multiplier(bu0), mu1 = scale_multiplier(bu1);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      mg[c] = scale_multiplier(bg[c]);
+      mu[c] = scale_multiplier(bu[c]);
+    }
     if (colok) {
       uint8_t* csr = p.cs + slab * (int64_t)W + c0;
-      __stcs(reinterpret_cast<unsigned short*>(csr), (unsigned short)(bg0 | (bg1 << 8)));
+      __stcs(reinterpret_cast<unsigned int*>(csr), bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
       if (ACT == kSwiGLU)
-        __stcs(reinterpret_cast<unsigned short*>(csr + N), (unsigned short)(bu0 | (bu1 << 8)));
+        __stcs(reinterpret_cast<unsigned int*>(csr + N),
+               bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
     }
-    unsigned short* qb = reinterpret_cast<unsigned short*>(p.cq + row0 * (int64_t)W + c0);
-    const int Whc = opaque(Wh);
+    unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
+    const int Wqc = opaque(Wq);
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
-      const uint32_t qg = e4m3x2(bf16_lo_p(DG[r]), mg0, bf16_hi_p(DG[r]), mg1);
+      const uint32_t qg = e4m3x2_2(bf16x2_to_f2_p(DG[r][0]), mg[0], mg[1]) |
+                          (e4m3x2_2(bf16x2_to_f2_p(DG[r][1]), mg[2], mg[3]) << 16);
       if (FULL || (colok && r < nrows)) {
-        __stcs(qb + r * Whc, (unsigned short)qg);
+        __stcs(qb + r * Wqc, qg);
         if (ACT == kSwiGLU) {
-          const uint32_t qu = e4m3x2(bf16_lo_p(DU[r]), mu0, bf16_hi_p(DU[r]), mu1);
-          __stcs(qb + r * Whc + (N >> 1), (unsigned short)qu);
+          const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(DU[r][0]), mu[0], mu[1]) |
+                              (e4m3x2_2(bf16x2_to_f2_p(DU[r][1]), mu[2], mu[3]) << 16);
+          __stcs(qb + r * Wqc + (N >> 2), qu);
         }
       }
     }
@@ -705,54 +847,74 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const float* sig, cons
 }
 
 template <int ACT, int DIRS, bool GROUPED>
-__global__ void __launch_bounds__(bwd_threads(ACT, DIRS), 1)
+__global__ void __launch_bounds__(Cfg<ACT, true>::kThreads, 1)
     act_bwd_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_dy, const Params p) {
-  constexpr int kWarps = bwd_warps(ACT);
-  constexpr int kOps = bwd_operands(ACT);
+  using C = Cfg<ACT, true>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  unsigned char* smem = align_smem(smem_raw);
-  float* sig_s = reinterpret_cast<float*>(smem + ring_bytes(kWarps, kOps));
-  int* cb_s = reinterpret_cast<int*>(smem + ring_bytes(kWarps, kOps) +
-                                     (ACT == kSwiGLU ? kSigBytes : 0));
-  int* ro_s = cb_s + (GROUPED ? ((p.E + 1 + 3) / 4) * 4 : 0);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      smem + ring_bytes(kWarps, kOps) + (ACT == kSwiGLU ? kSigBytes : 0) +
-      (GROUPED ? group_bytes(p.E) : 0));
-  const int64_t n_slabs = stage_and_validate<ACT == kSwiGLU, GROUPED>(p, sig_s, cb_s, ro_s);
-  if (n_slabs < 0) return;
+  const Smem m = carve<ACT, true>(smem_raw, GROUPED ? p.E : 0);
+  uint64_t* sig_bar = m.bars + C::kWarps * C::kSlots;
+  const int64_t n_slabs = stage_and_validate<C::kSig, GROUPED>(p, m, sig_bar);
+  if (n_slabs < 0) {
+    if (C::kSig && threadIdx.x == 0) mbar_wait(sig_bar, 0u);
+    return;
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n_items = n_slabs * p.n_tiles;
-  const int64_t first = (int64_t)blockIdx.x * kWarps + warp;
-  const int64_t stride = (int64_t)gridDim.x * kWarps;
+  const int64_t first = (int64_t)blockIdx.x * C::kWarps + warp;
+  const int64_t stride = (int64_t)gridDim.x * C::kWarps;
   const int count = first < n_items ? (int)((n_items - 1 - first) / stride + 1) : 0;
   const int K = 2 * count;
-  Ring ring{smem + warp * kSlots * kOps * kOperandHalfBytes, bars + warp * kSlots, kOps};
-  ring_prime<GROUPED>(p, cb_s, ro_s, ring, &tm_x, &tm_dy, first, stride, K, lane, ACT == kSwiGLU,
-                      true);
+  Ring<C::kOps, C::kSlots> ring;
+  ring.slots = m.ring + warp * C::kSlots * C::kOps * kOpHalfBytes;
+  ring.bars = m.bars + warp * C::kSlots;
+  ring.k_issue = 0;
+  ring.row0 = 0;
+  if (count > 0) ring.cur.init(first, stride, p.n_tiles);
+  ring_prime<C::kOps, C::kSlots, GROUPED>(p, m, ring, &tm_x, &tm_dy, K, lane);
+  if (C::kSig && !mbar_wait(sig_bar, 0u)) {
+    if (lane == 0) {
+      report_timeout(p, 4u);
+      ring_drain(ring, 0);
+    }
+    return;
+  }
+  // the row scales of each item are loaded one item ahead
+  Cursor cur;
+  int64_t row0 = 0;
+  int nrows = 0;
+  float sv = 0.0f;
+  if (count > 0) {
+    cur.init(first, stride, p.n_tiles);
+    slab_rows<GROUPED>(p, m, cur.slab, row0, nrows);
+    sv = lane < nrows ? __ldg(p.s + row0 + lane) : 0.0f;
+  }
   bool ok = true;
   for (int j = 0; j < count; ++j) {
-    const int64_t it = first + j * stride;
-    const int64_t slab = it / p.n_tiles;
-    const int tile = (int)(it - slab * p.n_tiles);
-    int64_t row0;
-    int nrows;
-    slab_rows<GROUPED>(p, cb_s, ro_s, slab, row0, nrows);
-    const bool full = nrows == 32 && (tile + 1) * kTileCols <= p.N;
-    const int64_t n1 = it + stride, n2 = it + 2 * stride;
-    if (full)
-      bwd_tile<ACT, DIRS, GROUPED, true>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
-                                         cb_s, ro_s, &tm_x, &tm_dy, n1, n2, K, ok);
-    else
-      bwd_tile<ACT, DIRS, GROUPED, false>(p, sig_s, ring, 2 * j, slab, tile, row0, nrows, lane,
-                                          cb_s, ro_s, &tm_x, &tm_dy, n1, n2, K, ok);
+    Cursor nx = cur;
+    nx.next();
+    int64_t row0n = 0;
+    int nrowsn = 0;
+    float svn = 0.0f;
+    if (j + 1 < count) {
+      slab_rows<GROUPED>(p, m, nx.slab, row0n, nrowsn);
+      svn = lane < nrowsn ? __ldg(p.s + row0n + lane) : 0.0f;
+    }
+    const bool full = nrows == 32 && (cur.tile + 1) * kTileCols <= p.N;
+    bwd_tile<ACT, DIRS, GROUPED>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, full, sv,
+                                 lane, &tm_x, &tm_dy, ok);
+    cur = nx;
+    row0 = row0n;
+    nrows = nrowsn;
+    sv = svn;
     if (!ok) {
       if (lane == 0) {
         report_timeout(p, 2u);
-        ring_drain(ring, 2 * j, K);
+        ring_drain(ring, 2 * j);
       }
       return;
     }
   }
 }
+
 }  // namespace moeact

@@ -277,7 +277,7 @@ def test_splits_to_offsets_status(cuda_device, splits, M, status):
 
 def test_splits_to_offsets_many_groups(cuda_device):
     g = np.random.default_rng(3)
-    m = (g.integers(0, 5, 4096) * 32 + g.integers(0, 3, 4096)).astype(np.int64)
+    m = (g.integers(0, 5, 2040) * 32 + g.integers(0, 3, 2040)).astype(np.int64)
     M = int(m.sum())
     st, ro, cb = oracle.splits_to_offsets(m, M)
     gro, gcb, gst = mg.splits_to_offsets(torch.from_numpy(m).to(cuda_device), M)

@@ -50,9 +50,9 @@ FwdVariant fwd_variant() {
   return {act_fwd_kernel<ACT, DIRS, STAGED, GROUPED>, Cfg<ACT, false>::kThreads,
           smem_bytes<ACT, false>(false, 0), Cfg<ACT, false>::kSig};
 }
-template <int ACT, int DIRS, bool GROUPED>
+template <int ACT, int DIRS, bool GROUPED, bool REREAD>
 BwdVariant bwd_variant() {
-  return {act_bwd_kernel<ACT, DIRS, GROUPED>, Cfg<ACT, true>::kThreads,
+  return {act_bwd_kernel<ACT, DIRS, GROUPED, REREAD>, Cfg<ACT, true>::kThreads,
           smem_bytes<ACT, true>(false, 0), Cfg<ACT, true>::kSig};
 }
 
@@ -68,12 +68,18 @@ void fwd_all(FwdVariant* out, int& n) {
   }
 }
 
+template <int ACT, bool GROUPED, bool REREAD>
+void bwd_all_rr(BwdVariant* out, int& n) {
+  out[n++] = bwd_variant<ACT, 0, GROUPED, REREAD>();
+  out[n++] = bwd_variant<ACT, kRow, GROUPED, REREAD>();
+  out[n++] = bwd_variant<ACT, kCol, GROUPED, REREAD>();
+  out[n++] = bwd_variant<ACT, kRow | kCol, GROUPED, REREAD>();
+}
+
 template <int ACT, bool GROUPED>
 void bwd_all(BwdVariant* out, int& n) {
-  out[n++] = bwd_variant<ACT, 0, GROUPED>();
-  out[n++] = bwd_variant<ACT, kRow, GROUPED>();
-  out[n++] = bwd_variant<ACT, kCol, GROUPED>();
-  out[n++] = bwd_variant<ACT, kRow | kCol, GROUPED>();
+  bwd_all_rr<ACT, GROUPED, false>(out, n);
+  bwd_all_rr<ACT, GROUPED, true>(out, n);
 }
 
 // Extra shared memory of a grouped call (its col-block offsets), at most.
@@ -103,7 +109,7 @@ moeact_status init_device(int dev) {
   }
 
   FwdVariant fv[32];
-  BwdVariant bv[32];
+  BwdVariant bv[40];
   int nf = 0, nb = 0;
   fwd_all<kSwiGLU, false>(fv, nf);
   fwd_all<kSwiGLU, true>(fv, nf);
@@ -231,12 +237,19 @@ FwdVariant pick_fwd(int dirs, bool staged) {
   return fwd_variant<ACT, kRow | kCol, false, GROUPED>();
 }
 
+// With dX written, the colwise pass re-reads it instead of keeping the whole
+// tile in registers.
+template <int ACT, bool GROUPED, bool REREAD>
+BwdVariant pick_bwd_rr(int dirs) {
+  if (dirs == 0) return bwd_variant<ACT, 0, GROUPED, REREAD>();
+  if (dirs == kRow) return bwd_variant<ACT, kRow, GROUPED, REREAD>();
+  if (dirs == kCol) return bwd_variant<ACT, kCol, GROUPED, REREAD>();
+  return bwd_variant<ACT, kRow | kCol, GROUPED, REREAD>();
+}
+
 template <int ACT, bool GROUPED>
-BwdVariant pick_bwd(int dirs) {
-  if (dirs == 0) return bwd_variant<ACT, 0, GROUPED>();
-  if (dirs == kRow) return bwd_variant<ACT, kRow, GROUPED>();
-  if (dirs == kCol) return bwd_variant<ACT, kCol, GROUPED>();
-  return bwd_variant<ACT, kRow | kCol, GROUPED>();
+BwdVariant pick_bwd(int dirs, bool reread) {
+  return reread ? pick_bwd_rr<ACT, GROUPED, true>(dirs) : pick_bwd_rr<ACT, GROUPED, false>(dirs);
 }
 
 // Tensor map of a bf16 [rows, width] matrix with a row stride of `ld`
@@ -363,8 +376,9 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   p.err = g_err_ptr[dev];
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
   BwdVariant v;
-  if (act == kSwiGLU) v = grouped ? pick_bwd<kSwiGLU, true>(dirs) : pick_bwd<kSwiGLU, false>(dirs);
-  else v = grouped ? pick_bwd<kSReLU, true>(dirs) : pick_bwd<kSReLU, false>(dirs);
+  const bool rr = dx != nullptr;
+  if (act == kSwiGLU) v = grouped ? pick_bwd<kSwiGLU, true>(dirs, rr) : pick_bwd<kSwiGLU, false>(dirs, rr);
+  else v = grouped ? pick_bwd<kSReLU, true>(dirs, rr) : pick_bwd<kSReLU, false>(dirs, rr);
   CUtensorMap tx, tdy;
   if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
   if ((st = make_map(&tdy, dy, N, M, lddy))) return st;

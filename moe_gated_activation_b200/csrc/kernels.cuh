@@ -652,6 +652,49 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------- backward row
+// The backward of one row's four columns (a lane's share): packed bf16
+// dgate/dup pairs and the row's dscale partial sum_c dY*h.
+template <int ACT>
+__device__ __forceinline__ void bwd_row(const float* sig, uint2 D, uint2 G, uint2 U, float sr,
+                                        uint32_t& dg0, uint32_t& dg1, uint32_t& du0,
+                                        uint32_t& du1, float& part) {
+  const float2 s2 = make_float2(sr, sr);
+  const float2 d01 = bf16x2_to_f2(D.x), d23 = bf16x2_to_f2(D.y);
+  const float2 p01 = mul2(d01, s2), p23 = mul2(d23, s2);
+  float2 h01, h23;
+  if (ACT == kSwiGLU) {
+    const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
+    float2 sg01, sg23;
+    sigma_pair(sig, G.x, sg01.x, sg01.y);
+    sigma_pair(sig, G.y, sg23.x, sg23.y);
+    const float2 si01 = mul2(bf16x2_to_f2(G.x), sg01), si23 = mul2(bf16x2_to_f2(G.y), sg23);
+    const float2 one = make_float2(1.0f, 1.0f);
+    const float2 ds01 = fma2(si01, sub2(one, sg01), sg01);
+    const float2 ds23 = fma2(si23, sub2(one, sg23), sg23);
+    const float2 dga = mul2(mul2(p01, u01), ds01), dgb = mul2(mul2(p23, u23), ds23);
+    const float2 dua = mul2(p01, si01), dub = mul2(p23, si23);
+    dg0 = pack_bf16x2(dga.x, dga.y);
+    dg1 = pack_bf16x2(dgb.x, dgb.y);
+    du0 = pack_bf16x2(dua.x, dua.y);
+    du1 = pack_bf16x2(dub.x, dub.y);
+    h01 = mul2(si01, u01);
+    h23 = mul2(si23, u23);
+  } else {
+    const float2 r01 = make_float2(relu_keep_nan(bf16_lo(G.x)), relu_keep_nan(bf16_hi(G.x)));
+    const float2 r23 = make_float2(relu_keep_nan(bf16_lo(G.y)), relu_keep_nan(bf16_hi(G.y)));
+    const float2 two = make_float2(2.0f, 2.0f);
+    const float2 dga = mul2(p01, mul2(two, r01)), dgb = mul2(p23, mul2(two, r23));
+    dg0 = pack_bf16x2(dga.x, dga.y);
+    dg1 = pack_bf16x2(dgb.x, dgb.y);
+    du0 = du1 = 0u;
+    h01 = mul2(r01, r01);
+    h23 = mul2(r23, r23);
+  }
+  part = __fmaf_rn(d23.y, h23.y, __fmaf_rn(d23.x, h23.x, __fmaf_rn(d01.y, h01.y,
+                                                                    __fmul_rn(d01.x, h01.x))));
+}
+
 // ------------------------------------------------------------- backward tile
 // dscale: each warp reduces its 32 rows x 128 columns to one partial per row
 // and stores it, lane = row, into the workspace at [tile][row] (plain stores,
@@ -846,7 +889,171 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
   }
 }
 
-template <int ACT, int DIRS, bool GROUPED>
+// The backward tile when dX is written (the usual case): the colwise pass
+// re-reads each lane's own just-written dX columns (program order makes a
+// thread's stores visible to its later loads; the 16 KiB per tile is still in
+// L2), so only one 16-row half of gradients is held in registers.  Colwise
+// maxima are accumulated on the fly.
+template <int ACT, int DIRS, bool GROUPED, bool FULL, int OPS, int SLOTS>
+__device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
+                                            Ring<OPS, SLOTS>& ring, int k0, int K, int64_t slab,
+                                            int tile, int64_t row0, int nrows, float sv, int lane,
+                                            const void* tm_x, const void* tm_dy, bool& ok_flag) {
+  const int N = p.N, W = p.W;
+  const int Wq = W >> 2;   // row stride in 32-bit words (codes) / 8-byte words (dx)
+  const int c0 = tile * kTileCols + 4 * lane;
+  const bool colok = c0 < N;
+  float ph[2];
+  uint32_t bh[2];
+  uint32_t acg[2] = {0u, 0u}, acu[2] = {0u, 0u};   // colwise maxima (packed bf16 magnitudes)
+  unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + c0);
+  uint2* dxb = reinterpret_cast<uint2*>(p.dx + row0 * (int64_t)W + c0);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k = k0 + h;
+    const int slot = k % SLOTS;
+    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / SLOTS) & 1u)) { ok_flag = false; return; }
+    const unsigned char* sm = ring.slots + slot * OPS * kOpHalfBytes + 8 * lane;
+    uint32_t DG[16][2], DU[16][2];
+    float P[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = 16 * h + i;
+      const uint2 D = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
+      const uint2 G = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
+      uint2 U = make_uint2(0u, 0u);
+      if (ACT == kSwiGLU) U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
+      const float sr = __shfl_sync(kFull, sv, r);
+      float part;
+      bwd_row<ACT>(m.sig, D, G, U, sr, DG[i][0], DG[i][1], DU[i][0], DU[i][1], part);
+      const bool live = FULL || r < nrows;
+      if (!FULL && !live) { DG[i][0] = DG[i][1] = DU[i][0] = DU[i][1] = 0u; part = 0.0f; }
+      P[i] = part;
+      if (FULL || (colok && live)) {
+        dxb[r * Wq] = make_uint2(DG[i][0], DG[i][1]);
+        if (ACT == kSwiGLU) dxb[r * Wq + (N >> 2)] = make_uint2(DU[i][0], DU[i][1]);
+      }
+      if (DIRS & kCol) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          acg[c] = __vmaxu2(acg[c], DG[i][c] & 0x7FFF7FFFu);
+          if (ACT == kSwiGLU) acu[c] = __vmaxu2(acu[c], DU[i][c] & 0x7FFF7FFFu);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && ring.k_issue < K) ring_issue<OPS, SLOTS, GROUPED>(p, m, ring, tm_x, tm_dy);
+    if (p.dscale != nullptr) {
+      bfly_sum_f32<8>(P, lane, 16);
+      bfly_sum_f32<4>(P, lane, 8);
+      bfly_sum_f32<2>(P, lane, 4);
+      bfly_sum_f32<1>(P, lane, 2);
+      ph[h] = __fadd_rn(P[0], __shfl_xor_sync(kFull, P[0], 1));
+    }
+    if (DIRS & kRow) {
+      uint32_t A[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t mg = __vmaxu2(DG[i][0] & 0x7FFF7FFFu, DG[i][1] & 0x7FFF7FFFu);
+        const uint32_t mu = __vmaxu2(DU[i][0] & 0x7FFF7FFFu, DU[i][1] & 0x7FFF7FFFu);
+        A[i] = __vmaxu2(__byte_perm(mg, mu, 0x5410), __byte_perm(mg, mu, 0x7632));
+      }
+      bfly_max_u16x2<8>(A, lane, 4);
+      bfly_max_u16x2<4>(A, lane, 2);
+      bfly_max_u16x2<2>(A, lane, 1);
+      const uint32_t bg0 = e8m0_from_amax(A[0] << 16), bu0 = e8m0_from_amax(A[0] & 0xFFFF0000u);
+      const uint32_t bg1 = e8m0_from_amax(A[1] << 16), bu1 = e8m0_from_amax(A[1] & 0xFFFF0000u);
+      bh[h] = bg0 | (bu0 << 8) | (bg1 << 16) | (bu1 << 24);
+      const uint32_t mg0 = scale_multiplier(bg0), mg1 = scale_multiplier(bg1);
+      const uint32_t mu0 = scale_multiplier(bu0), mu1 = scale_multiplier(bu1);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * h + i;
+        const int src = (lane & 24) | (i >> 1);
+        const uint32_t mg = __shfl_sync(kFull, (i & 1) ? mg1 : mg0, src);
+        const uint32_t qg = e4m3x2_2(bf16x2_to_f2(DG[i][0]), mg, mg) |
+                            (e4m3x2_2(bf16x2_to_f2(DG[i][1]), mg, mg) << 16);
+        uint32_t qu = 0;
+        if (ACT == kSwiGLU) {
+          const uint32_t mu = __shfl_sync(kFull, (i & 1) ? mu1 : mu0, src);
+          qu = e4m3x2_2(bf16x2_to_f2(DU[i][0]), mu, mu) |
+               (e4m3x2_2(bf16x2_to_f2(DU[i][1]), mu, mu) << 16);
+        }
+        if (FULL || (colok && r < nrows)) {
+          __stcs(rqb + r * Wq, qg);
+          if (ACT == kSwiGLU) __stcs(rqb + r * Wq + (N >> 2), qu);
+        }
+      }
+    }
+  }
+  if (p.dscale != nullptr) {
+    const int src = 2 * (lane & 15);
+    const float v0 = __shfl_sync(kFull, ph[0], src), v1 = __shfl_sync(kFull, ph[1], src);
+    if (lane < nrows) __stcg(p.part + (int64_t)tile * p.M + row0 + lane, lane < 16 ? v0 : v1);
+  }
+  if (DIRS & kRow) {
+    const uint32_t vg = gather_row_scales(bh[0], bh[1], lane, 0, 2);
+    const uint32_t vu = gather_row_scales(bh[0], bh[1], lane, 1, 3);
+    if (lane < nrows) {
+      const int nb = min(4, (N - tile * kTileCols) / 32);
+      uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
+      store_scales4(rsr, vg, nb);
+      if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
+    }
+  }
+  if (DIRS & kCol) {
+    uint32_t bg[4], bu[4], mg[4], mu[4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      bg[2 * c] = e8m0_from_amax(acg[c] << 16);
+      bg[2 * c + 1] = e8m0_from_amax(acg[c] & 0xFFFF0000u);
+      bu[2 * c] = e8m0_from_amax(acu[c] << 16);
+      bu[2 * c + 1] = e8m0_from_amax(acu[c] & 0xFFFF0000u);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      mg[c] = scale_multiplier(bg[c]);
+      mu[c] = scale_multiplier(bu[c]);
+    }
+    if (colok) {
+      uint8_t* csr = p.cs + slab * (int64_t)W + c0;
+      __stcs(reinterpret_cast<unsigned int*>(csr), bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
+      if (ACT == kSwiGLU)
+        __stcs(reinterpret_cast<unsigned int*>(csr + N),
+               bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
+    }
+    unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
+    const int Wqc = opaque(Wq);
+    // re-read the tile's dX in two batches of 16 rows (loads first, then the math)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint2 RG[16], RU[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * h + i;
+        const bool ok = FULL || (colok && r < nrows);
+        RG[i] = ok ? __ldcg(dxb + r * Wqc) : make_uint2(0u, 0u);
+        if (ACT == kSwiGLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (N >> 2)) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * h + i;
+        const uint32_t qg = e4m3x2_2(bf16x2_to_f2_p(RG[i].x), mg[0], mg[1]) |
+                            (e4m3x2_2(bf16x2_to_f2_p(RG[i].y), mg[2], mg[3]) << 16);
+        if (FULL || (colok && r < nrows)) {
+          __stcs(qb + r * Wqc, qg);
+          if (ACT == kSwiGLU) {
+            const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(RU[i].x), mu[0], mu[1]) |
+                                (e4m3x2_2(bf16x2_to_f2_p(RU[i].y), mu[2], mu[3]) << 16);
+            __stcs(qb + r * Wqc + (N >> 2), qu);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int ACT, int DIRS, bool GROUPED, bool REREAD>
 __global__ void __launch_bounds__(Cfg<ACT, true>::kThreads, 1)
     act_bwd_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_dy, const Params p) {
@@ -901,8 +1108,17 @@ __global__ void __launch_bounds__(Cfg<ACT, true>::kThreads, 1)
       svn = lane < nrowsn ? __ldg(p.s + row0n + lane) : 0.0f;
     }
     const bool full = nrows == 32 && (cur.tile + 1) * kTileCols <= p.N;
-    bwd_tile<ACT, DIRS, GROUPED>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, full, sv,
-                                 lane, &tm_x, &tm_dy, ok);
+    if (REREAD) {
+      if (full)
+        bwd_tile_rr<ACT, DIRS, GROUPED, true>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
+                                              nrows, sv, lane, &tm_x, &tm_dy, ok);
+      else
+        bwd_tile_rr<ACT, DIRS, GROUPED, false>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
+                                               nrows, sv, lane, &tm_x, &tm_dy, ok);
+    } else {
+      bwd_tile<ACT, DIRS, GROUPED>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, full,
+                                   sv, lane, &tm_x, &tm_dy, ok);
+    }
     cur = nx;
     row0 = row0n;
     nrows = nrowsn;

@@ -253,7 +253,7 @@ BwdVariant pick_bwd(int dirs, bool reread) {
 }
 
 // Tensor map of a bf16 [rows, width] matrix with a row stride of `ld`
-// elements, read in boxes of 64 columns x 16 rows; out-of-range elements read
+// elements, read in boxes of 128 columns x 16 rows; out-of-range elements read
 // as zero.  Encoded on the host for every call (no allocation).
 moeact_status make_map(CUtensorMap* map, const void* base, int64_t width, int64_t rows,
                        int64_t ld) {
@@ -267,6 +267,30 @@ moeact_status make_map(CUtensorMap* map, const void* base, int64_t width, int64_
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MOEACT_OK;
+}
+
+// Tensor map of a SwiGLU input [rows, 2N] (gate | up, row stride `ld`) as a
+// [rows][2][N] view, read in boxes of 128 columns x 1 half x 16 rows: columns
+// past N read as zero in the gate half as well as in the up half, so a ragged
+// last column tile never sees the up values through its gate box (used by the
+// backward, whose dscale sums across the lanes of a tile).
+moeact_status make_map_gated(CUtensorMap* map, const void* base, int64_t N, int64_t rows,
+                             int64_t ld) {
+  const cuuint64_t dims[3] = {(cuuint64_t)N, 2, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)(N * 2), (cuuint64_t)(ld * 2)};
+  const cuuint32_t box[3] = {(cuuint32_t)kTileCols, 1, (cuuint32_t)kHalfRows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOEACT_OK;
+}
+
+moeact_status make_x_map(CUtensorMap* map, int act, const void* x, int64_t N, int64_t rows,
+                         int64_t ld) {
+  return act == kSwiGLU ? make_map_gated(map, x, N, rows, ld) : make_map(map, x, N, rows, ld);
 }
 
 int64_t grid_for(int64_t slabs_upper, int n_tiles, int threads, int dev) {
@@ -380,7 +404,7 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   if (act == kSwiGLU) v = grouped ? pick_bwd<kSwiGLU, true>(dirs, rr) : pick_bwd<kSwiGLU, false>(dirs, rr);
   else v = grouped ? pick_bwd<kSReLU, true>(dirs, rr) : pick_bwd<kSReLU, false>(dirs, rr);
   CUtensorMap tx, tdy;
-  if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
+  if ((st = make_x_map(&tx, act, x, N, M, ldx))) return st;
   if ((st = make_map(&tdy, dy, N, M, lddy))) return st;
   const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
   v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(v.sig, grouped, p.E), cs>>>(tx, tdy, p);

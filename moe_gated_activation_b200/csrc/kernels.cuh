@@ -387,12 +387,23 @@ __device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
   const int x = r.cur.tile * kTileCols, y = (int)r.row0 + half * kHalfRows;
   mbar_expect_tx(bar, OPS * kOpHalfBytes);
   if (OPS == 3 || (OPS == 2 && tm_dy != nullptr)) {
-    // backward: dY, then x (gate), then up (SwiGLU)
+    // backward: dY, then x (gate), then up (SwiGLU).  A SwiGLU input has a 3-D
+    // map whose middle coordinate picks gate (0) or up (1), so that columns
+    // past N read as zero in both halves: the dscale sum runs across all the
+    // lanes of a tile, including those past N.  SReLU's map is 2-D, [rows][N].
     tma_load_2d(dst, tm_dy, x, y, bar);
-    tma_load_2d(dst + kOpHalfBytes, tm_x, x, y, bar);
-    if (OPS == 3) tma_load_2d(dst + 2 * kOpHalfBytes, tm_x, x + p.N, y, bar);
+    if (OPS == 3) {
+      tma_load_3d(dst + kOpHalfBytes, tm_x, x, 0, y, bar);
+      tma_load_3d(dst + 2 * kOpHalfBytes, tm_x, x, 1, y, bar);
+    } else {
+      tma_load_2d(dst + kOpHalfBytes, tm_x, x, y, bar);
+    }
   } else {
-    // forward: gate, then up (SwiGLU)
+    // forward: gate, then up (SwiGLU) from a 2-D [rows][width] map, width 2N
+    // for SwiGLU (measured faster than the 3-D map).  In a ragged last column
+    // tile the gate box reaches into the up half; the lanes past N compute on
+    // those values, but nothing they produce crosses into a column below N
+    // (rowwise blocks are 8-lane aligned) or is stored.
     tma_load_2d(dst, tm_x, x, y, bar);
     if (OPS == 2) tma_load_2d(dst + kOpHalfBytes, tm_x, x + p.N, y, bar);
   }
@@ -894,6 +905,133 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
 // thread's stores visible to its later loads; the 16 KiB per tile is still in
 // L2), so only one 16-row half of gradients is held in registers.  Colwise
 // maxima are accumulated on the fly.
+// One 16-row half of a backward tile: waits for its ring slot, computes dX for
+// the half (stored), the half's dscale partial (ph, rows 2(l&15) + {0,1}),
+// its rowwise scales (bh, this lane's reduced E8M0 bytes) and codes, and folds
+// the colwise maxima into acg / acu.  Returns false if the slot never landed.
+template <int ACT, int DIRS, bool GROUPED, bool FULL, int OPS, int SLOTS>
+__device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
+                                            Ring<OPS, SLOTS>& ring, int k0, int h, int K,
+                                            int nrows, float sv, int lane, bool colok, int Wq,
+                                            unsigned int* rqb, uint2* dxb, const void* tm_x,
+                                            const void* tm_dy, float& ph, uint32_t& bh,
+                                            uint32_t (&acg)[2], uint32_t (&acu)[2]) {
+  const int N = p.N;
+  // per-half copies the compiler cannot hoist out of the (rolled) half loop,
+  // so that the 16 row offsets are not kept live across it
+  const int Wqh = opaque(Wq), Nq = opaque(N >> 2);
+  const int nrh = nrows - 16 * h;   // rows of this half that exist
+  const int k = k0 + h;
+  const int slot = k % SLOTS;
+  if (!mbar_wait(ring.bars + slot, (uint32_t)(k / SLOTS) & 1u)) return false;
+  const unsigned char* sm = ring.slots + slot * OPS * kOpHalfBytes + 8 * lane;
+  uint32_t DG[16][2], DU[16][2];
+  float P[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = 16 * h + i;
+    const uint2 D = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
+    const uint2 G = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
+    uint2 U = make_uint2(0u, 0u);
+    if (ACT == kSwiGLU) U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
+    const float sr = __shfl_sync(kFull, sv, r);
+    float part;
+    bwd_row<ACT>(m.sig, D, G, U, sr, DG[i][0], DG[i][1], DU[i][0], DU[i][1], part);
+    const bool live = FULL || i < nrh;
+    // rows past the slab's end: past M they read as zero (and give zeros); in
+    // a grouped call they are the next group's rows, which must not count
+    if (GROUPED && !live) { DG[i][0] = DG[i][1] = DU[i][0] = DU[i][1] = 0u; part = 0.0f; }
+    P[i] = part;
+    if (FULL || (colok && live)) {
+      dxb[r * Wqh] = make_uint2(DG[i][0], DG[i][1]);
+      if (ACT == kSwiGLU) dxb[r * Wqh + Nq] = make_uint2(DU[i][0], DU[i][1]);
+    }
+    if (DIRS & kCol) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        acg[c] = __vmaxu2(acg[c], DG[i][c] & 0x7FFF7FFFu);
+        if (ACT == kSwiGLU) acu[c] = __vmaxu2(acu[c], DU[i][c] & 0x7FFF7FFFu);
+      }
+    }
+  }
+  __syncwarp();
+  if (lane == 0 && ring.k_issue < K) ring_issue<OPS, SLOTS, GROUPED>(p, m, ring, tm_x, tm_dy);
+  if (p.dscale != nullptr) {
+    bfly_sum_f32<8>(P, lane, 16);
+    bfly_sum_f32<4>(P, lane, 8);
+    bfly_sum_f32<2>(P, lane, 4);
+    bfly_sum_f32<1>(P, lane, 2);
+    ph = __fadd_rn(P[0], __shfl_xor_sync(kFull, P[0], 1));
+  }
+  if (DIRS & kRow) {
+    uint32_t A[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t mg = __vmaxu2(DG[i][0] & 0x7FFF7FFFu, DG[i][1] & 0x7FFF7FFFu);
+      const uint32_t mu = __vmaxu2(DU[i][0] & 0x7FFF7FFFu, DU[i][1] & 0x7FFF7FFFu);
+      A[i] = __vmaxu2(__byte_perm(mg, mu, 0x5410), __byte_perm(mg, mu, 0x7632));
+    }
+    bfly_max_u16x2<8>(A, lane, 4);
+    bfly_max_u16x2<4>(A, lane, 2);
+    bfly_max_u16x2<2>(A, lane, 1);
+    const uint32_t bg0 = e8m0_from_amax(A[0] << 16), bu0 = e8m0_from_amax(A[0] & 0xFFFF0000u);
+    const uint32_t bg1 = e8m0_from_amax(A[1] << 16), bu1 = e8m0_from_amax(A[1] & 0xFFFF0000u);
+    bh = bg0 | (bu0 << 8) | (bg1 << 16) | (bu1 << 24);
+    const uint32_t mg0 = scale_multiplier(bg0), mg1 = scale_multiplier(bg1);
+    const uint32_t mu0 = scale_multiplier(bu0), mu1 = scale_multiplier(bu1);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = 16 * h + i;
+      const int src = (lane & 24) | (i >> 1);
+      const uint32_t mg = __shfl_sync(kFull, (i & 1) ? mg1 : mg0, src);
+      const uint32_t qg = e4m3x2_2(bf16x2_to_f2(DG[i][0]), mg, mg) |
+                          (e4m3x2_2(bf16x2_to_f2(DG[i][1]), mg, mg) << 16);
+      uint32_t qu = 0;
+      if (ACT == kSwiGLU) {
+        const uint32_t mu = __shfl_sync(kFull, (i & 1) ? mu1 : mu0, src);
+        qu = e4m3x2_2(bf16x2_to_f2(DU[i][0]), mu, mu) |
+             (e4m3x2_2(bf16x2_to_f2(DU[i][1]), mu, mu) << 16);
+      }
+      if (FULL || (colok && i < nrh)) {
+        __stcs(rqb + r * Wqh, qg);
+        if (ACT == kSwiGLU) __stcs(rqb + r * Wqh + Nq, qu);
+      }
+    }
+  }
+  return true;
+}
+
+// Colwise codes of one 16-row half of a backward tile, from dX re-read out of
+// L2 (loads first, then the math).
+template <int ACT, bool FULL>
+__device__ __forceinline__ void bwd_colwise_half_rr(int h, int N, int nrows, bool colok,
+                                                    int Wqc, const uint2* dxb, unsigned int* qb,
+                                                    const uint32_t (&mg)[4],
+                                                    const uint32_t (&mu)[4]) {
+  uint2 RG[16], RU[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = 16 * h + i;
+    const bool ok = FULL || (colok && r < nrows);
+    RG[i] = ok ? __ldcg(dxb + r * Wqc) : make_uint2(0u, 0u);
+    if (ACT == kSwiGLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (N >> 2)) : make_uint2(0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = 16 * h + i;
+    const uint32_t qg = e4m3x2_2(bf16x2_to_f2_p(RG[i].x), mg[0], mg[1]) |
+                        (e4m3x2_2(bf16x2_to_f2_p(RG[i].y), mg[2], mg[3]) << 16);
+    if (FULL || (colok && r < nrows)) {
+      __stcs(qb + r * Wqc, qg);
+      if (ACT == kSwiGLU) {
+        const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(RU[i].x), mu[0], mu[1]) |
+                            (e4m3x2_2(bf16x2_to_f2_p(RU[i].y), mu[2], mu[3]) << 16);
+        __stcs(qb + r * Wqc + (N >> 2), qu);
+      }
+    }
+  }
+}
+
 template <int ACT, int DIRS, bool GROUPED, bool FULL, int OPS, int SLOTS>
 __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
                                             Ring<OPS, SLOTS>& ring, int k0, int K, int64_t slab,
@@ -903,88 +1041,25 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
   const int Wq = W >> 2;   // row stride in 32-bit words (codes) / 8-byte words (dx)
   const int c0 = tile * kTileCols + 4 * lane;
   const bool colok = c0 < N;
-  float ph[2];
-  uint32_t bh[2];
+  float ph[2] = {0.0f, 0.0f};
+  uint32_t bh[2] = {0u, 0u};
   uint32_t acg[2] = {0u, 0u}, acu[2] = {0u, 0u};   // colwise maxima (packed bf16 magnitudes)
   unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + c0);
   uint2* dxb = reinterpret_cast<uint2*>(p.dx + row0 * (int64_t)W + c0);
-#pragma unroll
+  // one copy of the half body (only scalars cross the halves): half the code
+  // for the instruction cache to hold.  Measured faster than two unrolled
+  // copies at every size, most of all when each warp sees only a few tiles
+  // and the code is fetched cold.
+#pragma unroll 1
   for (int h = 0; h < 2; ++h) {
-    const int k = k0 + h;
-    const int slot = k % SLOTS;
-    if (!mbar_wait(ring.bars + slot, (uint32_t)(k / SLOTS) & 1u)) { ok_flag = false; return; }
-    const unsigned char* sm = ring.slots + slot * OPS * kOpHalfBytes + 8 * lane;
-    uint32_t DG[16][2], DU[16][2];
-    float P[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int r = 16 * h + i;
-      const uint2 D = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
-      const uint2 G = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
-      uint2 U = make_uint2(0u, 0u);
-      if (ACT == kSwiGLU) U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
-      const float sr = __shfl_sync(kFull, sv, r);
-      float part;
-      bwd_row<ACT>(m.sig, D, G, U, sr, DG[i][0], DG[i][1], DU[i][0], DU[i][1], part);
-      const bool live = FULL || r < nrows;
-      if (!FULL && !live) { DG[i][0] = DG[i][1] = DU[i][0] = DU[i][1] = 0u; part = 0.0f; }
-      P[i] = part;
-      if (FULL || (colok && live)) {
-        dxb[r * Wq] = make_uint2(DG[i][0], DG[i][1]);
-        if (ACT == kSwiGLU) dxb[r * Wq + (N >> 2)] = make_uint2(DU[i][0], DU[i][1]);
-      }
-      if (DIRS & kCol) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          acg[c] = __vmaxu2(acg[c], DG[i][c] & 0x7FFF7FFFu);
-          if (ACT == kSwiGLU) acu[c] = __vmaxu2(acu[c], DU[i][c] & 0x7FFF7FFFu);
-        }
-      }
+    float v;
+    uint32_t b;
+    if (!bwd_half_rr<ACT, DIRS, GROUPED, FULL>(p, m, ring, k0, h, K, nrows, sv, lane, colok, Wq,
+                                               rqb, dxb, tm_x, tm_dy, v, b, acg, acu)) {
+      ok_flag = false;
+      return;
     }
-    __syncwarp();
-    if (lane == 0 && ring.k_issue < K) ring_issue<OPS, SLOTS, GROUPED>(p, m, ring, tm_x, tm_dy);
-    if (p.dscale != nullptr) {
-      bfly_sum_f32<8>(P, lane, 16);
-      bfly_sum_f32<4>(P, lane, 8);
-      bfly_sum_f32<2>(P, lane, 4);
-      bfly_sum_f32<1>(P, lane, 2);
-      ph[h] = __fadd_rn(P[0], __shfl_xor_sync(kFull, P[0], 1));
-    }
-    if (DIRS & kRow) {
-      uint32_t A[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t mg = __vmaxu2(DG[i][0] & 0x7FFF7FFFu, DG[i][1] & 0x7FFF7FFFu);
-        const uint32_t mu = __vmaxu2(DU[i][0] & 0x7FFF7FFFu, DU[i][1] & 0x7FFF7FFFu);
-        A[i] = __vmaxu2(__byte_perm(mg, mu, 0x5410), __byte_perm(mg, mu, 0x7632));
-      }
-      bfly_max_u16x2<8>(A, lane, 4);
-      bfly_max_u16x2<4>(A, lane, 2);
-      bfly_max_u16x2<2>(A, lane, 1);
-      const uint32_t bg0 = e8m0_from_amax(A[0] << 16), bu0 = e8m0_from_amax(A[0] & 0xFFFF0000u);
-      const uint32_t bg1 = e8m0_from_amax(A[1] << 16), bu1 = e8m0_from_amax(A[1] & 0xFFFF0000u);
-      bh[h] = bg0 | (bu0 << 8) | (bg1 << 16) | (bu1 << 24);
-      const uint32_t mg0 = scale_multiplier(bg0), mg1 = scale_multiplier(bg1);
-      const uint32_t mu0 = scale_multiplier(bu0), mu1 = scale_multiplier(bu1);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * h + i;
-        const int src = (lane & 24) | (i >> 1);
-        const uint32_t mg = __shfl_sync(kFull, (i & 1) ? mg1 : mg0, src);
-        const uint32_t qg = e4m3x2_2(bf16x2_to_f2(DG[i][0]), mg, mg) |
-                            (e4m3x2_2(bf16x2_to_f2(DG[i][1]), mg, mg) << 16);
-        uint32_t qu = 0;
-        if (ACT == kSwiGLU) {
-          const uint32_t mu = __shfl_sync(kFull, (i & 1) ? mu1 : mu0, src);
-          qu = e4m3x2_2(bf16x2_to_f2(DU[i][0]), mu, mu) |
-               (e4m3x2_2(bf16x2_to_f2(DU[i][1]), mu, mu) << 16);
-        }
-        if (FULL || (colok && r < nrows)) {
-          __stcs(rqb + r * Wq, qg);
-          if (ACT == kSwiGLU) __stcs(rqb + r * Wq + (N >> 2), qu);
-        }
-      }
-    }
+    if (h == 0) { ph[0] = v; bh[0] = b; } else { ph[1] = v; bh[1] = b; }
   }
   if (p.dscale != nullptr) {
     const int src = 2 * (lane & 15);
@@ -1024,35 +1099,14 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
     }
     unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
     const int Wqc = opaque(Wq);
-    // re-read the tile's dX in two batches of 16 rows (loads first, then the math)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint2 RG[16], RU[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * h + i;
-        const bool ok = FULL || (colok && r < nrows);
-        RG[i] = ok ? __ldcg(dxb + r * Wqc) : make_uint2(0u, 0u);
-        if (ACT == kSwiGLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (N >> 2)) : make_uint2(0u, 0u);
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * h + i;
-        const uint32_t qg = e4m3x2_2(bf16x2_to_f2_p(RG[i].x), mg[0], mg[1]) |
-                            (e4m3x2_2(bf16x2_to_f2_p(RG[i].y), mg[2], mg[3]) << 16);
-        if (FULL || (colok && r < nrows)) {
-          __stcs(qb + r * Wqc, qg);
-          if (ACT == kSwiGLU) {
-            const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(RU[i].x), mu[0], mu[1]) |
-                                (e4m3x2_2(bf16x2_to_f2_p(RU[i].y), mu[2], mu[3]) << 16);
-            __stcs(qb + r * Wqc + (N >> 2), qu);
-          }
-        }
-      }
-    }
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h)
+      bwd_colwise_half_rr<ACT, FULL>(h, N, nrows, colok, Wqc, dxb, qb, mg, mu);
   }
 }
 
+// REREAD: dX is written and the colwise pass re-reads it (from L2); without
+// it the whole tile stays in registers for the colwise pass.
 template <int ACT, int DIRS, bool GROUPED, bool REREAD>
 __global__ void __launch_bounds__(Cfg<ACT, true>::kThreads, 1)
     act_bwd_kernel(const __grid_constant__ CUtensorMap tm_x,

@@ -20,8 +20,8 @@ pytestmark = pytest.mark.gpu
 
 ACTS = {"swiglu": oracle.SWIGLU, "srelu": oracle.SRELU}
 DIRS = {"row": oracle.ROWWISE, "col": oracle.COLWISE, "both": oracle.ROWWISE | oracle.COLWISE}
-# several 64-column tiles, a ragged last tile (N % 64 == 32), partial last
-# 32-row slabs (M % 32 != 0) and a single-block case
+# several 128-column tiles, ragged last tiles (N % 128 in {32, 64, 96}),
+# partial last 32-row slabs (M % 32 != 0) and a single-block case
 SHAPES = [(32, 32), (96, 224), (100, 192), (257, 320), (64, 2048)]
 
 
@@ -90,6 +90,35 @@ def test_backward_parity(cuda_device, act, dirs, shape):
     assert_dscale(got.dscale, ref["dscale"], bound, what + " dscale")
 
 
+@pytest.mark.parametrize("grouped", [False, True])
+def test_backward_parity_many_tiles_per_warp(cuda_device, grouped):
+    """The shapes above give each warp of the persistent backward one or two
+    32x128 tiles; this one gives it more than four, so that the ring of each
+    warp wraps several times, with ragged rows, columns and groups."""
+    M, N = 16392, 1056
+    c = _case(M, N, "swiglu", seed=91)
+    xb, s, dyb = bf16_bits(c["x"]), c["s"].numpy(), bf16_bits(c["dy"])
+    x, sg, dy = c["x"].to(cuda_device), c["s"].to(cuda_device), c["dy"].to(cuda_device)
+    if grouped:
+        g = np.random.default_rng(5)
+        cut = np.sort(g.integers(0, M, 15))
+        m = np.diff(np.concatenate([[0], cut, [M]])).astype(np.int64)
+        _, ro, cb = oracle.splits_to_offsets(m, M)
+        gro, gcb, _ = mg.splits_to_offsets(torch.from_numpy(m).to(cuda_device), M)
+        got, st = mg.grouped_scaled_swiglu_mxfp8_bwd(dy, x, sg, gro, gcb, col_scale_rows=int(cb[-1]))
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        ref = oracle.grouped_act_bwd(dyb, xb, s, N, 3, ro, cb)
+    else:
+        got = _bwd("swiglu", dy, x, sg, 3)
+        torch.cuda.synchronize()
+        ref = oracle.act_bwd(dyb, xb, s, N, 3)
+    what = f"swiglu bwd many tiles grouped={grouped}"
+    compare_mx(got.mx, ref, what, exact=True)
+    assert np.array_equal(bf16_u16(got.dx), ref["dx"]), what + " dx"
+    assert_dscale(got.dscale, ref["dscale"], dscale_abs_bound(dyb, xb, s, N), what + " dscale")
+
+
 @pytest.mark.parametrize("want_dx,want_dscale", [(False, True), (True, False), (False, False)])
 def test_backward_optional_outputs(cuda_device, want_dx, want_dscale):
     M, N = 96, 224
@@ -154,6 +183,35 @@ def test_special_values_forward_and_backward(cuda_device, act):
     assert np.array_equal(np.isinf(gd), np.isinf(rd))
     bound = dscale_abs_bound(dyb, xb, sn, N, act == "swiglu")
     assert_dscale(gd[fin], rd[fin], bound[fin], "special dscale")
+
+
+def test_ragged_last_column_tile_sees_no_up_values(cuda_device):
+    """With N % 128 != 0 the last 128-column tile of the gate reaches past
+    column N-1.  Those columns must read as zero, not as the first up values:
+    here row 3's up half is +Inf in its first 96 columns and its dY is
+    positive, so its dscale is +Inf, which a NaN from an Inf gate times a zero
+    up would turn into NaN."""
+    M, N = 64, 160
+    c = _case(M, N, "swiglu", seed=23)
+    x, s, dy = c["x"].clone(), c["s"], c["dy"].clone()
+    x[3, N:N + 96] = float("inf")
+    x[3, :N] = 1.0
+    dy[3] = dy[3].abs() + 0.5
+    xb, sn, dyb = bf16_bits(x), s.numpy(), bf16_bits(dy)
+    ref = oracle.act_bwd(dyb, xb, sn, N, 3)
+    got = _bwd("swiglu", dy.to(cuda_device), x.to(cuda_device), s.to(cuda_device), 3)
+    torch.cuda.synchronize()
+    assert np.isposinf(ref["dscale"][3])
+    compare_mx(got.mx, ref, "ragged tile bwd", exact=True)
+    assert np.array_equal(bf16_u16(got.dx), ref["dx"])
+    gd = got.dscale.cpu().numpy()
+    assert np.isposinf(gd[3]), gd[3]
+    fin = np.isfinite(ref["dscale"])
+    assert_dscale(gd[fin], ref["dscale"][fin], dscale_abs_bound(dyb, xb, sn, N)[fin], "ragged dscale")
+    reff = oracle.act_fwd(xb, sn, N, 3)
+    gotf = _fwd("swiglu", x.to(cuda_device), s.to(cuda_device), 3)
+    torch.cuda.synchronize()
+    compare_mx(gotf, reff, "ragged tile fwd", exact=True)
 
 
 def test_strided_input_is_read_in_place_and_inputs_are_not_mutated(cuda_device):

@@ -159,6 +159,24 @@ def ncu_traffic(workload, kernel, dirs_name):
     return None
 
 
+def max_over_ranks(value, world, device):
+    """The largest `value` over all ranks (every rank gets it); with one rank,
+    `value` itself.  `device` is where the collective's tensor lives (cuda
+    for NCCL, cpu for gloo)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world, steps, step_bytes, total_ms):
+    """Whole-job throughput of `world` replicas: every rank processed
+    `steps` steps of `step_bytes` each; the job took the slowest rank's
+    `total_ms`."""
+    return world * steps * step_bytes / (total_ms * 1e-3) / 1e9
+
+
 def dist_setup(n_gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -291,11 +309,7 @@ def run_ours(args):
     splits_ms = [t[0] for t in times]
     fwd_ms = [t[1] for t in times]
     bwd_ms = [t[2] for t in times]
-    total_ms = sum(t[3] for t in times)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(t[3] for t in times), world, dev)
 
     # end to end through the public API with host buffers (pinned), H2D of the
     # step's inputs and D2H of every output inside the timed region
@@ -311,7 +325,7 @@ def run_ours(args):
     achieved = bm[dom] / (dom_us * 1e-6) / 1e9
     kname = "act_bwd_kernel" if dom == "bwd" else "act_fwd_kernel"
     traffic = ncu_traffic(args.workload, kname, args.dirs)
-    value = world * args.steps * step_bytes / (total_ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, args.steps, step_bytes, total_ms)
     out = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -400,15 +414,11 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
         one()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     E = int(inp["m_splits"].numel())
     bm = byte_model(M, N, E, dirs, S=S)
     step_bytes = bm["splits"] + bm["fwd"] + bm["bwd"]
-    return {"value": round(world * step_bytes * steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    return {"value": round(whole_job_gbs(world, steps, step_bytes, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4)}
 
@@ -485,7 +495,9 @@ def run_reference(args):
            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
            "data": "synthetic (seeded torch generators)",
            "config": {"workload": f"{wl.key}: {wl.title}", "M": wl.M, "N": wl.N,
-                      "dirs": args.dirs, "activation": "swiglu"},
+                      "groups": wl.groups, "dirs": args.dirs, "activation": "swiglu",
+                      "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
+                      "parallelism": "host cores (rank 0)"},
            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,

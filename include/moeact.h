@@ -63,7 +63,7 @@
  *
  * Ownership and execution: the caller allocates every input, output and
  * workspace on the device; the library allocates nothing per call (it keeps
- * one 32 KiB sigmoid table per device, built at moeact_init or at the first
+ * one 48 KiB sigmoid table per device, built at moeact_init or at the first
  * call on that device).  Calls are asynchronous on `stream` (a cudaStream_t
  * passed as void*, NULL = legacy default stream) and never synchronise the
  * host, except moeact_init.  Inputs are never written.  Outputs must not

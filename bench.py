@@ -249,26 +249,37 @@ def run_ours(args):
             bwd(ro, cb, st)
             ev[3].record(stream)
     else:
-        # the whole step captured once as a CUDA graph, with event-record nodes
-        # between the calls, and replayed once per step
-        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-        graph = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(graph, stream=side):
-                gev[0].record(side)
-                ro, cb, st = splits()
-                gev[1].record(side)
-                fwd(ro, cb, st)
-                gev[2].record(side)
-                bwd(ro, cb, st)
-                gev[3].record(side)
-        stream.wait_stream(side)
-        torch.cuda.synchronize()
+        # The step captured as a CUDA graph and replayed once per step.  The
+        # timed graph has event-record nodes only at its ends (an event node
+        # between two kernels costs a few microseconds); a second graph with
+        # event nodes between the calls gives the per-kernel times.
+        def capture(evs):
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(g, stream=side):
+                    evs[0].record(side)
+                    ro, cb, st = splits()
+                    if len(evs) == 4:
+                        evs[1].record(side)
+                    fwd(ro, cb, st)
+                    if len(evs) == 4:
+                        evs[2].record(side)
+                    bwd(ro, cb, st)
+                    evs[-1].record(side)
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            return g
 
-    def timed_steps(n, record):
-        """n steps, each after an L2 flush; returns per-step [splits, fwd, bwd, total] ms."""
+        sev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        graph = capture(sev)
+        graph_parts = capture(gev)
+
+    def timed_steps(n, record, parts=False):
+        """n steps, each after an L2 flush; returns per-step [splits, fwd, bwd, total] ms
+        (parts=False: the step graph, total only)."""
         out = []
         for i in range(n):
             do_flush(i)
@@ -277,12 +288,17 @@ def run_ours(args):
                 run_step(ev)
                 if record:
                     out.append(ev)
-            else:
-                graph.replay()
+            elif parts:
+                graph_parts.replay()
                 torch.cuda.synchronize()
                 if record:
                     out.append([gev[0].elapsed_time(gev[1]), gev[1].elapsed_time(gev[2]),
                                 gev[2].elapsed_time(gev[3]), gev[0].elapsed_time(gev[3])])
+            else:
+                graph.replay()
+                torch.cuda.synchronize()
+                if record:
+                    out.append([None, None, None, sev[0].elapsed_time(sev[1])])
         if args.eager:
             torch.cuda.synchronize()
             out = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
@@ -290,6 +306,8 @@ def run_ours(args):
         return out
 
     timed_steps(args.warmup, False)
+    if not args.eager:
+        timed_steps(args.warmup, False, parts=True)
     torch.cuda.synchronize()
     sampler = ClockSampler(dev)
     with sampler:
@@ -301,14 +319,17 @@ def run_ours(args):
         times = timed_steps(args.steps, True)
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
+        # per-kernel times: the same steps again, with event nodes between the calls
+        parts = times if args.eager else timed_steps(args.steps, True, parts=True)
+        torch.cuda.synchronize()
         sampler.active = False
         if world > 1:
             torch.distributed.barrier()
     if not args.eager:
-        del graph
-    splits_ms = [t[0] for t in times]
-    fwd_ms = [t[1] for t in times]
-    bwd_ms = [t[2] for t in times]
+        del graph, graph_parts
+    splits_ms = [t[0] for t in parts]
+    fwd_ms = [t[1] for t in parts]
+    bwd_ms = [t[2] for t in parts]
     total_ms = max_over_ranks(sum(t[3] for t in times), world, dev)
 
     # end to end through the public API with host buffers (pinned), H2D of the
@@ -342,7 +363,8 @@ def run_ours(args):
         "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
                    "dirs": args.dirs, "activation": "swiglu",
                    "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
-                   "launch": "eager" if args.eager else "one CUDA graph per step (event nodes between the calls)",
+                   "launch": "eager" if args.eager else "one CUDA graph per step (events at its ends only)",
+                   "kernel_times": "eager events" if args.eager else "a second timed pass of the same steps, with event nodes between the calls",
                    "l2": "flushed before every step (256 MiB written then read), outside the timed events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
@@ -359,7 +381,7 @@ def run_ours(args):
             "splits_to_offsets": {"us": round(1e3 * mean(splits_ms), 2)},
         },
         "wall_s_timed_region": round(wall, 4),
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,   # splits, fwd, bwd, dscale reduction per step
         "clocks": sampler.summary(),
         "e2e": e2e,
     }

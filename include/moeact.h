@@ -139,7 +139,10 @@ const char* moeact_last_error(void);
  *   colblk_offs  int64 [E+1] out: sum_{k<e} ceil(m_k/32), the first
  *                col-scale row of group e (device).
  *   status       int32 out (device): MOEACT_DEV_OK, or NEGATIVE_SPLIT /
- *                SPLIT_SUM, in which case no offset is written.
+ *                SPLIT_SUM, in which case row_offs[0] (and colblk_offs[0])
+ *                are set to -1 and nothing else is written: a grouped call
+ *                given these offsets reports MOEACT_DEV_BAD_OFFSETS and
+ *                writes nothing.
  * E = 0 is legal (offsets [0], M must be 0).  Element offsets of any array
  * are row_offs times its row length.
  * ------------------------------------------------------------------- */

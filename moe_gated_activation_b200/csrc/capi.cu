@@ -1,6 +1,7 @@
 // C ABI of libmoeact (declared in include/moeact.h): argument validation,
 // per-device set-up and kernel dispatch.  Argument checks happen on the host
 // before anything is launched; nothing here allocates device memory.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -466,7 +467,11 @@ moeact_status splits_to_offsets(const int64_t* m_splits, int32_t num_groups, int
   int dev;
   moeact_status st = ensure_ready(cs, &dev);
   if (st) return st;
-  splits_kernel<<<1, 1024, 0, cs>>>(m_splits, num_groups, total_rows, row_offs, colblk_offs, status);
+  // one thread per group up to 1024 (whole warps): a small E launches fewer
+  // threads and synchronises fewer warps
+  const int threads = (int)std::min<int64_t>(1024, std::max<int64_t>(32, ceil_div(num_groups, 32) * 32));
+  splits_kernel<<<1, threads, 0, cs>>>(m_splits, num_groups, total_rows, row_offs, colblk_offs,
+                                       status);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "splits_to_offsets launch");
   return MOEACT_OK;

@@ -333,6 +333,45 @@ def test_splits_to_offsets_status(cuda_device, splits, M, status):
     assert int(gst.item()) == status
 
 
+def test_failed_splits_leave_no_usable_offsets(cuda_device):
+    """Offsets buffers reused across calls: after a valid splits_to_offsets and
+    a grouped forward, bad splits (negative, or not summing to M) into the same
+    buffers must make the next grouped forward report bad offsets and write
+    nothing, not run on the earlier call's offsets."""
+    N, m = 64, np.array([32, 64, 0, 32], np.int64)
+    M = int(m.sum())
+    c = _case(M, N, "swiglu", seed=31)
+    x, s = c["x"].to(cuda_device), c["s"].to(cuda_device)
+    md = torch.from_numpy(m).to(cuda_device)
+    ro = torch.empty(len(m) + 1, dtype=torch.int64, device=cuda_device)
+    cb = torch.empty_like(ro)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    lib = _capi.lib()
+    stream = torch.cuda.current_stream(cuda_device).cuda_stream
+    _capi.call("splits_to_offsets", md.data_ptr(), len(m), M, ro.data_ptr(), cb.data_ptr(),
+               st.data_ptr(), stream)
+    good, gst = mg.grouped_scaled_swiglu_mxfp8_fwd(x, s, ro, cb, col_scale_rows=M // 32)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and int(gst.item()) == 0
+    for bad, code in (([32, -32, 64, 32], 1), ([32, 64, 0, 0], 2)):
+        mb = torch.tensor(bad, dtype=torch.int64, device=cuda_device)
+        _capi.call("splits_to_offsets", mb.data_ptr(), len(bad), M, ro.data_ptr(),
+                   cb.data_ptr(), st.data_ptr(), stream)
+        torch.cuda.synchronize()
+        assert int(st.item()) == code
+        outs = {k: torch.full_like(getattr(good, k).view(torch.uint8), 0xAB)
+                for k in ("row_codes", "row_scales", "col_codes", "col_scales")}
+        mx = _capi.MxOut(*(outs[k].data_ptr() for k in ("row_codes", "row_scales", "col_codes",
+                                                          "col_scales")))
+        st2 = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+        _capi.call("grouped_scaled_swiglu_mxfp8_fwd", x.data_ptr(), 2 * N, s.data_ptr(), M, N, 3,
+                   0, ro.data_ptr(), cb.data_ptr(), len(m), st2.data_ptr(), mx, stream)
+        torch.cuda.synchronize()
+        assert int(st2.item()) == _capi.DEV_BAD_OFFSETS
+        for o in outs.values():
+            assert bool((o == 0xAB).all())
+
+
 def test_splits_to_offsets_many_groups(cuda_device):
     g = np.random.default_rng(3)
     m = (g.integers(0, 5, 2040) * 32 + g.integers(0, 3, 2040)).astype(np.int64)

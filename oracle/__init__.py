@@ -89,6 +89,10 @@ def _load():
     lib.orc_grouped_act_bwd.argtypes = [I, P, I64, P, I64, P, I64, I64, I, P, P, I32,
                                         P, P, P, P, P, P]
     lib.orc_grouped_act_bwd.restype = I
+    lib.orc_scales_gemm_layout.argtypes = [P, I64, I64, P]
+    lib.orc_scales_gemm_layout.restype = None
+    lib.orc_col_scales_gemm_layout.argtypes = [P, I64, P, P, I32, P]
+    lib.orc_col_scales_gemm_layout.restype = I
     if lib.orc_sigma_init() != 0:
         raise RuntimeError("oracle: sigmoid table has uncertified roundings")
     _lib = lib
@@ -268,3 +272,27 @@ def grouped_act_bwd(dy_bits, x_bits, s, N, dirs, row_offs, colblk_offs, act=SWIG
     if rc:
         raise ValueError(f"oracle grouped_act_bwd failed ({rc})")
     return out
+
+
+# ---------------------------------------------------------------- GEMM-ready scales
+def scales_gemm_layout(S: np.ndarray) -> np.ndarray:
+    """E8M0 matrix [R, C] -> the 128 x 4 tiled GEMM layout (flat uint8,
+    ceil(R/128) * ceil(C/4) * 512 bytes, padding 0)."""
+    S = _c(S, np.uint8)
+    R, C = S.shape
+    out = np.zeros(((R + 127) // 128) * ((C + 3) // 4) * 512, np.uint8)
+    _load().orc_scales_gemm_layout(_ptr(S), R, C, _ptr(out))
+    return out
+
+
+def col_scales_gemm_layout(cs: np.ndarray, W: int, row_offs, colblk_offs) -> np.ndarray:
+    """Row-major colwise scales [S, W] of a grouped tensor -> per expert, the
+    transposed [W, m_e/32] matrix in the GEMM layout, experts in order."""
+    cs = _c(cs, np.uint8)
+    ro = _c(row_offs, np.int64)
+    co = _c(colblk_offs, np.int64)
+    E = ro.shape[0] - 1
+    out = np.zeros(max(1, int(ro[-1]) * W // 32), np.uint8)
+    if _load().orc_col_scales_gemm_layout(_ptr(cs), W, _ptr(ro), _ptr(co), E, _ptr(out)):
+        raise ValueError("GEMM layout needs W and every group's rows to be multiples of 128")
+    return out[:int(ro[-1]) * W // 32]

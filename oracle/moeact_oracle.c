@@ -442,3 +442,53 @@ int orc_grouped_act_bwd(int act, const uint16_t* dy, int64_t lddy, const uint16_
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* GEMM-ready scale layout.                                            */
+/* ------------------------------------------------------------------ */
+/* The consumer of the quantized grouped tensors is a block-scaled grouped
+ * GEMM (TransformerEngine PR #3238, sequence diagram: the activation feeds
+ * quantized grouped storage to the next grouped linear).  The pages give no
+ * layout for its scale factors; the reading taken is the one block-scaled
+ * tensor-core GEMMs read: the E8M0 matrix S[R][C] (one byte per 32 elements
+ * along the GEMM's K dimension) cut into tiles of 128 rows x 4 columns, 512
+ * bytes each, tiles stored in row-major order of (row tile, column tile);
+ * inside a tile, element (r, c) (r < 128, c < 4) is at byte
+ * (r % 32) * 16 + (r / 32) * 4 + c.  Positions past R or C (when R or C is
+ * not a whole number of tiles) are 0. */
+void orc_scales_gemm_layout(const uint8_t* S, int64_t R, int64_t C, uint8_t* out) {
+  int64_t rt = (R + 127) / 128, ct = (C + 3) / 4;
+  memset(out, 0, (size_t)(rt * ct * 512));
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t c = 0; c < C; ++c) {
+      int64_t tile = (r / 128) * ct + c / 4;
+      int64_t rr = r % 128, cc = c % 4;
+      out[tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + cc] = S[r * C + c];
+    }
+}
+
+/* Colwise scales in the GEMM layout.  The colwise-quantized tensor of an
+ * expert (m_e rows, W columns, 32x1 blocks) is read by the GEMM transposed:
+ * W rows and K = m_e, so its scale matrix is the transpose of the expert's
+ * [m_e/32][W] colwise scales, [W][m_e/32], laid out as above.  Experts
+ * follow one another in expert order.  cs holds the row-major colwise
+ * scales (expert e at rows colblk_offs[e] ..).  Returns 1 (nothing written)
+ * unless every expert's row count and W are multiples of 128, the shapes
+ * for which no tile needs padding. */
+int orc_col_scales_gemm_layout(const uint8_t* cs, int64_t W, const int64_t* row_offs,
+                               const int64_t* colblk_offs, int32_t E, uint8_t* out) {
+  if (W % 128) return 1;
+  for (int32_t e = 0; e < E; ++e)
+    if ((row_offs[e + 1] - row_offs[e]) % 128) return 1;
+  int64_t pos = 0;
+  for (int32_t e = 0; e < E; ++e) {
+    int64_t kb = (row_offs[e + 1] - row_offs[e]) / 32;   /* K blocks of expert e */
+    uint8_t* t = (uint8_t*)malloc((size_t)(W * kb > 0 ? W * kb : 1));
+    for (int64_t w = 0; w < W; ++w)
+      for (int64_t j = 0; j < kb; ++j) t[w * kb + j] = cs[(colblk_offs[e] + j) * W + w];
+    orc_scales_gemm_layout(t, W, kb, out + pos);
+    pos += (W / 128) * (kb / 4) * 512;
+    free(t);
+  }
+  return 0;
+}

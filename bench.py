@@ -224,13 +224,16 @@ def run_ours(args):
     def splits():
         return mg.splits_to_offsets(m_dev, M)
 
+    gemm = args.scales == "gemm"
+
     def fwd(ro, cb, st):
         return mg.grouped_scaled_swiglu_mxfp8_fwd(x, s, ro, cb, rowwise=rw, colwise=cw,
-                                                  col_scale_rows=S, status=st)
+                                                  col_scale_rows=S, status=st, gemm_scales=gemm)
 
     def bwd(ro, cb, st):
         return mg.grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, ro, cb, rowwise=rw, colwise=cw,
-                                                  col_scale_rows=S, workspace=ws, status=st)
+                                                  col_scale_rows=S, workspace=ws, status=st,
+                                                  gemm_scales=gemm)
 
     # eager warm-up
     for i in range(3):
@@ -361,7 +364,7 @@ def run_ours(args):
         "dtype": "f32",
         "data": "synthetic (seeded torch generators; shapes and statistics of the pages' workloads)",
         "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
-                   "dirs": args.dirs, "activation": "swiglu",
+                   "dirs": args.dirs, "scales": args.scales, "activation": "swiglu",
                    "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
                    "launch": "eager" if args.eager else "one CUDA graph per step (events at its ends only)",
                    "kernel_times": "eager events" if args.eager else "a second timed pass of the same steps, with event nodes between the calls",
@@ -411,10 +414,13 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
         dyd.copy_(dyh, non_blocking=True)
         md.copy_(mh, non_blocking=True)
         ro, cb, st = mg.splits_to_offsets(md, M)
+        gemm = args.scales == "gemm"
         f, fst = mg.grouped_scaled_swiglu_mxfp8_fwd(xd, sd, ro, cb, rowwise=rw, colwise=cw,
-                                                    col_scale_rows=S, status=st)
+                                                    col_scale_rows=S, status=st,
+                                                    gemm_scales=gemm)
         b, bst = mg.grouped_scaled_swiglu_mxfp8_bwd(dyd, xd, sd, ro, cb, rowwise=rw, colwise=cw,
-                                                    col_scale_rows=S, status=st)
+                                                    col_scale_rows=S, status=st,
+                                                    gemm_scales=gemm)
         outs = [t for t in (*f, *b.mx, b.dx, b.dscale, st) if t is not None and t.numel()]
         if outs_h is None:
             outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
@@ -534,6 +540,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--dirs", default="both", choices=list(DIRS))
+    ap.add_argument("--scales", default="rowmajor", choices=["rowmajor", "gemm"],
+                    help="E8M0 scale layout: row-major, or the GEMM-ready 128 x 4 tiles")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of CUDA graphs")

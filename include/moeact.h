@@ -109,18 +109,39 @@ typedef enum moeact_status {
 #define MOEACT_DEV_NEGATIVE_SPLIT 1   /* a split < 0 */
 #define MOEACT_DEV_SPLIT_SUM 2        /* splits do not sum to M */
 #define MOEACT_DEV_BAD_OFFSETS 3      /* offsets not those of valid splits */
+#define MOEACT_DEV_UNALIGNED_GROUPS 4 /* GEMM scale layout with a group whose rows
+                                         are not a multiple of 128 */
 
 /* Largest number of groups (experts) a grouped call accepts. */
 #define MOEACT_MAX_GROUPS 2040
 /* Largest M accepted (2^30 rows; TMA coordinates are 32-bit). */
 #define MOEACT_MAX_ROWS (((int64_t)1) << 30)
 
+/* Layouts of the E8M0 scale arrays (moeact_mx_out.scale_layout).
+ * ROWMAJOR: row scales [M, W/32], col scales [S, W], row-major (see Layouts).
+ * GEMM: the layout a block-scaled tensor-core GEMM reads its scale factors
+ *   in (the pages name the consumer, a block-scaled grouped GEMM, but give no
+ *   layout; this is the reading taken).  A scale matrix is cut into tiles of
+ *   128 rows x 4 scale columns, 512 bytes each, stored in row-major order of
+ *   (row tile, column tile); inside a tile, element (r, c) is at byte
+ *   (r % 32) * 16 + (r / 32) * 4 + c.  Row scales: the [M, W/32] matrix
+ *   (M * W / 32 bytes).  Col scales: each group's colwise data is read by
+ *   the GEMM transposed (W rows, K = the group's rows), so its scales are the
+ *   [W, m_e/32] matrix, tiled the same way, groups one after the other
+ *   (group e from byte row_offs[e] / 32 * W; M * W / 32 bytes in all).
+ *   Needs M, N and (grouped) every group's row count to be multiples of 128
+ *   -- whole tiles, no padding -- else MOEACT_EINVAL on the host or
+ *   MOEACT_DEV_UNALIGNED_GROUPS in the status word. */
+#define MOEACT_SCALES_ROWMAJOR 0
+#define MOEACT_SCALES_GEMM 1
+
 /* MXFP8 outputs of one call; a disabled direction's two pointers must be NULL. */
 typedef struct moeact_mx_out {
   uint8_t* row_codes;   /* [M, W]    E4M3, rowwise 1x32 blocks */
-  uint8_t* row_scales;  /* [M, W/32] E8M0 */
+  uint8_t* row_scales;  /* [M, W/32] E8M0 (in `scale_layout`) */
   uint8_t* col_codes;   /* [M, W]    E4M3, colwise 32x1 blocks */
-  uint8_t* col_scales;  /* [S, W]    E8M0 */
+  uint8_t* col_scales;  /* [S, W]    E8M0 (in `scale_layout`) */
+  int32_t scale_layout; /* MOEACT_SCALES_ROWMAJOR (0) or MOEACT_SCALES_GEMM */
 } moeact_mx_out;
 
 /* Build the sigmoid table on the current device and set up its kernels.

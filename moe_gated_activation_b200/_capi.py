@@ -16,13 +16,15 @@ LIB_PATH = os.path.join(_PKG, "libmoeact.so")
 
 OK, EINVAL, EALIGN, EUNSUPPORTED, ERANGE, ECUDA, EWORKSPACE = range(7)
 ROWWISE, COLWISE = 1, 2
-DEV_OK, DEV_NEGATIVE_SPLIT, DEV_SPLIT_SUM, DEV_BAD_OFFSETS = range(4)
+DEV_OK, DEV_NEGATIVE_SPLIT, DEV_SPLIT_SUM, DEV_BAD_OFFSETS, DEV_UNALIGNED_GROUPS = range(5)
+SCALES_ROWMAJOR, SCALES_GEMM = 0, 1
 MAX_GROUPS = 2040
 
 
 class MxOut(ctypes.Structure):
     _fields_ = [("row_codes", ctypes.c_void_p), ("row_scales", ctypes.c_void_p),
-                ("col_codes", ctypes.c_void_p), ("col_scales", ctypes.c_void_p)]
+                ("col_codes", ctypes.c_void_p), ("col_scales", ctypes.c_void_p),
+                ("scale_layout", ctypes.c_int32)]
 
 
 class MoeactError(RuntimeError):

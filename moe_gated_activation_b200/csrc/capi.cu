@@ -57,16 +57,22 @@ BwdVariant bwd_variant() {
           smem_bytes<ACT, true>(false, 0), Cfg<ACT, true>::kSig};
 }
 
+template <int ACT, bool GROUPED, int LAYOUT>
+void fwd_all_layout(FwdVariant* out, int& n) {
+  out[n++] = fwd_variant<ACT, kRow | LAYOUT, false, GROUPED>();
+  out[n++] = fwd_variant<ACT, kCol | LAYOUT, false, GROUPED>();
+  out[n++] = fwd_variant<ACT, kRow | kCol | LAYOUT, false, GROUPED>();
+  if (ACT == kSwiGLU) {
+    out[n++] = fwd_variant<ACT, kRow | LAYOUT, true, GROUPED>();
+    out[n++] = fwd_variant<ACT, kCol | LAYOUT, true, GROUPED>();
+    out[n++] = fwd_variant<ACT, kRow | kCol | LAYOUT, true, GROUPED>();
+  }
+}
+
 template <int ACT, bool GROUPED>
 void fwd_all(FwdVariant* out, int& n) {
-  out[n++] = fwd_variant<ACT, kRow, false, GROUPED>();
-  out[n++] = fwd_variant<ACT, kCol, false, GROUPED>();
-  out[n++] = fwd_variant<ACT, kRow | kCol, false, GROUPED>();
-  if (ACT == kSwiGLU) {
-    out[n++] = fwd_variant<ACT, kRow, true, GROUPED>();
-    out[n++] = fwd_variant<ACT, kCol, true, GROUPED>();
-    out[n++] = fwd_variant<ACT, kRow | kCol, true, GROUPED>();
-  }
+  fwd_all_layout<ACT, GROUPED, 0>(out, n);
+  fwd_all_layout<ACT, GROUPED, kGemm>(out, n);
 }
 
 template <int ACT, bool GROUPED, bool REREAD>
@@ -75,6 +81,9 @@ void bwd_all_rr(BwdVariant* out, int& n) {
   out[n++] = bwd_variant<ACT, kRow, GROUPED, REREAD>();
   out[n++] = bwd_variant<ACT, kCol, GROUPED, REREAD>();
   out[n++] = bwd_variant<ACT, kRow | kCol, GROUPED, REREAD>();
+  out[n++] = bwd_variant<ACT, kRow | kGemm, GROUPED, REREAD>();
+  out[n++] = bwd_variant<ACT, kCol | kGemm, GROUPED, REREAD>();
+  out[n++] = bwd_variant<ACT, kRow | kCol | kGemm, GROUPED, REREAD>();
 }
 
 template <int ACT, bool GROUPED>
@@ -109,8 +118,8 @@ moeact_status init_device(int dev) {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
 
-  FwdVariant fv[32];
-  BwdVariant bv[40];
+  FwdVariant fv[48];
+  BwdVariant bv[64];
   int nf = 0, nb = 0;
   fwd_all<kSwiGLU, false>(fv, nf);
   fwd_all<kSwiGLU, true>(fv, nf);
@@ -195,6 +204,16 @@ moeact_status check_mx(const moeact_mx_out& o, int dirs, bool allow_none) {
   return MOEACT_OK;
 }
 
+// The GEMM-ready scale layout is defined for whole 128 x 128 tiles only.
+moeact_status check_layout(const moeact_mx_out& o, int64_t M, int64_t N) {
+  if (o.scale_layout != MOEACT_SCALES_ROWMAJOR && o.scale_layout != MOEACT_SCALES_GEMM)
+    return fail(MOEACT_EINVAL, "scale_layout must be MOEACT_SCALES_ROWMAJOR or MOEACT_SCALES_GEMM");
+  if (o.scale_layout == MOEACT_SCALES_GEMM && (M % 128 != 0 || N % 128 != 0))
+    return fail(MOEACT_EINVAL, "the GEMM scale layout needs M and N to be multiples of 128 "
+                "(got M=%lld, N=%lld)", (long long)M, (long long)N);
+  return MOEACT_OK;
+}
+
 moeact_status check_shape(const void* x, int64_t ldx, const float* s, int64_t M, int64_t N,
                           int act) {
   if (!x || !s) return fail(MOEACT_EINVAL, "x and s are required");
@@ -228,24 +247,41 @@ size_t ws_bytes_needed(int64_t M, int64_t N) {
 // ------------------------------------------------------------ launches
 template <int ACT, bool GROUPED>
 FwdVariant pick_fwd(int dirs, bool staged) {
+  // dirs carries kGemm for the GEMM-ready scale layout
   if (ACT == kSwiGLU && staged) {
-    if (dirs == kRow) return fwd_variant<ACT, kRow, true, GROUPED>();
-    if (dirs == kCol) return fwd_variant<ACT, kCol, true, GROUPED>();
-    return fwd_variant<ACT, kRow | kCol, true, GROUPED>();
+    switch (dirs) {
+      case kRow: return fwd_variant<ACT, kRow, true, GROUPED>();
+      case kCol: return fwd_variant<ACT, kCol, true, GROUPED>();
+      case kRow | kCol: return fwd_variant<ACT, kRow | kCol, true, GROUPED>();
+      case kRow | kGemm: return fwd_variant<ACT, kRow | kGemm, true, GROUPED>();
+      case kCol | kGemm: return fwd_variant<ACT, kCol | kGemm, true, GROUPED>();
+      default: return fwd_variant<ACT, kRow | kCol | kGemm, true, GROUPED>();
+    }
   }
-  if (dirs == kRow) return fwd_variant<ACT, kRow, false, GROUPED>();
-  if (dirs == kCol) return fwd_variant<ACT, kCol, false, GROUPED>();
-  return fwd_variant<ACT, kRow | kCol, false, GROUPED>();
+  switch (dirs) {
+    case kRow: return fwd_variant<ACT, kRow, false, GROUPED>();
+    case kCol: return fwd_variant<ACT, kCol, false, GROUPED>();
+    case kRow | kCol: return fwd_variant<ACT, kRow | kCol, false, GROUPED>();
+    case kRow | kGemm: return fwd_variant<ACT, kRow | kGemm, false, GROUPED>();
+    case kCol | kGemm: return fwd_variant<ACT, kCol | kGemm, false, GROUPED>();
+    default: return fwd_variant<ACT, kRow | kCol | kGemm, false, GROUPED>();
+  }
 }
 
 // With dX written, the colwise pass re-reads it instead of keeping the whole
 // tile in registers.
 template <int ACT, bool GROUPED, bool REREAD>
 BwdVariant pick_bwd_rr(int dirs) {
-  if (dirs == 0) return bwd_variant<ACT, 0, GROUPED, REREAD>();
-  if (dirs == kRow) return bwd_variant<ACT, kRow, GROUPED, REREAD>();
-  if (dirs == kCol) return bwd_variant<ACT, kCol, GROUPED, REREAD>();
-  return bwd_variant<ACT, kRow | kCol, GROUPED, REREAD>();
+  // dirs carries kGemm for the GEMM-ready scale layout (never with dirs 0)
+  switch (dirs) {
+    case 0: return bwd_variant<ACT, 0, GROUPED, REREAD>();
+    case kRow: return bwd_variant<ACT, kRow, GROUPED, REREAD>();
+    case kCol: return bwd_variant<ACT, kCol, GROUPED, REREAD>();
+    case kRow | kCol: return bwd_variant<ACT, kRow | kCol, GROUPED, REREAD>();
+    case kRow | kGemm: return bwd_variant<ACT, kRow | kGemm, GROUPED, REREAD>();
+    case kCol | kGemm: return bwd_variant<ACT, kCol | kGemm, GROUPED, REREAD>();
+    default: return bwd_variant<ACT, kRow | kCol | kGemm, GROUPED, REREAD>();
+  }
 }
 
 template <int ACT, bool GROUPED>
@@ -311,6 +347,7 @@ moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, in
   moeact_status st = check_shape(x, ldx, s, M, N, act);
   if (st) return st;
   if ((st = check_mx(out, dirs, false))) return st;
+  if ((st = check_layout(out, M, N))) return st;
   if (staged != 0 && staged != 1) return fail(MOEACT_EINVAL, "staged_rounding must be 0 or 1");
   if (grouped && (st = check_groups(ro, cb, E, status))) return st;
   if (M == 0) return MOEACT_OK;
@@ -334,11 +371,15 @@ moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, in
   p.status = status;
   p.dense_slabs = ceil_div(M, 32);
   p.n_tiles = (int)ceil_div(N, kTileCols);
+  p.gemm_scales = out.scale_layout == MOEACT_SCALES_GEMM;
   p.err = g_err_ptr[dev];
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
   FwdVariant v;
-  if (act == kSwiGLU) v = grouped ? pick_fwd<kSwiGLU, true>(dirs, staged) : pick_fwd<kSwiGLU, false>(dirs, staged);
-  else v = grouped ? pick_fwd<kSReLU, true>(dirs, false) : pick_fwd<kSReLU, false>(dirs, false);
+  const int kdirs = dirs | (p.gemm_scales ? kGemm : 0);
+  if (act == kSwiGLU)
+    v = grouped ? pick_fwd<kSwiGLU, true>(kdirs, staged) : pick_fwd<kSwiGLU, false>(kdirs, staged);
+  else
+    v = grouped ? pick_fwd<kSReLU, true>(kdirs, false) : pick_fwd<kSReLU, false>(kdirs, false);
   CUtensorMap tx;
   if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
   const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
@@ -357,6 +398,7 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   moeact_status st = check_shape(x, ldx, s, M, N, act);
   if (st) return st;
   if ((st = check_mx(out, dirs, true))) return st;
+  if ((st = check_layout(out, M, N))) return st;
   if (!dy) return fail(MOEACT_EINVAL, "dy is required");
   if (lddy < N) return fail(MOEACT_EINVAL, "lddy (%lld) smaller than N", (long long)lddy);
   if (lddy % 8 != 0) return fail(MOEACT_EALIGN, "lddy must be a multiple of 8 elements");
@@ -398,12 +440,16 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   p.status = status;
   p.dense_slabs = ceil_div(M, 32);
   p.n_tiles = (int)ceil_div(N, kTileCols);
+  p.gemm_scales = out.scale_layout == MOEACT_SCALES_GEMM;
   p.err = g_err_ptr[dev];
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
   BwdVariant v;
   const bool rr = dx != nullptr;
-  if (act == kSwiGLU) v = grouped ? pick_bwd<kSwiGLU, true>(dirs, rr) : pick_bwd<kSwiGLU, false>(dirs, rr);
-  else v = grouped ? pick_bwd<kSReLU, true>(dirs, rr) : pick_bwd<kSReLU, false>(dirs, rr);
+  const int kdirs = dirs | ((p.gemm_scales && dirs) ? kGemm : 0);
+  if (act == kSwiGLU)
+    v = grouped ? pick_bwd<kSwiGLU, true>(kdirs, rr) : pick_bwd<kSwiGLU, false>(kdirs, rr);
+  else
+    v = grouped ? pick_bwd<kSReLU, true>(kdirs, rr) : pick_bwd<kSReLU, false>(kdirs, rr);
   CUtensorMap tx, tdy;
   if ((st = make_x_map(&tx, act, x, N, M, ldx))) return st;
   if ((st = make_map(&tdy, dy, N, M, lddy))) return st;

@@ -45,6 +45,10 @@ namespace moeact {
 enum Act : int { kSwiGLU = 0, kSReLU = 1 };
 constexpr int kRow = 1;
 constexpr int kCol = 2;
+// Kernel template flag carried in the DIRS bits: scales in the GEMM-ready
+// tiled layout (a compile-time choice, so the row-major kernels carry none of
+// its code).
+constexpr int kGemm = 4;
 constexpr int kTileCols = 128;   // columns of a warp-tile (4 per lane)
 
 // The table lives in device global memory of this module, one copy per
@@ -217,6 +221,7 @@ struct Params {
   int32_t* status;
   int64_t dense_slabs;
   int n_tiles;
+  int gemm_scales;    // scales in the GEMM-ready tiled layout (see gemm_row_scales_off)
   uint32_t* err;      // device error word (timeouts), never expected to be set
 };
 
@@ -314,15 +319,17 @@ __device__ __forceinline__ int64_t stage_and_validate(const Params& p, const Sme
         ok = (mm >= 0) && (r <= p.M) && (c - c0 == (mm + 31) / 32);
       }
       if (e == p.E) ok = ok && (r == p.M);
-      if (!ok) bad = 1;
+      if (!ok) bad |= 1;
+      if (p.gemm_scales && (r & 127)) bad |= 2;
       m.cb[e] = (int)c;
       m.ro[e] = (int)r;
     }
   }
-  bad = __syncthreads_or(bad);
+  const int bad_offsets = __syncthreads_or(bad & 1);
+  const int unaligned = __syncthreads_or(bad & 2);
   if (!GROUPED) return p.dense_slabs;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = bad ? 3 : 0;
-  return bad ? -1 : (int64_t)m.cb[p.E];
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = bad_offsets ? 3 : (unaligned ? 4 : 0);
+  return (bad_offsets || unaligned) ? -1 : (int64_t)m.cb[p.E];
 }
 
 // Rows of slab `slab`: first row and count (<= 32).
@@ -459,6 +466,49 @@ __device__ __forceinline__ void store_scales4(uint8_t* dst, uint32_t v, int nb) 
   }
 }
 
+// GEMM-ready scale layout: the E8M0 matrix cut into tiles of 128 rows x 4
+// scale columns (512 bytes), tiles in row-major order, element (r, c) of a
+// tile at byte (r % 32) * 16 + (r / 32) * 4 + c.  Used only when M, every
+// group's rows and N are multiples of 128, so that no tile is partial.
+// Byte offset of the four row scales of row r in scale columns 4t .. 4t+3
+// (tile column t) of a matrix with `nct` tile columns:
+__device__ __forceinline__ int64_t gemm_row_scales_off(int64_t r, int t, int nct) {
+  return ((((r >> 7) * nct + t)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2);
+}
+
+// Colwise scales in the GEMM layout: a group's colwise data is read by the
+// GEMM transposed ([W] rows, K = the group's rows), so its scales form the
+// [W][m_e / 32] matrix of the same tiled layout; groups follow one another,
+// group e's tiles starting at byte base = row_offs[e] / 32 * W (the same
+// place its row-major colwise scales start).  Byte offset of the scale of
+// column w, K block j (of the group), with kt = m_e / 128 tile columns:
+__device__ __forceinline__ int64_t gemm_col_scale_off(int64_t base, int w, int j, int kt) {
+  return base + ((int64_t)((w >> 7) * kt + (j >> 2)) << 9) + ((w & 31) << 4) +
+         (((w >> 5) & 3) << 2) + (j & 3);
+}
+
+// The group geometry of slab `slab` for gemm_col_scale_off: base, the slab's
+// K block j within its group, and the group's tile columns kt.
+template <bool GROUPED>
+__device__ __forceinline__ void gemm_col_geom(const Params& p, const Smem& m, int64_t slab,
+                                              int64_t& base, int& j, int& kt) {
+  if (!GROUPED) {
+    base = 0;
+    j = (int)slab;
+    kt = (int)(p.M >> 7);
+    return;
+  }
+  int lo = 0, hi = p.E - 1;
+  const int sl = (int)slab;
+  while (lo < hi) {   // largest e with cb[e] <= slab (as slab_rows)
+    const int mid = (lo + hi + 1) >> 1;
+    if (m.cb[mid] <= sl) lo = mid; else hi = mid - 1;
+  }
+  base = (int64_t)(m.ro[lo] >> 5) * p.W;
+  j = sl - m.cb[lo];
+  kt = (m.ro[lo + 1] - m.ro[lo]) >> 7;
+}
+
 // Gathers, for row `lane` of the tile, the four blocks' E8M0 bytes from the
 // lanes that reduced them: bytes `byte_lo` (rows 0-15) / `byte_hi` (rows
 // 16-31) of w[h] in lanes 8k + ((row & 15) >> 1).
@@ -567,7 +617,11 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
     const uint32_t v = gather_row_scales(bh[0], bh[1], lane, 0, 1);
     if (lane < nrows) {
       const int nb = min(4, (p.N - tile * kTileCols) / 32);
-      store_scales4(p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile, v, nb);
+      if (DIRS & kGemm)
+        __stcs(reinterpret_cast<unsigned int*>(
+                   p.rs + gemm_row_scales_off(row0 + lane, tile, p.n_tiles)), v);
+      else
+        store_scales4(p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile, v, nb);
     }
   }
   if (DIRS & kCol) {
@@ -582,9 +636,18 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
       b[c] = e8m0_from_amax(a[c] >> 1);
       mu[c] = scale_multiplier(b[c]);
     }
-    if (colok)
-      __stcs(reinterpret_cast<unsigned int*>(p.cs + slab * (int64_t)W + c0),
-             b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));
+    if (colok) {
+      if (DIRS & kGemm) {
+        int64_t base;
+        int j, kt;
+        gemm_col_geom<GROUPED>(p, m, slab, base, j, kt);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) p.cs[gemm_col_scale_off(base, c0 + c, j, kt)] = (uint8_t)b[c];
+      } else {
+        __stcs(reinterpret_cast<unsigned int*>(p.cs + slab * (int64_t)W + c0),
+               b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));
+      }
+    }
     unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
     const int Wqc = opaque(Wq);
 #pragma unroll
@@ -869,9 +932,18 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
     const uint32_t vu = gather_row_scales(bh[0], bh[1], lane, 1, 3);
     if (lane < nrows) {
       const int nb = min(4, (N - tile * kTileCols) / 32);
-      uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
-      store_scales4(rsr, vg, nb);
-      if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
+      if (DIRS & kGemm) {
+        const int nct = W >> 7;
+        __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row0 + lane, tile, nct)),
+               vg);
+        if (ACT == kSwiGLU)
+          __stcs(reinterpret_cast<unsigned int*>(
+                     p.rs + gemm_row_scales_off(row0 + lane, (N >> 7) + tile, nct)), vu);
+      } else {
+        uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
+        store_scales4(rsr, vg, nb);
+        if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
+      }
     }
   }
   if (DIRS & kCol) {
@@ -897,11 +969,23 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
       mu[c] = scale_multiplier(bu[c]);
     }
     if (colok) {
-      uint8_t* csr = p.cs + slab * (int64_t)W + c0;
-      __stcs(reinterpret_cast<unsigned int*>(csr), bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
-      if (ACT == kSwiGLU)
-        __stcs(reinterpret_cast<unsigned int*>(csr + N),
-               bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
+      if (DIRS & kGemm) {
+        int64_t base;
+        int j, kt;
+        gemm_col_geom<GROUPED>(p, m, slab, base, j, kt);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          p.cs[gemm_col_scale_off(base, c0 + c, j, kt)] = (uint8_t)bg[c];
+          if (ACT == kSwiGLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
+        }
+      } else {
+        uint8_t* csr = p.cs + slab * (int64_t)W + c0;
+        __stcs(reinterpret_cast<unsigned int*>(csr),
+               bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
+        if (ACT == kSwiGLU)
+          __stcs(reinterpret_cast<unsigned int*>(csr + N),
+                 bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
+      }
     }
     unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
     const int Wqc = opaque(Wq);
@@ -1092,9 +1176,18 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
     const uint32_t vu = gather_row_scales(bh[0], bh[1], lane, 1, 3);
     if (lane < nrows) {
       const int nb = min(4, (N - tile * kTileCols) / 32);
-      uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
-      store_scales4(rsr, vg, nb);
-      if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
+      if (DIRS & kGemm) {
+        const int nct = W >> 7;
+        __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row0 + lane, tile, nct)),
+               vg);
+        if (ACT == kSwiGLU)
+          __stcs(reinterpret_cast<unsigned int*>(
+                     p.rs + gemm_row_scales_off(row0 + lane, (N >> 7) + tile, nct)), vu);
+      } else {
+        uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
+        store_scales4(rsr, vg, nb);
+        if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
+      }
     }
   }
   if (DIRS & kCol) {
@@ -1112,11 +1205,23 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
       mu[c] = scale_multiplier(bu[c]);
     }
     if (colok) {
-      uint8_t* csr = p.cs + slab * (int64_t)W + c0;
-      __stcs(reinterpret_cast<unsigned int*>(csr), bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
-      if (ACT == kSwiGLU)
-        __stcs(reinterpret_cast<unsigned int*>(csr + N),
-               bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
+      if (DIRS & kGemm) {
+        int64_t base;
+        int j, kt;
+        gemm_col_geom<GROUPED>(p, m, slab, base, j, kt);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          p.cs[gemm_col_scale_off(base, c0 + c, j, kt)] = (uint8_t)bg[c];
+          if (ACT == kSwiGLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
+        }
+      } else {
+        uint8_t* csr = p.cs + slab * (int64_t)W + c0;
+        __stcs(reinterpret_cast<unsigned int*>(csr),
+               bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
+        if (ACT == kSwiGLU)
+          __stcs(reinterpret_cast<unsigned int*>(csr + N),
+                 bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
+      }
     }
     unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
     const int Wqc = opaque(Wq);

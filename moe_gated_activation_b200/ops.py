@@ -76,7 +76,7 @@ def _alloc_mx(M, W, dirs, device, col_rows):
     return rq, rs, cq, cs
 
 
-def _mx_struct(rq, rs, cq, cs, dirs):
+def _mx_struct(rq, rs, cq, cs, dirs, gemm_scales=False):
     if dirs & ROWWISE:
         r = (rq.data_ptr(), rs.data_ptr())
     else:
@@ -85,7 +85,8 @@ def _mx_struct(rq, rs, cq, cs, dirs):
         c = (cq.data_ptr(), cs.data_ptr())
     else:
         c = (None, None)
-    return _capi.MxOut(r[0], r[1], c[0], c[1])
+    layout = _capi.SCALES_GEMM if gemm_scales else _capi.SCALES_ROWMAJOR
+    return _capi.MxOut(r[0], r[1], c[0], c[1], layout)
 
 
 def _mx_result(rq, rs, cq, cs, col_rows_view=None):
@@ -112,7 +113,7 @@ def splits_to_offsets(m_splits: torch.Tensor, total_rows: int):
 
 
 # ------------------------------------------------------------------ forward
-def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None):
+def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False):
     swiglu = act == "swiglu"
     if N is None:
         N = x.shape[1] // 2 if swiglu else x.shape[1]
@@ -126,7 +127,7 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None):
         ro, cb, E, st, view = grouped
         col_rows = (M + 31) // 32 + E
     rq, rs, cq, cs = _alloc_mx(M, N, dirs, x.device, col_rows)
-    mx = _mx_struct(rq, rs, cq, cs, dirs)
+    mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales)
     stream = _stream(x.device)
     ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
     if grouped is None:
@@ -145,14 +146,17 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None):
     return _mx_result(rq, rs, cq, cs, view)
 
 
-def scaled_swiglu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, staged_rounding=False, N=None):
-    """MXFP8 of SwiGLU(x) * s; x bf16 [M, >=2N] packs [gate | up]."""
-    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding)
+def scaled_swiglu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, staged_rounding=False, N=None,
+                            gemm_scales=False):
+    """MXFP8 of SwiGLU(x) * s; x bf16 [M, >=2N] packs [gate | up].
+    gemm_scales: scales in the GEMM-ready tiled layout (moeact.h,
+    MOEACT_SCALES_GEMM; M and N multiples of 128)."""
+    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, gemm_scales=gemm_scales)
 
 
-def scaled_srelu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, N=None):
+def scaled_srelu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, N=None, gemm_scales=False):
     """MXFP8 of relu(x)^2 * s; x bf16 [M, >=N]."""
-    return _fwd("srelu", x, s, N, rowwise, colwise, False)
+    return _fwd("srelu", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales)
 
 
 def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
@@ -164,19 +168,20 @@ def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
 
 def grouped_scaled_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
                                     staged_rounding=False, status=None, col_scale_rows=None,
-                                    N=None):
+                                    N=None, gemm_scales=False):
     """Grouped forward: experts own the rows given by `row_offs` (from
     splits_to_offsets).  Returns (MXFP8, status).  Col scales hold
     ceil(M/32) + E rows unless `col_scale_rows` (sum of ceil(m_e/32), known on
     the host) is given."""
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
-    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, g), status
+    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, g,
+                gemm_scales=gemm_scales), status
 
 
 def grouped_scaled_srelu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
-                                   status=None, col_scale_rows=None, N=None):
+                                   status=None, col_scale_rows=None, N=None, gemm_scales=False):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
-    return _fwd("srelu", x, s, N, rowwise, colwise, False, g), status
+    return _fwd("srelu", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales), status
 
 
 # ------------------------------------------------------------------ backward
@@ -189,7 +194,8 @@ def bwd_workspace_bytes(M, N, num_groups=1):
 
 
 def _workspace(device, nbytes):
-    """A zero-filled workspace per (device, stream); the kernels leave it zeroed."""
+    """A workspace per (device, stream), reused across calls (the kernels need
+    no initial content in it)."""
     key = (device.index, torch.cuda.current_stream(device).cuda_stream)
     with _ws_lock:
         ws = _ws_cache.get(key)
@@ -199,7 +205,8 @@ def _workspace(device, nbytes):
     return ws
 
 
-def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, grouped=None):
+def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, grouped=None,
+         gemm_scales=False):
     swiglu = act == "swiglu"
     if N is None:
         N = dy.shape[1]
@@ -218,7 +225,7 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
         ro, cb, E, st, view = grouped
         col_rows = (M + 31) // 32 + E
     rq, rs, cq, cs = _alloc_mx(M, W, dirs, dev, col_rows)
-    mx = _mx_struct(rq, rs, cq, cs, dirs)
+    mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales)
     dx = torch.empty((M, W), dtype=torch.bfloat16, device=dev) if want_dx else None
     dscale = torch.empty(M, dtype=torch.float32, device=dev) if want_dscale else None
     nbytes = bwd_workspace_bytes(M, N, E)
@@ -240,30 +247,34 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
 
 
 def scaled_swiglu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
-                            want_dscale=True, workspace=None, N=None):
+                            want_dscale=True, workspace=None, N=None, gemm_scales=False):
     """Backward of the scaled SwiGLU: MXFP8 of [dgate | dup], bf16 dx, fp32 dscale."""
-    return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace)
+    return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
+                gemm_scales=gemm_scales)
 
 
 def scaled_srelu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
-                           want_dscale=True, workspace=None, N=None):
-    return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace)
+                           want_dscale=True, workspace=None, N=None, gemm_scales=False):
+    return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
+                gemm_scales=gemm_scales)
 
 
 def grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
                                     colwise=True, want_dx=True, want_dscale=True,
-                                    workspace=None, status=None, col_scale_rows=None, N=None):
+                                    workspace=None, status=None, col_scale_rows=None, N=None,
+                                    gemm_scales=False):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                g), status
+                g, gemm_scales=gemm_scales), status
 
 
 def grouped_scaled_srelu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
                                    colwise=True, want_dx=True, want_dscale=True,
-                                   workspace=None, status=None, col_scale_rows=None, N=None):
+                                   workspace=None, status=None, col_scale_rows=None, N=None,
+                                   gemm_scales=False):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                g), status
+                g, gemm_scales=gemm_scales), status
 
 
 # ------------------------------------------------------------------ misc

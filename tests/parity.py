@@ -106,3 +106,27 @@ def compare_mx(got, ref, what, exact=True):
         assert_codes(got.col_codes, ref["col_codes"], what + " col codes", exact)
     else:
         assert got.col_codes.numel() == 0 and got.col_scales.numel() == 0
+
+
+# ------------------------------------------------------------------ GEMM scale layout
+def unblock_rows(buf, R, C):
+    """Inverse of the GEMM-ready tiled scale layout for an [R, C] matrix with
+    R % 128 == 0 and C % 4 == 0 (tiles [R/128, C/4] of 32 x 4 x 4 bytes
+    ordered (r0, r1, c), row r = 128 t + 32 r1 + r0), via tensor reshapes."""
+    t = torch.as_tensor(np.asarray(buf)).reshape(R // 128, C // 4, 32, 4, 4)
+    return t.permute(0, 3, 2, 1, 4).reshape(R, C).numpy()
+
+
+def unblock_cols(buf, W, m_splits):
+    """Row-major colwise scales [sum m_e/32, W] from the GEMM-ready layout:
+    per group, tiles of the transposed [W, m_e/32] matrix."""
+    buf = np.asarray(buf).reshape(-1)
+    parts, pos = [], 0
+    for me in m_splits:
+        kb = int(me) // 32
+        n = W * kb
+        if n:
+            blk = unblock_rows(buf[pos:pos + n], W, kb)   # [W, m_e/32]
+            parts.append(np.ascontiguousarray(blk.T))
+        pos += n
+    return np.concatenate(parts) if parts else np.zeros((0, W), np.uint8)

@@ -138,3 +138,14 @@ def test_splits_to_offsets_argument_errors(lib):
     assert f(A16, 4, -1, A16, A16, A16, None) == _capi.EINVAL
     assert f(A16 + 4, 4, 64, A16, A16, A16, None) == _capi.EALIGN
     assert f(A16, 4, 1 << 40, A16, A16, A16, None) == _capi.ERANGE
+
+
+def test_gemm_scale_layout_argument_errors(lib):
+    gemm = lambda *p: _capi.MxOut(*p, _capi.SCALES_GEMM)
+    bad_layout = _capi.MxOut(A16, A16, None, None, 2)
+    assert fwd(lib, mx=bad_layout) == _capi.EINVAL
+    assert fwd(lib, M=256, N=96, ldx=192, mx=gemm(A16, A16, None, None)) == _capi.EINVAL
+    assert b"multiples of 128" in lib.moeact_last_error()
+    assert fwd(lib, M=100, N=256, mx=gemm(A16, A16, None, None)) == _capi.EINVAL
+    assert bwd(lib, M=96, N=128, ldx=256, lddy=128, mx=gemm(A16, A16, None, None)) == _capi.EINVAL
+    assert fwd(lib, M=0, N=256, mx=gemm(A16, A16, None, None)) == _capi.OK

@@ -89,6 +89,19 @@ def _load():
     lib.orc_grouped_act_bwd.argtypes = [I, P, I64, P, I64, P, I64, I64, I, P, P, I32,
                                         P, P, P, P, P, P]
     lib.orc_grouped_act_bwd.restype = I
+    F = ctypes.c_float
+    lib.orc_clamped_fwd.argtypes = [P, I64, P, I64, I64, I, F, F, P, P, P, P]
+    lib.orc_clamped_fwd.restype = I
+    lib.orc_clamped_values.argtypes = [P, I64, P, I64, I64, F, F, P]
+    lib.orc_clamped_values.restype = I
+    lib.orc_clamped_bwd.argtypes = [P, I64, P, I64, P, I64, I64, I, F, F, P, P, P, P, P, P]
+    lib.orc_clamped_bwd.restype = I
+    lib.orc_grouped_clamped_fwd.argtypes = [P, I64, P, I64, I64, I, F, F, P, P, I32,
+                                            P, P, P, P]
+    lib.orc_grouped_clamped_fwd.restype = I
+    lib.orc_grouped_clamped_bwd.argtypes = [P, I64, P, I64, P, I64, I64, I, F, F, P, P, I32,
+                                            P, P, P, P, P, P]
+    lib.orc_grouped_clamped_bwd.restype = I
     lib.orc_scales_gemm_layout.argtypes = [P, I64, I64, P]
     lib.orc_scales_gemm_layout.restype = None
     lib.orc_col_scales_gemm_layout.argtypes = [P, I64, P, P, I32, P]
@@ -296,3 +309,86 @@ def col_scales_gemm_layout(cs: np.ndarray, W: int, row_offs, colblk_offs) -> np.
     if _load().orc_col_scales_gemm_layout(_ptr(cs), W, _ptr(ro), _ptr(co), E, _ptr(out)):
         raise ValueError("GEMM layout needs W and every group's rows to be multiples of 128")
     return out[:int(ro[-1]) * W // 32]
+
+
+# ---------------------------------------------------------------- ClampedSwiGLU
+CLAMPED_ALPHA = 1.702   # defaults of the reading (the public gpt-oss clamped SwiGLU)
+CLAMPED_LIMIT = 7.0
+
+
+def _check_rc(rc, what):
+    if rc == 3:
+        raise ArithmeticError(f"oracle {what}: a sigma rounding could not be certified")
+    if rc:
+        raise ValueError(f"oracle {what} failed ({rc})")
+
+
+def clamped_fwd(x_bits, s, N, dirs, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT):
+    """Forward of the scaled ClampedSwiGLU: MXFP8 of h(x) * s, width N."""
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    M = x_bits.shape[0]
+    out = _alloc_mx(M, N, dirs)
+    _check_rc(_load().orc_clamped_fwd(_ptr(x_bits), x_bits.shape[1], _ptr(s), M, N, dirs,
+                                      alpha, limit, *_mx_ptrs(out)), "clamped_fwd")
+    return out
+
+
+def clamped_values(x_bits, s, N, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT):
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    M = x_bits.shape[0]
+    y = np.zeros((M, N), np.float32)
+    _check_rc(_load().orc_clamped_values(_ptr(x_bits), x_bits.shape[1], _ptr(s), M, N, alpha,
+                                         limit, _ptr(y)), "clamped_values")
+    return y
+
+
+def clamped_bwd(dy_bits, x_bits, s, N, dirs, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
+                want_dx=True, want_dscale=True):
+    dy_bits = _c(dy_bits, np.uint16)
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    M = x_bits.shape[0]
+    out = _alloc_mx(M, 2 * N, dirs)
+    out["dx"] = np.zeros((M, 2 * N), np.uint16) if want_dx else None
+    out["dscale"] = np.zeros(M, np.float32) if want_dscale else None
+    _check_rc(_load().orc_clamped_bwd(_ptr(dy_bits), dy_bits.shape[1], _ptr(x_bits),
+                                      x_bits.shape[1], _ptr(s), M, N, dirs, alpha, limit,
+                                      _ptr(out["dx"]), _ptr(out["dscale"]), *_mx_ptrs(out)),
+              "clamped_bwd")
+    return out
+
+
+def grouped_clamped_fwd(x_bits, s, N, dirs, row_offs, colblk_offs, alpha=CLAMPED_ALPHA,
+                        limit=CLAMPED_LIMIT):
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    ro = _c(row_offs, np.int64)
+    co = _c(colblk_offs, np.int64)
+    M = x_bits.shape[0]
+    out = _alloc_mx(M, N, dirs, colblk_rows=int(co[-1]))
+    _check_rc(_load().orc_grouped_clamped_fwd(_ptr(x_bits), x_bits.shape[1], _ptr(s), M, N,
+                                              dirs, alpha, limit, _ptr(ro), _ptr(co),
+                                              ro.shape[0] - 1, *_mx_ptrs(out)),
+              "grouped_clamped_fwd")
+    return out
+
+
+def grouped_clamped_bwd(dy_bits, x_bits, s, N, dirs, row_offs, colblk_offs,
+                        alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT):
+    dy_bits = _c(dy_bits, np.uint16)
+    x_bits = _c(x_bits, np.uint16)
+    s = _c(s, np.float32)
+    ro = _c(row_offs, np.int64)
+    co = _c(colblk_offs, np.int64)
+    M = x_bits.shape[0]
+    out = _alloc_mx(M, 2 * N, dirs, colblk_rows=int(co[-1]))
+    out["dx"] = np.zeros((M, 2 * N), np.uint16)
+    out["dscale"] = np.zeros(M, np.float32)
+    _check_rc(_load().orc_grouped_clamped_bwd(_ptr(dy_bits), dy_bits.shape[1], _ptr(x_bits),
+                                              x_bits.shape[1], _ptr(s), M, N, dirs, alpha,
+                                              limit, _ptr(ro), _ptr(co), ro.shape[0] - 1,
+                                              _ptr(out["dx"]), _ptr(out["dscale"]),
+                                              *_mx_ptrs(out)), "grouped_clamped_bwd")
+    return out

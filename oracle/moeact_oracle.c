@@ -444,6 +444,161 @@ int orc_grouped_act_bwd(int act, const uint16_t* dy, int64_t lddy, const uint16_
 }
 
 /* ------------------------------------------------------------------ */
+/* ClampedSwiGLU                                                       */
+/* ------------------------------------------------------------------ */
+/* The third per-row-scaled activation TransformerEngine PR #3238 names
+ * (Greptile summary: SReLU / SwiGLU / ClampedSwiGLU); the pages give no
+ * definition.  Reading taken (the clamped SwiGLU of the public gpt-oss
+ * models, alpha and limit as parameters), in fp32 steps, x = [gate | up]:
+ *   gc = min(g, L), uc = clamp(u, -L, L)   (NaN passes through)
+ *   z = RN(alpha * gc);  sig = correctly rounded sigma(z)
+ *   silu = RN(gc * sig);  v = RN(uc + 1);  h = RN(silu * v);  y = RN(h * s)
+ * Backward (the SwiGLU form with the slope alpha; clamped inputs get a zero
+ * gradient, as a clamp's gradient is):
+ *   p = RN(dY * s)
+ *   dsilu = g > L ? 0 : fma(RN(alpha * silu), RN(1 - sig), sig)
+ *   dgate = g > L ? +0 : bf16(RN(RN(p * v) * dsilu))
+ *   dup   = |u| > L ? +0 : bf16(RN(p * silu))
+ *   dscale = sum_j dY * h (binary64, rounded once).
+ * With alpha = 1 and L = +Inf it is SwiGLU with up + 1 in place of up. */
+typedef struct { float g, u, gc, uc, z, sig, silu, v, h; } orc_clamped_parts;
+
+static void clamped_parts(uint16_t gb, uint16_t ub, float alpha, float L,
+                          orc_clamped_parts* c, int* certified) {
+  c->g = orc_bf16_to_f32(gb);
+  c->u = orc_bf16_to_f32(ub);
+  c->gc = (c->g > L) ? L : c->g;
+  c->uc = (c->u > L) ? L : ((c->u < -L) ? -L : c->u);
+  c->z = alpha * c->gc;
+  int ok = 1;
+  if (isnan(c->z)) c->sig = c->z;
+  else if (isinf(c->z)) c->sig = c->z > 0 ? 1.0f : 0.0f;
+  else c->sig = sigma_certified(c->z, &ok);
+  if (!ok) *certified = 0;
+  c->silu = c->gc * c->sig;
+  c->v = c->uc + 1.0f;
+  c->h = c->silu * c->v;
+}
+
+static int clamped_args_ok(float alpha, float L) {
+  return alpha >= 0.8125f && alpha <= 2.0f && L > 0.0f;   /* L may be +Inf; NaN fails */
+}
+
+/* Forward: outputs as orc_act_fwd (width N).  Returns 1 on bad arguments,
+ * 3 if a sigma rounding could not be certified. */
+int orc_clamped_fwd(const uint16_t* x, int64_t ldx, const float* s, int64_t M, int64_t N,
+                    int dirs, float alpha, float limit,
+                    uint8_t* rq, uint8_t* rs, uint8_t* cq, uint8_t* cs) {
+  if (M < 0 || N <= 0 || N % 32 != 0 || !clamped_args_ok(alpha, limit)) return 1;
+  if (M == 0) return 0;
+  orc_fpenv env = orc_enter();
+  float* y = (float*)malloc((size_t)(M * N) * sizeof(float));
+  if (!y) { orc_leave(env); return 2; }
+  int cert = 1;
+  for (int64_t i = 0; i < M; ++i)
+    for (int64_t j = 0; j < N; ++j) {
+      orc_clamped_parts c;
+      clamped_parts(x[i * ldx + j], x[i * ldx + N + j], alpha, limit, &c, &cert);
+      y[i * N + j] = c.h * s[i];
+    }
+  mxfp8_quantize(y, M, N, dirs, rq, rs, cq, cs);
+  free(y);
+  orc_leave(env);
+  return cert ? 0 : 3;
+}
+
+/* The fp32 activation before quantization (for pins). */
+int orc_clamped_values(const uint16_t* x, int64_t ldx, const float* s, int64_t M, int64_t N,
+                       float alpha, float limit, float* y) {
+  if (!clamped_args_ok(alpha, limit)) return 1;
+  orc_fpenv env = orc_enter();
+  int cert = 1;
+  for (int64_t i = 0; i < M; ++i)
+    for (int64_t j = 0; j < N; ++j) {
+      orc_clamped_parts c;
+      clamped_parts(x[i * ldx + j], x[i * ldx + N + j], alpha, limit, &c, &cert);
+      y[i * N + j] = c.h * s[i];
+    }
+  orc_leave(env);
+  return cert ? 0 : 3;
+}
+
+/* Backward: dx bf16 [M, 2N] = [dgate | dup], dscale fp32 [M], MXFP8 of dx. */
+int orc_clamped_bwd(const uint16_t* dy, int64_t lddy, const uint16_t* x, int64_t ldx,
+                    const float* s, int64_t M, int64_t N, int dirs, float alpha, float limit,
+                    uint16_t* dx, float* dscale,
+                    uint8_t* rq, uint8_t* rs, uint8_t* cq, uint8_t* cs) {
+  if (M < 0 || N <= 0 || N % 32 != 0 || !clamped_args_ok(alpha, limit)) return 1;
+  if (M == 0) return 0;
+  orc_fpenv env = orc_enter();
+  int64_t W = 2 * N;
+  float* d = (float*)malloc((size_t)(M * W) * sizeof(float));
+  if (!d) { orc_leave(env); return 2; }
+  int cert = 1;
+  for (int64_t i = 0; i < M; ++i) {
+    double acc = 0.0;
+    for (int64_t j = 0; j < N; ++j) {
+      orc_clamped_parts c;
+      clamped_parts(x[i * ldx + j], x[i * ldx + N + j], alpha, limit, &c, &cert);
+      float gy = orc_bf16_to_f32(dy[i * lddy + j]);
+      float p = gy * s[i];
+      float dg = 0.0f, du = 0.0f;
+      if (!(c.g > limit)) {
+        float as = alpha * c.silu;
+        float dsilu = fmaf(as, 1.0f - c.sig, c.sig);   /* one rounding */
+        float t = p * c.v;
+        dg = bf16_round(t * dsilu);
+      }
+      if (!(c.u > limit || c.u < -limit)) du = bf16_round(p * c.silu);
+      d[i * W + j] = dg;
+      d[i * W + N + j] = du;
+      acc += (double)gy * (double)c.h;
+    }
+    if (dscale) dscale[i] = (float)acc;
+  }
+  if (dx)
+    for (int64_t k = 0; k < M * W; ++k) dx[k] = orc_f32_to_bf16(d[k]);
+  mxfp8_quantize(d, M, W, dirs, rq, rs, cq, cs);
+  free(d);
+  orc_leave(env);
+  return cert ? 0 : 3;
+}
+
+int orc_grouped_clamped_fwd(const uint16_t* x, int64_t ldx, const float* s, int64_t M,
+                            int64_t N, int dirs, float alpha, float limit,
+                            const int64_t* row_offs, const int64_t* colblk_offs, int32_t E,
+                            uint8_t* rq, uint8_t* rs, uint8_t* cq, uint8_t* cs) {
+  if (row_offs[E] != M) return 2;
+  for (int32_t e = 0; e < E; ++e) {
+    int64_t r0 = row_offs[e], me = row_offs[e + 1] - r0, c0 = colblk_offs[e];
+    int rc = orc_clamped_fwd(x + r0 * ldx, ldx, s + r0, me, N, dirs, alpha, limit,
+                             rq ? rq + r0 * N : NULL, rs ? rs + r0 * (N / 32) : NULL,
+                             cq ? cq + r0 * N : NULL, cs ? cs + c0 * N : NULL);
+    if (rc) return rc;
+  }
+  return 0;
+}
+
+int orc_grouped_clamped_bwd(const uint16_t* dy, int64_t lddy, const uint16_t* x, int64_t ldx,
+                            const float* s, int64_t M, int64_t N, int dirs, float alpha,
+                            float limit, const int64_t* row_offs, const int64_t* colblk_offs,
+                            int32_t E, uint16_t* dx, float* dscale,
+                            uint8_t* rq, uint8_t* rs, uint8_t* cq, uint8_t* cs) {
+  if (row_offs[E] != M) return 2;
+  int64_t W = 2 * N;
+  for (int32_t e = 0; e < E; ++e) {
+    int64_t r0 = row_offs[e], me = row_offs[e + 1] - r0, c0 = colblk_offs[e];
+    int rc = orc_clamped_bwd(dy + r0 * lddy, lddy, x + r0 * ldx, ldx, s + r0, me, N, dirs,
+                             alpha, limit, dx ? dx + r0 * W : NULL,
+                             dscale ? dscale + r0 : NULL, rq ? rq + r0 * W : NULL,
+                             rs ? rs + r0 * (W / 32) : NULL, cq ? cq + r0 * W : NULL,
+                             cs ? cs + c0 * W : NULL);
+    if (rc) return rc;
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* GEMM-ready scale layout.                                            */
 /* ------------------------------------------------------------------ */
 /* The consumer of the quantized grouped tensors is a block-scaled grouped

@@ -290,3 +290,63 @@ def bwd_values(dyb, xb, s, N, act="swiglu"):
         dx.append(d)
         dsc.append(math.nan if nan else float(acc))
     return dx, dsc
+
+
+# ------------------------------------------------------------ ClampedSwiGLU
+def fadd(a: float, b: float) -> float:
+    return fsub(a, -b)
+
+
+@functools.lru_cache(maxsize=None)
+def sigmoid_of(z: float) -> float:
+    """Correctly rounded fp32 sigma of an fp32 value z (decimal, 60 digits)."""
+    if math.isnan(z):
+        return math.nan
+    if math.isinf(z):
+        return 1.0 if z > 0 else 0.0
+    if z < -200:
+        return 0.0
+    if z > 200:
+        return 1.0
+    ctx = decimal.Context(prec=60)
+    e = ctx.exp(ctx.minus(decimal.Decimal(z)))
+    return round_f32(Fraction(ctx.divide(decimal.Decimal(1), ctx.add(decimal.Decimal(1), e))))
+
+
+def _clamped_parts(gb, ub, alpha, L):
+    g, u = bf16_value(gb), bf16_value(ub)
+    gc = L if g > L else g
+    uc = L if u > L else (-L if u < -L else u)
+    z = fmul(alpha, gc)
+    sig = sigmoid_of(z)
+    silu = fmul(gc, sig)
+    v = fadd(uc, 1.0)
+    return g, u, sig, silu, v, fmul(silu, v)
+
+
+def clamped_fwd_values(xb, s, N, alpha, L):
+    return [[fmul(_clamped_parts(row[j], row[N + j], alpha, L)[5], s[i]) for j in range(N)]
+            for i, row in enumerate(xb)]
+
+
+def clamped_bwd_values(dyb, xb, s, N, alpha, L):
+    dx, dsc = [], []
+    for i, row in enumerate(xb):
+        d = [0.0] * (2 * N)
+        acc, bad = Fraction(0), False
+        for j in range(N):
+            g, u, sig, silu, v, h = _clamped_parts(row[j], row[N + j], alpha, L)
+            gy = bf16_value(dyb[i][j])
+            p = fmul(gy, s[i])
+            if not g > L:
+                dsilu = ffma(fmul(alpha, silu), fsub(1.0, sig), sig)
+                d[j] = round_bf16_value(fmul(fmul(p, v), dsilu))
+            if not (u > L or u < -L):
+                d[N + j] = round_bf16_value(fmul(p, silu))
+            if any(math.isnan(t) or math.isinf(t) for t in (gy, h)):
+                bad = True
+            else:
+                acc += Fraction(gy) * Fraction(h)
+        dx.append(d)
+        dsc.append(math.nan if bad else float(acc))
+    return dx, dsc

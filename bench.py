@@ -159,6 +159,17 @@ def ncu_traffic(workload, kernel, dirs_name):
     return None
 
 
+def act_api(mg, act):
+    """(grouped forward, grouped backward, extra keyword arguments) of an
+    activation; ClampedSwiGLU at the default slope and limit."""
+    if act == "clamped":
+        mg.init_clamped()
+        return (mg.grouped_scaled_clamped_swiglu_mxfp8_fwd,
+                mg.grouped_scaled_clamped_swiglu_mxfp8_bwd,
+                {"alpha": mg.ops.CLAMPED_ALPHA, "limit": mg.ops.CLAMPED_LIMIT})
+    return mg.grouped_scaled_swiglu_mxfp8_fwd, mg.grouped_scaled_swiglu_mxfp8_bwd, {}
+
+
 def max_over_ranks(value, world, device):
     """The largest `value` over all ranks (every rank gets it); with one rank,
     `value` itself.  `device` is where the collective's tensor lives (cuda
@@ -225,15 +236,15 @@ def run_ours(args):
         return mg.splits_to_offsets(m_dev, M)
 
     gemm = args.scales == "gemm"
+    fwd_api, bwd_api, extra = act_api(mg, args.act)
 
     def fwd(ro, cb, st):
-        return mg.grouped_scaled_swiglu_mxfp8_fwd(x, s, ro, cb, rowwise=rw, colwise=cw,
-                                                  col_scale_rows=S, status=st, gemm_scales=gemm)
+        return fwd_api(x, s, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, status=st,
+                       gemm_scales=gemm, **extra)
 
     def bwd(ro, cb, st):
-        return mg.grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, ro, cb, rowwise=rw, colwise=cw,
-                                                  col_scale_rows=S, workspace=ws, status=st,
-                                                  gemm_scales=gemm)
+        return bwd_api(dy, x, s, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, workspace=ws,
+                       status=st, gemm_scales=gemm, **extra)
 
     # eager warm-up
     for i in range(3):
@@ -364,7 +375,7 @@ def run_ours(args):
         "dtype": "f32",
         "data": "synthetic (seeded torch generators; shapes and statistics of the pages' workloads)",
         "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
-                   "dirs": args.dirs, "scales": args.scales, "activation": "swiglu",
+                   "dirs": args.dirs, "scales": args.scales, "activation": args.act,
                    "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
                    "launch": "eager" if args.eager else "one CUDA graph per step (events at its ends only)",
                    "kernel_times": "eager events" if args.eager else "a second timed pass of the same steps, with event nodes between the calls",
@@ -397,50 +408,77 @@ def run_ours(args):
 
 
 def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
+    """The step through the public API with host buffers: every step copies its
+    inputs (X, s, dY, m_splits) from pinned host memory to the device, runs
+    splits_to_offsets, the forward and the backward, and copies every output
+    back to pinned host memory.  Three streams pipeline consecutive steps
+    (host->device copies of step i+1 and device->host copies of step i-1 run
+    while step i computes; the two copy directions use separate engines), with
+    double-buffered device inputs and host outputs.  Timed from the first copy
+    in to the last copy out."""
     M, N = wl.M, wl.N
     rw, cw = bool(dirs & 1), bool(dirs & 2)
-    xh = inp["x"].cpu().pin_memory()
-    sh = inp["s"].cpu().pin_memory()
-    dyh = inp["dy"].cpu().pin_memory()
-    mh = inp["m_splits"].clone().pin_memory()
-    xd, sd, dyd, md = (torch.empty_like(t, device=dev) for t in (xh, sh, dyh, mh))
-    h2d = sum(t.numel() * t.element_size() for t in (xh, sh, dyh, mh))
-    outs_h = None
+    gemm = args.scales == "gemm"
+    fwd_api, bwd_api, extra = act_api(mg, args.act)
+    hin = [inp["x"].cpu().pin_memory(), inp["s"].cpu().pin_memory(),
+           inp["dy"].cpu().pin_memory(), inp["m_splits"].clone().pin_memory()]
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    dbuf = [[torch.empty_like(t, device=dev) for t in hin] for _ in range(2)]
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    hout = [None, None]
 
-    def one():
-        nonlocal outs_h
-        xd.copy_(xh, non_blocking=True)
-        sd.copy_(sh, non_blocking=True)
-        dyd.copy_(dyh, non_blocking=True)
-        md.copy_(mh, non_blocking=True)
-        ro, cb, st = mg.splits_to_offsets(md, M)
-        gemm = args.scales == "gemm"
-        f, fst = mg.grouped_scaled_swiglu_mxfp8_fwd(xd, sd, ro, cb, rowwise=rw, colwise=cw,
-                                                    col_scale_rows=S, status=st,
-                                                    gemm_scales=gemm)
-        b, bst = mg.grouped_scaled_swiglu_mxfp8_bwd(dyd, xd, sd, ro, cb, rowwise=rw, colwise=cw,
-                                                    col_scale_rows=S, status=st,
-                                                    gemm_scales=gemm)
-        outs = [t for t in (*f, *b.mx, b.dx, b.dscale, st) if t is not None and t.numel()]
-        if outs_h is None:
-            outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-        for h, t in zip(outs_h, outs):
-            h.copy_(t, non_blocking=True)
-        return outs
+    def step(i, in_free, out_free):
+        """Enqueue step i; returns (inputs consumed, outputs copied) events."""
+        b = i & 1
+        xd, sd, dyd, md = dbuf[b]
+        with torch.cuda.stream(s_in):
+            if in_free[b] is not None:
+                s_in.wait_event(in_free[b])
+            for d, h in zip(dbuf[b], hin):
+                d.copy_(h, non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(loaded)
+            ro, cb, st = mg.splits_to_offsets(md, M)
+            f, _ = fwd_api(xd, sd, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, status=st,
+                           gemm_scales=gemm, **extra)
+            bw, _ = bwd_api(dyd, xd, sd, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S,
+                            status=st, gemm_scales=gemm, **extra)
+            outs = [t for t in (*f, *bw.mx, bw.dx, bw.dscale, st) if t is not None and t.numel()]
+            done = torch.cuda.Event()
+            done.record(s_comp)
+        if hout[b] is None:
+            hout[b] = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            if out_free[b] is not None:
+                s_out.wait_event(out_free[b])
+            for h, t in zip(hout[b], outs):
+                t.record_stream(s_out)
+                h.copy_(t, non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(s_out)
+        return done, copied, outs
 
-    outs = one()
+    in_free, out_free = [None, None], [None, None]
+    keep = []                                  # outputs of the last steps stay referenced
+    for i in range(4):                         # warm-up: host outputs, allocator pool
+        in_free[i & 1], out_free[i & 1], outs = step(i, in_free, out_free)
+        keep = (keep + [outs])[-2:]
     torch.cuda.synchronize()
     d2h = sum(t.numel() * t.element_size() for t in outs)
-    steps = max(1, min(args.steps, 20))
+    steps = max(2, min(args.steps, 20))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(steps):
+        in_free[i & 1], out_free[i & 1], outs = step(i, in_free, out_free)
+        keep = (keep + [outs])[-2:]
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     E = int(inp["m_splits"].numel())
@@ -448,7 +486,8 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
     step_bytes = bm["splits"] + bm["fwd"] + bm["bwd"]
     return {"value": round(whole_job_gbs(world, steps, step_bytes, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 4)}
+            "ms_per_step": round(ms / steps, 4),
+            "pipeline": "copy-in / compute / copy-out streams, double-buffered"}
 
 
 # ------------------------------------------------------------------ oracle timing
@@ -540,6 +579,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--dirs", default="both", choices=list(DIRS))
+    ap.add_argument("--act", default="swiglu", choices=["swiglu", "clamped"],
+                    help="activation: SwiGLU, or ClampedSwiGLU (alpha 1.702, limit 7)")
     ap.add_argument("--scales", default="rowmajor", choices=["rowmajor", "gemm"],
                     help="E8M0 scale layout: row-major, or the GEMM-ready 128 x 4 tiles")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

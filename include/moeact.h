@@ -275,6 +275,54 @@ moeact_status scaled_swiglu_mxfp8_bwd_noalloc(const void* dy, int64_t lddy, cons
                                               int dirs, void* dx, float* dscale,
                                               moeact_mx_out out, void* stream);
 
+/* ---------------------------------------------------------------------
+ * ClampedSwiGLU [TE: the third per-row-scaled activation of the fused
+ * grouped linear, Greptile summary; the pages name it without a definition,
+ * so this is a reading: the clamped SwiGLU of the public gpt-oss models,
+ * with the slope alpha and the limit L as arguments]:
+ *   gc = min(g, L), uc = clamp(u, -L, L)   (NaN passes through)
+ *   z = RN(alpha * gc); sig = correctly rounded fp32 sigma(z)
+ *   y = RN(RN(RN(gc * sig) * RN(uc + 1)) * s_row)
+ * Backward, the SwiGLU form with slope alpha; a clamped input gets a zero
+ * gradient (+0):
+ *   p = RN(dY * s); dsilu = fma(RN(alpha * RN(gc * sig)), RN(1 - sig), sig)
+ *   dgate = g > L ? 0 : bf16(RN(RN(p * RN(uc + 1)) * dsilu))
+ *   dup = |u| > L ? 0 : bf16(RN(p * RN(gc * sig)))
+ *   dscale_row = sum_j dY * h (h = RN(RN(gc * sig) * RN(uc + 1))).
+ * Layout, outputs, workspace and errors as for SwiGLU (x = [gate | up],
+ * W = 2N in the backward; no staged rounding).  alpha must lie in
+ * [0.8125, 2] and limit be > 0 (+Inf allowed), else MOEACT_EINVAL.  The
+ * first call with a given alpha on a device builds that alpha's sigmoid table
+ * (device memory, kept until exit; synchronises the device once; at most 8
+ * distinct alphas per device, else MOEACT_ERANGE); it must not be inside a
+ * stream capture (MOEACT_EUNSUPPORTED) -- call moeact_init_clamped(alpha)
+ * first.  With alpha = 1 and limit = +Inf it is SwiGLU with up + 1 for up.
+ * ------------------------------------------------------------------- */
+moeact_status moeact_init_clamped(float alpha);
+moeact_status scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                              int64_t M, int64_t N, int dirs, float alpha,
+                                              float limit, moeact_mx_out out, void* stream);
+moeact_status grouped_scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                                      int64_t M, int64_t N, int dirs,
+                                                      float alpha, float limit,
+                                                      const int64_t* row_offs,
+                                                      const int64_t* colblk_offs,
+                                                      int32_t num_groups, int32_t* status,
+                                                      moeact_mx_out out, void* stream);
+moeact_status scaled_clamped_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
+                                              int64_t ldx, const float* s, int64_t M, int64_t N,
+                                              int dirs, float alpha, float limit, void* dx,
+                                              float* dscale, moeact_mx_out out, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+moeact_status grouped_scaled_clamped_swiglu_mxfp8_bwd(
+    const void* dy, int64_t lddy, const void* x, int64_t ldx, const float* s, int64_t M,
+    int64_t N, int dirs, float alpha, float limit, const int64_t* row_offs,
+    const int64_t* colblk_offs, int32_t num_groups, int32_t* status, void* dx, float* dscale,
+    moeact_mx_out out, void* workspace, size_t workspace_bytes, void* stream);
+/* Test hook: the table of sigma(RN(alpha * g)) over all 65536 bf16 g, fp32
+ * [65536] (as moeact_sigmoid_dump). */
+moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream);
+
 /* Reads and clears this device's error word: non-zero if a kernel gave up
  * waiting for its own input copies (bit 0 forward, bit 1 backward) -- a
  * defensive bound that ends the kernel instead of letting it hang; never

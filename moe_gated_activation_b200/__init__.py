@@ -11,11 +11,17 @@ from .ops import (  # noqa: F401
     ROWWISE,
     Backward,
     bwd_workspace_bytes,
+    grouped_scaled_clamped_swiglu_mxfp8_bwd,
+    grouped_scaled_clamped_swiglu_mxfp8_fwd,
     grouped_scaled_srelu_mxfp8_bwd,
     grouped_scaled_srelu_mxfp8_fwd,
     grouped_scaled_swiglu_mxfp8_bwd,
     grouped_scaled_swiglu_mxfp8_fwd,
+    clamped_sigmoid_table,
     init,
+    init_clamped,
+    scaled_clamped_swiglu_mxfp8_bwd,
+    scaled_clamped_swiglu_mxfp8_fwd,
     scaled_srelu_mxfp8_bwd,
     scaled_srelu_mxfp8_fwd,
     scaled_swiglu_mxfp8_bwd,

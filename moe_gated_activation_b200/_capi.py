@@ -41,6 +41,7 @@ I64 = ctypes.c_int64
 I32 = ctypes.c_int32
 I = ctypes.c_int
 SZ = ctypes.c_size_t
+F = ctypes.c_float
 
 _SIGS = {
     "moeact_init": ([], I),
@@ -59,6 +60,15 @@ _SIGS = {
     "grouped_scaled_srelu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, P, P, I32, P, P, P,
                                         MxOut, P, SZ, P], I),
     "moeact_sigmoid_dump": ([P, P], I),
+    "moeact_init_clamped": ([F], I),
+    "scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, MxOut, P], I),
+    "grouped_scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, P, P, I32, P,
+                                                 MxOut, P], I),
+    "scaled_clamped_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, F, F, P, P, MxOut, P,
+                                         SZ, P], I),
+    "grouped_scaled_clamped_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, F, F, P, P, I32,
+                                                 P, P, P, MxOut, P, SZ, P], I),
+    "moeact_clamped_sigmoid_dump": ([F, P, P], I),
     "moeact_device_error": ([P], I),
     "scaled_swiglu_mxfp8_bwd_noalloc": ([P, I64, P, I64, P, I64, I64, I, P, P, MxOut, P], I),
 }

@@ -2,6 +2,7 @@
 // per-device set-up and kernel dispatch.  Argument checks happen on the host
 // before anything is launched; nothing here allocates device memory.
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -13,7 +14,8 @@
 #include <cuda_runtime.h>
 
 #include "../../include/moeact.h"
-#include "kernels.cuh"
+#include "host_kernels.cuh"
+#include "variants.cuh"
 
 namespace moeact {
 namespace {
@@ -39,64 +41,18 @@ int g_sms[kMaxDevices];
 std::mutex g_mu;
 __device__ int g_sigma_uncertain;
 
-using FwdFn = void (*)(const CUtensorMap, const Params);
-using BwdFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
-// smem_fixed: shared memory without group offsets; sig: the kernel carries the
-// sigmoid table, whose gap holds the group offsets (so they add nothing)
-struct FwdVariant { FwdFn fn; int threads; int smem_fixed; bool sig; };
-struct BwdVariant { BwdFn fn; int threads; int smem_fixed; bool sig; };
-
-template <int ACT, int DIRS, bool STAGED, bool GROUPED>
-FwdVariant fwd_variant() {
-  return {act_fwd_kernel<ACT, DIRS, STAGED, GROUPED>, Cfg<ACT, false>::kThreads,
-          smem_bytes<ACT, false>(false, 0), Cfg<ACT, false>::kSig};
-}
-template <int ACT, int DIRS, bool GROUPED, bool REREAD>
-BwdVariant bwd_variant() {
-  return {act_bwd_kernel<ACT, DIRS, GROUPED, REREAD>, Cfg<ACT, true>::kThreads,
-          smem_bytes<ACT, true>(false, 0), Cfg<ACT, true>::kSig};
-}
-
-template <int ACT, bool GROUPED, int LAYOUT>
-void fwd_all_layout(FwdVariant* out, int& n) {
-  out[n++] = fwd_variant<ACT, kRow | LAYOUT, false, GROUPED>();
-  out[n++] = fwd_variant<ACT, kCol | LAYOUT, false, GROUPED>();
-  out[n++] = fwd_variant<ACT, kRow | kCol | LAYOUT, false, GROUPED>();
-  if (ACT == kSwiGLU) {
-    out[n++] = fwd_variant<ACT, kRow | LAYOUT, true, GROUPED>();
-    out[n++] = fwd_variant<ACT, kCol | LAYOUT, true, GROUPED>();
-    out[n++] = fwd_variant<ACT, kRow | kCol | LAYOUT, true, GROUPED>();
-  }
-}
-
-template <int ACT, bool GROUPED>
-void fwd_all(FwdVariant* out, int& n) {
-  fwd_all_layout<ACT, GROUPED, 0>(out, n);
-  fwd_all_layout<ACT, GROUPED, kGemm>(out, n);
-}
-
-template <int ACT, bool GROUPED, bool REREAD>
-void bwd_all_rr(BwdVariant* out, int& n) {
-  out[n++] = bwd_variant<ACT, 0, GROUPED, REREAD>();
-  out[n++] = bwd_variant<ACT, kRow, GROUPED, REREAD>();
-  out[n++] = bwd_variant<ACT, kCol, GROUPED, REREAD>();
-  out[n++] = bwd_variant<ACT, kRow | kCol, GROUPED, REREAD>();
-  out[n++] = bwd_variant<ACT, kRow | kGemm, GROUPED, REREAD>();
-  out[n++] = bwd_variant<ACT, kCol | kGemm, GROUPED, REREAD>();
-  out[n++] = bwd_variant<ACT, kRow | kCol | kGemm, GROUPED, REREAD>();
-}
-
-template <int ACT, bool GROUPED>
-void bwd_all(BwdVariant* out, int& n) {
-  bwd_all_rr<ACT, GROUPED, false>(out, n);
-  bwd_all_rr<ACT, GROUPED, true>(out, n);
-}
+// The fused kernels of each activation (index kSwiGLU / kSReLU / kClamped),
+// filled once.
+FwdVariant g_fwd[3][kVariantSlots];
+BwdVariant g_bwd[3][kVariantSlots];
+bool g_tables_filled = false;
 
 // Extra shared memory of a grouped call (its col-block offsets), at most.
 constexpr int kGroupSmem = group_bytes(MOEACT_MAX_GROUPS);
 
 __device__ uint32_t g_err_word;
 uint32_t* g_err_ptr[kMaxDevices];
+float* g_sig_ptr[kMaxDevices];   // g_sigma_table on each device
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 moeact_status init_device(int dev) {
@@ -118,31 +74,41 @@ moeact_status init_device(int dev) {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
 
-  FwdVariant fv[48];
-  BwdVariant bv[64];
-  int nf = 0, nb = 0;
-  fwd_all<kSwiGLU, false>(fv, nf);
-  fwd_all<kSwiGLU, true>(fv, nf);
-  fwd_all<kSReLU, false>(fv, nf);
-  fwd_all<kSReLU, true>(fv, nf);
-  bwd_all<kSwiGLU, false>(bv, nb);
-  bwd_all<kSwiGLU, true>(bv, nb);
-  bwd_all<kSReLU, false>(bv, nb);
-  bwd_all<kSReLU, true>(bv, nb);
-  for (int i = 0; i < nf; ++i) {
-    e = cudaFuncSetAttribute(fv[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fv[i].smem_fixed + (fv[i].sig ? 0 : kGroupSmem));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  if (!g_tables_filled) {
+    fill_fwd_swiglu_dense(g_fwd[kSwiGLU]);
+    fill_fwd_swiglu_grouped(g_fwd[kSwiGLU]);
+    fill_bwd_swiglu_dense(g_bwd[kSwiGLU]);
+    fill_bwd_swiglu_grouped(g_bwd[kSwiGLU]);
+    fill_fwd_srelu_dense(g_fwd[kSReLU]);
+    fill_fwd_srelu_grouped(g_fwd[kSReLU]);
+    fill_bwd_srelu_dense(g_bwd[kSReLU]);
+    fill_bwd_srelu_grouped(g_bwd[kSReLU]);
+    fill_fwd_clamped_dense(g_fwd[kClamped]);
+    fill_fwd_clamped_grouped(g_fwd[kClamped]);
+    fill_bwd_clamped_dense(g_bwd[kClamped]);
+    fill_bwd_clamped_grouped(g_bwd[kClamped]);
+    g_tables_filled = true;
   }
-  for (int i = 0; i < nb; ++i) {
-    e = cudaFuncSetAttribute(bv[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bv[i].smem_fixed + (bv[i].sig ? 0 : kGroupSmem));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-  }
+  for (auto& tab : g_fwd)
+    for (const FwdVariant& v : tab) {
+      if (!v.fn) continue;
+      e = cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               v.smem_fixed + (v.sig ? 0 : kGroupSmem));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+  for (auto& tab : g_bwd)
+    for (const BwdVariant& v : tab) {
+      if (!v.fn) continue;
+      e = cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               v.smem_fixed + (v.sig ? 0 : kGroupSmem));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    }
   e = cudaFuncSetAttribute(sigma_table_dump, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSigBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   e = cudaGetSymbolAddress(reinterpret_cast<void**>(&g_err_ptr[dev]), g_err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+  e = cudaGetSymbolAddress(reinterpret_cast<void**>(&g_sig_ptr[dev]), g_sigma_table);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
 
   cudaStream_t st;
@@ -156,7 +122,8 @@ moeact_status init_device(int dev) {
     int* d_unc = nullptr;
     e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d_unc), g_sigma_uncertain);
     if (e == cudaSuccess) {
-      sigma_table_init<<<(kSigEntriesPadded + 255) / 256, 256, 0, st>>>(d_unc);
+      sigma_table_init<<<(kSigEntriesPadded + 255) / 256, 256, 0, st>>>(g_sig_ptr[dev], 1.0f,
+                                                                          d_unc);
       e = cudaGetLastError();
     }
   }
@@ -221,7 +188,7 @@ moeact_status check_shape(const void* x, int64_t ldx, const float* s, int64_t M,
   if (N <= 0 || N % 32 != 0) return fail(MOEACT_EINVAL, "N must be a positive multiple of 32 (got %lld)", (long long)N);
   if (M > MOEACT_MAX_ROWS) return fail(MOEACT_ERANGE, "M above 2^30");
   if (N > (1 << 24)) return fail(MOEACT_ERANGE, "N above 2^24");
-  const int64_t width = act == kSwiGLU ? 2 * N : N;
+  const int64_t width = act != kSReLU ? 2 * N : N;
   if (ldx < width) return fail(MOEACT_EINVAL, "ldx (%lld) smaller than the input width %lld", (long long)ldx, (long long)width);
   if (ldx % 8 != 0) return fail(MOEACT_EALIGN, "ldx must be a multiple of 8 elements");
   if (ldx > (((int64_t)1) << 40) || M * ldx > (((int64_t)1) << 61)) return fail(MOEACT_ERANGE, "input extent too large");
@@ -245,50 +212,6 @@ size_t ws_bytes_needed(int64_t M, int64_t N) {
 }
 
 // ------------------------------------------------------------ launches
-template <int ACT, bool GROUPED>
-FwdVariant pick_fwd(int dirs, bool staged) {
-  // dirs carries kGemm for the GEMM-ready scale layout
-  if (ACT == kSwiGLU && staged) {
-    switch (dirs) {
-      case kRow: return fwd_variant<ACT, kRow, true, GROUPED>();
-      case kCol: return fwd_variant<ACT, kCol, true, GROUPED>();
-      case kRow | kCol: return fwd_variant<ACT, kRow | kCol, true, GROUPED>();
-      case kRow | kGemm: return fwd_variant<ACT, kRow | kGemm, true, GROUPED>();
-      case kCol | kGemm: return fwd_variant<ACT, kCol | kGemm, true, GROUPED>();
-      default: return fwd_variant<ACT, kRow | kCol | kGemm, true, GROUPED>();
-    }
-  }
-  switch (dirs) {
-    case kRow: return fwd_variant<ACT, kRow, false, GROUPED>();
-    case kCol: return fwd_variant<ACT, kCol, false, GROUPED>();
-    case kRow | kCol: return fwd_variant<ACT, kRow | kCol, false, GROUPED>();
-    case kRow | kGemm: return fwd_variant<ACT, kRow | kGemm, false, GROUPED>();
-    case kCol | kGemm: return fwd_variant<ACT, kCol | kGemm, false, GROUPED>();
-    default: return fwd_variant<ACT, kRow | kCol | kGemm, false, GROUPED>();
-  }
-}
-
-// With dX written, the colwise pass re-reads it instead of keeping the whole
-// tile in registers.
-template <int ACT, bool GROUPED, bool REREAD>
-BwdVariant pick_bwd_rr(int dirs) {
-  // dirs carries kGemm for the GEMM-ready scale layout (never with dirs 0)
-  switch (dirs) {
-    case 0: return bwd_variant<ACT, 0, GROUPED, REREAD>();
-    case kRow: return bwd_variant<ACT, kRow, GROUPED, REREAD>();
-    case kCol: return bwd_variant<ACT, kCol, GROUPED, REREAD>();
-    case kRow | kCol: return bwd_variant<ACT, kRow | kCol, GROUPED, REREAD>();
-    case kRow | kGemm: return bwd_variant<ACT, kRow | kGemm, GROUPED, REREAD>();
-    case kCol | kGemm: return bwd_variant<ACT, kCol | kGemm, GROUPED, REREAD>();
-    default: return bwd_variant<ACT, kRow | kCol | kGemm, GROUPED, REREAD>();
-  }
-}
-
-template <int ACT, bool GROUPED>
-BwdVariant pick_bwd(int dirs, bool reread) {
-  return reread ? pick_bwd_rr<ACT, GROUPED, true>(dirs) : pick_bwd_rr<ACT, GROUPED, false>(dirs);
-}
-
 // Tensor map of a bf16 [rows, width] matrix with a row stride of `ld`
 // elements, read in boxes of 128 columns x 16 rows; out-of-range elements read
 // as zero.  Encoded on the host for every call (no allocation).
@@ -327,7 +250,7 @@ moeact_status make_map_gated(CUtensorMap* map, const void* base, int64_t N, int6
 
 moeact_status make_x_map(CUtensorMap* map, int act, const void* x, int64_t N, int64_t rows,
                          int64_t ld) {
-  return act == kSwiGLU ? make_map_gated(map, x, N, rows, ld) : make_map(map, x, N, rows, ld);
+  return act != kSReLU ? make_map_gated(map, x, N, rows, ld) : make_map(map, x, N, rows, ld);
 }
 
 int64_t grid_for(int64_t slabs_upper, int n_tiles, int threads, int dev) {
@@ -339,16 +262,130 @@ int64_t grid_for(int64_t slabs_upper, int n_tiles, int threads, int dev) {
 
 int group_smem(bool sig, bool grouped, int E) { return (grouped && !sig) ? group_bytes(E) : 0; }
 
-moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, int64_t M,
-                         int64_t N, int dirs, int staged, const int64_t* ro, const int64_t* cb,
+// ------------------------------------------------------------ ClampedSwiGLU
+// The slope alpha of ClampedSwiGLU is folded into its sigmoid table (one table
+// per alpha and device, built at the first call with that alpha, which
+// synchronises the device once), so alpha must keep the table's bf16 range
+// sufficient: for |g| < 2^-25, sigma(RN(alpha g)) rounds to 1/2 when alpha <=
+// 2, and for |g| >= 128 it is 0 or 1 when alpha >= 13/16.
+constexpr float kClampAlphaMin = 0.8125f, kClampAlphaMax = 2.0f;
+constexpr int kMaxAlphaTables = 8;
+struct AlphaTable {
+  uint32_t alpha_bits;
+  float* tab;
+};
+AlphaTable g_alpha_tab[kMaxDevices][kMaxAlphaTables];
+int g_n_alpha[kMaxDevices];
+
+moeact_status check_clamp_args(float alpha, float limit) {
+  if (!(alpha >= kClampAlphaMin && alpha <= kClampAlphaMax))
+    return fail(MOEACT_EINVAL, "alpha must lie in [0.8125, 2] (got %g)", (double)alpha);
+  if (!(limit > 0.0f)) return fail(MOEACT_EINVAL, "limit must be > 0 (got %g)", (double)limit);
+  return MOEACT_OK;
+}
+
+// The device table of sigma(RN(alpha * g)) for `alpha`, built on first use.
+moeact_status alpha_table(int dev, float alpha, cudaStream_t call_stream, const float** out) {
+  uint32_t bits;
+  std::memcpy(&bits, &alpha, 4);
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int i = 0; i < g_n_alpha[dev]; ++i)
+    if (g_alpha_tab[dev][i].alpha_bits == bits) {
+      *out = g_alpha_tab[dev][i].tab;
+      return MOEACT_OK;
+    }
+  if (g_n_alpha[dev] == kMaxAlphaTables)
+    return fail(MOEACT_ERANGE, "more than %d distinct alpha values on one device", kMaxAlphaTables);
+  cudaStreamCaptureStatus capt = cudaStreamCaptureStatusNone;
+  if (call_stream && cudaStreamIsCapturing(call_stream, &capt) == cudaSuccess &&
+      capt != cudaStreamCaptureStatusNone)
+    return fail(MOEACT_EUNSUPPORTED,
+                "first use of alpha %g inside a stream capture; call moeact_init_clamped() first",
+                (double)alpha);
+  float* tab = nullptr;
+  int* d_unc = nullptr;
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&tab), kSigBytes);
+  if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&d_unc), sizeof(int));
+  cudaStream_t st = nullptr;
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  int unc = -1;
+  if (e == cudaSuccess) e = cudaMemsetAsync(tab, 0, kSigBytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_unc, 0, sizeof(int), st);
+  if (e == cudaSuccess) {
+    sigma_table_init<<<(kSigEntriesPadded + 255) / 256, 256, 0, st>>>(tab, alpha, d_unc);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&unc, d_unc, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (st) cudaStreamDestroy(st);
+  if (d_unc) cudaFree(d_unc);
+  if (e != cudaSuccess || unc != 0) {
+    if (tab) cudaFree(tab);
+    if (e != cudaSuccess) return cuda_fail(e, "ClampedSwiGLU sigmoid table set-up");
+    return fail(MOEACT_ECUDA, "sigmoid table for alpha %g: %d entries could not be certified",
+                (double)alpha, unc);
+  }
+  g_alpha_tab[dev][g_n_alpha[dev]++] = {bits, tab};
+  *out = tab;
+  return MOEACT_OK;
+}
+
+// sigma(z) correctly rounded to fp32, for the sigmoid of a clamped gate: an
+// x87 extended evaluation (64-bit significand, error a few units of 2^-64)
+// rounded once, refused when it lies within 2^-56 (relative) of an fp32
+// rounding boundary (not expected to happen).
+bool sigmoid_f32_host(float z, float* out) {
+  if (std::isinf(z)) {
+    *out = z > 0 ? 1.0f : 0.0f;
+    return true;
+  }
+  const long double sl = 1.0L / (1.0L + expl(-(long double)z));
+  const float f = (float)sl;
+  const long double up = 0.5L * ((long double)f + (long double)nextafterf(f, INFINITY));
+  const long double dn = 0.5L * ((long double)f + (long double)nextafterf(f, -INFINITY));
+  const long double tol = fabsl(sl) * 0x1p-56L;
+  *out = f;
+  return fabsl(sl - up) > tol && fabsl(sl - dn) > tol;
+}
+
+// What a fused call computes: the activation and its parameters.
+struct ActArgs {
+  int act;
+  int staged;        // SwiGLU only
+  float alpha;       // ClampedSwiGLU only
+  float limit;       // ClampedSwiGLU only
+};
+
+ActArgs plain(int act, int staged = 0) { return {act, staged, 1.0f, INFINITY}; }
+
+// Fills the activation-dependent parameters (the sigmoid table to stage and
+// the clamp constants).
+moeact_status act_params(const ActArgs& a, int dev, cudaStream_t cs, Params& p) {
+  p.sig_src = g_sig_ptr[dev];
+  p.clamp_L = a.limit;
+  p.clamp_alpha = a.alpha;
+  p.clamp_sigL = 1.0f;
+  if (a.act != kClamped) return MOEACT_OK;
+  moeact_status st = alpha_table(dev, a.alpha, cs, &p.sig_src);
+  if (st) return st;
+  const float z = a.alpha * a.limit;   // RN(alpha * L), fp32
+  if (!sigmoid_f32_host(z, &p.clamp_sigL))
+    return fail(MOEACT_EUNSUPPORTED, "sigma(alpha * limit) could not be certified");
+  return MOEACT_OK;
+}
+
+moeact_status fwd_common(const ActArgs& a, const void* x, int64_t ldx, const float* s,
+                         int64_t M, int64_t N, int dirs, const int64_t* ro, const int64_t* cb,
                          int32_t E, int32_t* status, moeact_mx_out out, void* stream,
                          bool grouped) {
   t_err[0] = 0;
+  const int act = a.act, staged = a.staged;
   moeact_status st = check_shape(x, ldx, s, M, N, act);
   if (st) return st;
   if ((st = check_mx(out, dirs, false))) return st;
   if ((st = check_layout(out, M, N))) return st;
   if (staged != 0 && staged != 1) return fail(MOEACT_EINVAL, "staged_rounding must be 0 or 1");
+  if (act == kClamped && (st = check_clamp_args(a.alpha, a.limit))) return st;
   if (grouped && (st = check_groups(ro, cb, E, status))) return st;
   if (M == 0) return MOEACT_OK;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -373,15 +410,13 @@ moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, in
   p.n_tiles = (int)ceil_div(N, kTileCols);
   p.gemm_scales = out.scale_layout == MOEACT_SCALES_GEMM;
   p.err = g_err_ptr[dev];
+  if ((st = act_params(a, dev, cs, p))) return st;
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
-  FwdVariant v;
   const int kdirs = dirs | (p.gemm_scales ? kGemm : 0);
-  if (act == kSwiGLU)
-    v = grouped ? pick_fwd<kSwiGLU, true>(kdirs, staged) : pick_fwd<kSwiGLU, false>(kdirs, staged);
-  else
-    v = grouped ? pick_fwd<kSReLU, true>(kdirs, false) : pick_fwd<kSReLU, false>(kdirs, false);
+  const FwdVariant& v = g_fwd[act][fwd_slot(grouped, act == kSwiGLU && staged, kdirs)];
+  if (!v.fn) return fail(MOEACT_EUNSUPPORTED, "no forward kernel for this combination");
   CUtensorMap tx;
-  if ((st = make_map(&tx, x, act == kSwiGLU ? 2 * N : N, M, ldx))) return st;
+  if ((st = make_map(&tx, x, act != kSReLU ? 2 * N : N, M, ldx))) return st;
   const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
   v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(v.sig, grouped, p.E), cs>>>(tx, p);
   const cudaError_t e = cudaGetLastError();
@@ -389,12 +424,13 @@ moeact_status fwd_common(int act, const void* x, int64_t ldx, const float* s, in
   return MOEACT_OK;
 }
 
-moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, int64_t ldx,
-                         const float* s, int64_t M, int64_t N, int dirs, const int64_t* ro,
-                         const int64_t* cb, int32_t E, int32_t* status, void* dx,
-                         float* dscale, moeact_mx_out out, void* ws, size_t ws_bytes,
+moeact_status bwd_common(const ActArgs& a, const void* dy, int64_t lddy, const void* x,
+                         int64_t ldx, const float* s, int64_t M, int64_t N, int dirs,
+                         const int64_t* ro, const int64_t* cb, int32_t E, int32_t* status,
+                         void* dx, float* dscale, moeact_mx_out out, void* ws, size_t ws_bytes,
                          void* stream, bool grouped) {
   t_err[0] = 0;
+  const int act = a.act;
   moeact_status st = check_shape(x, ldx, s, M, N, act);
   if (st) return st;
   if ((st = check_mx(out, dirs, true))) return st;
@@ -407,6 +443,7 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   if (dx && !aligned(dx, 16)) return fail(MOEACT_EALIGN, "dx must be 16-byte aligned");
   if (dscale && !aligned(dscale, 4)) return fail(MOEACT_EALIGN, "dscale must be 4-byte aligned");
   if (dirs == 0 && !dx && !dscale) return fail(MOEACT_EINVAL, "nothing requested: dirs == 0 and no dx / dscale");
+  if (act == kClamped && (st = check_clamp_args(a.alpha, a.limit))) return st;
   if (grouped && (st = check_groups(ro, cb, E, status))) return st;
   const size_t ws_need = ws_bytes_needed(M, N);
   if (dscale) {
@@ -426,7 +463,7 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   p.s = s;
   p.M = M;
   p.N = (int)N;
-  p.W = (int)(act == kSwiGLU ? 2 * N : N);
+  p.W = (int)(act != kSReLU ? 2 * N : N);
   p.rq = out.row_codes;
   p.rs = out.row_scales;
   p.cq = out.col_codes;
@@ -442,14 +479,14 @@ moeact_status bwd_common(int act, const void* dy, int64_t lddy, const void* x, i
   p.n_tiles = (int)ceil_div(N, kTileCols);
   p.gemm_scales = out.scale_layout == MOEACT_SCALES_GEMM;
   p.err = g_err_ptr[dev];
+  if ((st = act_params(a, dev, cs, p))) return st;
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
-  BwdVariant v;
+  // with dX written, the colwise pass re-reads it instead of keeping the
+  // whole tile in registers
   const bool rr = dx != nullptr;
   const int kdirs = dirs | ((p.gemm_scales && dirs) ? kGemm : 0);
-  if (act == kSwiGLU)
-    v = grouped ? pick_bwd<kSwiGLU, true>(kdirs, rr) : pick_bwd<kSwiGLU, false>(kdirs, rr);
-  else
-    v = grouped ? pick_bwd<kSReLU, true>(kdirs, rr) : pick_bwd<kSReLU, false>(kdirs, rr);
+  const BwdVariant& v = g_bwd[act][bwd_slot(grouped, rr, kdirs)];
+  if (!v.fn) return fail(MOEACT_EUNSUPPORTED, "no backward kernel for this combination");
   CUtensorMap tx, tdy;
   if ((st = make_x_map(&tx, act, x, N, M, ldx))) return st;
   if ((st = make_map(&tdy, dy, N, M, lddy))) return st;
@@ -526,14 +563,14 @@ moeact_status splits_to_offsets(const int64_t* m_splits, int32_t num_groups, int
 moeact_status scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s, int64_t M,
                                       int64_t N, int dirs, int staged_rounding,
                                       moeact_mx_out out, void* stream) {
-  return fwd_common(kSwiGLU, x, ldx, s, M, N, dirs, staged_rounding, nullptr, nullptr, 0,
+  return fwd_common(plain(kSwiGLU, staged_rounding), x, ldx, s, M, N, dirs, nullptr, nullptr, 0,
                     nullptr, out, stream, false);
 }
 
 moeact_status scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s, int64_t M,
                                      int64_t N, int dirs, moeact_mx_out out, void* stream) {
-  return fwd_common(kSReLU, x, ldx, s, M, N, dirs, 0, nullptr, nullptr, 0, nullptr, out, stream,
-                    false);
+  return fwd_common(plain(kSReLU), x, ldx, s, M, N, dirs, nullptr, nullptr, 0, nullptr, out,
+                    stream, false);
 }
 
 moeact_status grouped_scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
@@ -542,8 +579,8 @@ moeact_status grouped_scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const 
                                               const int64_t* colblk_offs, int32_t num_groups,
                                               int32_t* status, moeact_mx_out out,
                                               void* stream) {
-  return fwd_common(kSwiGLU, x, ldx, s, M, N, dirs, staged_rounding, row_offs, colblk_offs,
-                    num_groups, status, out, stream, true);
+  return fwd_common(plain(kSwiGLU, staged_rounding), x, ldx, s, M, N, dirs, row_offs,
+                    colblk_offs, num_groups, status, out, stream, true);
 }
 
 moeact_status grouped_scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
@@ -551,8 +588,8 @@ moeact_status grouped_scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const f
                                              const int64_t* row_offs,
                                              const int64_t* colblk_offs, int32_t num_groups,
                                              int32_t* status, moeact_mx_out out, void* stream) {
-  return fwd_common(kSReLU, x, ldx, s, M, N, dirs, 0, row_offs, colblk_offs, num_groups, status,
-                    out, stream, true);
+  return fwd_common(plain(kSReLU), x, ldx, s, M, N, dirs, row_offs, colblk_offs, num_groups,
+                    status, out, stream, true);
 }
 
 size_t scaled_act_mxfp8_bwd_workspace_size(int64_t M, int64_t N, int32_t num_groups) {
@@ -565,7 +602,7 @@ moeact_status scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* 
                                       const float* s, int64_t M, int64_t N, int dirs, void* dx,
                                       float* dscale, moeact_mx_out out, void* workspace,
                                       size_t workspace_bytes, void* stream) {
-  return bwd_common(kSwiGLU, dy, lddy, x, ldx, s, M, N, dirs, nullptr, nullptr, 0, nullptr, dx,
+  return bwd_common(plain(kSwiGLU), dy, lddy, x, ldx, s, M, N, dirs, nullptr, nullptr, 0, nullptr, dx,
                     dscale, out, workspace, workspace_bytes, stream, false);
 }
 
@@ -573,7 +610,7 @@ moeact_status scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x
                                      const float* s, int64_t M, int64_t N, int dirs, void* dx,
                                      float* dscale, moeact_mx_out out, void* workspace,
                                      size_t workspace_bytes, void* stream) {
-  return bwd_common(kSReLU, dy, lddy, x, ldx, s, M, N, dirs, nullptr, nullptr, 0, nullptr, dx,
+  return bwd_common(plain(kSReLU), dy, lddy, x, ldx, s, M, N, dirs, nullptr, nullptr, 0, nullptr, dx,
                     dscale, out, workspace, workspace_bytes, stream, false);
 }
 
@@ -584,7 +621,7 @@ moeact_status grouped_scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, cons
                                               int32_t* status, void* dx, float* dscale,
                                               moeact_mx_out out, void* workspace,
                                               size_t workspace_bytes, void* stream) {
-  return bwd_common(kSwiGLU, dy, lddy, x, ldx, s, M, N, dirs, row_offs, colblk_offs, num_groups,
+  return bwd_common(plain(kSwiGLU), dy, lddy, x, ldx, s, M, N, dirs, row_offs, colblk_offs, num_groups,
                     status, dx, dscale, out, workspace, workspace_bytes, stream, true);
 }
 
@@ -595,8 +632,74 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
                                              int32_t* status, void* dx, float* dscale,
                                              moeact_mx_out out, void* workspace,
                                              size_t workspace_bytes, void* stream) {
-  return bwd_common(kSReLU, dy, lddy, x, ldx, s, M, N, dirs, row_offs, colblk_offs, num_groups,
+  return bwd_common(plain(kSReLU), dy, lddy, x, ldx, s, M, N, dirs, row_offs, colblk_offs, num_groups,
                     status, dx, dscale, out, workspace, workspace_bytes, stream, true);
+}
+
+// ---------------------------------------------------------------- ClampedSwiGLU
+moeact_status moeact_init_clamped(float alpha) {
+  t_err[0] = 0;
+  moeact_status st = check_clamp_args(alpha, 1.0f);
+  if (st) return st;
+  int dev;
+  if ((st = ensure_ready(nullptr, &dev))) return st;
+  const float* tab;
+  return alpha_table(dev, alpha, nullptr, &tab);
+}
+
+moeact_status scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                              int64_t M, int64_t N, int dirs, float alpha,
+                                              float limit, moeact_mx_out out, void* stream) {
+  return fwd_common({kClamped, 0, alpha, limit}, x, ldx, s, M, N, dirs, nullptr, nullptr, 0,
+                    nullptr, out, stream, false);
+}
+
+moeact_status grouped_scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
+                                                      int64_t M, int64_t N, int dirs,
+                                                      float alpha, float limit,
+                                                      const int64_t* row_offs,
+                                                      const int64_t* colblk_offs,
+                                                      int32_t num_groups, int32_t* status,
+                                                      moeact_mx_out out, void* stream) {
+  return fwd_common({kClamped, 0, alpha, limit}, x, ldx, s, M, N, dirs, row_offs, colblk_offs,
+                    num_groups, status, out, stream, true);
+}
+
+moeact_status scaled_clamped_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
+                                              int64_t ldx, const float* s, int64_t M, int64_t N,
+                                              int dirs, float alpha, float limit, void* dx,
+                                              float* dscale, moeact_mx_out out, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  return bwd_common({kClamped, 0, alpha, limit}, dy, lddy, x, ldx, s, M, N, dirs, nullptr,
+                    nullptr, 0, nullptr, dx, dscale, out, workspace, workspace_bytes, stream,
+                    false);
+}
+
+moeact_status grouped_scaled_clamped_swiglu_mxfp8_bwd(
+    const void* dy, int64_t lddy, const void* x, int64_t ldx, const float* s, int64_t M,
+    int64_t N, int dirs, float alpha, float limit, const int64_t* row_offs,
+    const int64_t* colblk_offs, int32_t num_groups, int32_t* status, void* dx, float* dscale,
+    moeact_mx_out out, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common({kClamped, 0, alpha, limit}, dy, lddy, x, ldx, s, M, N, dirs, row_offs,
+                    colblk_offs, num_groups, status, dx, dscale, out, workspace, workspace_bytes,
+                    stream, true);
+}
+
+moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream) {
+  t_err[0] = 0;
+  if (!out) return fail(MOEACT_EINVAL, "out is required");
+  if (!aligned(out, 4)) return fail(MOEACT_EALIGN, "out must be 4-byte aligned");
+  moeact_status st = check_clamp_args(alpha, 1.0f);
+  if (st) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int dev;
+  if ((st = ensure_ready(cs, &dev))) return st;
+  const float* tab;
+  if ((st = alpha_table(dev, alpha, cs, &tab))) return st;
+  sigma_table_dump<<<128, 256, kSigBytes, cs>>>(tab, out);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sigmoid dump launch");
+  return MOEACT_OK;
 }
 
 moeact_status moeact_device_error(uint32_t* flags) {
@@ -624,7 +727,7 @@ moeact_status moeact_sigmoid_dump(float* out, void* stream) {
   int dev;
   moeact_status st = ensure_ready(cs, &dev);
   if (st) return st;
-  sigma_table_dump<<<128, 256, kSigBytes, cs>>>(out);
+  sigma_table_dump<<<128, 256, kSigBytes, cs>>>(g_sig_ptr[dev], out);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sigmoid dump launch");
   return MOEACT_OK;

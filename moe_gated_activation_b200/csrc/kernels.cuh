@@ -1,7 +1,6 @@
 // Kernels of libmoeact (sm_100a).
 //
-// * sigma_table_init  -- builds the correctly rounded fp32 sigmoid table once
-//                        per device (binary64 evaluation + rounding check).
+// (The sigmoid tables and their set-up kernel are in sigma.cuh.)
 // * splits_kernel     -- m_splits -> row / col-block offsets and a status
 //                        (TransformerEngine PR #3238, Greptile summary:
 //                        splits_to_offsets_multi computes all offsets once).
@@ -14,24 +13,22 @@
 //                        grad_scales; pytorch/ao PR #4743, API).
 //
 // Work decomposition (both fused kernels).  A work item is one warp-tile:
-// 32 rows (one colwise block, never crossing an expert boundary) x 64
-// columns; lane l owns columns 2l and 2l+1 for all 32 rows, so the colwise
-// amax is a per-lane loop over registers and the rowwise 1x32 amax is a
-// 16-lane reduction.  The grid is persistent (one CTA per SM, the sigmoid
-// table staged once per CTA in shared memory); warps walk the items
-// slab-major so that neighbouring warps read neighbouring columns of the same
-// rows.
+// 32 rows (one colwise block, never crossing an expert boundary) x 128
+// columns; lane l owns columns 4l .. 4l+3 for all 32 rows, so the colwise
+// amax is a per-lane loop over registers and the rowwise 1x32 amax is an
+// 8-lane reduction.  The grid is persistent (one CTA per SM, the sigmoid
+// table staged once per CTA in shared memory).
 //
 // Data movement.  Each warp owns a ring of shared-memory slots, each holding
-// one 16-row half of a warp-tile's inputs ([16 x 64] bf16 per operand), filled
-// by TMA (cp.async.bulk.tensor, no multicast) and signalled through one
-// mbarrier per slot.  Lane 0 keeps two half-tiles in flight ahead of the one
-// being computed, so the warp never waits on global-memory latency and the
-// inputs never occupy registers; rows and columns outside the tensor arrive
-// as zeros.  Lanes read their two columns of each row from shared memory
-// (conflict-free: a warp reads one 128-byte row).  Codes, scales and
-// gradients are stored directly, 64 (codes) or 128 (bf16) contiguous bytes
-// per warp per row; full tiles take a path without bounds predicates.
+// one 16-row half of a warp-tile's inputs ([16 x 128] bf16 per operand),
+// filled by TMA (cp.async.bulk.tensor, no multicast) and signalled through
+// one mbarrier per slot; lane 0 refills a slot as soon as it is consumed, so
+// the loads of the next half-tiles overlap the math of the current one, and
+// rows and columns outside the tensor arrive as zeros.  Lanes read their four
+// columns of each row from shared memory (a warp reads one 256-byte row).
+// Codes, scales and gradients are stored directly, 128 (codes) or 256 (bf16)
+// contiguous bytes per warp per row; full tiles take a path without bounds
+// predicates.
 #pragma once
 
 #include <cstdint>
@@ -42,7 +39,7 @@
 
 namespace moeact {
 
-enum Act : int { kSwiGLU = 0, kSReLU = 1 };
+enum Act : int { kSwiGLU = 0, kSReLU = 1, kClamped = 2 };   // kClamped: ClampedSwiGLU
 constexpr int kRow = 1;
 constexpr int kCol = 2;
 // Kernel template flag carried in the DIRS bits: scales in the GEMM-ready
@@ -51,151 +48,8 @@ constexpr int kCol = 2;
 constexpr int kGemm = 4;
 constexpr int kTileCols = 128;   // columns of a warp-tile (4 per lane)
 
-// The table lives in device global memory of this module, one copy per
-// device, written by sigma_table_init before any activation kernel reads it,
-// already in the shared-memory layout (positive gates at [0, 4097), negative
-// at [8192, 12289)) so that a kernel stages it with one bulk copy.
-__device__ __align__(16) float g_sigma_table[kSigBytes / 4];
-
 __host__ __device__ constexpr int sig_slot(int i) {
   return i < (int)kSigPerSign ? i : i - (int)kSigPerSign + kSigNegOffset;
-}
-
-// Builds the table.  For |g| < 2^-9, sigma(g) = 1/2 + g/4 - g^3/48 + O(g^5):
-// hi = 1/2 + g/4 is exact in binary64 and the rest is far smaller than any
-// distance from hi to an fp32 rounding boundary except when hi sits exactly on
-// one (a midpoint), where binary64 cannot see the remainder; there the
-// remainder's sign (that of -g) decides.  Elsewhere the table comes from
-// binary64 exp and division (error < 2^-51 relative), and entries whose
-// binary64 value lies within 2^-48 (relative) of a rounding boundary are
-// counted as uncertain (none are expected: the closest true value stays
-// 2^-37 away).
-__global__ void sigma_table_init(int* uncertain) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= kSigEntries) return;
-  const uint32_t neg = i >= (int)kSigPerSign ? 1u : 0u;
-  const uint32_t mag = (uint32_t)i - neg * kSigPerSign + kSigLo;
-  const float g = __uint_as_float(((neg << 15) | mag) << 16);
-  if (fabsf(g) < 0x1p-9f) {
-    const double hi = 0.5 + 0.25 * (double)g;
-    const float d = __double2float_rd(hi), u = __double2float_ru(hi);
-    float f;
-    if (d == u) {
-      f = d;
-    } else if (hi == 0.5 * ((double)d + (double)u)) {
-      f = g > 0.0f ? d : u;
-    } else {
-      f = __double2float_rn(hi);
-    }
-    g_sigma_table[sig_slot(i)] = f;
-    return;
-  }
-  const double sd = 1.0 / (1.0 + exp(-(double)g));
-  const float f = __double2float_rn(sd);
-  const double up = 0.5 * ((double)f + (double)nextafterf(f, __int_as_float(0x7F800000)));
-  const double dn = 0.5 * ((double)f + (double)nextafterf(f, __int_as_float(0xFF800000)));
-  const double tol = fabs(sd) * 0x1p-48;
-  if (!(fabs(sd - up) > tol && fabs(sd - dn) > tol)) atomicAdd(uncertain, 1);
-  g_sigma_table[sig_slot(i)] = f;
-}
-
-// Expands the table to all 65536 bf16 patterns (test hook), through the same
-// shared-memory layout and pair lookup the fused kernels use: thread t looks
-// up the packed pair (2t, 2t + 1).
-__global__ void sigma_table_dump(float* out) {
-  extern __shared__ __align__(16) float tab[];
-  for (int i = threadIdx.x; i < kSigBytes / 4; i += blockDim.x) tab[i] = g_sigma_table[i];
-  __syncthreads();
-  const uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < 32768) {
-    float a, b;
-    sigma_pair(tab, (2 * t) | ((2 * t + 1) << 16), a, b);
-    out[2 * t] = a;
-    out[2 * t + 1] = b;
-  }
-}
-
-// ---------------------------------------------------------------- offsets
-// One CTA of 1024 threads; thread t owns a contiguous chunk of the groups.
-__global__ void __launch_bounds__(1024) splits_kernel(const int64_t* __restrict__ m, int E,
-                                                      int64_t M, int64_t* __restrict__ ro,
-                                                      int64_t* __restrict__ cb,
-                                                      int32_t* __restrict__ status) {
-  __shared__ long long s_r[32], s_c[32];
-  __shared__ int s_neg, s_big;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  if (t == 0) { s_neg = 0; s_big = 0; }
-  __syncthreads();
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = min(E, t * per), e1 = min(E, e0 + per);
-  long long r = 0, c = 0;
-  int neg = 0, big = 0;
-  for (int e = e0; e < e1; ++e) {
-    const long long v = m[e];
-    if (v < 0) neg = 1;
-    else if (v > M) big = 1;
-    else { r += v; c += (v + 31) / 32; }
-  }
-  if (neg) atomicOr(&s_neg, 1);
-  if (big) atomicOr(&s_big, 1);
-  // block-wide exclusive scan of (r, c)
-  long long ir = r, ic = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long yr = __shfl_up_sync(kFull, ir, o), yc = __shfl_up_sync(kFull, ic, o);
-    if (lane >= o) { ir += yr; ic += yc; }
-  }
-  if (lane == 31) { s_r[warp] = ir; s_c[warp] = ic; }
-  __syncthreads();
-  if (warp == 0) {
-    long long wr = lane < (int)(blockDim.x >> 5) ? s_r[lane] : 0;
-    long long wc = lane < (int)(blockDim.x >> 5) ? s_c[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long yr = __shfl_up_sync(kFull, wr, o), yc = __shfl_up_sync(kFull, wc, o);
-      if (lane >= o) { wr += yr; wc += yc; }
-    }
-    s_r[lane] = wr; s_c[lane] = wc;   // inclusive over warps
-  }
-  __syncthreads();
-  const long long total = s_r[(blockDim.x >> 5) - 1];
-  int st = 0;
-  if (s_neg) st = 1;
-  else if (s_big || total != M) st = 2;
-  if (t == 0) *status = st;
-  if (st) {
-    // no offsets for bad splits: mark them invalid, so that a grouped call
-    // given them reports MOEACT_DEV_BAD_OFFSETS and writes nothing (instead
-    // of running on offsets left by an earlier call)
-    if (t == 0) {
-      ro[0] = -1;
-      if (cb) cb[0] = -1;
-    }
-    return;
-  }
-  long long base_r = (warp ? s_r[warp - 1] : 0) + ir - r;
-  long long base_c = (warp ? s_c[warp - 1] : 0) + ic - c;
-  for (int e = e0; e < e1; ++e) {
-    ro[e] = base_r;
-    if (cb) cb[e] = base_c;
-    const long long v = m[e];
-    base_r += v;
-    base_c += (v + 31) / 32;
-  }
-  if (t == 0) { ro[E] = total; if (cb) cb[E] = s_c[(blockDim.x >> 5) - 1]; }
-}
-
-// ---------------------------------------------------------------- dscale sum
-// dscale[row] = sum over tiles t = 0, 1, ... of part[t][row], in that order.
-__global__ void __launch_bounds__(256) dscale_reduce_kernel(const float* __restrict__ part,
-                                                            int n_tiles, int64_t M,
-                                                            float* __restrict__ dscale) {
-  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= M) return;
-  float acc = 0.0f;
-#pragma unroll 8
-  for (int t = 0; t < n_tiles; ++t) acc = __fadd_rn(acc, __ldcg(part + (int64_t)t * M + row));
-  dscale[row] = acc;
 }
 
 // ---------------------------------------------------------------- fused kernels
@@ -222,6 +76,12 @@ struct Params {
   int64_t dense_slabs;
   int n_tiles;
   int gemm_scales;    // scales in the GEMM-ready tiled layout (see gemm_row_scales_off)
+  const float* sig_src;   // the sigmoid table to stage (device memory, shared-memory layout)
+  // ClampedSwiGLU: gate and up limit L, slope alpha (folded into sig_src),
+  // and sigma(RN(alpha * L)), the sigmoid of a clamped gate
+  float clamp_L;
+  float clamp_alpha;
+  float clamp_sigL;
   uint32_t* err;      // device error word (timeouts), never expected to be set
 };
 
@@ -233,7 +93,7 @@ constexpr int kRowBytes = kTileCols * 2;                   // 256 B of a bf16 ti
 // warp, chosen so that rings + sigmoid table fit the 227 KiB of shared memory.
 template <int ACT, bool BWD>
 struct Cfg {
-  static constexpr bool kSig = ACT == kSwiGLU;
+  static constexpr bool kSig = ACT != kSReLU;   // gated: sigmoid table, gate + up
   static constexpr int kOps = BWD ? (kSig ? 3 : 2) : (kSig ? 2 : 1);
   static constexpr int kWarps = BWD ? (kSig ? 7 : 8) : 8;
   static constexpr int kSlots = (!BWD && !kSig) ? 3 : 2;
@@ -303,8 +163,8 @@ __device__ __forceinline__ int64_t stage_and_validate(const Params& p, const Sme
     mbar_init(sig_bar, 1);
     mbar_init_fence();
     mbar_expect_tx(sig_bar, 2 * kSigHalfBytes);
-    bulk_load(m.sig, g_sigma_table, kSigHalfBytes, sig_bar);
-    bulk_load(m.sig + kSigNegOffset, g_sigma_table + kSigNegOffset, kSigHalfBytes, sig_bar);
+    bulk_load(m.sig, p.sig_src, kSigHalfBytes, sig_bar);
+    bulk_load(m.sig + kSigNegOffset, p.sig_src + kSigNegOffset, kSigHalfBytes, sig_bar);
   }
   int bad = 0;
   if (GROUPED) {
@@ -526,6 +386,66 @@ __device__ __forceinline__ uint32_t gather_row_scales(uint32_t w0, uint32_t w1, 
   return v;
 }
 
+// ------------------------------------------------------------- ClampedSwiGLU
+// NaN-propagating min / max (one instruction each).
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// A pair of gates (fp32, with their sigmoids from the table) clamped at L: a
+// gate above L becomes L and takes sigma(RN(alpha * L)); NaN passes through.
+__device__ __forceinline__ void clamp_gates(float2& g, float2& sg, const Params& p) {
+  sg.x = g.x > p.clamp_L ? p.clamp_sigL : sg.x;
+  sg.y = g.y > p.clamp_L ? p.clamp_sigL : sg.y;
+  g.x = min_nan(g.x, p.clamp_L);
+  g.y = min_nan(g.y, p.clamp_L);
+}
+
+// clamp(u, -L, L) + 1 for a pair of ups (NaN passes through).
+__device__ __forceinline__ float2 clamped_up_plus_one(float2 u, float L) {
+  return make_float2(__fadd_rn(max_nan(min_nan(u.x, L), -L), 1.0f),
+                     __fadd_rn(max_nan(min_nan(u.y, L), -L), 1.0f));
+}
+
+// Backward of ClampedSwiGLU for the four columns of a lane in one row (p =
+// dY * s): the SwiGLU form with slope alpha, dsilu = fma(RN(alpha * silu),
+// 1 - sig, sig); a clamped gate or up gets a zero gradient.
+__device__ __forceinline__ void clamped_bwd_math(const Params& p, const float* sig, uint2 G,
+                                                 uint2 U, float2 p01, float2 p23, float2& dg01,
+                                                 float2& dg23, float2& du01, float2& du23,
+                                                 float2& h01, float2& h23) {
+  const float L = p.clamp_L;
+  const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
+  float2 sg01, sg23;
+  sigma_pair(sig, G.x, sg01.x, sg01.y);
+  sigma_pair(sig, G.y, sg23.x, sg23.y);
+  float2 g01 = bf16x2_to_f2(G.x), g23 = bf16x2_to_f2(G.y);
+  const bool cg0 = g01.x > L, cg1 = g01.y > L, cg2 = g23.x > L, cg3 = g23.y > L;
+  clamp_gates(g01, sg01, p);
+  clamp_gates(g23, sg23, p);
+  const float2 si01 = mul2(g01, sg01), si23 = mul2(g23, sg23);
+  const float2 v01 = clamped_up_plus_one(u01, L), v23 = clamped_up_plus_one(u23, L);
+  const float2 one = make_float2(1.0f, 1.0f), a2 = make_float2(p.clamp_alpha, p.clamp_alpha);
+  const float2 ds01 = fma2(mul2(a2, si01), sub2(one, sg01), sg01);
+  const float2 ds23 = fma2(mul2(a2, si23), sub2(one, sg23), sg23);
+  const float2 dga = mul2(mul2(p01, v01), ds01), dgb = mul2(mul2(p23, v23), ds23);
+  const float2 dua = mul2(p01, si01), dub = mul2(p23, si23);
+  const auto cu = [L](float u) { return fabsf(u) > L; };
+  dg01 = make_float2(cg0 ? 0.0f : dga.x, cg1 ? 0.0f : dga.y);
+  dg23 = make_float2(cg2 ? 0.0f : dgb.x, cg3 ? 0.0f : dgb.y);
+  du01 = make_float2(cu(u01.x) ? 0.0f : dua.x, cu(u01.y) ? 0.0f : dua.y);
+  du23 = make_float2(cu(u23.x) ? 0.0f : dub.x, cu(u23.y) ? 0.0f : dub.y);
+  h01 = mul2(si01, v01);
+  h23 = mul2(si23, v23);
+}
+
 // ------------------------------------------------------------- forward tile
 // Lane l owns columns 4l .. 4l+3 of a 32 x 128 warp-tile; a rowwise block is
 // 8 lanes.  Rowwise work runs per 16-row half: after the 3-step butterfly
@@ -557,7 +477,18 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
       const float sr = __shfl_sync(kFull, sv, r);
       const float2 s2 = make_float2(sr, sr);
       float2 h01, h23;
-      if (ACT == kSwiGLU) {
+      if (ACT == kClamped) {
+        const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
+        float2 sg01, sg23;
+        sigma_pair(m.sig, G.x, sg01.x, sg01.y);
+        sigma_pair(m.sig, G.y, sg23.x, sg23.y);
+        float2 g01 = bf16x2_to_f2(G.x), g23 = bf16x2_to_f2(G.y);
+        clamp_gates(g01, sg01, p);
+        clamp_gates(g23, sg23, p);
+        const float2 si01 = mul2(g01, sg01), si23 = mul2(g23, sg23);
+        h01 = mul2(si01, clamped_up_plus_one(bf16x2_to_f2(U.x), p.clamp_L));
+        h23 = mul2(si23, clamped_up_plus_one(bf16x2_to_f2(U.y), p.clamp_L));
+      } else if (ACT == kSwiGLU) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
         float2 sg01, sg23;
         sigma_pair(m.sig, G.x, sg01.x, sg01.y);
@@ -751,14 +682,21 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
 // The backward of one row's four columns (a lane's share): packed bf16
 // dgate/dup pairs and the row's dscale partial sum_c dY*h.
 template <int ACT>
-__device__ __forceinline__ void bwd_row(const float* sig, uint2 D, uint2 G, uint2 U, float sr,
-                                        uint32_t& dg0, uint32_t& dg1, uint32_t& du0,
-                                        uint32_t& du1, float& part) {
+__device__ __forceinline__ void bwd_row(const Params& p, const float* sig, uint2 D, uint2 G,
+                                        uint2 U, float sr, uint32_t& dg0, uint32_t& dg1,
+                                        uint32_t& du0, uint32_t& du1, float& part) {
   const float2 s2 = make_float2(sr, sr);
   const float2 d01 = bf16x2_to_f2(D.x), d23 = bf16x2_to_f2(D.y);
   const float2 p01 = mul2(d01, s2), p23 = mul2(d23, s2);
   float2 h01, h23;
-  if (ACT == kSwiGLU) {
+  if (ACT == kClamped) {
+    float2 dga, dgb, dua, dub;
+    clamped_bwd_math(p, sig, G, U, p01, p23, dga, dgb, dua, dub, h01, h23);
+    dg0 = pack_bf16x2(dga.x, dga.y);
+    dg1 = pack_bf16x2(dgb.x, dgb.y);
+    du0 = pack_bf16x2(dua.x, dua.y);
+    du1 = pack_bf16x2(dub.x, dub.y);
+  } else if (ACT == kSwiGLU) {
     const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
     float2 sg01, sg23;
     sigma_pair(sig, G.x, sg01.x, sg01.y);
@@ -832,7 +770,10 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
       const float2 d01 = bf16x2_to_f2(D.x), d23 = bf16x2_to_f2(D.y);
       const float2 p01 = mul2(d01, s2), p23 = mul2(d23, s2);
       float2 dg01, dg23, du01, du23, h01, h23;
-      if (ACT == kSwiGLU) {
+      if (ACT == kClamped) {
+        const uint2 U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
+        clamped_bwd_math(p, m.sig, G, U, p01, p23, dg01, dg23, du01, du23, h01, h23);
+      } else if (ACT == kSwiGLU) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
         const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
         float2 sg01, sg23;
@@ -861,14 +802,14 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
       const bool live = FULL || r < nrows;
       DG[r][0] = live ? pack_bf16x2(dg01.x, dg01.y) : 0u;
       DG[r][1] = live ? pack_bf16x2(dg23.x, dg23.y) : 0u;
-      DU[r][0] = (live && ACT == kSwiGLU) ? pack_bf16x2(du01.x, du01.y) : 0u;
-      DU[r][1] = (live && ACT == kSwiGLU) ? pack_bf16x2(du23.x, du23.y) : 0u;
+      DU[r][0] = (live && ACT != kSReLU) ? pack_bf16x2(du01.x, du01.y) : 0u;
+      DU[r][1] = (live && ACT != kSReLU) ? pack_bf16x2(du23.x, du23.y) : 0u;
       P[i] = live ? __fmaf_rn(d23.y, h23.y, __fmaf_rn(d23.x, h23.x,
                               __fmaf_rn(d01.y, h01.y, __fmul_rn(d01.x, h01.x))))
                   : 0.0f;
       if (p.dx != nullptr && (FULL || (colok && r < nrows))) {
         __stcs(dxb + r * Wq, make_uint2(DG[r][0], DG[r][1]));
-        if (ACT == kSwiGLU) __stcs(dxb + r * Wq + (N >> 2), make_uint2(DU[r][0], DU[r][1]));
+        if (ACT != kSReLU) __stcs(dxb + r * Wq + (N >> 2), make_uint2(DU[r][0], DU[r][1]));
       }
     }
     __syncwarp();
@@ -909,14 +850,14 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
         const uint32_t qg = e4m3x2_2(bf16x2_to_f2(DG[r][0]), mg, mg) |
                             (e4m3x2_2(bf16x2_to_f2(DG[r][1]), mg, mg) << 16);
         uint32_t qu = 0;
-        if (ACT == kSwiGLU) {
+        if (ACT != kSReLU) {
           const uint32_t mu = __shfl_sync(kFull, (i & 1) ? mu1 : mu0, src);
           qu = e4m3x2_2(bf16x2_to_f2(DU[r][0]), mu, mu) |
                (e4m3x2_2(bf16x2_to_f2(DU[r][1]), mu, mu) << 16);
         }
         if (FULL || (colok && r < nrows)) {
           __stcs(rqb + r * Wq, qg);
-          if (ACT == kSwiGLU) __stcs(rqb + r * Wq + (N >> 2), qu);
+          if (ACT != kSReLU) __stcs(rqb + r * Wq + (N >> 2), qu);
         }
       }
     }
@@ -936,13 +877,13 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
         const int nct = W >> 7;
         __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row0 + lane, tile, nct)),
                vg);
-        if (ACT == kSwiGLU)
+        if (ACT != kSReLU)
           __stcs(reinterpret_cast<unsigned int*>(
                      p.rs + gemm_row_scales_off(row0 + lane, (N >> 7) + tile, nct)), vu);
       } else {
         uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
         store_scales4(rsr, vg, nb);
-        if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
+        if (ACT != kSReLU) store_scales4(rsr + N / 32, vu, nb);
       }
     }
   }
@@ -976,13 +917,13 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           p.cs[gemm_col_scale_off(base, c0 + c, j, kt)] = (uint8_t)bg[c];
-          if (ACT == kSwiGLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
+          if (ACT != kSReLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
         }
       } else {
         uint8_t* csr = p.cs + slab * (int64_t)W + c0;
         __stcs(reinterpret_cast<unsigned int*>(csr),
                bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
-        if (ACT == kSwiGLU)
+        if (ACT != kSReLU)
           __stcs(reinterpret_cast<unsigned int*>(csr + N),
                  bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
       }
@@ -995,7 +936,7 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
                           (e4m3x2_2(bf16x2_to_f2_p(DG[r][1]), mg[2], mg[3]) << 16);
       if (FULL || (colok && r < nrows)) {
         __stcs(qb + r * Wqc, qg);
-        if (ACT == kSwiGLU) {
+        if (ACT != kSReLU) {
           const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(DU[r][0]), mu[0], mu[1]) |
                               (e4m3x2_2(bf16x2_to_f2_p(DU[r][1]), mu[2], mu[3]) << 16);
           __stcs(qb + r * Wqc + (N >> 2), qu);
@@ -1038,10 +979,10 @@ __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
     const uint2 D = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
     const uint2 G = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
     uint2 U = make_uint2(0u, 0u);
-    if (ACT == kSwiGLU) U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
+    if (ACT != kSReLU) U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
     const float sr = __shfl_sync(kFull, sv, r);
     float part;
-    bwd_row<ACT>(m.sig, D, G, U, sr, DG[i][0], DG[i][1], DU[i][0], DU[i][1], part);
+    bwd_row<ACT>(p, m.sig, D, G, U, sr, DG[i][0], DG[i][1], DU[i][0], DU[i][1], part);
     const bool live = FULL || i < nrh;
     // rows past the slab's end: past M they read as zero (and give zeros); in
     // a grouped call they are the next group's rows, which must not count
@@ -1049,13 +990,13 @@ __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
     P[i] = part;
     if (FULL || (colok && live)) {
       dxb[r * Wqh] = make_uint2(DG[i][0], DG[i][1]);
-      if (ACT == kSwiGLU) dxb[r * Wqh + Nq] = make_uint2(DU[i][0], DU[i][1]);
+      if (ACT != kSReLU) dxb[r * Wqh + Nq] = make_uint2(DU[i][0], DU[i][1]);
     }
     if (DIRS & kCol) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         acg[c] = __vmaxu2(acg[c], DG[i][c] & 0x7FFF7FFFu);
-        if (ACT == kSwiGLU) acu[c] = __vmaxu2(acu[c], DU[i][c] & 0x7FFF7FFFu);
+        if (ACT != kSReLU) acu[c] = __vmaxu2(acu[c], DU[i][c] & 0x7FFF7FFFu);
       }
     }
   }
@@ -1092,14 +1033,14 @@ __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
       const uint32_t qg = e4m3x2_2(bf16x2_to_f2(DG[i][0]), mg, mg) |
                           (e4m3x2_2(bf16x2_to_f2(DG[i][1]), mg, mg) << 16);
       uint32_t qu = 0;
-      if (ACT == kSwiGLU) {
+      if (ACT != kSReLU) {
         const uint32_t mu = __shfl_sync(kFull, (i & 1) ? mu1 : mu0, src);
         qu = e4m3x2_2(bf16x2_to_f2(DU[i][0]), mu, mu) |
              (e4m3x2_2(bf16x2_to_f2(DU[i][1]), mu, mu) << 16);
       }
       if (FULL || (colok && i < nrh)) {
         __stcs(rqb + r * Wqh, qg);
-        if (ACT == kSwiGLU) __stcs(rqb + r * Wqh + Nq, qu);
+        if (ACT != kSReLU) __stcs(rqb + r * Wqh + Nq, qu);
       }
     }
   }
@@ -1119,7 +1060,7 @@ __device__ __forceinline__ void bwd_colwise_half_rr(int h, int N, int nrows, boo
     const int r = 16 * h + i;
     const bool ok = FULL || (colok && r < nrows);
     RG[i] = ok ? __ldcg(dxb + r * Wqc) : make_uint2(0u, 0u);
-    if (ACT == kSwiGLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (N >> 2)) : make_uint2(0u, 0u);
+    if (ACT != kSReLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (N >> 2)) : make_uint2(0u, 0u);
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -1128,7 +1069,7 @@ __device__ __forceinline__ void bwd_colwise_half_rr(int h, int N, int nrows, boo
                         (e4m3x2_2(bf16x2_to_f2_p(RG[i].y), mg[2], mg[3]) << 16);
     if (FULL || (colok && r < nrows)) {
       __stcs(qb + r * Wqc, qg);
-      if (ACT == kSwiGLU) {
+      if (ACT != kSReLU) {
         const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(RU[i].x), mu[0], mu[1]) |
                             (e4m3x2_2(bf16x2_to_f2_p(RU[i].y), mu[2], mu[3]) << 16);
         __stcs(qb + r * Wqc + (N >> 2), qu);
@@ -1180,13 +1121,13 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
         const int nct = W >> 7;
         __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row0 + lane, tile, nct)),
                vg);
-        if (ACT == kSwiGLU)
+        if (ACT != kSReLU)
           __stcs(reinterpret_cast<unsigned int*>(
                      p.rs + gemm_row_scales_off(row0 + lane, (N >> 7) + tile, nct)), vu);
       } else {
         uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
         store_scales4(rsr, vg, nb);
-        if (ACT == kSwiGLU) store_scales4(rsr + N / 32, vu, nb);
+        if (ACT != kSReLU) store_scales4(rsr + N / 32, vu, nb);
       }
     }
   }
@@ -1212,13 +1153,13 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           p.cs[gemm_col_scale_off(base, c0 + c, j, kt)] = (uint8_t)bg[c];
-          if (ACT == kSwiGLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
+          if (ACT != kSReLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
         }
       } else {
         uint8_t* csr = p.cs + slab * (int64_t)W + c0;
         __stcs(reinterpret_cast<unsigned int*>(csr),
                bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
-        if (ACT == kSwiGLU)
+        if (ACT != kSReLU)
           __stcs(reinterpret_cast<unsigned int*>(csr + N),
                  bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
       }

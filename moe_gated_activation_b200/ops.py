@@ -113,8 +113,8 @@ def splits_to_offsets(m_splits: torch.Tensor, total_rows: int):
 
 
 # ------------------------------------------------------------------ forward
-def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False):
-    swiglu = act == "swiglu"
+def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False, clamp=None):
+    swiglu = act != "srelu"        # gated: x = [gate | up]
     if N is None:
         N = x.shape[1] // 2 if swiglu else x.shape[1]
     _check_rows(x, "x", torch.bfloat16, 2 * N if swiglu else N)
@@ -130,7 +130,15 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
     mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales)
     stream = _stream(x.device)
     ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
-    if grouped is None:
+    if act == "clamped":
+        alpha, limit = clamp
+        if grouped is None:
+            _capi.call("scaled_clamped_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs,
+                       alpha, limit, mx, stream)
+        else:
+            _capi.call("grouped_scaled_clamped_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N,
+                       dirs, alpha, limit, _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
+    elif grouped is None:
         if swiglu:
             _capi.call("scaled_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs, int(staged),
                        mx, stream)
@@ -206,8 +214,8 @@ def _workspace(device, nbytes):
 
 
 def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, grouped=None,
-         gemm_scales=False):
-    swiglu = act == "swiglu"
+         gemm_scales=False, clamp=None):
+    swiglu = act != "srelu"        # gated: x = [gate | up], W = 2N
     if N is None:
         N = dy.shape[1]
     _check_rows(x, "x", torch.bfloat16, 2 * N if swiglu else N)
@@ -237,7 +245,14 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
     lddy = dy.stride(0) if M > 1 else max(dy.stride(0), dy.shape[1])
     common = (_ptr(dy), lddy, _ptr(x), ldx, _ptr(s), M, N, dirs)
     tail = (mx, _ptr(ws), ws.numel() if ws is not None else 0, stream)
-    if grouped is None:
+    if act == "clamped":
+        common = common + tuple(clamp)
+        if grouped is None:
+            _capi.call("scaled_clamped_swiglu_mxfp8_bwd", *common, _ptr(dx), _ptr(dscale), *tail)
+        else:
+            _capi.call("grouped_scaled_clamped_swiglu_mxfp8_bwd", *common, _ptr(ro), _ptr(cb), E,
+                       _ptr(st), _ptr(dx), _ptr(dscale), *tail)
+    elif grouped is None:
         name = "scaled_swiglu_mxfp8_bwd" if swiglu else "scaled_srelu_mxfp8_bwd"
         _capi.call(name, *common, _ptr(dx), _ptr(dscale), *tail)
     else:
@@ -275,6 +290,57 @@ def grouped_scaled_srelu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=T
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
                 g, gemm_scales=gemm_scales), status
+
+
+# ------------------------------------------------------------------ ClampedSwiGLU
+CLAMPED_ALPHA = 1.702   # defaults of the reading (the public gpt-oss clamped SwiGLU)
+CLAMPED_LIMIT = 7.0
+
+
+def scaled_clamped_swiglu_mxfp8_fwd(x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
+                                    rowwise=True, colwise=True, N=None, gemm_scales=False):
+    """MXFP8 of ClampedSwiGLU(x) * s (moeact.h); x bf16 [M, >=2N] packs [gate | up]."""
+    return _fwd("clamped", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales,
+                clamp=(alpha, limit))
+
+
+def grouped_scaled_clamped_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, alpha=CLAMPED_ALPHA,
+                                            limit=CLAMPED_LIMIT, rowwise=True, colwise=True,
+                                            status=None, col_scale_rows=None, N=None,
+                                            gemm_scales=False):
+    g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
+    return _fwd("clamped", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales,
+                clamp=(alpha, limit)), status
+
+
+def scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
+                                    rowwise=True, colwise=True, want_dx=True, want_dscale=True,
+                                    workspace=None, N=None, gemm_scales=False):
+    return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
+                gemm_scales=gemm_scales, clamp=(alpha, limit))
+
+
+def grouped_scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *,
+                                            alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
+                                            rowwise=True, colwise=True, want_dx=True,
+                                            want_dscale=True, workspace=None, status=None,
+                                            col_scale_rows=None, N=None, gemm_scales=False):
+    g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
+    return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, g,
+                gemm_scales=gemm_scales, clamp=(alpha, limit)), status
+
+
+def init_clamped(alpha=CLAMPED_ALPHA):
+    """Build the sigmoid table of a ClampedSwiGLU slope on the current device
+    (the first call with that alpha would; this one may precede a capture)."""
+    _capi.call("moeact_init_clamped", alpha)
+
+
+def clamped_sigmoid_table(alpha=CLAMPED_ALPHA, device="cuda"):
+    """fp32 sigma(RN(alpha * g)) for all 65536 bf16 g, as the kernels compute it."""
+    out = torch.empty(65536, dtype=torch.float32, device=device)
+    _capi.call("moeact_clamped_sigmoid_dump", alpha, _ptr(out), _stream(out.device))
+    return out
 
 
 # ------------------------------------------------------------------ misc

@@ -102,6 +102,8 @@ def _load():
     lib.orc_grouped_clamped_bwd.argtypes = [P, I64, P, I64, P, I64, I64, I, F, F, P, P, I32,
                                             P, P, P, P, P, P]
     lib.orc_grouped_clamped_bwd.restype = I
+    lib.orc_clamped_sigmoid.argtypes = [F, ctypes.c_uint16, ctypes.POINTER(I)]
+    lib.orc_clamped_sigmoid.restype = F
     lib.orc_scales_gemm_layout.argtypes = [P, I64, I64, P]
     lib.orc_scales_gemm_layout.restype = None
     lib.orc_col_scales_gemm_layout.argtypes = [P, I64, P, P, I32, P]
@@ -391,4 +393,15 @@ def grouped_clamped_bwd(dy_bits, x_bits, s, N, dirs, row_offs, colblk_offs,
                                               limit, _ptr(ro), _ptr(co), ro.shape[0] - 1,
                                               _ptr(out["dx"]), _ptr(out["dscale"]),
                                               *_mx_ptrs(out)), "grouped_clamped_bwd")
+    return out
+
+
+def clamped_sigmoid_table(alpha=CLAMPED_ALPHA) -> np.ndarray:
+    """sigma(RN(alpha * g)) for all 65536 bf16 g (fp32, correctly rounded)."""
+    lib = _load()
+    ok = ctypes.c_int(1)
+    out = np.array([lib.orc_clamped_sigmoid(alpha, b, ctypes.byref(ok)) for b in range(65536)],
+                   np.float32)
+    if not ok.value:
+        raise ArithmeticError("a sigma rounding could not be certified")
     return out

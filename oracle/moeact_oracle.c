@@ -480,6 +480,21 @@ static void clamped_parts(uint16_t gb, uint16_t ub, float alpha, float L,
   c->h = c->silu * c->v;
 }
 
+/* sigma(RN(alpha * g)) for the bf16 gate g (no clamp), for the table pin;
+ * *certified is cleared if the rounding could not be certified. */
+float orc_clamped_sigmoid(float alpha, uint16_t gbits, int* certified) {
+  orc_fpenv env = orc_enter();
+  float z = alpha * orc_bf16_to_f32(gbits);
+  float r;
+  int ok = 1;
+  if (isnan(z)) r = z;
+  else if (isinf(z)) r = z > 0 ? 1.0f : 0.0f;
+  else r = sigma_certified(z, &ok);
+  if (!ok) *certified = 0;
+  orc_leave(env);
+  return r;
+}
+
 static int clamped_args_ok(float alpha, float L) {
   return alpha >= 0.8125f && alpha <= 2.0f && L > 0.0f;   /* L may be +Inf; NaN fails */
 }

@@ -409,6 +409,37 @@ def test_grouped_forward_backward_parity(cuda_device, act, name):
                   "grouped dscale")
 
 
+@pytest.mark.parametrize("act", ["swiglu", "srelu"])
+def test_grouped_parity_at_the_group_limit(cuda_device, act):
+    """MOEACT_MAX_GROUPS groups (the most offsets the kernels stage in shared
+    memory: in the sigmoid table's gap for SwiGLU, after the rings for SReLU),
+    ragged sizes 0..40 with many empty groups."""
+    N = 64
+    g = np.random.default_rng(17)
+    m = g.integers(0, 41, _capi.MAX_GROUPS).astype(np.int64)
+    m[g.random(_capi.MAX_GROUPS) < 0.3] = 0
+    M = int(m.sum())
+    c = _case(M, N, act, seed=19)
+    xb, s, dyb = bf16_bits(c["x"]), c["s"].numpy(), bf16_bits(c["dy"])
+    _, ro, cb = oracle.splits_to_offsets(m, M)
+    gro, gcb, gst = mg.splits_to_offsets(torch.from_numpy(m).to(cuda_device), M)
+    x, sg, dy = c["x"].to(cuda_device), c["s"].to(cuda_device), c["dy"].to(cuda_device)
+    S = int(cb[-1])
+    fwd = mg.grouped_scaled_swiglu_mxfp8_fwd if act == "swiglu" else mg.grouped_scaled_srelu_mxfp8_fwd
+    bwd = mg.grouped_scaled_swiglu_mxfp8_bwd if act == "swiglu" else mg.grouped_scaled_srelu_mxfp8_bwd
+    got, st = fwd(x, sg, gro, gcb, col_scale_rows=S)
+    gotb, stb = bwd(dy, x, sg, gro, gcb, col_scale_rows=S)
+    torch.cuda.synchronize()
+    assert int(gst.item()) == 0 and int(st.item()) == 0 and int(stb.item()) == 0
+    ref = oracle.grouped_act_fwd(xb, s, N, 3, ro, cb, act=ACTS[act])
+    compare_mx(got, ref, f"{act} fwd at {_capi.MAX_GROUPS} groups", exact=True)
+    refb = oracle.grouped_act_bwd(dyb, xb, s, N, 3, ro, cb, act=ACTS[act])
+    compare_mx(gotb.mx, refb, f"{act} bwd at {_capi.MAX_GROUPS} groups", exact=True)
+    assert np.array_equal(bf16_u16(gotb.dx), refb["dx"])
+    assert_dscale(gotb.dscale, refb["dscale"], dscale_abs_bound(dyb, xb, s, N, act == "swiglu"),
+                  "dscale at the group limit")
+
+
 def test_grouped_equals_dense_for_aligned_splits(cuda_device):
     N = 128
     m = np.array([96, 0, 32, 128, 0, 64], np.int64)

@@ -157,3 +157,22 @@ def test_argument_range():
     for alpha, L in ((0.5, 7.0), (2.5, 7.0), (1.0, 0.0), (1.0, -1.0), (1.0, float("nan"))):
         with pytest.raises(ValueError):
             oracle.clamped_fwd(xb, s, 32, BOTH, alpha=alpha, limit=L)
+
+
+def test_sigmoid_table_of_a_slope():
+    """sigma(RN(alpha * g)) over bf16 g: alpha = 1 gives the SwiGLU table;
+    for alpha = 1.702 a sample of gates (every 97th pattern, and the window
+    edges) against the exact reference."""
+    t1 = oracle.clamped_sigmoid_table(1.0)
+    ref = oracle.sigmoid_table()
+    fin = ~np.isnan(ref)
+    assert np.array_equal(t1.view(np.uint32)[fin], ref.view(np.uint32)[fin])
+    alpha = float(np.float32(1.702))
+    t = oracle.clamped_sigmoid_table(alpha)
+    sample = sorted(set(range(0, 65536, 97)) | {0x3300, 0x32FF, 0x42FF, 0x4300, 0xB300, 0xC2FF})
+    for b in sample:
+        g = naive_ref.bf16_value(b)
+        if math.isnan(g):
+            continue
+        want = naive_ref.sigmoid_of(naive_ref.fmul(alpha, g))
+        assert float(t[b]) == want, (hex(b), float(t[b]), want)

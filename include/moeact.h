@@ -142,6 +142,13 @@ typedef struct moeact_mx_out {
   uint8_t* col_codes;   /* [M, W]    E4M3, colwise 32x1 blocks */
   uint8_t* col_scales;  /* [S, W]    E8M0 (in `scale_layout`) */
   int32_t scale_layout; /* MOEACT_SCALES_ROWMAJOR (0) or MOEACT_SCALES_GEMM */
+  /* Optional device int32 (4-byte aligned), NULL for none: when it is
+   * non-zero at the time the call's kernels run, the call writes nothing
+   * (codes, scales, dX, dscale and the status word keep their contents), so
+   * that a captured CUDA graph can skip the work on some replays without
+   * changing any pointer [the device no-op flag of the pages' graph-safe
+   * paths].  It is read on the device, in stream order. */
+  const int32_t* noop_flag;
 } moeact_mx_out;
 
 /* Build the sigmoid table on the current device and set up its kernels.

@@ -24,7 +24,7 @@ MAX_GROUPS = 2040
 class MxOut(ctypes.Structure):
     _fields_ = [("row_codes", ctypes.c_void_p), ("row_scales", ctypes.c_void_p),
                 ("col_codes", ctypes.c_void_p), ("col_scales", ctypes.c_void_p),
-                ("scale_layout", ctypes.c_int32)]
+                ("scale_layout", ctypes.c_int32), ("noop_flag", ctypes.c_void_p)]
 
 
 class MoeactError(RuntimeError):

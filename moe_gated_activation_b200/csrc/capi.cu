@@ -168,6 +168,7 @@ moeact_status check_mx(const moeact_mx_out& o, int dirs, bool allow_none) {
   const void* ps[4] = {o.row_codes, o.row_scales, o.col_codes, o.col_scales};
   for (const void* p : ps)
     if (p && !aligned(p, 16)) return fail(MOEACT_EALIGN, "MXFP8 output pointers must be 16-byte aligned");
+  if (o.noop_flag && !aligned(o.noop_flag, 4)) return fail(MOEACT_EALIGN, "noop_flag must be 4-byte aligned");
   return MOEACT_OK;
 }
 
@@ -409,6 +410,7 @@ moeact_status fwd_common(const ActArgs& a, const void* x, int64_t ldx, const flo
   p.dense_slabs = ceil_div(M, 32);
   p.n_tiles = (int)ceil_div(N, kTileCols);
   p.gemm_scales = out.scale_layout == MOEACT_SCALES_GEMM;
+  p.noop = out.noop_flag;
   p.err = g_err_ptr[dev];
   if ((st = act_params(a, dev, cs, p))) return st;
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
@@ -478,6 +480,7 @@ moeact_status bwd_common(const ActArgs& a, const void* dy, int64_t lddy, const v
   p.dense_slabs = ceil_div(M, 32);
   p.n_tiles = (int)ceil_div(N, kTileCols);
   p.gemm_scales = out.scale_layout == MOEACT_SCALES_GEMM;
+  p.noop = out.noop_flag;
   p.err = g_err_ptr[dev];
   if ((st = act_params(a, dev, cs, p))) return st;
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
@@ -495,7 +498,8 @@ moeact_status bwd_common(const ActArgs& a, const void* dy, int64_t lddy, const v
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   if (dscale) {
-    dscale_reduce_kernel<<<(unsigned)ceil_div(M, 256), 256, 0, cs>>>(p.part, p.n_tiles, M, dscale);
+    dscale_reduce_kernel<<<(unsigned)ceil_div(M, 256), 256, 0, cs>>>(p.part, p.n_tiles, M, dscale,
+                                                                      p.noop);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "dscale reduction launch");
   }

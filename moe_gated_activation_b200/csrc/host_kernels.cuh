@@ -146,7 +146,9 @@ __global__ void __launch_bounds__(1024) splits_kernel(const int64_t* __restrict_
 // dscale[row] = sum over tiles t = 0, 1, ... of part[t][row], in that order.
 __global__ void __launch_bounds__(256) dscale_reduce_kernel(const float* __restrict__ part,
                                                             int n_tiles, int64_t M,
-                                                            float* __restrict__ dscale) {
+                                                            float* __restrict__ dscale,
+                                                            const int32_t* noop) {
+  if (noop != nullptr && *noop != 0) return;
   const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= M) return;
   float acc = 0.0f;

@@ -76,7 +76,7 @@ def _alloc_mx(M, W, dirs, device, col_rows):
     return rq, rs, cq, cs
 
 
-def _mx_struct(rq, rs, cq, cs, dirs, gemm_scales=False):
+def _mx_struct(rq, rs, cq, cs, dirs, gemm_scales=False, noop_flag=None):
     if dirs & ROWWISE:
         r = (rq.data_ptr(), rs.data_ptr())
     else:
@@ -86,7 +86,10 @@ def _mx_struct(rq, rs, cq, cs, dirs, gemm_scales=False):
     else:
         c = (None, None)
     layout = _capi.SCALES_GEMM if gemm_scales else _capi.SCALES_ROWMAJOR
-    return _capi.MxOut(r[0], r[1], c[0], c[1], layout)
+    if noop_flag is not None and (noop_flag.dtype != torch.int32 or not noop_flag.is_cuda):
+        raise ValueError("noop_flag must be an int32 CUDA tensor")
+    return _capi.MxOut(r[0], r[1], c[0], c[1], layout,
+                       noop_flag.data_ptr() if noop_flag is not None else None)
 
 
 def _mx_result(rq, rs, cq, cs, col_rows_view=None):
@@ -113,7 +116,8 @@ def splits_to_offsets(m_splits: torch.Tensor, total_rows: int):
 
 
 # ------------------------------------------------------------------ forward
-def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False, clamp=None):
+def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False, clamp=None,
+         noop_flag=None):
     swiglu = act != "srelu"        # gated: x = [gate | up]
     if N is None:
         N = x.shape[1] // 2 if swiglu else x.shape[1]
@@ -127,7 +131,7 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
         ro, cb, E, st, view = grouped
         col_rows = (M + 31) // 32 + E
     rq, rs, cq, cs = _alloc_mx(M, N, dirs, x.device, col_rows)
-    mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales)
+    mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales, noop_flag)
     stream = _stream(x.device)
     ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
     if act == "clamped":
@@ -155,16 +159,19 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
 
 
 def scaled_swiglu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, staged_rounding=False, N=None,
-                            gemm_scales=False):
+                            gemm_scales=False, noop_flag=None):
     """MXFP8 of SwiGLU(x) * s; x bf16 [M, >=2N] packs [gate | up].
     gemm_scales: scales in the GEMM-ready tiled layout (moeact.h,
     MOEACT_SCALES_GEMM; M and N multiples of 128)."""
-    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, gemm_scales=gemm_scales)
+    return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, gemm_scales=gemm_scales,
+                noop_flag=noop_flag)
 
 
-def scaled_srelu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, N=None, gemm_scales=False):
+def scaled_srelu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, N=None, gemm_scales=False,
+                           noop_flag=None):
     """MXFP8 of relu(x)^2 * s; x bf16 [M, >=N]."""
-    return _fwd("srelu", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales)
+    return _fwd("srelu", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales,
+                noop_flag=noop_flag)
 
 
 def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
@@ -176,20 +183,22 @@ def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
 
 def grouped_scaled_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
                                     staged_rounding=False, status=None, col_scale_rows=None,
-                                    N=None, gemm_scales=False):
+                                    N=None, gemm_scales=False, noop_flag=None):
     """Grouped forward: experts own the rows given by `row_offs` (from
     splits_to_offsets).  Returns (MXFP8, status).  Col scales hold
     ceil(M/32) + E rows unless `col_scale_rows` (sum of ceil(m_e/32), known on
     the host) is given."""
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, g,
-                gemm_scales=gemm_scales), status
+                gemm_scales=gemm_scales, noop_flag=noop_flag), status
 
 
 def grouped_scaled_srelu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
-                                   status=None, col_scale_rows=None, N=None, gemm_scales=False):
+                                   status=None, col_scale_rows=None, N=None, gemm_scales=False,
+                                   noop_flag=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
-    return _fwd("srelu", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales), status
+    return _fwd("srelu", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales,
+                noop_flag=noop_flag), status
 
 
 # ------------------------------------------------------------------ backward
@@ -214,7 +223,7 @@ def _workspace(device, nbytes):
 
 
 def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, grouped=None,
-         gemm_scales=False, clamp=None):
+         gemm_scales=False, clamp=None, noop_flag=None):
     swiglu = act != "srelu"        # gated: x = [gate | up], W = 2N
     if N is None:
         N = dy.shape[1]
@@ -233,7 +242,7 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
         ro, cb, E, st, view = grouped
         col_rows = (M + 31) // 32 + E
     rq, rs, cq, cs = _alloc_mx(M, W, dirs, dev, col_rows)
-    mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales)
+    mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales, noop_flag)
     dx = torch.empty((M, W), dtype=torch.bfloat16, device=dev) if want_dx else None
     dscale = torch.empty(M, dtype=torch.float32, device=dev) if want_dscale else None
     nbytes = bwd_workspace_bytes(M, N, E)
@@ -262,34 +271,36 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
 
 
 def scaled_swiglu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
-                            want_dscale=True, workspace=None, N=None, gemm_scales=False):
+                            want_dscale=True, workspace=None, N=None, gemm_scales=False,
+                            noop_flag=None):
     """Backward of the scaled SwiGLU: MXFP8 of [dgate | dup], bf16 dx, fp32 dscale."""
     return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales)
+                gemm_scales=gemm_scales, noop_flag=noop_flag)
 
 
 def scaled_srelu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
-                           want_dscale=True, workspace=None, N=None, gemm_scales=False):
+                           want_dscale=True, workspace=None, N=None, gemm_scales=False,
+                           noop_flag=None):
     return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales)
+                gemm_scales=gemm_scales, noop_flag=noop_flag)
 
 
 def grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
                                     colwise=True, want_dx=True, want_dscale=True,
                                     workspace=None, status=None, col_scale_rows=None, N=None,
-                                    gemm_scales=False):
+                                    gemm_scales=False, noop_flag=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                g, gemm_scales=gemm_scales), status
+                g, gemm_scales=gemm_scales, noop_flag=noop_flag), status
 
 
 def grouped_scaled_srelu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
                                    colwise=True, want_dx=True, want_dscale=True,
                                    workspace=None, status=None, col_scale_rows=None, N=None,
-                                   gemm_scales=False):
+                                   gemm_scales=False, noop_flag=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                g, gemm_scales=gemm_scales), status
+                g, gemm_scales=gemm_scales, noop_flag=noop_flag), status
 
 
 # ------------------------------------------------------------------ ClampedSwiGLU
@@ -298,36 +309,38 @@ CLAMPED_LIMIT = 7.0
 
 
 def scaled_clamped_swiglu_mxfp8_fwd(x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
-                                    rowwise=True, colwise=True, N=None, gemm_scales=False):
+                                    rowwise=True, colwise=True, N=None, gemm_scales=False,
+                                    noop_flag=None):
     """MXFP8 of ClampedSwiGLU(x) * s (moeact.h); x bf16 [M, >=2N] packs [gate | up]."""
     return _fwd("clamped", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales,
-                clamp=(alpha, limit))
+                clamp=(alpha, limit), noop_flag=noop_flag)
 
 
 def grouped_scaled_clamped_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, alpha=CLAMPED_ALPHA,
                                             limit=CLAMPED_LIMIT, rowwise=True, colwise=True,
                                             status=None, col_scale_rows=None, N=None,
-                                            gemm_scales=False):
+                                            gemm_scales=False, noop_flag=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _fwd("clamped", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales,
-                clamp=(alpha, limit)), status
+                clamp=(alpha, limit), noop_flag=noop_flag), status
 
 
 def scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
                                     rowwise=True, colwise=True, want_dx=True, want_dscale=True,
-                                    workspace=None, N=None, gemm_scales=False):
+                                    workspace=None, N=None, gemm_scales=False, noop_flag=None):
     return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales, clamp=(alpha, limit))
+                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag)
 
 
 def grouped_scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *,
                                             alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
                                             rowwise=True, colwise=True, want_dx=True,
                                             want_dscale=True, workspace=None, status=None,
-                                            col_scale_rows=None, N=None, gemm_scales=False):
+                                            col_scale_rows=None, N=None, gemm_scales=False,
+                                            noop_flag=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, g,
-                gemm_scales=gemm_scales, clamp=(alpha, limit)), status
+                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag), status
 
 
 def init_clamped(alpha=CLAMPED_ALPHA):

@@ -149,3 +149,8 @@ def test_gemm_scale_layout_argument_errors(lib):
     assert fwd(lib, M=100, N=256, mx=gemm(A16, A16, None, None)) == _capi.EINVAL
     assert bwd(lib, M=96, N=128, ldx=256, lddy=128, mx=gemm(A16, A16, None, None)) == _capi.EINVAL
     assert fwd(lib, M=0, N=256, mx=gemm(A16, A16, None, None)) == _capi.OK
+
+
+def test_noop_flag_alignment(lib):
+    mx = _capi.MxOut(A16, A16, None, None, _capi.SCALES_ROWMAJOR, A16 + 2)
+    assert fwd(lib, mx=mx) == _capi.EALIGN

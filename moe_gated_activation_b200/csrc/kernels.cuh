@@ -1049,24 +1049,31 @@ __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
   return true;
 }
 
-// Colwise codes of one 16-row half of a backward tile, from dX re-read out of
-// L2 (loads first, then the math).
+// Colwise codes of a backward tile from dX re-read out of L2, in four chunks
+// of 8 rows with double-buffered loads: the loads of the next chunk are in
+// flight while the current one is quantized and stored, so one load latency
+// per tile is exposed instead of one per chunk.
 template <int ACT, bool FULL>
-__device__ __forceinline__ void bwd_colwise_half_rr(int h, int N, int nrows, bool colok,
-                                                    int Wqc, const uint2* dxb, unsigned int* qb,
-                                                    const uint32_t (&mg)[4],
-                                                    const uint32_t (&mu)[4]) {
-  uint2 RG[16], RU[16];
+__device__ __forceinline__ void bwd_colwise_load8(int q, int N, int nrows, bool colok, int Wqc,
+                                                  const uint2* dxb, uint2 (&RG)[8],
+                                                  uint2 (&RU)[8]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int r = 16 * h + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = 8 * q + i;
     const bool ok = FULL || (colok && r < nrows);
     RG[i] = ok ? __ldcg(dxb + r * Wqc) : make_uint2(0u, 0u);
     if (ACT != kSReLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (N >> 2)) : make_uint2(0u, 0u);
   }
+}
+
+template <int ACT, bool FULL>
+__device__ __forceinline__ void bwd_colwise_store8(int q, int N, int nrows, bool colok, int Wqc,
+                                                   unsigned int* qb, const uint2 (&RG)[8],
+                                                   const uint2 (&RU)[8], const uint32_t (&mg)[4],
+                                                   const uint32_t (&mu)[4]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int r = 16 * h + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = 8 * q + i;
     const uint32_t qg = e4m3x2_2(bf16x2_to_f2_p(RG[i].x), mg[0], mg[1]) |
                         (e4m3x2_2(bf16x2_to_f2_p(RG[i].y), mg[2], mg[3]) << 16);
     if (FULL || (colok && r < nrows)) {
@@ -1077,6 +1084,21 @@ __device__ __forceinline__ void bwd_colwise_half_rr(int h, int N, int nrows, boo
         __stcs(qb + r * Wqc + (N >> 2), qu);
       }
     }
+  }
+}
+
+template <int ACT, bool FULL>
+__device__ __forceinline__ void bwd_colwise_rr(int N, int nrows, bool colok, int Wqc,
+                                               const uint2* dxb, unsigned int* qb,
+                                               const uint32_t (&mg)[4], const uint32_t (&mu)[4]) {
+  uint2 AG[8], AU[8], BG[8], BU[8];
+  bwd_colwise_load8<ACT, FULL>(0, N, nrows, colok, Wqc, dxb, AG, AU);
+#pragma unroll 1
+  for (int q = 0; q < 4; q += 2) {
+    bwd_colwise_load8<ACT, FULL>(q + 1, N, nrows, colok, Wqc, dxb, BG, BU);
+    bwd_colwise_store8<ACT, FULL>(q, N, nrows, colok, Wqc, qb, AG, AU, mg, mu);
+    if (q + 2 < 4) bwd_colwise_load8<ACT, FULL>(q + 2, N, nrows, colok, Wqc, dxb, AG, AU);
+    bwd_colwise_store8<ACT, FULL>(q + 1, N, nrows, colok, Wqc, qb, BG, BU, mg, mu);
   }
 }
 
@@ -1168,9 +1190,7 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
     }
     unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
     const int Wqc = opaque(Wq);
-#pragma unroll 1
-    for (int h = 0; h < 2; ++h)
-      bwd_colwise_half_rr<ACT, FULL>(h, N, nrows, colok, Wqc, dxb, qb, mg, mu);
+    bwd_colwise_rr<ACT, FULL>(N, nrows, colok, Wqc, dxb, qb, mg, mu);
   }
 }
 

@@ -7,7 +7,9 @@ package never imports the product.
 
 The arithmetic lives in ``moeact_oracle.c`` (plain C, IEEE binary32 steps in the
 order the method states, binary128 for the sigmoid, binary64 for sums); this
-module only compiles it with gcc and marshals numpy arrays through ctypes.
+module only compiles it with gcc and marshals numpy arrays through ctypes (and,
+for inputs whose gate and up columns are interleaved, rearranges columns around
+those calls).
 
 Array conventions (all numpy, C-contiguous):
   bf16 data is passed as ``uint16`` bit patterns; fp32 as ``float32``;
@@ -405,3 +407,86 @@ def clamped_sigmoid_table(alpha=CLAMPED_ALPHA) -> np.ndarray:
     if not ok.value:
         raise ArithmeticError("a sigma rounding could not be certified")
     return out
+
+
+# ---------------------------------------------------------------- interleaved gate / up
+# TE PR #3238, Important Files Changed (swiglu.py row): the GLU interleave
+# reshaping of the gated input moves into the scaled_swiglu / scaled_dswiglu
+# kernels.  The block order and size are a reading: the 2N columns hold G gate
+# columns, then the G up columns paired with them, repeated N / G times; dX
+# comes back in the same order, and its MXFP8 blocks run along the stored
+# columns.  The functions below only rearrange columns and then call the
+# oracle's halves-layout functions and quantizer.
+def glu_halves(x_bits, N, G):
+    """An interleaved gated input [M, >= 2N] as [gate | up] halves [M, 2N]."""
+    x = np.asarray(x_bits)
+    M = x.shape[0]
+    blocks = x[:, :2 * N].reshape(M, N // G, 2, G)
+    return np.ascontiguousarray(np.concatenate(
+        [blocks[:, :, 0, :].reshape(M, N), blocks[:, :, 1, :].reshape(M, N)], axis=1))
+
+
+def glu_interleave(a, N, G):
+    """[gate | up] halves [M, 2N] -> the interleaved column order."""
+    a = np.asarray(a)
+    M = a.shape[0]
+    g = a[:, :N].reshape(M, N // G, 1, G)
+    u = a[:, N:2 * N].reshape(M, N // G, 1, G)
+    return np.ascontiguousarray(np.concatenate([g, u], axis=2).reshape(M, 2 * N))
+
+
+def _quantize_grouped(y, dirs, row_offs=None, colblk_offs=None):
+    """MXFP8 of y [M, W]; with offsets, each group's rows on their own
+    (colwise blocks end at group boundaries, col scales at colblk_offs[e])."""
+    if row_offs is None:
+        return mxfp8_quantize(y, dirs)
+    ro = _c(row_offs, np.int64)
+    co = _c(colblk_offs, np.int64)
+    M, W = y.shape
+    out = _alloc_mx(M, W, dirs, colblk_rows=int(co[-1]))
+    for e in range(ro.shape[0] - 1):
+        r0, r1 = int(ro[e]), int(ro[e + 1])
+        if r1 == r0:
+            continue
+        q = mxfp8_quantize(y[r0:r1], dirs)
+        if dirs & ROWWISE:
+            out["row_codes"][r0:r1] = q["row_codes"]
+            out["row_scales"][r0:r1] = q["row_scales"]
+        if dirs & COLWISE:
+            out["col_codes"][r0:r1] = q["col_codes"]
+            c0 = int(co[e])
+            out["col_scales"][c0:c0 + q["col_scales"].shape[0]] = q["col_scales"]
+    return out
+
+
+def interleaved_fwd(x_bits, s, N, dirs, G, act="swiglu", staged=False, row_offs=None,
+                    colblk_offs=None, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT):
+    """Forward of a gated activation whose input interleaves gate and up in
+    blocks of G columns (act "swiglu" or "clamped"; grouped with offsets)."""
+    xc = glu_halves(x_bits, N, G)
+    grouped = row_offs is not None
+    if act == "clamped":
+        if grouped:
+            return grouped_clamped_fwd(xc, s, N, dirs, row_offs, colblk_offs, alpha, limit)
+        return clamped_fwd(xc, s, N, dirs, alpha, limit)
+    if grouped:
+        return grouped_act_fwd(xc, s, N, dirs, row_offs, colblk_offs, SWIGLU, staged)
+    return act_fwd(xc, s, N, dirs, SWIGLU, staged)
+
+
+def interleaved_bwd(dy_bits, x_bits, s, N, dirs, G, act="swiglu", row_offs=None,
+                    colblk_offs=None, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT):
+    """Backward with interleaved gate / up: dx [M, 2N] in the interleaved
+    order, dscale, and the MXFP8 of that dx (of its bf16 values)."""
+    xc = glu_halves(x_bits, N, G)
+    if act == "clamped":
+        r = clamped_bwd(dy_bits, xc, s, N, 0, alpha, limit)
+    else:
+        r = act_bwd(dy_bits, xc, s, N, 0, SWIGLU)
+    dx = glu_interleave(r["dx"], N, G)
+    y = (dx.astype(np.uint32) << 16).view(np.float32)
+    out = _quantize_grouped(y, dirs, row_offs, colblk_offs)
+    out["dx"] = dx
+    out["dscale"] = r["dscale"]
+    return out
+

@@ -159,15 +159,17 @@ def ncu_traffic(workload, kernel, dirs_name):
     return None
 
 
-def act_api(mg, act):
+def act_api(mg, act, glu_interleave=0):
     """(grouped forward, grouped backward, extra keyword arguments) of an
-    activation; ClampedSwiGLU at the default slope and limit."""
+    activation; ClampedSwiGLU at the default slope and limit; gate and up
+    interleaved in blocks of `glu_interleave` columns when it is non-zero."""
+    extra = {"glu_interleave": glu_interleave} if glu_interleave else {}
     if act == "clamped":
         mg.init_clamped()
+        extra.update(alpha=mg.ops.CLAMPED_ALPHA, limit=mg.ops.CLAMPED_LIMIT)
         return (mg.grouped_scaled_clamped_swiglu_mxfp8_fwd,
-                mg.grouped_scaled_clamped_swiglu_mxfp8_bwd,
-                {"alpha": mg.ops.CLAMPED_ALPHA, "limit": mg.ops.CLAMPED_LIMIT})
-    return mg.grouped_scaled_swiglu_mxfp8_fwd, mg.grouped_scaled_swiglu_mxfp8_bwd, {}
+                mg.grouped_scaled_clamped_swiglu_mxfp8_bwd, extra)
+    return mg.grouped_scaled_swiglu_mxfp8_fwd, mg.grouped_scaled_swiglu_mxfp8_bwd, extra
 
 
 def max_over_ranks(value, world, device):
@@ -236,7 +238,7 @@ def run_ours(args):
         return mg.splits_to_offsets(m_dev, M)
 
     gemm = args.scales == "gemm"
-    fwd_api, bwd_api, extra = act_api(mg, args.act)
+    fwd_api, bwd_api, extra = act_api(mg, args.act, args.glu_interleave)
 
     def fwd(ro, cb, st):
         return fwd_api(x, s, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, status=st,
@@ -376,6 +378,7 @@ def run_ours(args):
         "data": "synthetic (seeded torch generators; shapes and statistics of the pages' workloads)",
         "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
                    "dirs": args.dirs, "scales": args.scales, "activation": args.act,
+                   "glu_interleave": args.glu_interleave,
                    "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
                    "launch": "eager" if args.eager else "one CUDA graph per step (events at its ends only)",
                    "kernel_times": "eager events" if args.eager else "a second timed pass of the same steps, with event nodes between the calls",
@@ -419,7 +422,7 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
     M, N = wl.M, wl.N
     rw, cw = bool(dirs & 1), bool(dirs & 2)
     gemm = args.scales == "gemm"
-    fwd_api, bwd_api, extra = act_api(mg, args.act)
+    fwd_api, bwd_api, extra = act_api(mg, args.act, args.glu_interleave)
     hin = [inp["x"].cpu().pin_memory(), inp["s"].cpu().pin_memory(),
            inp["dy"].cpu().pin_memory(), inp["m_splits"].clone().pin_memory()]
     h2d = sum(t.numel() * t.element_size() for t in hin)
@@ -583,6 +586,8 @@ def main():
                     help="activation: SwiGLU, or ClampedSwiGLU (alpha 1.702, limit 7)")
     ap.add_argument("--scales", default="rowmajor", choices=["rowmajor", "gemm"],
                     help="E8M0 scale layout: row-major, or the GEMM-ready 128 x 4 tiles")
+    ap.add_argument("--glu-interleave", type=int, default=0,
+                    help="gate / up interleaved in blocks of G columns (0: [gate | up] halves)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of CUDA graphs")

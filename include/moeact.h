@@ -45,6 +45,18 @@
  * Layouts (all row-major, byte offsets from the given pointers):
  *   x        bf16 [M, ldx]; SwiGLU reads gate = x[:, 0:N], up = x[:, N:2N]
  *            (ldx >= 2N); SReLU reads x[:, 0:N] (ldx >= N).
+ *   glu_interleave  (gated calls) G = 0: the [gate | up] halves above.
+ *            G > 0: the 2N columns hold G gate columns, then the G up
+ *            columns that pair with them, repeated N/G times: gate column j
+ *            at (j / G) * 2G + j % G, its up column G further on [TE:
+ *            Important Files Changed, swiglu.py row -- the GLU interleave
+ *            reshaping now happens inside the scaled_swiglu / scaled_dswiglu
+ *            kernels; the block order and granularity are a reading].  G
+ *            must be 32, 64 or a multiple of 128 and divide N (G = N is the
+ *            halves layout), else MOEACT_EINVAL.  The
+ *            backward writes dx and the MXFP8 of [dgate | dup] in the same
+ *            interleaved column order, with the 1x32 blocks taken along the
+ *            stored columns (so each block is all dgate or all dup).
  *   dy       bf16 [M, lddy], first N columns (lddy >= N).
  *   s        fp32 [M] per-row scale (routing probability).
  *   W        width of the quantized tensor: N in the forward; 2N (SwiGLU,
@@ -181,12 +193,13 @@ moeact_status splits_to_offsets(const int64_t* m_splits, int32_t num_groups,
 /* ---------------------------------------------------------------------
  * Forward, dense [AO: gated_act_mxfp8_forward, plus TE's per-row scale].
  *   x [M, ldx] bf16, s [M] fp32, N % 32 == 0, dirs != 0; staged_rounding
- *   0/1 [VO].  M == 0 returns MOEACT_OK without launching.
+ *   0/1 [VO]; glu_interleave as under Layouts (0: [gate | up]).  M == 0
+ *   returns MOEACT_OK without launching.
  * ------------------------------------------------------------------- */
 moeact_status scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                       int64_t M, int64_t N, int dirs,
-                                      int staged_rounding, moeact_mx_out out,
-                                      void* stream);
+                                      int staged_rounding, int32_t glu_interleave,
+                                      moeact_mx_out out, void* stream);
 moeact_status scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                      int64_t M, int64_t N, int dirs,
                                      moeact_mx_out out, void* stream);
@@ -200,7 +213,7 @@ moeact_status scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
  * ------------------------------------------------------------------- */
 moeact_status grouped_scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                               int64_t M, int64_t N, int dirs,
-                                              int staged_rounding,
+                                              int staged_rounding, int32_t glu_interleave,
                                               const int64_t* row_offs,
                                               const int64_t* colblk_offs,
                                               int32_t num_groups, int32_t* status,
@@ -231,7 +244,7 @@ size_t scaled_act_mxfp8_bwd_workspace_size(int64_t M, int64_t N, int32_t num_gro
 
 moeact_status scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
                                       int64_t ldx, const float* s, int64_t M, int64_t N,
-                                      int dirs, void* dx, float* dscale,
+                                      int dirs, int32_t glu_interleave, void* dx, float* dscale,
                                       moeact_mx_out out, void* workspace,
                                       size_t workspace_bytes, void* stream);
 moeact_status scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
@@ -241,7 +254,7 @@ moeact_status scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x
                                      size_t workspace_bytes, void* stream);
 moeact_status grouped_scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
                                               int64_t ldx, const float* s, int64_t M,
-                                              int64_t N, int dirs,
+                                              int64_t N, int dirs, int32_t glu_interleave,
                                               const int64_t* row_offs,
                                               const int64_t* colblk_offs,
                                               int32_t num_groups, int32_t* status,
@@ -266,7 +279,7 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
  * allocator and cannot pass this library a workspace.  The paper has no
  * counterpart; this is a convenience of this library.
  *   Arguments, outputs and results are those of scaled_swiglu_mxfp8_bwd
- *   without the workspace: the dscale partial sums go to a 16 MiB array built
+ *   with glu_interleave = 0 and without the workspace: the dscale partial sums go to a 16 MiB array built
  *   into the library (held by every GPU that loads it, until exit), so with
  *   dscale requested ceil(N/128) * M must not exceed 4194304 (else
  *   MOEACT_ERANGE, nothing launched).  Allocates nothing.
@@ -296,8 +309,9 @@ moeact_status scaled_swiglu_mxfp8_bwd_noalloc(const void* dy, int64_t lddy, cons
  *   dgate = g > L ? 0 : bf16(RN(RN(p * RN(uc + 1)) * dsilu))
  *   dup = |u| > L ? 0 : bf16(RN(p * RN(gc * sig)))
  *   dscale_row = sum_j dY * h (h = RN(RN(gc * sig) * RN(uc + 1))).
- * Layout, outputs, workspace and errors as for SwiGLU (x = [gate | up],
- * W = 2N in the backward; no staged rounding).  alpha must lie in
+ * Layout, outputs, workspace and errors as for SwiGLU (x = [gate | up] or
+ * interleaved by glu_interleave, W = 2N in the backward; no staged
+ * rounding).  alpha must lie in
  * [0.8125, 2] and limit be > 0 (+Inf allowed), else MOEACT_EINVAL.  The
  * first call with a given alpha on a device builds that alpha's sigmoid table
  * (device memory, kept until exit; synchronises the device once; at most 8
@@ -308,24 +322,28 @@ moeact_status scaled_swiglu_mxfp8_bwd_noalloc(const void* dy, int64_t lddy, cons
 moeact_status moeact_init_clamped(float alpha);
 moeact_status scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                               int64_t M, int64_t N, int dirs, float alpha,
-                                              float limit, moeact_mx_out out, void* stream);
+                                              float limit, int32_t glu_interleave,
+                                              moeact_mx_out out, void* stream);
 moeact_status grouped_scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                                       int64_t M, int64_t N, int dirs,
                                                       float alpha, float limit,
+                                                      int32_t glu_interleave,
                                                       const int64_t* row_offs,
                                                       const int64_t* colblk_offs,
                                                       int32_t num_groups, int32_t* status,
                                                       moeact_mx_out out, void* stream);
 moeact_status scaled_clamped_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
                                               int64_t ldx, const float* s, int64_t M, int64_t N,
-                                              int dirs, float alpha, float limit, void* dx,
-                                              float* dscale, moeact_mx_out out, void* workspace,
+                                              int dirs, float alpha, float limit,
+                                              int32_t glu_interleave, void* dx, float* dscale,
+                                              moeact_mx_out out, void* workspace,
                                               size_t workspace_bytes, void* stream);
 moeact_status grouped_scaled_clamped_swiglu_mxfp8_bwd(
     const void* dy, int64_t lddy, const void* x, int64_t ldx, const float* s, int64_t M,
-    int64_t N, int dirs, float alpha, float limit, const int64_t* row_offs,
-    const int64_t* colblk_offs, int32_t num_groups, int32_t* status, void* dx, float* dscale,
-    moeact_mx_out out, void* workspace, size_t workspace_bytes, void* stream);
+    int64_t N, int dirs, float alpha, float limit, int32_t glu_interleave,
+    const int64_t* row_offs, const int64_t* colblk_offs, int32_t num_groups, int32_t* status,
+    void* dx, float* dscale, moeact_mx_out out, void* workspace, size_t workspace_bytes,
+    void* stream);
 /* Test hook: the table of sigma(RN(alpha * g)) over all 65536 bf16 g, fp32
  * [65536] (as moeact_sigmoid_dump). */
 moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream);

@@ -48,26 +48,27 @@ _SIGS = {
     "moeact_status_string": ([I], ctypes.c_char_p),
     "moeact_last_error": ([], ctypes.c_char_p),
     "splits_to_offsets": ([P, I32, I64, P, P, P, P], I),
-    "scaled_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, I, MxOut, P], I),
+    "scaled_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, I, I32, MxOut, P], I),
     "scaled_srelu_mxfp8_fwd": ([P, I64, P, I64, I64, I, MxOut, P], I),
-    "grouped_scaled_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, I, P, P, I32, P, MxOut, P], I),
+    "grouped_scaled_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, I, I32, P, P, I32, P, MxOut, P],
+                                        I),
     "grouped_scaled_srelu_mxfp8_fwd": ([P, I64, P, I64, I64, I, P, P, I32, P, MxOut, P], I),
     "scaled_act_mxfp8_bwd_workspace_size": ([I64, I64, I32], SZ),
-    "scaled_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, P, P, MxOut, P, SZ, P], I),
+    "scaled_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, I32, P, P, MxOut, P, SZ, P], I),
     "scaled_srelu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, P, P, MxOut, P, SZ, P], I),
-    "grouped_scaled_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, P, P, I32, P, P, P,
+    "grouped_scaled_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, I32, P, P, I32, P, P, P,
                                          MxOut, P, SZ, P], I),
     "grouped_scaled_srelu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, P, P, I32, P, P, P,
                                         MxOut, P, SZ, P], I),
     "moeact_sigmoid_dump": ([P, P], I),
     "moeact_init_clamped": ([F], I),
-    "scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, MxOut, P], I),
-    "grouped_scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, P, P, I32, P,
+    "scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, I32, MxOut, P], I),
+    "grouped_scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, I32, P, P, I32, P,
                                                  MxOut, P], I),
-    "scaled_clamped_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, F, F, P, P, MxOut, P,
-                                         SZ, P], I),
-    "grouped_scaled_clamped_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, F, F, P, P, I32,
-                                                 P, P, P, MxOut, P, SZ, P], I),
+    "scaled_clamped_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, F, F, I32, P, P, MxOut,
+                                         P, SZ, P], I),
+    "grouped_scaled_clamped_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, F, F, I32, P, P,
+                                                 I32, P, P, P, MxOut, P, SZ, P], I),
     "moeact_clamped_sigmoid_dump": ([F, P, P], I),
     "moeact_device_error": ([P], I),
     "scaled_swiglu_mxfp8_bwd_noalloc": ([P, I64, P, I64, P, I64, I64, I, P, P, MxOut, P], I),

@@ -43,8 +43,8 @@ __device__ int g_sigma_uncertain;
 
 // The fused kernels of each activation (index kSwiGLU / kSReLU / kClamped),
 // filled once.
-FwdVariant g_fwd[3][kVariantSlots];
-BwdVariant g_bwd[3][kVariantSlots];
+FwdVariant g_fwd[3][kFwdSlots];
+BwdVariant g_bwd[3][kBwdSlots];
 bool g_tables_filled = false;
 
 // Extra shared memory of a grouped call (its col-block offsets), at most.
@@ -77,6 +77,8 @@ moeact_status init_device(int dev) {
   if (!g_tables_filled) {
     fill_fwd_swiglu_dense(g_fwd[kSwiGLU]);
     fill_fwd_swiglu_grouped(g_fwd[kSwiGLU]);
+    fill_fwd_swiglu_ilv_dense(g_fwd[kSwiGLU]);
+    fill_fwd_swiglu_ilv_grouped(g_fwd[kSwiGLU]);
     fill_bwd_swiglu_dense(g_bwd[kSwiGLU]);
     fill_bwd_swiglu_grouped(g_bwd[kSwiGLU]);
     fill_fwd_srelu_dense(g_fwd[kSReLU]);
@@ -85,6 +87,8 @@ moeact_status init_device(int dev) {
     fill_bwd_srelu_grouped(g_bwd[kSReLU]);
     fill_fwd_clamped_dense(g_fwd[kClamped]);
     fill_fwd_clamped_grouped(g_fwd[kClamped]);
+    fill_fwd_clamped_ilv_dense(g_fwd[kClamped]);
+    fill_fwd_clamped_ilv_grouped(g_fwd[kClamped]);
     fill_bwd_clamped_dense(g_bwd[kClamped]);
     fill_bwd_clamped_grouped(g_bwd[kClamped]);
     g_tables_filled = true;
@@ -249,9 +253,34 @@ moeact_status make_map_gated(CUtensorMap* map, const void* base, int64_t N, int6
   return MOEACT_OK;
 }
 
-moeact_status make_x_map(CUtensorMap* map, int act, const void* x, int64_t N, int64_t rows,
-                         int64_t ld) {
-  return act != kSReLU ? make_map_gated(map, x, N, rows, ld) : make_map(map, x, N, rows, ld);
+// Tensor map of a gated input whose gate and up columns alternate in blocks
+// of G (G gate columns, then their G up columns, repeated) as a
+// [rows][N/G][2][G] view.  Its box gathers 128 columns of one kind (gate or
+// up) x 16 rows: {128, 1, 1, 16} when G is a multiple of 128, {G, 1, 128/G,
+// 16} when G is 32 or 64, so the half-tile lands in shared memory as the
+// same dense [16][128] block as with [gate | up] halves.
+moeact_status make_map_ilv(CUtensorMap* map, const void* base, int64_t N, int64_t G,
+                           int64_t rows, int64_t ld) {
+  const cuuint64_t dims[4] = {(cuuint64_t)G, 2, (cuuint64_t)(N / G), (cuuint64_t)rows};
+  const cuuint64_t strides[3] = {(cuuint64_t)(G * 2), (cuuint64_t)(G * 4), (cuuint64_t)(ld * 2)};
+  const cuuint32_t box[4] = {(cuuint32_t)std::min<int64_t>(G, kTileCols), 1,
+                             (cuuint32_t)std::max<int64_t>(1, kTileCols / G),
+                             (cuuint32_t)kHalfRows};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOEACT_OK;
+}
+
+// The backward's map of x: SReLU [rows][N]; gated [rows][2][N] or, with an
+// interleave G, [rows][N/G][2][G].
+moeact_status make_x_map(CUtensorMap* map, int act, const void* x, int64_t N, int ilv,
+                         int64_t rows, int64_t ld) {
+  if (act == kSReLU) return make_map(map, x, N, rows, ld);
+  return ilv ? make_map_ilv(map, x, N, ilv, rows, ld) : make_map_gated(map, x, N, rows, ld);
 }
 
 int64_t grid_for(int64_t slabs_upper, int n_tiles, int threads, int dev) {
@@ -355,9 +384,30 @@ struct ActArgs {
   int staged;        // SwiGLU only
   float alpha;       // ClampedSwiGLU only
   float limit;       // ClampedSwiGLU only
+  int32_t ilv;       // gated: interleave block of gate / up columns (0: halves)
 };
 
-ActArgs plain(int act, int staged = 0) { return {act, staged, 1.0f, INFINITY}; }
+ActArgs plain(int act, int staged = 0, int32_t ilv = 0) {
+  return {act, staged, 1.0f, INFINITY, ilv};
+}
+
+// The interleave of a gated input: 0 ([gate | up] halves), or G columns of
+// gate then G of up, with G = 32, 64 or a multiple of 128 dividing N (G = N
+// is the halves layout).  On success *norm is 0 for halves, else G.
+moeact_status check_ilv(int act, int64_t N, int32_t G, int32_t* norm) {
+  *norm = 0;
+  if (G == 0) return MOEACT_OK;
+  if (act == kSReLU) return fail(MOEACT_EINVAL, "glu_interleave applies to gated activations only");
+  if (G < 0 || G % 32 != 0 || N % G != 0)
+    return fail(MOEACT_EINVAL, "glu_interleave (%d) must be a positive multiple of 32 dividing N",
+                (int)G);
+  if (G == N) return MOEACT_OK;
+  if (G != 32 && G != 64 && G % kTileCols != 0)
+    return fail(MOEACT_EINVAL, "glu_interleave (%d) must be 32, 64 or a multiple of 128",
+                (int)G);
+  *norm = G;
+  return MOEACT_OK;
+}
 
 // Fills the activation-dependent parameters (the sigmoid table to stage and
 // the clamp constants).
@@ -387,6 +437,8 @@ moeact_status fwd_common(const ActArgs& a, const void* x, int64_t ldx, const flo
   if ((st = check_layout(out, M, N))) return st;
   if (staged != 0 && staged != 1) return fail(MOEACT_EINVAL, "staged_rounding must be 0 or 1");
   if (act == kClamped && (st = check_clamp_args(a.alpha, a.limit))) return st;
+  int32_t ilv;
+  if ((st = check_ilv(act, N, a.ilv, &ilv))) return st;
   if (grouped && (st = check_groups(ro, cb, E, status))) return st;
   if (M == 0) return MOEACT_OK;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -399,6 +451,8 @@ moeact_status fwd_common(const ActArgs& a, const void* x, int64_t ldx, const flo
   p.M = M;
   p.N = (int)N;
   p.W = (int)N;
+  p.ilv = ilv;
+  p.up = ilv ? ilv : (int)N;
   p.rq = out.row_codes;
   p.rs = out.row_scales;
   p.cq = out.col_codes;
@@ -414,11 +468,13 @@ moeact_status fwd_common(const ActArgs& a, const void* x, int64_t ldx, const flo
   p.err = g_err_ptr[dev];
   if ((st = act_params(a, dev, cs, p))) return st;
   const int64_t slabs_upper = grouped ? ceil_div(M, 32) + E : ceil_div(M, 32);
-  const int kdirs = dirs | (p.gemm_scales ? kGemm : 0);
+  const int kdirs = dirs | (p.gemm_scales ? kGemm : 0) | (ilv ? kIlv : 0);
   const FwdVariant& v = g_fwd[act][fwd_slot(grouped, act == kSwiGLU && staged, kdirs)];
   if (!v.fn) return fail(MOEACT_EUNSUPPORTED, "no forward kernel for this combination");
   CUtensorMap tx;
-  if ((st = make_map(&tx, x, act != kSReLU ? 2 * N : N, M, ldx))) return st;
+  if (ilv) st = make_map_ilv(&tx, x, N, ilv, M, ldx);
+  else st = make_map(&tx, x, act != kSReLU ? 2 * N : N, M, ldx);
+  if (st) return st;
   const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
   v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(v.sig, grouped, p.E), cs>>>(tx, p);
   const cudaError_t e = cudaGetLastError();
@@ -446,6 +502,8 @@ moeact_status bwd_common(const ActArgs& a, const void* dy, int64_t lddy, const v
   if (dscale && !aligned(dscale, 4)) return fail(MOEACT_EALIGN, "dscale must be 4-byte aligned");
   if (dirs == 0 && !dx && !dscale) return fail(MOEACT_EINVAL, "nothing requested: dirs == 0 and no dx / dscale");
   if (act == kClamped && (st = check_clamp_args(a.alpha, a.limit))) return st;
+  int32_t ilv;
+  if ((st = check_ilv(act, N, a.ilv, &ilv))) return st;
   if (grouped && (st = check_groups(ro, cb, E, status))) return st;
   const size_t ws_need = ws_bytes_needed(M, N);
   if (dscale) {
@@ -466,6 +524,8 @@ moeact_status bwd_common(const ActArgs& a, const void* dy, int64_t lddy, const v
   p.M = M;
   p.N = (int)N;
   p.W = (int)(act != kSReLU ? 2 * N : N);
+  p.ilv = ilv;
+  p.up = ilv ? ilv : (int)N;
   p.rq = out.row_codes;
   p.rs = out.row_scales;
   p.cq = out.col_codes;
@@ -491,7 +551,7 @@ moeact_status bwd_common(const ActArgs& a, const void* dy, int64_t lddy, const v
   const BwdVariant& v = g_bwd[act][bwd_slot(grouped, rr, kdirs)];
   if (!v.fn) return fail(MOEACT_EUNSUPPORTED, "no backward kernel for this combination");
   CUtensorMap tx, tdy;
-  if ((st = make_x_map(&tx, act, x, N, M, ldx))) return st;
+  if ((st = make_x_map(&tx, act, x, N, ilv, M, ldx))) return st;
   if ((st = make_map(&tdy, dy, N, M, lddy))) return st;
   const int64_t blocks = grid_for(slabs_upper, p.n_tiles, v.threads, dev);
   v.fn<<<(unsigned)blocks, v.threads, v.smem_fixed + group_smem(v.sig, grouped, p.E), cs>>>(tx, tdy, p);
@@ -566,9 +626,9 @@ moeact_status splits_to_offsets(const int64_t* m_splits, int32_t num_groups, int
 
 moeact_status scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s, int64_t M,
                                       int64_t N, int dirs, int staged_rounding,
-                                      moeact_mx_out out, void* stream) {
-  return fwd_common(plain(kSwiGLU, staged_rounding), x, ldx, s, M, N, dirs, nullptr, nullptr, 0,
-                    nullptr, out, stream, false);
+                                      int32_t glu_interleave, moeact_mx_out out, void* stream) {
+  return fwd_common(plain(kSwiGLU, staged_rounding, glu_interleave), x, ldx, s, M, N, dirs,
+                    nullptr, nullptr, 0, nullptr, out, stream, false);
 }
 
 moeact_status scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s, int64_t M,
@@ -579,12 +639,13 @@ moeact_status scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
 
 moeact_status grouped_scaled_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                               int64_t M, int64_t N, int dirs,
-                                              int staged_rounding, const int64_t* row_offs,
+                                              int staged_rounding, int32_t glu_interleave,
+                                              const int64_t* row_offs,
                                               const int64_t* colblk_offs, int32_t num_groups,
                                               int32_t* status, moeact_mx_out out,
                                               void* stream) {
-  return fwd_common(plain(kSwiGLU, staged_rounding), x, ldx, s, M, N, dirs, row_offs,
-                    colblk_offs, num_groups, status, out, stream, true);
+  return fwd_common(plain(kSwiGLU, staged_rounding, glu_interleave), x, ldx, s, M, N, dirs,
+                    row_offs, colblk_offs, num_groups, status, out, stream, true);
 }
 
 moeact_status grouped_scaled_srelu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
@@ -603,11 +664,13 @@ size_t scaled_act_mxfp8_bwd_workspace_size(int64_t M, int64_t N, int32_t num_gro
 }
 
 moeact_status scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x, int64_t ldx,
-                                      const float* s, int64_t M, int64_t N, int dirs, void* dx,
-                                      float* dscale, moeact_mx_out out, void* workspace,
-                                      size_t workspace_bytes, void* stream) {
-  return bwd_common(plain(kSwiGLU), dy, lddy, x, ldx, s, M, N, dirs, nullptr, nullptr, 0, nullptr, dx,
-                    dscale, out, workspace, workspace_bytes, stream, false);
+                                      const float* s, int64_t M, int64_t N, int dirs,
+                                      int32_t glu_interleave, void* dx, float* dscale,
+                                      moeact_mx_out out, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  return bwd_common(plain(kSwiGLU, 0, glu_interleave), dy, lddy, x, ldx, s, M, N, dirs, nullptr,
+                    nullptr, 0, nullptr, dx, dscale, out, workspace, workspace_bytes, stream,
+                    false);
 }
 
 moeact_status scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x, int64_t ldx,
@@ -620,13 +683,15 @@ moeact_status scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x
 
 moeact_status grouped_scaled_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
                                               int64_t ldx, const float* s, int64_t M, int64_t N,
-                                              int dirs, const int64_t* row_offs,
+                                              int dirs, int32_t glu_interleave,
+                                              const int64_t* row_offs,
                                               const int64_t* colblk_offs, int32_t num_groups,
                                               int32_t* status, void* dx, float* dscale,
                                               moeact_mx_out out, void* workspace,
                                               size_t workspace_bytes, void* stream) {
-  return bwd_common(plain(kSwiGLU), dy, lddy, x, ldx, s, M, N, dirs, row_offs, colblk_offs, num_groups,
-                    status, dx, dscale, out, workspace, workspace_bytes, stream, true);
+  return bwd_common(plain(kSwiGLU, 0, glu_interleave), dy, lddy, x, ldx, s, M, N, dirs, row_offs,
+                    colblk_offs, num_groups, status, dx, dscale, out, workspace, workspace_bytes,
+                    stream, true);
 }
 
 moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
@@ -653,40 +718,44 @@ moeact_status moeact_init_clamped(float alpha) {
 
 moeact_status scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                               int64_t M, int64_t N, int dirs, float alpha,
-                                              float limit, moeact_mx_out out, void* stream) {
-  return fwd_common({kClamped, 0, alpha, limit}, x, ldx, s, M, N, dirs, nullptr, nullptr, 0,
-                    nullptr, out, stream, false);
+                                              float limit, int32_t glu_interleave,
+                                              moeact_mx_out out, void* stream) {
+  return fwd_common({kClamped, 0, alpha, limit, glu_interleave}, x, ldx, s, M, N, dirs, nullptr,
+                    nullptr, 0, nullptr, out, stream, false);
 }
 
 moeact_status grouped_scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                                       int64_t M, int64_t N, int dirs,
                                                       float alpha, float limit,
+                                                      int32_t glu_interleave,
                                                       const int64_t* row_offs,
                                                       const int64_t* colblk_offs,
                                                       int32_t num_groups, int32_t* status,
                                                       moeact_mx_out out, void* stream) {
-  return fwd_common({kClamped, 0, alpha, limit}, x, ldx, s, M, N, dirs, row_offs, colblk_offs,
-                    num_groups, status, out, stream, true);
+  return fwd_common({kClamped, 0, alpha, limit, glu_interleave}, x, ldx, s, M, N, dirs, row_offs,
+                    colblk_offs, num_groups, status, out, stream, true);
 }
 
 moeact_status scaled_clamped_swiglu_mxfp8_bwd(const void* dy, int64_t lddy, const void* x,
                                               int64_t ldx, const float* s, int64_t M, int64_t N,
-                                              int dirs, float alpha, float limit, void* dx,
-                                              float* dscale, moeact_mx_out out, void* workspace,
+                                              int dirs, float alpha, float limit,
+                                              int32_t glu_interleave, void* dx, float* dscale,
+                                              moeact_mx_out out, void* workspace,
                                               size_t workspace_bytes, void* stream) {
-  return bwd_common({kClamped, 0, alpha, limit}, dy, lddy, x, ldx, s, M, N, dirs, nullptr,
-                    nullptr, 0, nullptr, dx, dscale, out, workspace, workspace_bytes, stream,
-                    false);
+  return bwd_common({kClamped, 0, alpha, limit, glu_interleave}, dy, lddy, x, ldx, s, M, N, dirs,
+                    nullptr, nullptr, 0, nullptr, dx, dscale, out, workspace, workspace_bytes,
+                    stream, false);
 }
 
 moeact_status grouped_scaled_clamped_swiglu_mxfp8_bwd(
     const void* dy, int64_t lddy, const void* x, int64_t ldx, const float* s, int64_t M,
-    int64_t N, int dirs, float alpha, float limit, const int64_t* row_offs,
-    const int64_t* colblk_offs, int32_t num_groups, int32_t* status, void* dx, float* dscale,
-    moeact_mx_out out, void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_common({kClamped, 0, alpha, limit}, dy, lddy, x, ldx, s, M, N, dirs, row_offs,
-                    colblk_offs, num_groups, status, dx, dscale, out, workspace, workspace_bytes,
-                    stream, true);
+    int64_t N, int dirs, float alpha, float limit, int32_t glu_interleave,
+    const int64_t* row_offs, const int64_t* colblk_offs, int32_t num_groups, int32_t* status,
+    void* dx, float* dscale, moeact_mx_out out, void* workspace, size_t workspace_bytes,
+    void* stream) {
+  return bwd_common({kClamped, 0, alpha, limit, glu_interleave}, dy, lddy, x, ldx, s, M, N, dirs,
+                    row_offs, colblk_offs, num_groups, status, dx, dscale, out, workspace,
+                    workspace_bytes, stream, true);
 }
 
 moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream) {
@@ -793,6 +862,6 @@ extern "C" moeact_status scaled_swiglu_mxfp8_bwd_noalloc(
     if (st != MOEACT_OK) return st;
     ws_bytes = kNoAllocScratchBytes;
   }
-  return scaled_swiglu_mxfp8_bwd(dy, lddy, x, ldx, s, M, N, dirs, dx, dscale, out, ws, ws_bytes,
-                                 stream);
+  return scaled_swiglu_mxfp8_bwd(dy, lddy, x, ldx, s, M, N, dirs, 0, dx, dscale, out, ws,
+                                 ws_bytes, stream);
 }

@@ -228,6 +228,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, int x, int z, int w,
+                                            int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];"
+      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(z), "r"(w),
+        "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- warp butterflies
 // "Transposed" butterfly: each lane holds one value per row for 2*HALF rows;
 // after the step it holds HALF partial reductions, over lanes {l, l ^ off},

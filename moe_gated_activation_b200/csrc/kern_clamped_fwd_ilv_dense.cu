@@ -1,0 +1,7 @@
+// Instantiates every dense fused forward kernel of ClampedSwiGLU for an input whose
+// gate and up columns are interleaved in blocks (see variants.cuh).
+#include "variants.cuh"
+
+namespace moeact {
+void fill_fwd_clamped_ilv_dense(FwdVariant* t) { fill_fwd<kClamped, false, false, true>(t); }
+}  // namespace moeact

@@ -1,0 +1,7 @@
+// Instantiates every grouped fused forward kernel of SwiGLU for an input whose
+// gate and up columns are interleaved in blocks (see variants.cuh).
+#include "variants.cuh"
+
+namespace moeact {
+void fill_fwd_swiglu_ilv_grouped(FwdVariant* t) { fill_fwd<kSwiGLU, true, true, true>(t); }
+}  // namespace moeact

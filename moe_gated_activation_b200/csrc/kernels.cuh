@@ -46,6 +46,10 @@ constexpr int kCol = 2;
 // tiled layout (a compile-time choice, so the row-major kernels carry none of
 // its code).
 constexpr int kGemm = 4;
+// Forward template flag in the DIRS bits: gate and up interleaved in blocks
+// (loads through a 4-D map), so the halves layout's forward keeps its own
+// instantiation, untouched by the interleaved load code.
+constexpr int kIlv = 8;
 constexpr int kTileCols = 128;   // columns of a warp-tile (4 per lane)
 
 __host__ __device__ constexpr int sig_slot(int i) {
@@ -83,6 +87,11 @@ struct Params {
   float clamp_alpha;
   float clamp_sigL;
   const int32_t* noop;   // nullable: a non-zero flag makes the call write nothing
+  // Gated layouts of x and dX (width 2N): ilv == 0 is [gate | up] halves;
+  // ilv = G > 0 is G gate columns, then the G matching up columns, repeated.
+  // up = the stored distance from a gate column to its up column (N or G).
+  int ilv;
+  int up;
   uint32_t* err;      // device error word (timeouts), never expected to be set
 };
 
@@ -260,7 +269,8 @@ struct Ring {
   int k_issue;       // next half-tile to issue
 };
 
-template <int OPS, int SLOTS, bool GROUPED>
+// FWD_ILV: a forward whose input interleaves gate and up in blocks (kIlv).
+template <int OPS, int SLOTS, bool GROUPED, bool FWD_ILV = false>
 __device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
                                            Ring<OPS, SLOTS>& r, const void* tm_x,
                                            const void* tm_dy) {
@@ -282,11 +292,22 @@ __device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
     // lanes of a tile, including those past N.  SReLU's map is 2-D, [rows][N].
     tma_load_2d(dst, tm_dy, x, y, bar);
     if (OPS == 3) {
-      tma_load_3d(dst + kOpHalfBytes, tm_x, x, 0, y, bar);
-      tma_load_3d(dst + 2 * kOpHalfBytes, tm_x, x, 1, y, bar);
+      if (p.ilv) {
+        tma_load_4d(dst + kOpHalfBytes, tm_x, x % p.ilv, 0, x / p.ilv, y, bar);
+        tma_load_4d(dst + 2 * kOpHalfBytes, tm_x, x % p.ilv, 1, x / p.ilv, y, bar);
+      } else {
+        tma_load_3d(dst + kOpHalfBytes, tm_x, x, 0, y, bar);
+        tma_load_3d(dst + 2 * kOpHalfBytes, tm_x, x, 1, y, bar);
+      }
     } else {
       tma_load_2d(dst + kOpHalfBytes, tm_x, x, y, bar);
     }
+  } else if (FWD_ILV) {
+    // forward, interleaved gate / up blocks: a 4-D map [rows][N/G][2][G]
+    // whose box gathers the tile's 128 gate (then up) columns into the same
+    // dense [16][128] half-tile as the 2-D case
+    tma_load_4d(dst, tm_x, x % p.ilv, 0, x / p.ilv, y, bar);
+    tma_load_4d(dst + kOpHalfBytes, tm_x, x % p.ilv, 1, x / p.ilv, y, bar);
   } else {
     // forward: gate, then up (SwiGLU) from a 2-D [rows][width] map, width 2N
     // for SwiGLU (measured faster than the 3-D map).  In a ragged last column
@@ -385,6 +406,54 @@ __device__ __forceinline__ uint32_t gather_row_scales(uint32_t w0, uint32_t w1, 
     v |= (((lane < 16 ? a : b) >> sh) & 0xFFu) << (8 * k);
   }
   return v;
+}
+
+// Stored column, in a gated tensor of width 2N (x, dX and the MXFP8 of dX),
+// of gate column c; its up column is `p.up` further on.  [gate | up] halves
+// (ilv == 0) keep c; interleaved blocks of G put it at (c / G) 2G + c % G.
+__device__ __forceinline__ int glu_col(const Params& p, int c) {
+  return p.ilv ? (c / p.ilv) * 2 * p.ilv + c % p.ilv : c;
+}
+
+// Row scales of row `row` of a backward tile: vg / vu hold the E8M0 bytes of
+// the tile's four dgate / dup blocks (block 0 in the low byte), nb of which
+// exist.  With [gate | up] halves or an interleave of 128 columns or more,
+// each set of four stays adjacent (dup's `p.up` columns after dgate's); an
+// interleave of 32 or 64 columns alternates them within the 8 adjacent scale
+// bytes of the tile's 256 stored columns.
+template <int ACT, int DIRS>
+__device__ __forceinline__ void store_bwd_row_scales(const Params& p, int64_t row, int tile,
+                                                     uint32_t vg, uint32_t vu, int nb) {
+  const int W = p.W;
+  if (ACT == kSReLU || p.ilv == 0 || p.ilv >= kTileCols) {
+    const int sc = glu_col(p, tile * kTileCols);   // stored column of the tile's dgate
+    if (DIRS & kGemm) {
+      const int nct = W >> 7;
+      __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row, sc >> 7, nct)), vg);
+      if (ACT != kSReLU)
+        __stcs(reinterpret_cast<unsigned int*>(
+                   p.rs + gemm_row_scales_off(row, (sc + p.up) >> 7, nct)), vu);
+    } else {
+      uint8_t* rsr = p.rs + row * (int64_t)(W / 32) + sc / 32;
+      store_scales4(rsr, vg, nb);
+      if (ACT != kSReLU) store_scales4(rsr + p.up / 32, vu, nb);
+    }
+  } else {
+    // G = 32: g0 u0 g1 u1 | g2 u2 g3 u3;  G = 64: g0 g1 u0 u1 | g2 g3 u2 u3
+    const bool g32 = p.ilv == 32;
+    const uint32_t w0 = __byte_perm(vg, vu, g32 ? 0x5140 : 0x5410);
+    const uint32_t w1 = __byte_perm(vg, vu, g32 ? 0x7362 : 0x7632);
+    if (DIRS & kGemm) {
+      const int nct = W >> 7;
+      __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row, 2 * tile, nct)), w0);
+      __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row, 2 * tile + 1, nct)),
+             w1);
+    } else {
+      uint8_t* rsr = p.rs + row * (int64_t)(W / 32) + 8 * tile;
+      store_scales4(rsr, w0, min(4, 2 * nb));
+      if (nb > 2) store_scales4(rsr + 4, w1, 2 * nb - 4);
+    }
+  }
 }
 
 // ------------------------------------------------------------- ClampedSwiGLU
@@ -520,7 +589,8 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
     }
     // the slot is consumed: refill it with the half-tile SLOTS ahead
     __syncwarp();
-    if (lane == 0 && ring.k_issue < K) ring_issue<OPS, SLOTS, GROUPED>(p, m, ring, tm_x, nullptr);
+    if (lane == 0 && ring.k_issue < K)
+      ring_issue<OPS, SLOTS, GROUPED, (DIRS & kIlv) != 0>(p, m, ring, tm_x, nullptr);
     if (DIRS & kRow) {
       uint32_t A[16];
 #pragma unroll
@@ -592,14 +662,15 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
 }
 
 // Sets up the warp's ring (barriers initialised by lane 0) and primes it.
-template <int OPS, int SLOTS, bool GROUPED>
+template <int OPS, int SLOTS, bool GROUPED, bool FWD_ILV = false>
 __device__ __forceinline__ void ring_prime(const Params& p, const Smem& m, Ring<OPS, SLOTS>& r,
                                            const void* tm_x, const void* tm_dy, int K,
                                            int lane) {
   if (lane == 0) {
     for (int i = 0; i < SLOTS; ++i) mbar_init(r.bars + i, 1);
     mbar_init_fence();
-    while (r.k_issue < K && r.k_issue < SLOTS) ring_issue<OPS, SLOTS, GROUPED>(p, m, r, tm_x, tm_dy);
+    while (r.k_issue < K && r.k_issue < SLOTS)
+      ring_issue<OPS, SLOTS, GROUPED, FWD_ILV>(p, m, r, tm_x, tm_dy);
   }
   __syncwarp();
 }
@@ -630,7 +701,7 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
   ring.k_issue = 0;
   ring.row0 = 0;
   if (count > 0) ring.cur.init(first, stride, p.n_tiles);
-  ring_prime<C::kOps, C::kSlots, GROUPED>(p, m, ring, &tm_x, nullptr, K, lane);
+  ring_prime<C::kOps, C::kSlots, GROUPED, (DIRS & kIlv) != 0>(p, m, ring, &tm_x, nullptr, K, lane);
   if (C::kSig && !mbar_wait(sig_bar, 0u)) {
     if (lane == 0) {
       report_timeout(p, 4u);
@@ -749,12 +820,13 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
   const int Wq = W >> 2;   // code row stride in 32-bit words
   const int c0 = tile * kTileCols + 4 * lane;
   const bool colok = c0 < N;
+  const int cs0 = glu_col(p, c0), Uq = p.up >> 2;   // stored column; up offset in words
 
   uint32_t DG[32][2], DU[32][2];
   float ph[2];
   uint32_t bh[2];
-  unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + c0);
-  uint2* dxb = reinterpret_cast<uint2*>(p.dx + row0 * (int64_t)W + c0);
+  unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + cs0);
+  uint2* dxb = reinterpret_cast<uint2*>(p.dx + row0 * (int64_t)W + cs0);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int k = k0 + h;
@@ -811,7 +883,7 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
                   : 0.0f;
       if (p.dx != nullptr && (FULL || (colok && r < nrows))) {
         __stcs(dxb + r * Wq, make_uint2(DG[r][0], DG[r][1]));
-        if (ACT != kSReLU) __stcs(dxb + r * Wq + (N >> 2), make_uint2(DU[r][0], DU[r][1]));
+        if (ACT != kSReLU) __stcs(dxb + r * Wq + Uq, make_uint2(DU[r][0], DU[r][1]));
       }
     }
     __syncwarp();
@@ -859,7 +931,7 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
         }
         if (FULL || (colok && r < nrows)) {
           __stcs(rqb + r * Wq, qg);
-          if (ACT != kSReLU) __stcs(rqb + r * Wq + (N >> 2), qu);
+          if (ACT != kSReLU) __stcs(rqb + r * Wq + Uq, qu);
         }
       }
     }
@@ -873,21 +945,9 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
     // lane l stores the block scales of row l (dgate blocks, then dup blocks)
     const uint32_t vg = gather_row_scales(bh[0], bh[1], lane, 0, 2);
     const uint32_t vu = gather_row_scales(bh[0], bh[1], lane, 1, 3);
-    if (lane < nrows) {
-      const int nb = min(4, (N - tile * kTileCols) / 32);
-      if (DIRS & kGemm) {
-        const int nct = W >> 7;
-        __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row0 + lane, tile, nct)),
-               vg);
-        if (ACT != kSReLU)
-          __stcs(reinterpret_cast<unsigned int*>(
-                     p.rs + gemm_row_scales_off(row0 + lane, (N >> 7) + tile, nct)), vu);
-      } else {
-        uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
-        store_scales4(rsr, vg, nb);
-        if (ACT != kSReLU) store_scales4(rsr + N / 32, vu, nb);
-      }
-    }
+    if (lane < nrows)
+      store_bwd_row_scales<ACT, DIRS>(p, row0 + lane, tile, vg, vu,
+                                      min(4, (N - tile * kTileCols) / 32));
   }
   if (DIRS & kCol) {
     uint32_t ag[2] = {0u, 0u}, au[2] = {0u, 0u};
@@ -918,19 +978,20 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
         gemm_col_geom<GROUPED>(p, m, slab, base, j, kt);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          p.cs[gemm_col_scale_off(base, c0 + c, j, kt)] = (uint8_t)bg[c];
-          if (ACT != kSReLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
+          p.cs[gemm_col_scale_off(base, cs0 + c, j, kt)] = (uint8_t)bg[c];
+          if (ACT != kSReLU)
+            p.cs[gemm_col_scale_off(base, cs0 + p.up + c, j, kt)] = (uint8_t)bu[c];
         }
       } else {
-        uint8_t* csr = p.cs + slab * (int64_t)W + c0;
+        uint8_t* csr = p.cs + slab * (int64_t)W + cs0;
         __stcs(reinterpret_cast<unsigned int*>(csr),
                bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
         if (ACT != kSReLU)
-          __stcs(reinterpret_cast<unsigned int*>(csr + N),
+          __stcs(reinterpret_cast<unsigned int*>(csr + p.up),
                  bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
       }
     }
-    unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
+    unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + cs0);
     const int Wqc = opaque(Wq);
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
@@ -941,7 +1002,7 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
         if (ACT != kSReLU) {
           const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(DU[r][0]), mu[0], mu[1]) |
                               (e4m3x2_2(bf16x2_to_f2_p(DU[r][1]), mu[2], mu[3]) << 16);
-          __stcs(qb + r * Wqc + (N >> 2), qu);
+          __stcs(qb + r * Wqc + Uq, qu);
         }
       }
     }
@@ -964,10 +1025,9 @@ __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
                                             unsigned int* rqb, uint2* dxb, const void* tm_x,
                                             const void* tm_dy, float& ph, uint32_t& bh,
                                             uint32_t (&acg)[2], uint32_t (&acu)[2]) {
-  const int N = p.N;
   // per-half copies the compiler cannot hoist out of the (rolled) half loop,
   // so that the 16 row offsets are not kept live across it
-  const int Wqh = opaque(Wq), Nq = opaque(N >> 2);
+  const int Wqh = opaque(Wq), Nq = opaque(p.up >> 2);
   const int nrh = nrows - 16 * h;   // rows of this half that exist
   const int k = k0 + h;
   const int slot = k % SLOTS;
@@ -1054,7 +1114,7 @@ __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
 // flight while the current one is quantized and stored, so one load latency
 // per tile is exposed instead of one per chunk.
 template <int ACT, bool FULL>
-__device__ __forceinline__ void bwd_colwise_load8(int q, int N, int nrows, bool colok, int Wqc,
+__device__ __forceinline__ void bwd_colwise_load8(int q, int U, int nrows, bool colok, int Wqc,
                                                   const uint2* dxb, uint2 (&RG)[8],
                                                   uint2 (&RU)[8]) {
 #pragma unroll
@@ -1062,12 +1122,12 @@ __device__ __forceinline__ void bwd_colwise_load8(int q, int N, int nrows, bool 
     const int r = 8 * q + i;
     const bool ok = FULL || (colok && r < nrows);
     RG[i] = ok ? __ldcg(dxb + r * Wqc) : make_uint2(0u, 0u);
-    if (ACT != kSReLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (N >> 2)) : make_uint2(0u, 0u);
+    if (ACT != kSReLU) RU[i] = ok ? __ldcg(dxb + r * Wqc + (U >> 2)) : make_uint2(0u, 0u);
   }
 }
 
 template <int ACT, bool FULL>
-__device__ __forceinline__ void bwd_colwise_store8(int q, int N, int nrows, bool colok, int Wqc,
+__device__ __forceinline__ void bwd_colwise_store8(int q, int U, int nrows, bool colok, int Wqc,
                                                    unsigned int* qb, const uint2 (&RG)[8],
                                                    const uint2 (&RU)[8], const uint32_t (&mg)[4],
                                                    const uint32_t (&mu)[4]) {
@@ -1081,24 +1141,37 @@ __device__ __forceinline__ void bwd_colwise_store8(int q, int N, int nrows, bool
       if (ACT != kSReLU) {
         const uint32_t qu = e4m3x2_2(bf16x2_to_f2_p(RU[i].x), mu[0], mu[1]) |
                             (e4m3x2_2(bf16x2_to_f2_p(RU[i].y), mu[2], mu[3]) << 16);
-        __stcs(qb + r * Wqc + (N >> 2), qu);
+        __stcs(qb + r * Wqc + (U >> 2), qu);
       }
     }
   }
 }
 
 template <int ACT, bool FULL>
-__device__ __forceinline__ void bwd_colwise_rr(int N, int nrows, bool colok, int Wqc,
+__device__ __forceinline__ void bwd_colwise_rr(int U, int nrows, bool colok, int Wqc,
                                                const uint2* dxb, unsigned int* qb,
                                                const uint32_t (&mg)[4], const uint32_t (&mu)[4]) {
   uint2 AG[8], AU[8], BG[8], BU[8];
-  bwd_colwise_load8<ACT, FULL>(0, N, nrows, colok, Wqc, dxb, AG, AU);
+  if (ACT == kClamped) {
+    // ClampedSwiGLU's larger row body leaves fewer registers: 16 rows at a
+    // time, loads first, nothing carried across the loop (the overlapped
+    // form below spills there and measured slower)
+#pragma unroll 1
+    for (int q = 0; q < 4; q += 2) {
+      bwd_colwise_load8<ACT, FULL>(q, U, nrows, colok, Wqc, dxb, AG, AU);
+      bwd_colwise_load8<ACT, FULL>(q + 1, U, nrows, colok, Wqc, dxb, BG, BU);
+      bwd_colwise_store8<ACT, FULL>(q, U, nrows, colok, Wqc, qb, AG, AU, mg, mu);
+      bwd_colwise_store8<ACT, FULL>(q + 1, U, nrows, colok, Wqc, qb, BG, BU, mg, mu);
+    }
+    return;
+  }
+  bwd_colwise_load8<ACT, FULL>(0, U, nrows, colok, Wqc, dxb, AG, AU);
 #pragma unroll 1
   for (int q = 0; q < 4; q += 2) {
-    bwd_colwise_load8<ACT, FULL>(q + 1, N, nrows, colok, Wqc, dxb, BG, BU);
-    bwd_colwise_store8<ACT, FULL>(q, N, nrows, colok, Wqc, qb, AG, AU, mg, mu);
-    if (q + 2 < 4) bwd_colwise_load8<ACT, FULL>(q + 2, N, nrows, colok, Wqc, dxb, AG, AU);
-    bwd_colwise_store8<ACT, FULL>(q + 1, N, nrows, colok, Wqc, qb, BG, BU, mg, mu);
+    bwd_colwise_load8<ACT, FULL>(q + 1, U, nrows, colok, Wqc, dxb, BG, BU);
+    bwd_colwise_store8<ACT, FULL>(q, U, nrows, colok, Wqc, qb, AG, AU, mg, mu);
+    if (q + 2 < 4) bwd_colwise_load8<ACT, FULL>(q + 2, U, nrows, colok, Wqc, dxb, AG, AU);
+    bwd_colwise_store8<ACT, FULL>(q + 1, U, nrows, colok, Wqc, qb, BG, BU, mg, mu);
   }
 }
 
@@ -1111,11 +1184,12 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
   const int Wq = W >> 2;   // row stride in 32-bit words (codes) / 8-byte words (dx)
   const int c0 = tile * kTileCols + 4 * lane;
   const bool colok = c0 < N;
+  const int cs0 = glu_col(p, c0);   // stored column of the lane's first dgate column
   float ph[2] = {0.0f, 0.0f};
   uint32_t bh[2] = {0u, 0u};
   uint32_t acg[2] = {0u, 0u}, acu[2] = {0u, 0u};   // colwise maxima (packed bf16 magnitudes)
-  unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + c0);
-  uint2* dxb = reinterpret_cast<uint2*>(p.dx + row0 * (int64_t)W + c0);
+  unsigned int* rqb = reinterpret_cast<unsigned int*>(p.rq + row0 * (int64_t)W + cs0);
+  uint2* dxb = reinterpret_cast<uint2*>(p.dx + row0 * (int64_t)W + cs0);
   // one copy of the half body (only scalars cross the halves): half the code
   // for the instruction cache to hold.  Measured faster than two unrolled
   // copies at every size, most of all when each warp sees only a few tiles
@@ -1139,21 +1213,9 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
   if (DIRS & kRow) {
     const uint32_t vg = gather_row_scales(bh[0], bh[1], lane, 0, 2);
     const uint32_t vu = gather_row_scales(bh[0], bh[1], lane, 1, 3);
-    if (lane < nrows) {
-      const int nb = min(4, (N - tile * kTileCols) / 32);
-      if (DIRS & kGemm) {
-        const int nct = W >> 7;
-        __stcs(reinterpret_cast<unsigned int*>(p.rs + gemm_row_scales_off(row0 + lane, tile, nct)),
-               vg);
-        if (ACT != kSReLU)
-          __stcs(reinterpret_cast<unsigned int*>(
-                     p.rs + gemm_row_scales_off(row0 + lane, (N >> 7) + tile, nct)), vu);
-      } else {
-        uint8_t* rsr = p.rs + (row0 + lane) * (int64_t)(W / 32) + 4 * tile;
-        store_scales4(rsr, vg, nb);
-        if (ACT != kSReLU) store_scales4(rsr + N / 32, vu, nb);
-      }
-    }
+    if (lane < nrows)
+      store_bwd_row_scales<ACT, DIRS>(p, row0 + lane, tile, vg, vu,
+                                      min(4, (N - tile * kTileCols) / 32));
   }
   if (DIRS & kCol) {
     uint32_t bg[4], bu[4], mg[4], mu[4];
@@ -1176,21 +1238,22 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
         gemm_col_geom<GROUPED>(p, m, slab, base, j, kt);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          p.cs[gemm_col_scale_off(base, c0 + c, j, kt)] = (uint8_t)bg[c];
-          if (ACT != kSReLU) p.cs[gemm_col_scale_off(base, N + c0 + c, j, kt)] = (uint8_t)bu[c];
+          p.cs[gemm_col_scale_off(base, cs0 + c, j, kt)] = (uint8_t)bg[c];
+          if (ACT != kSReLU)
+            p.cs[gemm_col_scale_off(base, cs0 + p.up + c, j, kt)] = (uint8_t)bu[c];
         }
       } else {
-        uint8_t* csr = p.cs + slab * (int64_t)W + c0;
+        uint8_t* csr = p.cs + slab * (int64_t)W + cs0;
         __stcs(reinterpret_cast<unsigned int*>(csr),
                bg[0] | (bg[1] << 8) | (bg[2] << 16) | (bg[3] << 24));
         if (ACT != kSReLU)
-          __stcs(reinterpret_cast<unsigned int*>(csr + N),
+          __stcs(reinterpret_cast<unsigned int*>(csr + p.up),
                  bu[0] | (bu[1] << 8) | (bu[2] << 16) | (bu[3] << 24));
       }
     }
-    unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + c0);
+    unsigned int* qb = reinterpret_cast<unsigned int*>(p.cq + row0 * (int64_t)W + cs0);
     const int Wqc = opaque(Wq);
-    bwd_colwise_rr<ACT, FULL>(N, nrows, colok, Wqc, dxb, qb, mg, mu);
+    bwd_colwise_rr<ACT, FULL>(p.up, nrows, colok, Wqc, dxb, qb, mg, mu);
   }
 }
 

@@ -14,11 +14,13 @@ using BwdFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
 struct FwdVariant { FwdFn fn; int threads; int smem_fixed; bool sig; };
 struct BwdVariant { BwdFn fn; int threads; int smem_fixed; bool sig; };
 
-// Table slots: forward by (grouped, staged, dirs | layout), backward by
-// (grouped, dX re-read, dirs | layout); kdirs = ROWWISE/COLWISE bits | kGemm.
-constexpr int kVariantSlots = 32;
+// Table slots: forward by (grouped, staged, dirs | layout | interleave),
+// backward by (grouped, dX re-read, dirs | layout); kdirs = ROWWISE/COLWISE
+// bits | kGemm (| kIlv, forward only).
+constexpr int kFwdSlots = 64;
+constexpr int kBwdSlots = 32;
 inline int fwd_slot(bool grouped, bool staged, int kdirs) {
-  return ((grouped ? 2 : 0) + (staged ? 1 : 0)) * 8 + kdirs;
+  return ((grouped ? 2 : 0) + (staged ? 1 : 0)) * 16 + kdirs;
 }
 inline int bwd_slot(bool grouped, bool reread, int kdirs) {
   return ((grouped ? 2 : 0) + (reread ? 1 : 0)) * 8 + kdirs;
@@ -39,16 +41,17 @@ void put_bwd(BwdVariant* t) {
 }
 
 // Every forward variant of one activation, dense or grouped (STAGED: also
-// the staged-rounding ones).
-template <int ACT, bool STAGED, bool GROUPED>
+// the staged-rounding ones; ILV: the interleaved gate / up input's).
+template <int ACT, bool STAGED, bool GROUPED, bool ILV = false>
 void fill_fwd(FwdVariant* t) {
+  constexpr int I = ILV ? kIlv : 0;
 #define MOEACT_FWD_DIRS(ST, G)                              \
-  put_fwd<ACT, kRow, ST, G>(t);                             \
-  put_fwd<ACT, kCol, ST, G>(t);                             \
-  put_fwd<ACT, kRow | kCol, ST, G>(t);                      \
-  put_fwd<ACT, kRow | kGemm, ST, G>(t);                     \
-  put_fwd<ACT, kCol | kGemm, ST, G>(t);                     \
-  put_fwd<ACT, kRow | kCol | kGemm, ST, G>(t);
+  put_fwd<ACT, I | kRow, ST, G>(t);                         \
+  put_fwd<ACT, I | kCol, ST, G>(t);                         \
+  put_fwd<ACT, I | kRow | kCol, ST, G>(t);                  \
+  put_fwd<ACT, I | kRow | kGemm, ST, G>(t);                 \
+  put_fwd<ACT, I | kCol | kGemm, ST, G>(t);                 \
+  put_fwd<ACT, I | kRow | kCol | kGemm, ST, G>(t);
   MOEACT_FWD_DIRS(false, GROUPED)
   if constexpr (STAGED) {
     MOEACT_FWD_DIRS(true, GROUPED)
@@ -72,10 +75,14 @@ void fill_bwd(BwdVariant* t) {
 #undef MOEACT_BWD_DIRS
 }
 
-// Defined in kern_<activation>_<pass>_<dense|grouped>.cu; each fills its
-// entries of a kVariantSlots table (unused slots stay zero).
+// Defined in kern_<activation>_<pass>[_ilv]_<dense|grouped>.cu; each fills
+// its entries of a kFwdSlots / kBwdSlots table (unused slots stay zero).
 void fill_fwd_swiglu_dense(FwdVariant* t);
 void fill_fwd_swiglu_grouped(FwdVariant* t);
+void fill_fwd_swiglu_ilv_dense(FwdVariant* t);
+void fill_fwd_swiglu_ilv_grouped(FwdVariant* t);
+void fill_fwd_clamped_ilv_dense(FwdVariant* t);
+void fill_fwd_clamped_ilv_grouped(FwdVariant* t);
 void fill_bwd_swiglu_dense(BwdVariant* t);
 void fill_bwd_swiglu_grouped(BwdVariant* t);
 void fill_fwd_srelu_dense(FwdVariant* t);

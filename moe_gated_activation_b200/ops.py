@@ -98,6 +98,15 @@ def _mx_result(rq, rs, cq, cs, col_rows_view=None):
     return MXFP8(rq.view(torch.float8_e4m3fn), cq.view(torch.float8_e4m3fn), rs, cs)
 
 
+def _ilv(glu_interleave, gated):
+    """The glu_interleave argument: 0 for [gate | up] halves, else the block
+    size G of interleaved gate / up columns (gated activations only)."""
+    g = 0 if glu_interleave is None else int(glu_interleave)
+    if g and not gated:
+        raise ValueError("glu_interleave applies to gated activations only")
+    return g
+
+
 # ------------------------------------------------------------------ offsets
 def splits_to_offsets(m_splits: torch.Tensor, total_rows: int):
     """(row_offs, colblk_offs, status) int64/int64/int32 device tensors for the
@@ -117,7 +126,7 @@ def splits_to_offsets(m_splits: torch.Tensor, total_rows: int):
 
 # ------------------------------------------------------------------ forward
 def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False, clamp=None,
-         noop_flag=None):
+         noop_flag=None, glu_interleave=0):
     swiglu = act != "srelu"        # gated: x = [gate | up]
     if N is None:
         N = x.shape[1] // 2 if swiglu else x.shape[1]
@@ -134,24 +143,25 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
     mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales, noop_flag)
     stream = _stream(x.device)
     ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
+    ilv = _ilv(glu_interleave, swiglu)
     if act == "clamped":
         alpha, limit = clamp
         if grouped is None:
             _capi.call("scaled_clamped_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs,
-                       alpha, limit, mx, stream)
+                       alpha, limit, ilv, mx, stream)
         else:
             _capi.call("grouped_scaled_clamped_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N,
-                       dirs, alpha, limit, _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
+                       dirs, alpha, limit, ilv, _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
     elif grouped is None:
         if swiglu:
             _capi.call("scaled_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs, int(staged),
-                       mx, stream)
+                       ilv, mx, stream)
         else:
             _capi.call("scaled_srelu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs, mx, stream)
     else:
         if swiglu:
             _capi.call("grouped_scaled_swiglu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs,
-                       int(staged), _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
+                       int(staged), ilv, _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
         else:
             _capi.call("grouped_scaled_srelu_mxfp8_fwd", _ptr(x), ldx, _ptr(s), M, N, dirs,
                        _ptr(ro), _ptr(cb), E, _ptr(st), mx, stream)
@@ -159,12 +169,15 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
 
 
 def scaled_swiglu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, staged_rounding=False, N=None,
-                            gemm_scales=False, noop_flag=None):
+                            gemm_scales=False, noop_flag=None, glu_interleave=None):
     """MXFP8 of SwiGLU(x) * s; x bf16 [M, >=2N] packs [gate | up].
     gemm_scales: scales in the GEMM-ready tiled layout (moeact.h,
-    MOEACT_SCALES_GEMM; M and N multiples of 128)."""
+    MOEACT_SCALES_GEMM; M and N multiples of 128).
+    glu_interleave: G > 0 reads x as G gate columns, then their G up
+    columns, repeated (G = 32, 64 or a multiple of 128 dividing N); the
+    backward writes dx and its MXFP8 in the same column order."""
     return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, gemm_scales=gemm_scales,
-                noop_flag=noop_flag)
+                noop_flag=noop_flag, glu_interleave=glu_interleave)
 
 
 def scaled_srelu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, N=None, gemm_scales=False,
@@ -183,14 +196,16 @@ def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
 
 def grouped_scaled_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
                                     staged_rounding=False, status=None, col_scale_rows=None,
-                                    N=None, gemm_scales=False, noop_flag=None):
+                                    N=None, gemm_scales=False, noop_flag=None,
+                                    glu_interleave=None):
     """Grouped forward: experts own the rows given by `row_offs` (from
     splits_to_offsets).  Returns (MXFP8, status).  Col scales hold
     ceil(M/32) + E rows unless `col_scale_rows` (sum of ceil(m_e/32), known on
     the host) is given."""
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, g,
-                gemm_scales=gemm_scales, noop_flag=noop_flag), status
+                gemm_scales=gemm_scales, noop_flag=noop_flag,
+                glu_interleave=glu_interleave), status
 
 
 def grouped_scaled_srelu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
@@ -223,7 +238,7 @@ def _workspace(device, nbytes):
 
 
 def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, grouped=None,
-         gemm_scales=False, clamp=None, noop_flag=None):
+         gemm_scales=False, clamp=None, noop_flag=None, glu_interleave=0):
     swiglu = act != "srelu"        # gated: x = [gate | up], W = 2N
     if N is None:
         N = dy.shape[1]
@@ -254,8 +269,10 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
     lddy = dy.stride(0) if M > 1 else max(dy.stride(0), dy.shape[1])
     common = (_ptr(dy), lddy, _ptr(x), ldx, _ptr(s), M, N, dirs)
     tail = (mx, _ptr(ws), ws.numel() if ws is not None else 0, stream)
+    if swiglu:
+        clamp_args = tuple(clamp) if act == "clamped" else ()
+        common = common + clamp_args + (_ilv(glu_interleave, True),)
     if act == "clamped":
-        common = common + tuple(clamp)
         if grouped is None:
             _capi.call("scaled_clamped_swiglu_mxfp8_bwd", *common, _ptr(dx), _ptr(dscale), *tail)
         else:
@@ -272,10 +289,11 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
 
 def scaled_swiglu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
                             want_dscale=True, workspace=None, N=None, gemm_scales=False,
-                            noop_flag=None):
+                            noop_flag=None, glu_interleave=None):
     """Backward of the scaled SwiGLU: MXFP8 of [dgate | dup], bf16 dx, fp32 dscale."""
     return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales, noop_flag=noop_flag)
+                gemm_scales=gemm_scales, noop_flag=noop_flag,
+                glu_interleave=glu_interleave)
 
 
 def scaled_srelu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
@@ -288,10 +306,11 @@ def scaled_srelu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True
 def grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
                                     colwise=True, want_dx=True, want_dscale=True,
                                     workspace=None, status=None, col_scale_rows=None, N=None,
-                                    gemm_scales=False, noop_flag=None):
+                                    gemm_scales=False, noop_flag=None, glu_interleave=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                g, gemm_scales=gemm_scales, noop_flag=noop_flag), status
+                g, gemm_scales=gemm_scales, noop_flag=noop_flag,
+                glu_interleave=glu_interleave), status
 
 
 def grouped_scaled_srelu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
@@ -310,26 +329,31 @@ CLAMPED_LIMIT = 7.0
 
 def scaled_clamped_swiglu_mxfp8_fwd(x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
                                     rowwise=True, colwise=True, N=None, gemm_scales=False,
-                                    noop_flag=None):
+                                    noop_flag=None, glu_interleave=None):
     """MXFP8 of ClampedSwiGLU(x) * s (moeact.h); x bf16 [M, >=2N] packs [gate | up]."""
     return _fwd("clamped", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales,
-                clamp=(alpha, limit), noop_flag=noop_flag)
+                clamp=(alpha, limit), noop_flag=noop_flag,
+                glu_interleave=glu_interleave)
 
 
 def grouped_scaled_clamped_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, alpha=CLAMPED_ALPHA,
                                             limit=CLAMPED_LIMIT, rowwise=True, colwise=True,
                                             status=None, col_scale_rows=None, N=None,
-                                            gemm_scales=False, noop_flag=None):
+                                            gemm_scales=False, noop_flag=None,
+                                            glu_interleave=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _fwd("clamped", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales,
-                clamp=(alpha, limit), noop_flag=noop_flag), status
+                clamp=(alpha, limit), noop_flag=noop_flag,
+                glu_interleave=glu_interleave), status
 
 
 def scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
                                     rowwise=True, colwise=True, want_dx=True, want_dscale=True,
-                                    workspace=None, N=None, gemm_scales=False, noop_flag=None):
+                                    workspace=None, N=None, gemm_scales=False, noop_flag=None,
+                                    glu_interleave=None):
     return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag)
+                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag,
+                glu_interleave=glu_interleave)
 
 
 def grouped_scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *,
@@ -337,10 +361,11 @@ def grouped_scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *,
                                             rowwise=True, colwise=True, want_dx=True,
                                             want_dscale=True, workspace=None, status=None,
                                             col_scale_rows=None, N=None, gemm_scales=False,
-                                            noop_flag=None):
+                                            noop_flag=None, glu_interleave=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, g,
-                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag), status
+                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag,
+                glu_interleave=glu_interleave), status
 
 
 def init_clamped(alpha=CLAMPED_ALPHA):

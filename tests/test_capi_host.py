@@ -54,8 +54,8 @@ MX_ROW = _capi.MxOut(A16, A16, None, None)
 MX_BOTH = _capi.MxOut(A16, A16, A16, A16)
 
 
-def fwd(lib, x=A16, ldx=512, s=A16, M=64, N=256, dirs=1, staged=0, mx=MX_ROW):
-    return lib.scaled_swiglu_mxfp8_fwd(x, ldx, s, M, N, dirs, staged, mx, None)
+def fwd(lib, x=A16, ldx=512, s=A16, M=64, N=256, dirs=1, staged=0, mx=MX_ROW, ilv=0):
+    return lib.scaled_swiglu_mxfp8_fwd(x, ldx, s, M, N, dirs, staged, ilv, mx, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -89,9 +89,9 @@ def test_empty_input_is_ok_without_launch(lib):
 
 
 def bwd(lib, dy=A16, lddy=256, x=A16, ldx=512, s=A16, M=64, N=256, dirs=1, dx=A16, dscale=A16,
-        mx=MX_ROW, ws=A16, wsb=1 << 30):
-    return lib.scaled_swiglu_mxfp8_bwd(dy, lddy, x, ldx, s, M, N, dirs, dx, dscale, mx, ws, wsb,
-                                       None)
+        mx=MX_ROW, ws=A16, wsb=1 << 30, ilv=0):
+    return lib.scaled_swiglu_mxfp8_bwd(dy, lddy, x, ldx, s, M, N, dirs, ilv, dx, dscale, mx, ws,
+                                       wsb, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -121,7 +121,7 @@ def test_backward_workspace_only_needed_for_dscale(lib):
 
 def test_grouped_argument_errors(lib):
     f = lib.grouped_scaled_swiglu_mxfp8_fwd
-    args = lambda ro=A16, cb=A16, E=4, st=A16: (A16, 512, A16, 64, 256, 1, 0, ro, cb, E, st,
+    args = lambda ro=A16, cb=A16, E=4, st=A16: (A16, 512, A16, 64, 256, 1, 0, 0, ro, cb, E, st,
                                                  MX_ROW, None)
     assert f(*args(ro=None)) == _capi.EINVAL
     assert f(*args(st=None)) == _capi.EINVAL
@@ -154,3 +154,24 @@ def test_gemm_scale_layout_argument_errors(lib):
 def test_noop_flag_alignment(lib):
     mx = _capi.MxOut(A16, A16, None, None, _capi.SCALES_ROWMAJOR, A16 + 2)
     assert fwd(lib, mx=mx) == _capi.EALIGN
+
+
+@pytest.mark.parametrize("ilv,N,status", [
+    (16, 256, _capi.EINVAL),      # not a multiple of 32
+    (-32, 256, _capi.EINVAL),
+    (96, 384, _capi.EINVAL),      # divides N, but neither 32, 64 nor a multiple of 128
+    (256, 384, _capi.EINVAL),     # does not divide N
+    (64, 96, _capi.EINVAL),       # does not divide N
+    (32, 256, _capi.OK),          # M = 0: checked, nothing launched
+    (64, 192, _capi.OK),
+    (128, 384, _capi.OK),
+    (96, 96, _capi.OK),           # G = N is the halves layout
+])
+def test_glu_interleave_arguments(lib, ilv, N, status):
+    """glu_interleave: 32, 64 or a multiple of 128 dividing N, or 0 / N."""
+    assert fwd(lib, M=0, N=N, ldx=2 * N, ilv=ilv) == status
+    assert bwd(lib, M=0, N=N, ldx=2 * N, lddy=N, ilv=ilv) == status
+    clamped = lib.scaled_clamped_swiglu_mxfp8_fwd(A16, 2 * N, A16, 0, N, 1, 1.702, 7.0, ilv,
+                                                  MX_ROW, None)
+    assert clamped == status
+

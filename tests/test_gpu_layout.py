@@ -120,7 +120,7 @@ def test_unaligned_groups_set_status_and_write_nothing(cuda_device):
     st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     stream = torch.cuda.current_stream(cuda_device).cuda_stream
     _capi.call("grouped_scaled_swiglu_mxfp8_fwd", x.data_ptr(), 2 * N, sg.data_ptr(), M, N, 3, 0,
-               gro.data_ptr(), gcb.data_ptr(), len(m), st.data_ptr(), mx, stream)
+               0, gro.data_ptr(), gcb.data_ptr(), len(m), st.data_ptr(), mx, stream)
     torch.cuda.synchronize()
     assert int(gst.item()) == 0
     assert int(st.item()) == _capi.DEV_UNALIGNED_GROUPS

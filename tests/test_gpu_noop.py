@@ -52,12 +52,13 @@ def test_set_flag_writes_nothing(cuda_device, grouped):
         if call == "fwd":
             if grouped:
                 _capi.call("grouped_scaled_swiglu_mxfp8_fwd", x.data_ptr(), 2 * N, s.data_ptr(), M,
-                           N, 3, 0, ro.data_ptr(), cb.data_ptr(), 3, o["st"].data_ptr(), mx, stream)
+                           N, 3, 0, 0, ro.data_ptr(), cb.data_ptr(), 3, o["st"].data_ptr(), mx,
+                           stream)
             else:
                 _capi.call("scaled_swiglu_mxfp8_fwd", x.data_ptr(), 2 * N, s.data_ptr(), M, N, 3, 0,
-                           mx, stream)
+                           0, mx, stream)
         else:
-            args = [dy.data_ptr(), N, x.data_ptr(), 2 * N, s.data_ptr(), M, N, 3]
+            args = [dy.data_ptr(), N, x.data_ptr(), 2 * N, s.data_ptr(), M, N, 3, 0]
             if grouped:
                 _capi.call("grouped_scaled_swiglu_mxfp8_bwd", *args, ro.data_ptr(), cb.data_ptr(),
                            3, o["st"].data_ptr(), o["dx"].data_ptr(), o["dscale"].data_ptr(), mx,

@@ -257,7 +257,7 @@ def test_outputs_stay_inside_their_buffers(cuda_device):
     mx = _capi.MxOut(bufs["rq"][1], bufs["rs"][1], bufs["cq"][1], bufs["cs"][1])
     stream = torch.cuda.current_stream(cuda_device).cuda_stream
     _capi.call("scaled_swiglu_mxfp8_bwd", dy.data_ptr(), N, x.data_ptr(), 2 * N, s.data_ptr(),
-               M, N, 3, dxb[1], dsb[1], mx, ws.data_ptr(), ws.numel(), stream)
+               M, N, 3, 0, dxb[1], dsb[1], mx, ws.data_ptr(), ws.numel(), stream)
     torch.cuda.synchronize()
     for name, (buf, _), n in [(k, bufs[k], sizes[k]) for k in sizes] + \
             [("dx", dxb, M * W * 2), ("dscale", dsb, M * 4)]:
@@ -269,7 +269,7 @@ def test_outputs_stay_inside_their_buffers(cuda_device):
     # the same workspace serves the next call (its counters are back at zero)
     dsb2 = guarded(M * 4)
     _capi.call("scaled_swiglu_mxfp8_bwd", dy.data_ptr(), N, x.data_ptr(), 2 * N, s.data_ptr(),
-               M, N, 0, None, dsb2[1], _capi.MxOut(None, None, None, None), ws.data_ptr(),
+               M, N, 0, 0, None, dsb2[1], _capi.MxOut(None, None, None, None), ws.data_ptr(),
                ws.numel(), stream)
     torch.cuda.synchronize()
     a = dsb[0][pad:pad + 4 * M].cpu()
@@ -365,7 +365,7 @@ def test_failed_splits_leave_no_usable_offsets(cuda_device):
                                                           "col_scales")))
         st2 = torch.zeros(1, dtype=torch.int32, device=cuda_device)
         _capi.call("grouped_scaled_swiglu_mxfp8_fwd", x.data_ptr(), 2 * N, s.data_ptr(), M, N, 3,
-                   0, ro.data_ptr(), cb.data_ptr(), len(m), st2.data_ptr(), mx, stream)
+                   0, 0, ro.data_ptr(), cb.data_ptr(), len(m), st2.data_ptr(), mx, stream)
         torch.cuda.synchronize()
         assert int(st2.item()) == _capi.DEV_BAD_OFFSETS
         for o in outs.values():
@@ -476,7 +476,7 @@ def test_grouped_bad_offsets_set_status_and_write_nothing(cuda_device, corrupt):
     rs = torch.full((M, N // 32), 0x5A, dtype=torch.uint8, device=cuda_device)
     stt = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     _capi.call("grouped_scaled_swiglu_mxfp8_fwd", x.data_ptr(), 2 * N, s.data_ptr(), M, N, 1, 0,
-               gro.data_ptr(), gcb.data_ptr(), 3, stt.data_ptr(),
+               0, gro.data_ptr(), gcb.data_ptr(), 3, stt.data_ptr(),
                _capi.MxOut(rq.data_ptr(), rs.data_ptr(), None, None),
                torch.cuda.current_stream(cuda_device).cuda_stream)
     torch.cuda.synchronize()

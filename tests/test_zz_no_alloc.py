@@ -39,8 +39,10 @@ def _run(name, case, dev, workspace=None):
     M, N = dy.shape
     o, mx = _outputs(M, N, dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
-    args = [dy.data_ptr(), N, x.data_ptr(), 2 * N, s.data_ptr(), M, N, 3, o["dx"].data_ptr(),
-            o["dscale"].data_ptr(), mx]
+    args = [dy.data_ptr(), N, x.data_ptr(), 2 * N, s.data_ptr(), M, N, 3]
+    if workspace is not None:
+        args.append(0)   # glu_interleave: [gate | up] halves (the no-alloc call has no such argument)
+    args += [o["dx"].data_ptr(), o["dscale"].data_ptr(), mx]
     if workspace is not None:
         args += [workspace.data_ptr(), workspace.numel()]
     _capi.call(name, *args, stream)

@@ -526,14 +526,21 @@ def cpu_baseline(wl, dirs, budget_s=10.0):
     oracle.sigmoid_table()
     rows = _calibrate_rows(oracle, wl, dirs, budget_s)
     xb, s, dyb = _oracle_sample(wl, dirs, rows)
+    # whole passes over the sample until the budget is spent (a workload
+    # smaller than the budget is passed over several times)
+    passes = 0
     t0 = time.perf_counter()
-    _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
-    dt = time.perf_counter() - t0
+    while True:
+        _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= 0.9 * budget_s:
+            break
     bm = byte_model(rows, wl.N, 1, dirs)
-    return {"value": round((bm["fwd"] + bm["bwd"]) / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"rows [0, {rows}) of {wl.M} ({wl.key}), forward + backward, "
-                      f"dirs={dirs}, {dt:.1f} s single-threaded"}
+    return {"value": round(passes * (bm["fwd"] + bm["bwd"]) / dt / 1e9, 4), "unit": "GB/s",
+            "cores": 1, "kind": "oracle",
+            "sample": f"rows [0, {rows}) of {wl.M} ({wl.key}) x {passes} pass(es), forward + "
+                      f"backward, dirs={dirs}, {dt:.1f} s single-threaded"}
 
 
 def run_reference(args):

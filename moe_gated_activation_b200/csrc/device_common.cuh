@@ -194,7 +194,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
-// 1-D bulk copy (no multicast) of `bytes` (a multiple of 16, both addresses
+// 1-D bulk copy (this CTA only) of `bytes` (a multiple of 16, both addresses
 // 16-byte aligned) from global to shared memory, completing on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
@@ -204,7 +204,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// 2-D TMA tile load (no multicast) of box {x .. x+bx, y .. y+by} into shared
+// 2-D TMA tile load (this CTA only) of box {x .. x+bx, y .. y+by} into shared
 // memory, completing on `bar`; rows and columns outside the tensor read zero.
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y,
                                             uint64_t* bar) {

@@ -21,7 +21,7 @@
 //
 // Data movement.  Each warp owns a ring of shared-memory slots, each holding
 // one 16-row half of a warp-tile's inputs ([16 x 128] bf16 per operand),
-// filled by TMA (cp.async.bulk.tensor, no multicast) and signalled through
+// filled by TMA (cp.async.bulk.tensor, this CTA only) and signalled through
 // one mbarrier per slot; lane 0 refills a slot as soon as it is consumed, so
 // the loads of the next half-tiles overlap the math of the current one, and
 // rows and columns outside the tensor arrive as zeros.  Lanes read their four

@@ -333,9 +333,6 @@ __device__ __forceinline__ void ring_drain(const Ring<OPS, SLOTS>& r, int k_next
     mbar_wait(r.bars + (k % SLOTS), (uint32_t)(k / SLOTS) & 1u);
 }
 
-// Magnitude bits shifted left by one: ordering of |v| with NaN above +Inf
-// (an integer max over them is a NaN-propagating amax); e8m0 takes them >> 1.
-__device__ __forceinline__ uint32_t mag2(float v) { return __float_as_uint(v) << 1; }
 
 // Stores the E8M0 bytes of one row's blocks [4*tile, 4*tile + nb) (packed in
 // v, block 0 in the low byte): one 32-bit store when all four exist and the
@@ -469,6 +466,13 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return r;
 }
 
+// Three-input form (sm_100): NaN if any input is NaN, else the largest.
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // A pair of gates (fp32, with their sigmoids from the table) clamped at L: a
 // gate above L becomes L and takes sigma(RN(alpha * L)); NaN passes through.
 __device__ __forceinline__ void clamp_gates(float2& g, float2& sg, const Params& p) {
@@ -592,16 +596,19 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
     if (lane == 0 && ring.k_issue < K)
       ring_issue<OPS, SLOTS, GROUPED, (DIRS & kIlv) != 0>(p, m, ring, tm_x, nullptr);
     if (DIRS & kRow) {
+      // per-row amax of the lane's 4 values as the bits of a non-negative
+      // float (NaN above +Inf), so the butterfly can take integer maxima
       uint32_t A[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = 16 * h + i;
-        A[i] = max(__vimax3_u32(mag2(Y[r][0]), mag2(Y[r][1]), mag2(Y[r][2])), mag2(Y[r][3]));
+        A[i] = __float_as_uint(max_nan(max3_nan(fabsf(Y[r][0]), fabsf(Y[r][1]), fabsf(Y[r][2])),
+                                       fabsf(Y[r][3])));
       }
       bfly_max_u32<8>(A, lane, 4);
       bfly_max_u32<4>(A, lane, 2);
       bfly_max_u32<2>(A, lane, 1);
-      const uint32_t b0 = e8m0_from_amax(A[0] >> 1), b1 = e8m0_from_amax(A[1] >> 1);
+      const uint32_t b0 = e8m0_from_amax(A[0]), b1 = e8m0_from_amax(A[1]);
       bh[h] = b0 | (b1 << 8);
       const uint32_t m0 = scale_multiplier(b0), m1 = scale_multiplier(b1);
 #pragma unroll
@@ -627,15 +634,15 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
     }
   }
   if (DIRS & kCol) {
-    uint32_t a[4] = {0u, 0u, 0u, 0u};
+    float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int r = 0; r < 32; r += 2)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) a[c] = __vimax3_u32(a[c], mag2(Y[r][c]), mag2(Y[r + 1][c]));
+      for (int c = 0; c < 4; ++c) a[c] = max3_nan(a[c], fabsf(Y[r][c]), fabsf(Y[r + 1][c]));
     uint32_t b[4], mu[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      b[c] = e8m0_from_amax(a[c] >> 1);
+      b[c] = e8m0_from_amax(__float_as_uint(a[c]));
       mu[c] = scale_multiplier(b[c]);
     }
     if (colok) {

@@ -349,9 +349,11 @@ moeact_status grouped_scaled_clamped_swiglu_mxfp8_bwd(
 moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream);
 
 /* Reads and clears this device's error word: non-zero if a kernel gave up
- * waiting for its own input copies (bit 0 forward, bit 1 backward) -- a
- * defensive bound that ends the kernel instead of letting it hang; never
- * expected in normal operation.  Synchronous.  No counterpart on the pages. */
+ * waiting for its own input copies (bit 0 forward, bit 1 backward, bit 2 the
+ * sigmoid table's copy) -- a defensive bound that ends the kernel instead of
+ * letting it hang -- or found its shared-memory sigmoid table outside the
+ * 16-bit address range its lookups use (bit 3); never expected in normal
+ * operation.  Synchronous.  No counterpart on the pages. */
 moeact_status moeact_device_error(uint32_t* flags);
 
 /* ---------------------------------------------------------------------

@@ -55,6 +55,33 @@ __device__ __forceinline__ void sigma_pair(const float* tab, uint32_t G, float& 
   s_hi = *reinterpret_cast<const float*>(tb + (off >> 16));
 }
 
+// The same pair lookup on a table in shared memory whose highest address is
+// below 64 KiB, with the table's address folded into one constant, `key`
+// (sigma_key): both 16-bit lanes of c * 4 + key + sign bits are then the two
+// entries' shared-memory addresses.  The low lane's c * 4 + key always
+// carries exactly one into the high lane (its low half of key is
+// T - 4 lo + 2^16 for a table at T, and 4 c - 4 lo + T < 2^16), which the
+// high half of key pre-subtracts; the sign bits add 32 KiB to a lane without
+// a carry (T + 4 (hi - lo) + 32 KiB + 4 < 2^16 for T < 16 KiB).
+__host__ __device__ constexpr uint32_t sigma_key(uint32_t T) {
+  return ((T - 4u * kSigLo) & 0xFFFFu) | (((T - 4u * kSigLo - 1u) & 0xFFFFu) << 16);
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sigma_pair_s(uint32_t key, uint32_t G, float& s_lo,
+                                             float& s_hi) {
+  const uint32_t lo2 = kSigLo * 0x10001u, hi2 = kSigHi * 0x10001u;
+  const uint32_t c = __vimin3_u16x2(__vimax3_u16x2(G & 0x7FFF7FFFu, lo2, lo2), hi2, hi2);
+  const uint32_t a = c * 4u + key + (G & 0x80008000u);
+  s_lo = lds_f32(a & 0xFFFFu);
+  s_hi = lds_f32(a >> 16);
+}
+
 // ---------------------------------------------------------------- bf16
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

@@ -64,9 +64,10 @@ __global__ void sigma_table_dump(const float* src, float* out) {
   for (int i = threadIdx.x; i < kSigBytes / 4; i += blockDim.x) tab[i] = src[i];
   __syncthreads();
   const uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < 32768) {
+  const uint32_t T = smem_addr(tab);
+  if (t < 32768 && T + kSigBytes <= 0x10000u) {
     float a, b;
-    sigma_pair(tab, (2 * t) | ((2 * t + 1) << 16), a, b);
+    sigma_pair_s(sigma_key(T), (2 * t) | ((2 * t + 1) << 16), a, b);
     out[2 * t] = a;
     out[2 * t + 1] = b;
   }

@@ -104,6 +104,9 @@ constexpr int kRowBytes = kTileCols * 2;                   // 256 B of a bf16 ti
 template <int ACT, bool BWD>
 struct Cfg {
   static constexpr bool kSig = ACT != kSReLU;   // gated: sigmoid table, gate + up
+  // the table first in shared memory, looked up by 16-bit addresses
+  // (sigma_pair_s): the SwiGLU forward, where it measured faster
+  static constexpr bool kSigFront = !BWD && ACT == kSwiGLU;
   static constexpr int kOps = BWD ? (kSig ? 3 : 2) : (kSig ? 2 : 1);
   static constexpr int kWarps = BWD ? (kSig ? 7 : 8) : 8;
   static constexpr int kSlots = (!BWD && !kSig) ? 3 : 2;
@@ -119,12 +122,20 @@ constexpr int kGapCb = 4100;
 constexpr int kGapRo = 6144;
 __host__ __device__ constexpr int group_bytes(int E) { return 2 * ((E + 1 + 3) / 4) * 16; }
 
-// Shared memory of a CTA: 128 B of alignment slack, the ring, the table (or
-// the group offsets), the mbarriers.
+// Shared memory of a CTA: 128 B of alignment slack, then the sigmoid table
+// (padded to 1 KiB) and the ring (Cfg::kSigFront: the SwiGLU forward), or the
+// ring and the table (the other gated kernels), or the ring and the group
+// offsets (SReLU); then the mbarriers.  A table in front has shared-memory
+// addresses that fit in 16 bits (see sigma_pair_s); the backward and the
+// ClampedSwiGLU forward measured slower with that order, and look their
+// table up through its pointer.
+constexpr int kSigRegion = (kSigBytes + 1023) / 1024 * 1024;
 template <int ACT, bool BWD>
 __host__ __device__ constexpr int smem_bytes(bool grouped, int E) {
   using C = Cfg<ACT, BWD>;
-  return 128 + C::kRing + (C::kSig ? kSigBytes : (grouped ? group_bytes(E) : 0)) + C::kBars * 8;
+  return 128 + C::kRing +
+         (C::kSig ? (C::kSigFront ? kSigRegion : kSigBytes) : (grouped ? group_bytes(E) : 0)) +
+         C::kBars * 8;
 }
 
 __device__ __forceinline__ unsigned char* align_smem(unsigned char* p) {
@@ -134,6 +145,7 @@ __device__ __forceinline__ unsigned char* align_smem(unsigned char* p) {
 struct Smem {
   unsigned char* ring;
   float* sig;
+  uint32_t sig_key;   // kSigFront: sigma_pair_s's constant for this table's address
   int* cb;
   int* ro;
   uint64_t* bars;
@@ -144,15 +156,26 @@ __device__ __forceinline__ Smem carve(unsigned char* raw, int E) {
   using C = Cfg<ACT, BWD>;
   Smem m;
   unsigned char* base = align_smem(raw);
-  m.ring = base;
-  unsigned char* after = base + C::kRing;
-  if (C::kSig) {
-    m.sig = reinterpret_cast<float*>(after);
+  unsigned char* after;
+  if (C::kSigFront) {
+    m.sig = reinterpret_cast<float*>(base);
+    m.sig_key = sigma_key(smem_addr(base));
     m.cb = reinterpret_cast<int*>(m.sig + kGapCb);
     m.ro = reinterpret_cast<int*>(m.sig + kGapRo);
-    after += kSigBytes;
+    m.ring = base + kSigRegion;
+    after = m.ring + C::kRing;
+  } else if (C::kSig) {
+    m.ring = base;
+    m.sig = reinterpret_cast<float*>(base + C::kRing);
+    m.sig_key = 0;
+    m.cb = reinterpret_cast<int*>(m.sig + kGapCb);
+    m.ro = reinterpret_cast<int*>(m.sig + kGapRo);
+    after = base + C::kRing + kSigBytes;
   } else {
+    m.ring = base;
+    after = base + C::kRing;
     m.sig = nullptr;
+    m.sig_key = 0;
     m.cb = reinterpret_cast<int*>(after);
     m.ro = m.cb + ((E + 1 + 3) / 4) * 4;
     after += group_bytes(E);
@@ -323,6 +346,17 @@ __device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
 
 __device__ __forceinline__ void report_timeout(const Params& p, uint32_t code) {
   atomicOr(p.err, code);
+}
+
+// The sigmoid lookups address the table with 16-bit shared-memory addresses
+// (sigma_pair_s); a CTA whose table would end above 64 KiB (not expected:
+// the table starts the dynamic shared memory) records error bit 3 and does
+// nothing, before any copy is issued.
+template <bool FRONT>
+__device__ __forceinline__ bool sig_table_addressable(const Params& p, const Smem& m) {
+  if (!FRONT || smem_addr(m.sig) + kSigBytes <= 0x10000u) return true;
+  if (threadIdx.x == 0) report_timeout(p, 8u);
+  return false;
 }
 
 // After a timeout: bounded waits for the copies still in flight into the
@@ -565,8 +599,8 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
       } else if (ACT == kSwiGLU) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
         float2 sg01, sg23;
-        sigma_pair(m.sig, G.x, sg01.x, sg01.y);
-        sigma_pair(m.sig, G.y, sg23.x, sg23.y);
+        sigma_pair_s(m.sig_key, G.x, sg01.x, sg01.y);
+        sigma_pair_s(m.sig_key, G.y, sg23.x, sg23.y);
         const float2 si01 = mul2(bf16x2_to_f2(G.x), sg01), si23 = mul2(bf16x2_to_f2(G.y), sg23);
         const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
         if (STAGED) {
@@ -689,6 +723,7 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
   if (p.noop != nullptr && *p.noop != 0) return;   // a skipped replay: nothing issued yet
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const Smem m = carve<ACT, false>(smem_raw, GROUPED ? p.E : 0);
+  if (!sig_table_addressable<C::kSigFront>(p, m)) return;
   uint64_t* sig_bar = m.bars + C::kWarps * C::kSlots;
   const int64_t n_slabs = stage_and_validate<C::kSig, GROUPED>(p, m, sig_bar);
   if (n_slabs < 0) {

@@ -67,6 +67,9 @@ __host__ __device__ constexpr uint32_t sigma_key(uint32_t T) {
   return ((T - 4u * kSigLo) & 0xFFFFu) | (((T - 4u * kSigLo - 1u) & 0xFFFFu) << 16);
 }
 
+// A plain (non-volatile) shared load: ordered after the table's copy only
+// through its address, which the callers derive from data read after the
+// copy's barrier.
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;
   asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));

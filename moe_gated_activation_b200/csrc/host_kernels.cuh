@@ -64,7 +64,10 @@ __global__ void sigma_table_dump(const float* src, float* out) {
   for (int i = threadIdx.x; i < kSigBytes / 4; i += blockDim.x) tab[i] = src[i];
   __syncthreads();
   const uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
-  const uint32_t T = smem_addr(tab);
+  // the table's address passes through a volatile move after the barrier, so
+  // the lookups (plain ld.shared statements) cannot be scheduled before it
+  uint32_t T;
+  asm volatile("mov.u32 %0, %1;" : "=r"(T) : "r"(smem_addr(tab)));
   if (t < 32768 && T + kSigBytes <= 0x10000u) {
     float a, b;
     sigma_pair_s(sigma_key(T), (2 * t) | ((2 * t + 1) << 16), a, b);

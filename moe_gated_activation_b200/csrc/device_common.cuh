@@ -35,13 +35,6 @@ constexpr int kSigNegOffset = 8192;
 constexpr int kSigBytes = (kSigNegOffset + kSigPerSign + 3) / 4 * 16;   // 49168
 constexpr int kSigHalfBytes = (kSigPerSign + 3) / 4 * 16;                 // 16400
 
-__device__ __forceinline__ float sigma_lookup(const float* tab, uint32_t b16) {
-  uint32_t a = b16 & 0x7FFFu;
-  a = min(max(a, kSigLo), kSigHi) - kSigLo;
-  a += (b16 & 0x8000u) ? kSigNegOffset : 0u;
-  return tab[a];
-}
-
 // sigma of both bf16 values of a packed pair: both byte offsets are computed
 // at once in 16-bit lanes (clamp of the magnitude, minus the range start,
 // times 4, plus the sign bit as the 32 KiB offset of the negative half).
@@ -133,15 +126,6 @@ __device__ __forceinline__ uint32_t scale_multiplier(uint32_t b) {
   return b < 254u ? (254u - b) << 23 : (b == 254u ? 0x00400000u : kNanScale);
 }
 
-// Two values -> two E4M3 codes (a in the low byte): nearest even of v * 2^(127-b),
-// saturating.  For the NaN scale (b = 255) the multiplier is a NaN, the
-// product is NaN and the conversion gives the E4M3 NaN code 0x7F.
-__device__ __forceinline__ uint32_t e4m3x2(float a, uint32_t ma, float b, uint32_t mb) {
-  const float2 v = make_float2(__fmul_rn(a, __uint_as_float(ma)),
-                               __fmul_rn(b, __uint_as_float(mb)));
-  return (uint32_t)__nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, __NV_E4M3);
-}
-
 // A copy of v the compiler cannot see through: used so that a later pass
 // recomputes per-row addresses instead of keeping an earlier pass's live.
 __device__ __forceinline__ int opaque(int v) {
@@ -181,13 +165,15 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t v) { return make_float2(bf16_lo(v), bf16_hi(v)); }
 __device__ __forceinline__ float2 bf16x2_to_f2_p(uint32_t v) { return make_float2(bf16_lo_p(v), bf16_hi_p(v)); }
 
-// E4M3 codes of v * (ma, mb) (low byte: x), as e4m3x2 with a packed multiply.
+// Two E4M3 codes (low byte: v.x): nearest even of v.x * ma and v.y * mb
+// (ma, mb the bit patterns of the multipliers 2^(127-b)), saturating, through
+// one packed multiply.  For the NaN scale (b = 255) the multiplier is a NaN,
+// the product is NaN and the conversion gives the E4M3 NaN code 0x7F.
 __device__ __forceinline__ uint32_t e4m3x2_2(float2 v, uint32_t ma, uint32_t mb) {
   const float2 q = mul2(v, make_float2(__uint_as_float(ma), __uint_as_float(mb)));
   return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
 }
 
-__device__ __forceinline__ uint32_t f32_mag(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
 
 // ---------------------------------------------------------------- TMA / mbarrier
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

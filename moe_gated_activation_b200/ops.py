@@ -144,6 +144,14 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
     stream = _stream(x.device)
     ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
     ilv = _ilv(glu_interleave, swiglu)
+    if M == 0:
+        # nothing to compute (the library launches nothing either); empty
+        # tensors may have null data pointers, which the C ABI rejects
+        if dirs == 0:
+            raise ValueError("at least one of rowwise / colwise is required")
+        if grouped is not None:
+            st.zero_()
+        return _mx_result(rq, rs, cq, cs, view)
     if act == "clamped":
         alpha, limit = clamp
         if grouped is None:
@@ -267,6 +275,13 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
     stream = _stream(dev)
     ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
     lddy = dy.stride(0) if M > 1 else max(dy.stride(0), dy.shape[1])
+    if M == 0:
+        _ilv(glu_interleave, swiglu)
+        if dirs == 0 and not want_dx and not want_dscale:
+            raise ValueError("nothing requested: no direction, dx or dscale")
+        if grouped is not None:
+            st.zero_()
+        return Backward(_mx_result(rq, rs, cq, cs, view), dx, dscale)
     common = (_ptr(dy), lddy, _ptr(x), ldx, _ptr(s), M, N, dirs)
     tail = (mx, _ptr(ws), ws.numel() if ws is not None else 0, stream)
     if swiglu:

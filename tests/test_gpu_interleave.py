@@ -146,3 +146,51 @@ def test_bad_interleave(cuda_device):
             mg.scaled_swiglu_mxfp8_fwd(x, sg, glu_interleave=G)
         with pytest.raises(_capi.MoeactError):
             mg.scaled_swiglu_mxfp8_bwd(dy, x, sg, glu_interleave=G)
+
+
+def test_strided_input_and_g_equal_n(cuda_device):
+    """x with a row stride wider than 2N, and G = N (the halves layout)."""
+    M, N, G = 64, 256, 32
+    (xb, s, dyb), (x, sg, dy) = _case(M, N, 404, cuda_device)
+    wide = torch.zeros(M, 2 * N + 64, dtype=torch.bfloat16, device=cuda_device)
+    wide[:, :2 * N] = x
+    xs = wide[:, :2 * N]
+    got = mg.scaled_swiglu_mxfp8_fwd(xs, sg, glu_interleave=G)
+    gotb = mg.scaled_swiglu_mxfp8_bwd(dy, xs, sg, glu_interleave=G)
+    halves = mg.scaled_swiglu_mxfp8_fwd(x, sg, glu_interleave=N)
+    torch.cuda.synchronize()
+    compare_mx(got, oracle.interleaved_fwd(xb, s, N, 3, G), "strided fwd")
+    ref = oracle.interleaved_bwd(dyb, xb, s, N, 3, G)
+    compare_mx(gotb.mx, ref, "strided bwd")
+    assert np.array_equal(bf16_u16(gotb.dx), ref["dx"])
+    compare_mx(halves, oracle.act_fwd(xb, s, N, 3), "G = N")
+
+
+def test_noop_flag_and_empty_input(cuda_device):
+    """A set no-op flag writes nothing with an interleaved input either; an
+    empty input launches nothing."""
+    M, N, G = 64, 256, 64
+    (_, _, _), (x, sg, dy) = _case(M, N, 505, cuda_device)
+    flag = torch.ones(1, dtype=torch.int32, device=cuda_device)
+    stream = torch.cuda.current_stream(cuda_device).cuda_stream
+    ws = torch.zeros(mg.bwd_workspace_bytes(M, N), dtype=torch.uint8, device=cuda_device)
+    for W in (N, 2 * N):
+        u8_ = dict(dtype=torch.uint8, device=cuda_device)
+        o = [torch.full((M, W), 0xA5, **u8_), torch.full((M, W // 32), 0xA5, **u8_),
+             torch.full((M, W), 0xA5, **u8_), torch.full(((M + 31) // 32, W), 0xA5, **u8_)]
+        dx = torch.full((M, 2 * N), -7.0, dtype=torch.bfloat16, device=cuda_device)
+        dscale = torch.full((M,), -7.0, device=cuda_device)
+        mx = _capi.MxOut(*(t.data_ptr() for t in o), _capi.SCALES_ROWMAJOR, flag.data_ptr())
+        if W == N:
+            _capi.call("scaled_swiglu_mxfp8_fwd", x.data_ptr(), 2 * N, sg.data_ptr(), M, N, 3, 0,
+                       G, mx, stream)
+        else:
+            _capi.call("scaled_swiglu_mxfp8_bwd", dy.data_ptr(), N, x.data_ptr(), 2 * N,
+                       sg.data_ptr(), M, N, 3, G, dx.data_ptr(), dscale.data_ptr(), mx,
+                       ws.data_ptr(), ws.numel(), stream)
+        torch.cuda.synchronize()
+        assert all(bool((t == 0xA5).all()) for t in o)
+        assert bool((dx == -7.0).all()) and bool((dscale == -7.0).all())
+    e = mg.scaled_swiglu_mxfp8_fwd(x[:0], sg[:0], glu_interleave=G)
+    torch.cuda.synchronize()
+    assert e.row_codes.numel() == 0

@@ -482,3 +482,23 @@ def test_grouped_bad_offsets_set_status_and_write_nothing(cuda_device, corrupt):
     torch.cuda.synchronize()
     assert int(stt.item()) == _capi.DEV_BAD_OFFSETS
     assert bool((rq == 0x5A).all()) and bool((rs == 0x5A).all())
+
+
+def test_empty_inputs_through_the_python_api(cuda_device):
+    """M = 0 through the tensor API (empty tensors may have null data
+    pointers): empty outputs, no error, and a grouped call's status word 0."""
+    N = 128
+    x = torch.empty(0, 2 * N, dtype=torch.bfloat16, device=cuda_device)
+    s = torch.empty(0, dtype=torch.float32, device=cuda_device)
+    dy = torch.empty(0, N, dtype=torch.bfloat16, device=cuda_device)
+    f = mg.scaled_swiglu_mxfp8_fwd(x, s)
+    b = mg.scaled_swiglu_mxfp8_bwd(dy, x, s)
+    m = torch.zeros(3, dtype=torch.int64, device=cuda_device)
+    ro, cb, st = mg.splits_to_offsets(m, 0)
+    gf, gst = mg.grouped_scaled_swiglu_mxfp8_fwd(x, s, ro, cb, glu_interleave=32)
+    gb, gbst = mg.grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, ro, cb)
+    torch.cuda.synchronize()
+    assert f.row_codes.shape == (0, N) and f.col_scales.shape[0] == 0
+    assert b.dx.shape == (0, 2 * N) and b.dscale.shape == (0,)
+    assert int(st.item()) == 0 and int(gst.item()) == 0 and int(gbst.item()) == 0
+    assert gf.row_codes.numel() == 0 and gb.mx.row_codes.numel() == 0

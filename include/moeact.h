@@ -165,7 +165,10 @@ typedef struct moeact_mx_out {
 
 /* Build the sigmoid table on the current device and set up its kernels.
  * Optional: the first call on a device does it, but that first call must not
- * be inside a stream capture.  Synchronises the current device once. */
+ * be inside a stream capture.  Synchronises the current device once.
+ * MOEACT_EUNSUPPORTED if the device is not sm_100, or if its dynamic shared
+ * memory starts too high for the 16-bit table addressing of the SwiGLU
+ * forward (not expected on sm_100). */
 moeact_status moeact_init(void);
 
 /* Static text of a status; thread-local detail of the last failure. */

@@ -40,6 +40,7 @@ std::atomic<bool> g_ready[kMaxDevices];
 int g_sms[kMaxDevices];
 std::mutex g_mu;
 __device__ int g_sigma_uncertain;
+__device__ uint32_t g_smem_base;
 
 // The fused kernels of each activation (index kSwiGLU / kSReLU / kClamped),
 // filled once.
@@ -134,11 +135,28 @@ moeact_status init_device(int dev) {
   if (e == cudaSuccess)
     e = cudaMemcpyFromSymbolAsync(&unc, g_sigma_uncertain, sizeof(int), 0,
                                   cudaMemcpyDeviceToHost, st);
+  uint32_t smem_base = 0xFFFFFFFFu;
+  if (e == cudaSuccess) {
+    uint32_t* d_base = nullptr;
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d_base), g_smem_base);
+    if (e == cudaSuccess) {
+      smem_base_probe<<<1, 32, 1024, st>>>(d_base);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess)
+      e = cudaMemcpyFromSymbolAsync(&smem_base, g_smem_base, sizeof(uint32_t), 0,
+                                    cudaMemcpyDeviceToHost, st);
+  }
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   cudaStreamDestroy(st);
   if (e != cudaSuccess) return cuda_fail(e, "sigmoid table set-up");
   if (unc != 0)
     return fail(MOEACT_ECUDA, "sigmoid table: %d entries could not be certified", unc);
+  // the forward's table sits at the (128-byte aligned) start of dynamic
+  // shared memory and is looked up by 16-bit addresses
+  if (smem_base + 127u + (uint32_t)kSigBytes > 0x10000u)
+    return fail(MOEACT_EUNSUPPORTED, "dynamic shared memory starts at %u: above the 16-bit "
+                "range the sigmoid lookups use", smem_base);
   g_ready[dev].store(true);
   return MOEACT_OK;
 }

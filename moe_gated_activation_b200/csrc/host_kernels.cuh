@@ -76,6 +76,15 @@ __global__ void sigma_table_dump(const float* src, float* out) {
   }
 }
 
+// Shared-memory address at which dynamic shared memory begins (thread 0
+// writes it to *out).  The fused kernels have no static shared memory, so
+// theirs begins at the same address; the SwiGLU forward needs its sigmoid
+// table, placed there, to end below 64 KiB.
+__global__ void smem_base_probe(uint32_t* out) {
+  extern __shared__ __align__(128) unsigned char raw[];
+  if (threadIdx.x == 0) *out = smem_addr(raw);
+}
+
 // ---------------------------------------------------------------- offsets
 // One CTA of 1024 threads; thread t owns a contiguous chunk of the groups.
 __global__ void __launch_bounds__(1024) splits_kernel(const int64_t* __restrict__ m, int E,

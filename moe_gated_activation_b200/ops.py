@@ -4,6 +4,10 @@ These functions only allocate outputs with torch, check dtypes/strides and pass
 pointers and the current CUDA stream to libmoeact (include/moeact.h); every
 step of the computation runs in the library's sm_100a kernels.
 
+Every fused call takes ``out=``: caller-owned buffers (an ``MXFP8`` for the
+forward, a ``Backward`` for the backward) that the kernels write in place,
+for CUDA-graph replay without pointer changes.
+
 Return convention (pytorch/ao PR #4743, section "API"): an ``MXFP8`` tuple
 (row_codes, col_codes, row_scales, col_scales); a disabled direction comes back
 zero-sized.  Codes are ``torch.float8_e4m3fn`` [M, W] (same row-major layout
@@ -76,6 +80,36 @@ def _alloc_mx(M, W, dirs, device, col_rows):
     return rq, rs, cq, cs
 
 
+def _take_mx(out, M, W, dirs, device, col_rows):
+    """Caller-owned MXFP8 buffers (`out=`): the requested directions' tensors,
+    contiguous on `device`, codes uint8 or float8_e4m3fn [M, W], row scales
+    uint8 [M, W/32], col scales uint8 [>= col_rows, W].  The library writes
+    into them in place, so a captured CUDA graph can replay into the same
+    buffers (TE PR #3238: an output= argument for graph-replayed quantization)."""
+    e = torch.empty(0, dtype=torch.uint8, device=device)
+
+    def take(t, name, shape, min_rows=False):
+        if t is None:
+            raise ValueError(f"out.{name} is required for the requested direction")
+        if t.device != device or not t.is_contiguous():
+            raise ValueError(f"out.{name} must be contiguous on {device}")
+        if t.dtype == torch.float8_e4m3fn:
+            t = t.view(torch.uint8)
+        if t.dtype != torch.uint8:
+            raise TypeError(f"out.{name} must be uint8 (or float8_e4m3fn codes)")
+        ok = (t.dim() == 2 and t.shape[1] == shape[1] and t.shape[0] >= shape[0]) if min_rows \
+            else tuple(t.shape) == tuple(shape)
+        if not ok:
+            raise ValueError(f"out.{name} has shape {tuple(t.shape)}, {tuple(shape)} needed")
+        return t
+
+    rq = take(out.row_codes, "row_codes", (M, W)) if dirs & ROWWISE else e
+    rs = take(out.row_scales, "row_scales", (M, W // 32)) if dirs & ROWWISE else e
+    cq = take(out.col_codes, "col_codes", (M, W)) if dirs & COLWISE else e
+    cs = take(out.col_scales, "col_scales", (col_rows, W), min_rows=True) if dirs & COLWISE else e
+    return rq, rs, cq, cs
+
+
 def _mx_struct(rq, rs, cq, cs, dirs, gemm_scales=False, noop_flag=None):
     if dirs & ROWWISE:
         r = (rq.data_ptr(), rs.data_ptr())
@@ -126,7 +160,7 @@ def splits_to_offsets(m_splits: torch.Tensor, total_rows: int):
 
 # ------------------------------------------------------------------ forward
 def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False, clamp=None,
-         noop_flag=None, glu_interleave=0):
+         noop_flag=None, glu_interleave=0, out=None):
     swiglu = act != "srelu"        # gated: x = [gate | up]
     if N is None:
         N = x.shape[1] // 2 if swiglu else x.shape[1]
@@ -139,7 +173,10 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
     else:
         ro, cb, E, st, view = grouped
         col_rows = (M + 31) // 32 + E
-    rq, rs, cq, cs = _alloc_mx(M, N, dirs, x.device, col_rows)
+    if out is None:
+        rq, rs, cq, cs = _alloc_mx(M, N, dirs, x.device, col_rows)
+    else:
+        rq, rs, cq, cs = _take_mx(out, M, N, dirs, x.device, col_rows)
     mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales, noop_flag)
     stream = _stream(x.device)
     ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
@@ -177,7 +214,7 @@ def _fwd(act, x, s, N, rowwise, colwise, staged, grouped=None, gemm_scales=False
 
 
 def scaled_swiglu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, staged_rounding=False, N=None,
-                            gemm_scales=False, noop_flag=None, glu_interleave=None):
+                            gemm_scales=False, noop_flag=None, glu_interleave=None, out=None):
     """MXFP8 of SwiGLU(x) * s; x bf16 [M, >=2N] packs [gate | up].
     gemm_scales: scales in the GEMM-ready tiled layout (moeact.h,
     MOEACT_SCALES_GEMM; M and N multiples of 128).
@@ -185,14 +222,14 @@ def scaled_swiglu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, staged_rounding
     columns, repeated (G = 32, 64 or a multiple of 128 dividing N); the
     backward writes dx and its MXFP8 in the same column order."""
     return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, gemm_scales=gemm_scales,
-                noop_flag=noop_flag, glu_interleave=glu_interleave)
+                noop_flag=noop_flag, out=out, glu_interleave=glu_interleave)
 
 
 def scaled_srelu_mxfp8_fwd(x, s, *, rowwise=True, colwise=True, N=None, gemm_scales=False,
-                           noop_flag=None):
+                           noop_flag=None, out=None):
     """MXFP8 of relu(x)^2 * s; x bf16 [M, >=N]."""
     return _fwd("srelu", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales,
-                noop_flag=noop_flag)
+                noop_flag=noop_flag, out=out)
 
 
 def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
@@ -205,23 +242,23 @@ def _grouped_args(row_offs, colblk_offs, status, col_scale_rows, device):
 def grouped_scaled_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
                                     staged_rounding=False, status=None, col_scale_rows=None,
                                     N=None, gemm_scales=False, noop_flag=None,
-                                    glu_interleave=None):
+                                    glu_interleave=None, out=None):
     """Grouped forward: experts own the rows given by `row_offs` (from
     splits_to_offsets).  Returns (MXFP8, status).  Col scales hold
     ceil(M/32) + E rows unless `col_scale_rows` (sum of ceil(m_e/32), known on
     the host) is given."""
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _fwd("swiglu", x, s, N, rowwise, colwise, staged_rounding, g,
-                gemm_scales=gemm_scales, noop_flag=noop_flag,
+                gemm_scales=gemm_scales, noop_flag=noop_flag, out=out,
                 glu_interleave=glu_interleave), status
 
 
 def grouped_scaled_srelu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, rowwise=True, colwise=True,
                                    status=None, col_scale_rows=None, N=None, gemm_scales=False,
-                                   noop_flag=None):
+                                   noop_flag=None, out=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _fwd("srelu", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales,
-                noop_flag=noop_flag), status
+                noop_flag=noop_flag, out=out), status
 
 
 # ------------------------------------------------------------------ backward
@@ -246,7 +283,7 @@ def _workspace(device, nbytes):
 
 
 def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, grouped=None,
-         gemm_scales=False, clamp=None, noop_flag=None, glu_interleave=0):
+         gemm_scales=False, clamp=None, noop_flag=None, glu_interleave=0, out=None):
     swiglu = act != "srelu"        # gated: x = [gate | up], W = 2N
     if N is None:
         N = dy.shape[1]
@@ -264,10 +301,22 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
     else:
         ro, cb, E, st, view = grouped
         col_rows = (M + 31) // 32 + E
-    rq, rs, cq, cs = _alloc_mx(M, W, dirs, dev, col_rows)
+    if out is None:
+        rq, rs, cq, cs = _alloc_mx(M, W, dirs, dev, col_rows)
+        dx = torch.empty((M, W), dtype=torch.bfloat16, device=dev) if want_dx else None
+        dscale = torch.empty(M, dtype=torch.float32, device=dev) if want_dscale else None
+    else:
+        # caller-owned buffers: dx / dscale are computed when given
+        rq, rs, cq, cs = _take_mx(out.mx, M, W, dirs, dev, col_rows)
+        dx, dscale = out.dx, out.dscale
+        if dx is not None and (dx.dtype != torch.bfloat16 or tuple(dx.shape) != (M, W)
+                               or not dx.is_contiguous() or dx.device != dev):
+            raise ValueError(f"out.dx must be a contiguous bf16 [{M}, {W}] tensor on {dev}")
+        if dscale is not None and (dscale.dtype != torch.float32 or tuple(dscale.shape) != (M,)
+                                   or not dscale.is_contiguous() or dscale.device != dev):
+            raise ValueError(f"out.dscale must be a contiguous fp32 [{M}] tensor on {dev}")
+        want_dx, want_dscale = dx is not None, dscale is not None
     mx = _mx_struct(rq, rs, cq, cs, dirs, gemm_scales, noop_flag)
-    dx = torch.empty((M, W), dtype=torch.bfloat16, device=dev) if want_dx else None
-    dscale = torch.empty(M, dtype=torch.float32, device=dev) if want_dscale else None
     nbytes = bwd_workspace_bytes(M, N, E)
     ws = None
     if want_dscale:
@@ -304,37 +353,38 @@ def _bwd(act, dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, gr
 
 def scaled_swiglu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
                             want_dscale=True, workspace=None, N=None, gemm_scales=False,
-                            noop_flag=None, glu_interleave=None):
+                            noop_flag=None, glu_interleave=None, out=None):
     """Backward of the scaled SwiGLU: MXFP8 of [dgate | dup], bf16 dx, fp32 dscale."""
     return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales, noop_flag=noop_flag,
+                gemm_scales=gemm_scales, noop_flag=noop_flag, out=out,
                 glu_interleave=glu_interleave)
 
 
 def scaled_srelu_mxfp8_bwd(dy, x, s, *, rowwise=True, colwise=True, want_dx=True,
                            want_dscale=True, workspace=None, N=None, gemm_scales=False,
-                           noop_flag=None):
+                           noop_flag=None, out=None):
     return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales, noop_flag=noop_flag)
+                gemm_scales=gemm_scales, noop_flag=noop_flag, out=out)
 
 
 def grouped_scaled_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
                                     colwise=True, want_dx=True, want_dscale=True,
                                     workspace=None, status=None, col_scale_rows=None, N=None,
-                                    gemm_scales=False, noop_flag=None, glu_interleave=None):
+                                    gemm_scales=False, noop_flag=None, glu_interleave=None,
+                                    out=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("swiglu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                g, gemm_scales=gemm_scales, noop_flag=noop_flag,
+                g, gemm_scales=gemm_scales, noop_flag=noop_flag, out=out,
                 glu_interleave=glu_interleave), status
 
 
 def grouped_scaled_srelu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *, rowwise=True,
                                    colwise=True, want_dx=True, want_dscale=True,
                                    workspace=None, status=None, col_scale_rows=None, N=None,
-                                   gemm_scales=False, noop_flag=None):
+                                   gemm_scales=False, noop_flag=None, out=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("srelu", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                g, gemm_scales=gemm_scales, noop_flag=noop_flag), status
+                g, gemm_scales=gemm_scales, noop_flag=noop_flag, out=out), status
 
 
 # ------------------------------------------------------------------ ClampedSwiGLU
@@ -344,10 +394,10 @@ CLAMPED_LIMIT = 7.0
 
 def scaled_clamped_swiglu_mxfp8_fwd(x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
                                     rowwise=True, colwise=True, N=None, gemm_scales=False,
-                                    noop_flag=None, glu_interleave=None):
+                                    noop_flag=None, glu_interleave=None, out=None):
     """MXFP8 of ClampedSwiGLU(x) * s (moeact.h); x bf16 [M, >=2N] packs [gate | up]."""
     return _fwd("clamped", x, s, N, rowwise, colwise, False, gemm_scales=gemm_scales,
-                clamp=(alpha, limit), noop_flag=noop_flag,
+                clamp=(alpha, limit), noop_flag=noop_flag, out=out,
                 glu_interleave=glu_interleave)
 
 
@@ -355,19 +405,19 @@ def grouped_scaled_clamped_swiglu_mxfp8_fwd(x, s, row_offs, colblk_offs, *, alph
                                             limit=CLAMPED_LIMIT, rowwise=True, colwise=True,
                                             status=None, col_scale_rows=None, N=None,
                                             gemm_scales=False, noop_flag=None,
-                                            glu_interleave=None):
+                                            glu_interleave=None, out=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _fwd("clamped", x, s, N, rowwise, colwise, False, g, gemm_scales=gemm_scales,
-                clamp=(alpha, limit), noop_flag=noop_flag,
+                clamp=(alpha, limit), noop_flag=noop_flag, out=out,
                 glu_interleave=glu_interleave), status
 
 
 def scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, *, alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT,
                                     rowwise=True, colwise=True, want_dx=True, want_dscale=True,
                                     workspace=None, N=None, gemm_scales=False, noop_flag=None,
-                                    glu_interleave=None):
+                                    glu_interleave=None, out=None):
     return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace,
-                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag,
+                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag, out=out,
                 glu_interleave=glu_interleave)
 
 
@@ -376,10 +426,10 @@ def grouped_scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *,
                                             rowwise=True, colwise=True, want_dx=True,
                                             want_dscale=True, workspace=None, status=None,
                                             col_scale_rows=None, N=None, gemm_scales=False,
-                                            noop_flag=None, glu_interleave=None):
+                                            noop_flag=None, glu_interleave=None, out=None):
     g, status = _grouped_args(row_offs, colblk_offs, status, col_scale_rows, x.device)
     return _bwd("clamped", dy, x, s, N, rowwise, colwise, want_dx, want_dscale, workspace, g,
-                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag,
+                gemm_scales=gemm_scales, clamp=(alpha, limit), noop_flag=noop_flag, out=out,
                 glu_interleave=glu_interleave), status
 
 

@@ -159,17 +159,26 @@ def ncu_traffic(workload, kernel, dirs_name):
     return None
 
 
-def act_api(mg, act, glu_interleave=0):
-    """(grouped forward, grouped backward, extra keyword arguments) of an
-    activation; ClampedSwiGLU at the default slope and limit; gate and up
-    interleaved in blocks of `glu_interleave` columns when it is non-zero."""
+def act_api(mg, act, glu_interleave=0, staged=False):
+    """(grouped forward, grouped backward, forward and backward extra keyword
+    arguments) of an activation; ClampedSwiGLU at the default slope and limit;
+    gate and up interleaved in blocks of `glu_interleave` columns when it is
+    non-zero; SwiGLU's forward with staged rounding when `staged`."""
+    if act == "srelu":
+        if glu_interleave or staged:
+            raise SystemExit("SReLU takes neither --glu-interleave nor --staged")
+        return mg.grouped_scaled_srelu_mxfp8_fwd, mg.grouped_scaled_srelu_mxfp8_bwd, {}, {}
     extra = {"glu_interleave": glu_interleave} if glu_interleave else {}
     if act == "clamped":
+        if staged:
+            raise SystemExit("ClampedSwiGLU has no staged rounding")
         mg.init_clamped()
         extra.update(alpha=mg.ops.CLAMPED_ALPHA, limit=mg.ops.CLAMPED_LIMIT)
         return (mg.grouped_scaled_clamped_swiglu_mxfp8_fwd,
-                mg.grouped_scaled_clamped_swiglu_mxfp8_bwd, extra)
-    return mg.grouped_scaled_swiglu_mxfp8_fwd, mg.grouped_scaled_swiglu_mxfp8_bwd, extra
+                mg.grouped_scaled_clamped_swiglu_mxfp8_bwd, extra, dict(extra))
+    fwd_extra = dict(extra, staged_rounding=True) if staged else dict(extra)
+    return (mg.grouped_scaled_swiglu_mxfp8_fwd, mg.grouped_scaled_swiglu_mxfp8_bwd, fwd_extra,
+            extra)
 
 
 def max_over_ranks(value, world, device):
@@ -214,16 +223,19 @@ def run_ours(args):
     mg.init()
     wl = WORKLOADS[args.workload]
     dirs = DIRS[args.dirs]
-    inp = make_inputs(wl, device=dev)
+    srelu = args.act == "srelu"
+    if srelu and not wl.srelu_N:
+        raise SystemExit(f"workload {wl.key} has no SReLU input")
+    inp = make_inputs(wl, device=dev, srelu=srelu)
     x, s, dy = inp["x"], inp["s"], inp["dy"]
     assert dy is not None, "the benchmark workload needs a backward (dY)"
     m_host = inp["m_splits"]
     m_dev = m_host.to(dev)
     E = int(m_host.numel())
     S = int(((m_host + 31) // 32).sum())
-    M, N = wl.M, wl.N
+    M, N = wl.M, (wl.srelu_N if srelu else wl.N)
     rw, cw = bool(dirs & 1), bool(dirs & 2)
-    bm = byte_model(M, N, E, dirs, S=S)
+    bm = byte_model(M, N, E, dirs, srelu=srelu, S=S)
     step_bytes = bm["splits"] + bm["fwd"] + bm["bwd"]
 
     stream = torch.cuda.current_stream(dev)
@@ -238,15 +250,16 @@ def run_ours(args):
         return mg.splits_to_offsets(m_dev, M)
 
     gemm = args.scales == "gemm"
-    fwd_api, bwd_api, extra = act_api(mg, args.act, args.glu_interleave)
+    fwd_api, bwd_api, fwd_extra, bwd_extra = act_api(mg, args.act, args.glu_interleave,
+                                                     args.staged)
 
     def fwd(ro, cb, st):
         return fwd_api(x, s, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, status=st,
-                       gemm_scales=gemm, **extra)
+                       gemm_scales=gemm, **fwd_extra)
 
     def bwd(ro, cb, st):
         return bwd_api(dy, x, s, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, workspace=ws,
-                       status=st, gemm_scales=gemm, **extra)
+                       status=st, gemm_scales=gemm, **bwd_extra)
 
     # eager warm-up
     for i in range(3):
@@ -378,7 +391,7 @@ def run_ours(args):
         "data": "synthetic (seeded torch generators; shapes and statistics of the pages' workloads)",
         "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
                    "dirs": args.dirs, "scales": args.scales, "activation": args.act,
-                   "glu_interleave": args.glu_interleave,
+                   "staged_rounding": bool(args.staged), "glu_interleave": args.glu_interleave,
                    "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
                    "launch": "eager" if args.eager else "one CUDA graph per step (events at its ends only)",
                    "kernel_times": "eager events" if args.eager else "a second timed pass of the same steps, with event nodes between the calls",
@@ -403,7 +416,8 @@ def run_ours(args):
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, dirs, budget_s=args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(wl, dirs, budget_s=args.cpu_seconds, act=args.act,
+                                           staged=args.staged)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
@@ -419,10 +433,12 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
     while step i computes; the two copy directions use separate engines), with
     double-buffered device inputs and host outputs.  Timed from the first copy
     in to the last copy out."""
-    M, N = wl.M, wl.N
+    srelu = args.act == "srelu"
+    M, N = wl.M, (wl.srelu_N if srelu else wl.N)
     rw, cw = bool(dirs & 1), bool(dirs & 2)
     gemm = args.scales == "gemm"
-    fwd_api, bwd_api, extra = act_api(mg, args.act, args.glu_interleave)
+    fwd_api, bwd_api, fwd_extra, bwd_extra = act_api(mg, args.act, args.glu_interleave,
+                                                     args.staged)
     hin = [inp["x"].cpu().pin_memory(), inp["s"].cpu().pin_memory(),
            inp["dy"].cpu().pin_memory(), inp["m_splits"].clone().pin_memory()]
     h2d = sum(t.numel() * t.element_size() for t in hin)
@@ -445,9 +461,9 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
             s_comp.wait_event(loaded)
             ro, cb, st = mg.splits_to_offsets(md, M)
             f, _ = fwd_api(xd, sd, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, status=st,
-                           gemm_scales=gemm, **extra)
+                           gemm_scales=gemm, **fwd_extra)
             bw, _ = bwd_api(dyd, xd, sd, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S,
-                            status=st, gemm_scales=gemm, **extra)
+                            status=st, gemm_scales=gemm, **bwd_extra)
             outs = [t for t in (*f, *bw.mx, bw.dx, bw.dscale, st) if t is not None and t.numel()]
             done = torch.cuda.Event()
             done.record(s_comp)
@@ -485,7 +501,7 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     E = int(inp["m_splits"].numel())
-    bm = byte_model(M, N, E, dirs, S=S)
+    bm = byte_model(M, N, E, dirs, srelu=srelu, S=S)
     step_bytes = bm["splits"] + bm["fwd"] + bm["bwd"]
     return {"value": round(whole_job_gbs(world, steps, step_bytes, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
@@ -494,53 +510,64 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
 
 
 # ------------------------------------------------------------------ oracle timing
-def _oracle_sample(wl, dirs, rows):
+def _oracle_sample(wl, dirs, rows, act="swiglu"):
     """Inputs of the first `rows` rows of the workload, as numpy bit arrays."""
     from moe_gated_activation_b200.workloads import bf16_bits, make_inputs
-    inp = make_inputs(wl, device="cpu") if wl.M * wl.N <= (1 << 26) else None
+    srelu = act == "srelu"
+    N = wl.srelu_N if srelu else wl.N
+    inp = make_inputs(wl, device="cpu", srelu=srelu) if wl.M * N <= (1 << 26) else None
     if inp is None:
         # large workloads: draw the same law for a sample of rows only
         from moe_gated_activation_b200.workloads import random_case
-        c = random_case(rows, wl.N, wl.seed, std=wl.x_std)
+        c = random_case(rows, N, wl.seed, std=wl.x_std, width=N if srelu else 2 * N)
         return bf16_bits(c["x"]), c["s"].numpy(), bf16_bits(c["dy"])
     return (bf16_bits(inp["x"][:rows]), inp["s"][:rows].numpy().copy(),
             bf16_bits(inp["dy"][:rows]))
 
 
-def _oracle_step(oracle, xb, s, dyb, N, dirs):
-    oracle.act_fwd(xb, s, N, dirs)
-    oracle.act_bwd(dyb, xb, s, N, dirs)
+def _oracle_step(oracle, xb, s, dyb, N, dirs, act="swiglu", staged=False):
+    if act == "clamped":
+        oracle.clamped_fwd(xb, s, N, dirs)
+        oracle.clamped_bwd(dyb, xb, s, N, dirs)
+        return
+    a = oracle.SRELU if act == "srelu" else oracle.SWIGLU
+    oracle.act_fwd(xb, s, N, dirs, act=a, staged=staged)
+    oracle.act_bwd(dyb, xb, s, N, dirs, act=a)
 
 
-def _calibrate_rows(oracle, wl, dirs, budget_s):
-    xb, s, dyb = _oracle_sample(wl, dirs, 32)
+def _calibrate_rows(oracle, wl, dirs, budget_s, act="swiglu", staged=False):
+    xb, s, dyb = _oracle_sample(wl, dirs, 32, act)
+    N = wl.srelu_N if act == "srelu" else wl.N
     t0 = time.perf_counter()
-    _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+    _oracle_step(oracle, xb, s, dyb, N, dirs, act, staged)
     per32 = max(time.perf_counter() - t0, 1e-4)
     rows = int(budget_s / per32) * 32
     return max(32, min(wl.M, rows))
 
 
-def cpu_baseline(wl, dirs, budget_s=10.0):
+def cpu_baseline(wl, dirs, budget_s=10.0, act="swiglu", staged=False):
     import oracle
     oracle.sigmoid_table()
-    rows = _calibrate_rows(oracle, wl, dirs, budget_s)
-    xb, s, dyb = _oracle_sample(wl, dirs, rows)
+    srelu = act == "srelu"
+    N = wl.srelu_N if srelu else wl.N
+    rows = _calibrate_rows(oracle, wl, dirs, budget_s, act, staged)
+    xb, s, dyb = _oracle_sample(wl, dirs, rows, act)
     # whole passes over the sample until the budget is spent (a workload
     # smaller than the budget is passed over several times)
     passes = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+        _oracle_step(oracle, xb, s, dyb, N, dirs, act, staged)
         passes += 1
         dt = time.perf_counter() - t0
         if dt >= 0.9 * budget_s:
             break
-    bm = byte_model(rows, wl.N, 1, dirs)
+    bm = byte_model(rows, N, 1, dirs, srelu=srelu)
     return {"value": round(passes * (bm["fwd"] + bm["bwd"]) / dt / 1e9, 4), "unit": "GB/s",
             "cores": 1, "kind": "oracle",
-            "sample": f"rows [0, {rows}) of {wl.M} ({wl.key}) x {passes} pass(es), forward + "
-                      f"backward, dirs={dirs}, {dt:.1f} s single-threaded"}
+            "sample": f"rows [0, {rows}) of {wl.M} ({wl.key}) x {passes} pass(es), {act}"
+                      f"{' staged' if staged else ''} forward + backward, dirs={dirs}, "
+                      f"{dt:.1f} s single-threaded"}
 
 
 def run_reference(args):
@@ -589,8 +616,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--dirs", default="both", choices=list(DIRS))
-    ap.add_argument("--act", default="swiglu", choices=["swiglu", "clamped"],
-                    help="activation: SwiGLU, or ClampedSwiGLU (alpha 1.702, limit 7)")
+    ap.add_argument("--act", default="swiglu", choices=["swiglu", "clamped", "srelu"],
+                    help="activation: SwiGLU, ClampedSwiGLU (alpha 1.702, limit 7), or SReLU "
+                         "(on the workload's own SReLU input; c4 has one)")
+    ap.add_argument("--staged", action="store_true",
+                    help="SwiGLU forward with staged rounding (silu and h rounded to bf16)")
     ap.add_argument("--scales", default="rowmajor", choices=["rowmajor", "gemm"],
                     help="E8M0 scale layout: row-major, or the GEMM-ready 128 x 4 tiles")
     ap.add_argument("--glu-interleave", type=int, default=0,

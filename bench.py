@@ -374,7 +374,11 @@ def run_ours(args):
     dom_us = bwd_us if dom == "bwd" else fwd_us
     achieved = bm[dom] / (dom_us * 1e-6) / 1e9
     kname = "act_bwd_kernel" if dom == "bwd" else "act_fwd_kernel"
-    traffic = ncu_traffic(args.workload, kname, args.dirs)
+    # the profiled launches are the default variant (SwiGLU, halves layout,
+    # row-major scales, no staged rounding); other variants report none
+    default_variant = (args.act == "swiglu" and not args.staged and not args.glu_interleave
+                       and args.scales == "rowmajor")
+    traffic = ncu_traffic(args.workload, kname, args.dirs) if default_variant else None
     value = whole_job_gbs(world, args.steps, step_bytes, total_ms)
     out = {
         "metric": METRIC,

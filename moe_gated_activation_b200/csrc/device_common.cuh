@@ -88,10 +88,6 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf16_lo_p(uint32_t v) { return __uint_as_float(__byte_perm(v, 0u, 0x1044)); }
 __device__ __forceinline__ float bf16_hi_p(uint32_t v) { return __uint_as_float(__byte_perm(v, 0u, 0x3244)); }
 
-__device__ __forceinline__ float bf16_round(float v) {
-  return __bfloat162float(__float2bfloat16_rn(v));
-}
-
 // Two fp32 values -> packed bf16x2 (a in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);

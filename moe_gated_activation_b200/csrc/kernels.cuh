@@ -604,10 +604,13 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
         const float2 si01 = mul2(bf16x2_to_f2(G.x), sg01), si23 = mul2(bf16x2_to_f2(G.y), sg23);
         const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
         if (STAGED) {
-          h01 = mul2(make_float2(bf16_round(si01.x), bf16_round(si01.y)), u01);
-          h23 = mul2(make_float2(bf16_round(si23.x), bf16_round(si23.y)), u23);
-          h01 = make_float2(bf16_round(h01.x), bf16_round(h01.y));
-          h23 = make_float2(bf16_round(h23.x), bf16_round(h23.y));
+          // a = bf16(silu), h = bf16(a * u) (the product is exact in fp32),
+          // each pair rounded by one packed conversion
+          const float2 a01 = bf16x2_to_f2(pack_bf16x2(si01.x, si01.y));
+          const float2 a23 = bf16x2_to_f2(pack_bf16x2(si23.x, si23.y));
+          const float2 p01 = mul2(a01, u01), p23 = mul2(a23, u23);
+          h01 = bf16x2_to_f2(pack_bf16x2(p01.x, p01.y));
+          h23 = bf16x2_to_f2(pack_bf16x2(p23.x, p23.y));
         } else {
           h01 = mul2(si01, u01);
           h23 = mul2(si23, u23);

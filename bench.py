@@ -369,6 +369,7 @@ def run_ours(args):
 
     peak, peak_kind = measured_peak()
     mean = lambda v: sum(v) / len(v)
+    median = lambda v: sorted(v)[len(v) // 2]
     fwd_us, bwd_us = 1e3 * mean(fwd_ms), 1e3 * mean(bwd_ms)
     dom = "bwd" if bwd_us >= fwd_us else "fwd"
     dom_us = bwd_us if dom == "bwd" else fwd_us
@@ -406,10 +407,12 @@ def run_ours(args):
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes": bm[dom]},
         "kernels": {
-            "fwd": {"us": round(fwd_us, 2), "bytes": bm["fwd"],
+            "fwd": {"us": round(fwd_us, 2), "us_median": round(1e3 * median(fwd_ms), 2),
+                    "us_min": round(1e3 * min(fwd_ms), 2), "bytes": bm["fwd"],
                     "gbs": round(bm["fwd"] / (fwd_us * 1e-6) / 1e9, 1),
                     "frac": round(bm["fwd"] / (fwd_us * 1e-6) / 1e9 / peak, 4)},
-            "bwd": {"us": round(bwd_us, 2), "bytes": bm["bwd"],
+            "bwd": {"us": round(bwd_us, 2), "us_median": round(1e3 * median(bwd_ms), 2),
+                    "us_min": round(1e3 * min(bwd_ms), 2), "bytes": bm["bwd"],
                     "gbs": round(bm["bwd"] / (bwd_us * 1e-6) / 1e9, 1),
                     "frac": round(bm["bwd"] / (bwd_us * 1e-6) / 1e9 / peak, 4)},
             "splits_to_offsets": {"us": round(1e3 * mean(splits_ms), 2)},

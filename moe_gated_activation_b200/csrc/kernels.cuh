@@ -535,7 +535,6 @@ __device__ __forceinline__ void clamped_bwd_math(const Params& p, const float* s
   sigma_pair(sig, G.x, sg01.x, sg01.y);
   sigma_pair(sig, G.y, sg23.x, sg23.y);
   float2 g01 = bf16x2_to_f2(G.x), g23 = bf16x2_to_f2(G.y);
-  const bool cg0 = g01.x > L, cg1 = g01.y > L, cg2 = g23.x > L, cg3 = g23.y > L;
   clamp_gates(g01, sg01, p);
   clamp_gates(g23, sg23, p);
   const float2 si01 = mul2(g01, sg01), si23 = mul2(g23, sg23);
@@ -546,8 +545,11 @@ __device__ __forceinline__ void clamped_bwd_math(const Params& p, const float* s
   const float2 dga = mul2(mul2(p01, v01), ds01), dgb = mul2(mul2(p23, v23), ds23);
   const float2 dua = mul2(p01, si01), dub = mul2(p23, si23);
   const auto cu = [L](float u) { return fabsf(u) > L; };
-  dg01 = make_float2(cg0 ? 0.0f : dga.x, cg1 ? 0.0f : dga.y);
-  dg23 = make_float2(cg2 ? 0.0f : dgb.x, cg3 ? 0.0f : dgb.y);
+  // the gate comparisons are made here, from the input bits, rather than
+  // kept from the clamp (fewer values live across the math)
+  const auto cg = [L](float g) { return g > L; };
+  dg01 = make_float2(cg(bf16_lo_p(G.x)) ? 0.0f : dga.x, cg(bf16_hi_p(G.x)) ? 0.0f : dga.y);
+  dg23 = make_float2(cg(bf16_lo_p(G.y)) ? 0.0f : dgb.x, cg(bf16_hi_p(G.y)) ? 0.0f : dgb.y);
   du01 = make_float2(cu(u01.x) ? 0.0f : dua.x, cu(u01.y) ? 0.0f : dua.y);
   du23 = make_float2(cu(u23.x) ? 0.0f : dub.x, cu(u23.y) ? 0.0f : dub.y);
   h01 = mul2(si01, v01);

@@ -8,20 +8,20 @@ group.  The metric is algorithmic bytes / device time (GB/s), the byte model of
 the pytorch/ao PR #4743 performance table extended with the per-row scale and
 the backward's bf16 dX and dscale.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5]
                     [--dirs both|row|col] [--impl ours|reference]
 
-N > 1 runs under torchrun: every rank runs its own replica of the workload on
-its GPU (rows are independent; there is no exchange step), and the device time
-is the max over ranks.  L2 is flushed (written then read, 256 MiB) before every
-timed step, outside the timed events.
+The default workload is the largest single-GPU one (c5: X bf16 [131072, 16384],
+32 Zipf-skewed experts).  N > 1 runs under torchrun: every rank runs its own
+replica of the workload on its GPU (rows are independent; there is no exchange
+step), and the device time is the max over ranks.  L2 is flushed (written then
+read, 256 MiB) before every timed step, outside the timed events.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import sys
@@ -208,6 +208,28 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+# ------------------------------------------------------------------ config
+def workload_config(args, wl, M, N, E, world):
+    """The `config` of a bench line: the same dict for both arms."""
+    return {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
+            "dirs": args.dirs, "scales": args.scales, "activation": args.act,
+            "staged_rounding": bool(args.staged), "glu_interleave": args.glu_interleave,
+            "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
+            "l2": "flushed before every timed step (256 MiB written then read), outside the "
+                  "timed events",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def device_error_word():
+    """The library's device error word (reading clears it): non-zero if a
+    kernel gave up a bounded wait, i.e. its outputs are incomplete."""
+    import ctypes
+    from moe_gated_activation_b200 import _capi
+    v = ctypes.c_uint32(0)
+    _capi.call("moeact_device_error", ctypes.byref(v))
+    return v.value
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import moe_gated_activation_b200 as mg
@@ -261,82 +283,84 @@ def run_ours(args):
         return bwd_api(dy, x, s, ro, cb, rowwise=rw, colwise=cw, col_scale_rows=S, workspace=ws,
                        status=st, gemm_scales=gemm, **bwd_extra)
 
-    # eager warm-up
+    # eager warm-up; the offsets of the warm-up stay for the per-kernel graphs
     for i in range(3):
-        ro, cb, st = splits()
-        fwd(ro, cb, st)
-        bwd(ro, cb, st)
+        ro0, cb0, st0 = splits()
+        fwd(ro0, cb0, st0)
+        bwd(ro0, cb0, st0)
     torch.cuda.synchronize()
+    if int(st0.item()) != 0:
+        raise SystemExit(f"device status {int(st0.item())} from the warm-up step")
+
+    def capture(body):
+        """`body` captured as one CUDA graph between two event-record nodes."""
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                ev[0].record(side)
+                out = body()
+                ev[1].record(side)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        return g, ev, out
 
     if args.eager:
-        def run_step(ev):
-            ev[0].record(stream)
+        def step_body():
             ro, cb, st = splits()
-            ev[1].record(stream)
             fwd(ro, cb, st)
-            ev[2].record(stream)
             bwd(ro, cb, st)
-            ev[3].record(stream)
+            return st
+        graphs = None
     else:
-        # The step captured as a CUDA graph and replayed once per step.  The
-        # timed graph has event-record nodes only at its ends (an event node
-        # between two kernels costs a few microseconds); a second graph with
-        # event nodes between the calls gives the per-kernel times.
-        def capture(evs):
-            g = torch.cuda.CUDAGraph()
-            side = torch.cuda.Stream(dev)
-            side.wait_stream(stream)
-            with torch.cuda.stream(side):
-                with torch.cuda.graph(g, stream=side):
-                    evs[0].record(side)
-                    ro, cb, st = splits()
-                    if len(evs) == 4:
-                        evs[1].record(side)
-                    fwd(ro, cb, st)
-                    if len(evs) == 4:
-                        evs[2].record(side)
-                    bwd(ro, cb, st)
-                    evs[-1].record(side)
-            stream.wait_stream(side)
-            torch.cuda.synchronize()
-            return g
+        # The step as one CUDA graph with event nodes only at its ends (the
+        # headline); each call of the step as a graph of its own, timed the
+        # same way, for the per-kernel times (an event node between two
+        # kernels of one graph would add a few microseconds to each).
+        def step_body():
+            ro, cb, st = splits()
+            fwd(ro, cb, st)
+            bwd(ro, cb, st)
+            return st
+        graphs = {"step": capture(step_body),
+                  "splits": capture(splits),
+                  "fwd": capture(lambda: fwd(ro0, cb0, st0)),
+                  "bwd": capture(lambda: bwd(ro0, cb0, st0))}
 
-        sev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-        graph = capture(sev)
-        graph_parts = capture(gev)
-
-    def timed_steps(n, record, parts=False):
-        """n steps, each after an L2 flush; returns per-step [splits, fwd, bwd, total] ms
-        (parts=False: the step graph, total only)."""
+    def timed(name, n, record):
+        """n replays of graph `name` (eager: n calls), each after an L2 flush;
+        the device time of each in ms."""
         out = []
         for i in range(n):
             do_flush(i)
-            if args.eager:
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-                run_step(ev)
-                if record:
-                    out.append(ev)
-            elif parts:
-                graph_parts.replay()
-                torch.cuda.synchronize()
-                if record:
-                    out.append([gev[0].elapsed_time(gev[1]), gev[1].elapsed_time(gev[2]),
-                                gev[2].elapsed_time(gev[3]), gev[0].elapsed_time(gev[3])])
+            if graphs is None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                if name == "step":
+                    step_body()
+                elif name == "splits":
+                    splits()
+                elif name == "fwd":
+                    fwd(ro0, cb0, st0)
+                else:
+                    bwd(ro0, cb0, st0)
+                e1.record(stream)
+                e1.synchronize()
+                ms = e0.elapsed_time(e1)
             else:
-                graph.replay()
+                g, ev, _ = graphs[name]
+                g.replay()
                 torch.cuda.synchronize()
-                if record:
-                    out.append([None, None, None, sev[0].elapsed_time(sev[1])])
-        if args.eager:
-            torch.cuda.synchronize()
-            out = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
-                    e[0].elapsed_time(e[3])] for e in out]
+                ms = ev[0].elapsed_time(ev[1])
+            if record:
+                out.append(ms)
         return out
 
-    timed_steps(args.warmup, False)
-    if not args.eager:
-        timed_steps(args.warmup, False, parts=True)
+    for name in ("step", "splits", "fwd", "bwd"):
+        timed(name, args.warmup, False)
     torch.cuda.synchronize()
     sampler = ClockSampler(dev)
     with sampler:
@@ -345,32 +369,37 @@ def run_ours(args):
         torch.cuda.synchronize()
         sampler.active = True
         wall0 = time.perf_counter()
-        times = timed_steps(args.steps, True)
+        times = timed("step", args.steps, True)
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
-        # per-kernel times: the same steps again, with event nodes between the calls
-        parts = times if args.eager else timed_steps(args.steps, True, parts=True)
+        # per-kernel times: each call alone, the same number of replays
+        parts = {k: timed(k, args.steps, True) for k in ("splits", "fwd", "bwd")}
         torch.cuda.synchronize()
         sampler.active = False
         if world > 1:
             torch.distributed.barrier()
-    if not args.eager:
-        del graph, graph_parts
-    splits_ms = [t[0] for t in parts]
-    fwd_ms = [t[1] for t in parts]
-    bwd_ms = [t[2] for t in parts]
-    total_ms = max_over_ranks(sum(t[3] for t in times), world, dev)
+    total_ms = max_over_ranks(sum(times), world, dev)
+    # a kernel that gave up a bounded wait leaves its outputs incomplete: no number
+    err = device_error_word()
+    st_step = graphs["step"][2] if graphs is not None else st0
+    if err != 0 or int(st_step.item()) != 0 or int(st0.item()) != 0:
+        raise SystemExit(f"device error word {err:#x}, status {int(st_step.item())}: "
+                         "the timed kernels did not complete their work")
+    graphs = None
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
     # end to end through the public API with host buffers (pinned), H2D of the
     # step's inputs and D2H of every output inside the timed region
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world)
+        e2e = run_e2e(mg, wl, inp, dev, dirs, S, args, world)
+        if device_error_word() != 0:
+            raise SystemExit("device error word set during the end-to-end run")
 
     peak, peak_kind = measured_peak()
     mean = lambda v: sum(v) / len(v)
-    median = lambda v: sorted(v)[len(v) // 2]
-    fwd_us, bwd_us = 1e3 * mean(fwd_ms), 1e3 * mean(bwd_ms)
+    fwd_us, bwd_us = 1e3 * mean(parts["fwd"]), 1e3 * mean(parts["bwd"])
     dom = "bwd" if bwd_us >= fwd_us else "fwd"
     dom_us = bwd_us if dom == "bwd" else fwd_us
     achieved = bm[dom] / (dom_us * 1e-6) / 1e9
@@ -380,7 +409,24 @@ def run_ours(args):
     default_variant = (args.act == "swiglu" and not args.staged and not args.glu_interleave
                        and args.scales == "rowmajor")
     traffic = ncu_traffic(args.workload, kname, args.dirs) if default_variant else None
+
+    def kstats(name):
+        v = parts[name]
+        us = 1e3 * mean(v)
+        d = {"us": round(us, 2), "us_median": round(1e3 * statistics.median(v), 2),
+             "us_min": round(1e3 * min(v), 2)}
+        if name in bm and name != "splits":
+            d.update(bytes=bm[name], gbs=round(bm[name] / (us * 1e-6) / 1e9, 1),
+                     frac=round(bm[name] / (us * 1e-6) / 1e9 / peak, 4))
+        return d
+
     value = whole_job_gbs(world, args.steps, step_bytes, total_ms)
+    config = workload_config(args, wl, M, N, E, world)
+    config.update(
+        launch="eager" if args.eager else "one CUDA graph per step (event nodes at its ends only)",
+        kernel_times="each call alone (its own CUDA graph, event nodes at its ends), after an "
+                     "L2 flush, as many replays as timed steps; `us` is the mean, which the "
+                     "roofline uses; bwd = act_bwd_kernel + dscale_reduce_kernel")
     out = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -394,69 +440,63 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic (seeded torch generators; shapes and statistics of the pages' workloads)",
-        "config": {"workload": f"{wl.key}: {wl.title}", "M": M, "N": N, "groups": E,
-                   "dirs": args.dirs, "scales": args.scales, "activation": args.act,
-                   "staged_rounding": bool(args.staged), "glu_interleave": args.glu_interleave,
-                   "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
-                   "launch": "eager" if args.eager else "one CUDA graph per step (events at its ends only)",
-                   "kernel_times": "eager events" if args.eager else "a second timed pass of the same steps, with event nodes between the calls",
-                   "l2": "flushed before every step (256 MiB written then read), outside the timed events",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": config,
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes": bm[dom]},
-        "kernels": {
-            "fwd": {"us": round(fwd_us, 2), "us_median": round(1e3 * median(fwd_ms), 2),
-                    "us_min": round(1e3 * min(fwd_ms), 2), "bytes": bm["fwd"],
-                    "gbs": round(bm["fwd"] / (fwd_us * 1e-6) / 1e9, 1),
-                    "frac": round(bm["fwd"] / (fwd_us * 1e-6) / 1e9 / peak, 4)},
-            "bwd": {"us": round(bwd_us, 2), "us_median": round(1e3 * median(bwd_ms), 2),
-                    "us_min": round(1e3 * min(bwd_ms), 2), "bytes": bm["bwd"],
-                    "gbs": round(bm["bwd"] / (bwd_us * 1e-6) / 1e9, 1),
-                    "frac": round(bm["bwd"] / (bwd_us * 1e-6) / 1e9 / peak, 4)},
-            "splits_to_offsets": {"us": round(1e3 * mean(splits_ms), 2)},
-        },
+                     "algorithmic_bytes": bm[dom], "time_stat": "mean"},
+        "kernels": {"fwd": kstats("fwd"), "bwd": kstats("bwd"),
+                    "splits_to_offsets": kstats("splits")},
         "wall_s_timed_region": round(wall, 4),
         "gpu_launches": 4 * args.steps,   # splits, fwd, bwd, dscale reduction per step
+        "device_error_word": 0,
         "clocks": sampler.summary(),
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, dirs, budget_s=args.cpu_seconds, act=args.act,
-                                           staged=args.staged)
+        out["cpu_baseline"] = cpu_baseline(wl, dirs, inp, budget_s=args.cpu_seconds,
+                                           act=args.act, staged=args.staged)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(out))
 
 
-def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
+def run_e2e(mg, wl, inp, dev, dirs, S, args, world):
     """The step through the public API with host buffers: every step copies its
     inputs (X, s, dY, m_splits) from pinned host memory to the device, runs
     splits_to_offsets, the forward and the backward, and copies every output
     back to pinned host memory.  Three streams pipeline consecutive steps
     (host->device copies of step i+1 and device->host copies of step i-1 run
     while step i computes; the two copy directions use separate engines), with
-    double-buffered device inputs and host outputs.  Timed from the first copy
-    in to the last copy out."""
+    double-buffered device inputs.  The host output buffers are double-buffered
+    too when a step's outputs are small (<= 4 GiB), else shared by all steps
+    (nothing reads them on the host, and the copies into them are serialised
+    on one stream), which keeps pinned host memory bounded at the largest
+    workloads.  Timed from the first copy in to the last copy out."""
     srelu = args.act == "srelu"
     M, N = wl.M, (wl.srelu_N if srelu else wl.N)
     rw, cw = bool(dirs & 1), bool(dirs & 2)
     gemm = args.scales == "gemm"
     fwd_api, bwd_api, fwd_extra, bwd_extra = act_api(mg, args.act, args.glu_interleave,
                                                      args.staged)
-    hin = [inp["x"].cpu().pin_memory(), inp["s"].cpu().pin_memory(),
-           inp["dy"].cpu().pin_memory(), inp["m_splits"].clone().pin_memory()]
+
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    hin = [pinned_copy(inp["x"]), pinned_copy(inp["s"]), pinned_copy(inp["dy"]),
+           inp["m_splits"].clone().pin_memory()]
     h2d = sum(t.numel() * t.element_size() for t in hin)
     dbuf = [[torch.empty_like(t, device=dev) for t in hin] for _ in range(2)]
     s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     hout = [None, None]
+    shared_out = [False]
 
     def step(i, in_free, out_free):
-        """Enqueue step i; returns (inputs consumed, outputs copied) events."""
+        """Enqueue step i; returns (outputs computed, outputs copied) events."""
         b = i & 1
-        xd, sd, dyd, md = dbuf[b]
         with torch.cuda.stream(s_in):
             if in_free[b] is not None:
                 s_in.wait_event(in_free[b])
@@ -464,6 +504,7 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
                 d.copy_(h, non_blocking=True)
             loaded = torch.cuda.Event()
             loaded.record(s_in)
+        xd, sd, dyd, md = dbuf[b]
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(loaded)
             ro, cb, st = mg.splits_to_offsets(md, M)
@@ -474,8 +515,12 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
             outs = [t for t in (*f, *bw.mx, bw.dx, bw.dscale, st) if t is not None and t.numel()]
             done = torch.cuda.Event()
             done.record(s_comp)
-        if hout[b] is None:
-            hout[b] = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        if hout[0] is None:
+            nbytes = sum(t.numel() * t.element_size() for t in outs)
+            shared_out[0] = nbytes > (4 << 30)
+            hout[0] = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+            hout[1] = hout[0] if shared_out[0] else \
+                [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
         with torch.cuda.stream(s_out):
             s_out.wait_event(done)
             if out_free[b] is not None:
@@ -489,12 +534,14 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
 
     in_free, out_free = [None, None], [None, None]
     keep = []                                  # outputs of the last steps stay referenced
-    for i in range(4):                         # warm-up: host outputs, allocator pool
+    for i in range(3):                         # warm-up: host outputs, allocator pool
         in_free[i & 1], out_free[i & 1], outs = step(i, in_free, out_free)
         keep = (keep + [outs])[-2:]
     torch.cuda.synchronize()
     d2h = sum(t.numel() * t.element_size() for t in outs)
-    steps = max(2, min(args.steps, 20))
+    # a bounded number of steps (at the largest workload a step moves ~17 GB
+    # over PCIe)
+    steps = max(2, min(args.steps, 20 if d2h + h2d <= (4 << 30) else 6))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -510,26 +557,27 @@ def run_e2e(mg, wl, inp, dev, stream, dirs, S, args, world):
     E = int(inp["m_splits"].numel())
     bm = byte_model(M, N, E, dirs, srelu=srelu, S=S)
     step_bytes = bm["splits"] + bm["fwd"] + bm["bwd"]
+    pipe = "copy-in / compute / copy-out streams, double-buffered device inputs, " + \
+        ("one host output buffer for all steps" if shared_out[0] else
+         "double-buffered host outputs")
     return {"value": round(whole_job_gbs(world, steps, step_bytes, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 4),
-            "pipeline": "copy-in / compute / copy-out streams, double-buffered"}
+            "ms_per_step": round(ms / steps, 4), "pipeline": pipe}
 
 
 # ------------------------------------------------------------------ oracle timing
-def _oracle_sample(wl, dirs, rows, act="swiglu"):
-    """Inputs of the first `rows` rows of the workload, as numpy bit arrays."""
-    from moe_gated_activation_b200.workloads import bf16_bits, make_inputs
-    srelu = act == "srelu"
-    N = wl.srelu_N if srelu else wl.N
-    inp = make_inputs(wl, device="cpu", srelu=srelu) if wl.M * N <= (1 << 26) else None
-    if inp is None:
-        # large workloads: draw the same law for a sample of rows only
-        from moe_gated_activation_b200.workloads import random_case
-        c = random_case(rows, N, wl.seed, std=wl.x_std, width=N if srelu else 2 * N)
-        return bf16_bits(c["x"]), c["s"].numpy(), bf16_bits(c["dy"])
-    return (bf16_bits(inp["x"][:rows]), inp["s"][:rows].numpy().copy(),
-            bf16_bits(inp["dy"][:rows]))
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def _oracle_rows(x, s, dy, rows):
+    """The first `rows` rows of the inputs (torch tensors on any device), as
+    numpy bit arrays for the oracle."""
+    from moe_gated_activation_b200.workloads import bf16_bits
+    return (bf16_bits(x[:rows]), s[:rows].cpu().numpy().copy(), bf16_bits(dy[:rows]))
 
 
 def _oracle_step(oracle, xb, s, dyb, N, dirs, act="swiglu", staged=False):
@@ -542,43 +590,88 @@ def _oracle_step(oracle, xb, s, dyb, N, dirs, act="swiglu", staged=False):
     oracle.act_bwd(dyb, xb, s, N, dirs, act=a)
 
 
-def _calibrate_rows(oracle, wl, dirs, budget_s, act="swiglu", staged=False):
-    xb, s, dyb = _oracle_sample(wl, dirs, 32, act)
-    N = wl.srelu_N if act == "srelu" else wl.N
+class OraclePool:
+    """The oracle over independent 32-row slabs on `cores` host threads: the
+    sample's rows are cut into one chunk of whole 32-row slabs per thread
+    (a slab is a complete set of colwise blocks, so each chunk is a complete
+    problem), and each thread runs the oracle's forward and backward on its
+    chunk.  The oracle's C calls release the interpreter lock, so the threads
+    run in parallel; the oracle itself is unchanged (single-threaded per
+    call)."""
+
+    def __init__(self, oracle, xb, s, dyb, N, dirs, act, staged, cores):
+        import concurrent.futures
+        rows = xb.shape[0]
+        n = max(1, min(cores, rows // 32))
+        per = (rows // 32 + n - 1) // n * 32
+        self.chunks = [(xb[i:i + per], s[i:i + per], dyb[i:i + per])
+                       for i in range(0, rows, per)]
+        self.threads = len(self.chunks)
+        self.ex = concurrent.futures.ThreadPoolExecutor(self.threads)
+        self.args = (oracle, N, dirs, act, staged)
+
+    def step(self):
+        oracle, N, dirs, act, staged = self.args
+        futs = [self.ex.submit(_oracle_step, oracle, xb, s, dyb, N, dirs, act, staged)
+                for xb, s, dyb in self.chunks]
+        for f in futs:
+            f.result()
+
+    def close(self):
+        self.ex.shutdown()
+
+
+def _sample_rows(oracle, x, s, dy, N, dirs, seconds, cores, M, act="swiglu", staged=False):
+    """Rows of a sample the oracle passes over in about `seconds` on `cores`
+    threads: single-thread time of 32 rows, scaled by the thread count;
+    whole 32-row slabs, at least one per thread where the workload has them,
+    at most 2^28 input elements (host memory)."""
+    xb, sv, dyb = _oracle_rows(x, s, dy, 32)
     t0 = time.perf_counter()
-    _oracle_step(oracle, xb, s, dyb, N, dirs, act, staged)
+    _oracle_step(oracle, xb, sv, dyb, N, dirs, act, staged)
     per32 = max(time.perf_counter() - t0, 1e-4)
-    rows = int(budget_s / per32) * 32
-    return max(32, min(wl.M, rows))
+    rows = int(seconds * cores / per32) * 32
+    cap = max(32, ((1 << 28) // max(1, x.shape[1])) // 32 * 32)
+    return max(32, min(M, rows, cap))
 
 
-def cpu_baseline(wl, dirs, budget_s=10.0, act="swiglu", staged=False):
+def cpu_baseline(wl, dirs, inp, budget_s=10.0, act="swiglu", staged=False):
+    """The oracle on the first rows of the GPU arm's own inputs, on every host
+    core, for about `budget_s` seconds."""
     import oracle
     oracle.sigmoid_table()
     srelu = act == "srelu"
     N = wl.srelu_N if srelu else wl.N
-    rows = _calibrate_rows(oracle, wl, dirs, budget_s, act, staged)
-    xb, s, dyb = _oracle_sample(wl, dirs, rows, act)
+    cores = host_cores()
+    rows = _sample_rows(oracle, inp["x"], inp["s"], inp["dy"], N, dirs, budget_s / 2, cores,
+                        wl.M, act, staged)
+    xb, s, dyb = _oracle_rows(inp["x"], inp["s"], inp["dy"], rows)
+    pool = OraclePool(oracle, xb, s, dyb, N, dirs, act, staged, cores)
     # whole passes over the sample until the budget is spent (a workload
     # smaller than the budget is passed over several times)
     passes = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_step(oracle, xb, s, dyb, N, dirs, act, staged)
+        pool.step()
         passes += 1
         dt = time.perf_counter() - t0
         if dt >= 0.9 * budget_s:
             break
+    pool.close()
     bm = byte_model(rows, N, 1, dirs, srelu=srelu)
     return {"value": round(passes * (bm["fwd"] + bm["bwd"]) / dt / 1e9, 4), "unit": "GB/s",
-            "cores": 1, "kind": "oracle",
-            "sample": f"rows [0, {rows}) of {wl.M} ({wl.key}) x {passes} pass(es), {act}"
-                      f"{' staged' if staged else ''} forward + backward, dirs={dirs}, "
-                      f"{dt:.1f} s single-threaded"}
+            "cores": pool.threads, "host_cores": cores, "kind": "oracle",
+            "sample": f"rows [0, {rows}) of {wl.M} ({wl.key}, the timed arm's own inputs) x "
+                      f"{passes} pass(es), {act}{' staged' if staged else ''} forward + "
+                      f"backward, dirs={dirs}, {dt:.1f} s on {pool.threads} threads "
+                      f"(32-row slabs)"}
 
 
 def run_reference(args):
-    from moe_gated_activation_b200.workloads import WORKLOADS
+    """The reference arm: the C oracle (the only runnable definition of the
+    method; the pages hold no implementation) on the machine's host cores, over
+    a bounded sample of the workload's rows per step."""
+    from moe_gated_activation_b200.workloads import WORKLOADS, make_inputs
     import oracle
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -586,31 +679,40 @@ def run_reference(args):
         return
     wl = WORKLOADS[args.workload]
     dirs = DIRS[args.dirs]
+    srelu = args.act == "srelu"
+    N = wl.srelu_N if srelu else wl.N
+    # the same seeded inputs as the GPU arm (drawn on the GPU when there is one)
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(wl, device=gen_dev, srelu=srelu)
+    E = int(inp["m_splits"].numel())
     oracle.sigmoid_table()
+    cores = host_cores()
     per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
-    rows = _calibrate_rows(oracle, wl, dirs, per_step)
-    xb, s, dyb = _oracle_sample(wl, dirs, rows)
+    rows = _sample_rows(oracle, inp["x"], inp["s"], inp["dy"], N, dirs, per_step, cores, wl.M,
+                        args.act, args.staged)
+    xb, s, dyb = _oracle_rows(inp["x"], inp["s"], inp["dy"], rows)
+    del inp
+    pool = OraclePool(oracle, xb, s, dyb, N, dirs, args.act, args.staged, cores)
     for _ in range(args.warmup):
-        _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+        pool.step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_step(oracle, xb, s, dyb, wl.N, dirs)
+        pool.step()
     dt = time.perf_counter() - t0
-    bm = byte_model(rows, wl.N, 1, dirs)
+    pool.close()
+    bm = byte_model(rows, N, 1, dirs, srelu=srelu)
     value = args.steps * (bm["fwd"] + bm["bwd"]) / dt / 1e9
-    sample = (f"rows [0, {rows}) of {wl.M} ({wl.key}) per step, forward + backward, "
-              f"single-threaded C oracle")
+    sample = (f"rows [0, {rows}) of {wl.M} ({wl.key}) per step, forward + backward, C oracle "
+              f"on {pool.threads} host threads (32-row slabs)")
     out = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-           "data": "synthetic (seeded torch generators)",
-           "config": {"workload": f"{wl.key}: {wl.title}", "M": wl.M, "N": wl.N,
-                      "groups": wl.groups, "dirs": args.dirs, "activation": "swiglu",
-                      "step": "splits_to_offsets + grouped fwd + grouped bwd (dx, dscale)",
-                      "parallelism": "host cores (rank 0)"},
-           "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
-                            "kind": "oracle", "sample": sample},
+           "data": "synthetic (seeded torch generators; shapes and statistics of the pages' "
+                   "workloads)",
+           "config": workload_config(args, wl, wl.M, N, E, 1),
+           "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": pool.threads,
+                            "host_cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
@@ -621,7 +723,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "c5"])
+    ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--dirs", default="both", choices=list(DIRS))
     ap.add_argument("--act", default="swiglu", choices=["swiglu", "clamped", "srelu"],
                     help="activation: SwiGLU, ClampedSwiGLU (alpha 1.702, limit 7), or SReLU "

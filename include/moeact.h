@@ -285,9 +285,12 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
  *   with glu_interleave = 0 and without the workspace: the dscale partial sums go to a 16 MiB array built
  *   into the library (held by every GPU that loads it, until exit), so with
  *   dscale requested ceil(N/128) * M must not exceed 4194304 (else
- *   MOEACT_ERANGE, nothing launched).  Allocates nothing.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   MOEACT_ERANGE, nothing launched; shapes are checked first, as for
+ *   scaled_swiglu_mxfp8_bwd).  Allocates nothing.
+ *   The array's device address is looked up (cudaGetSymbolAddress) with the
+ *   rest of the per-device set-up, by moeact_init() or the first call of any
+ *   entry point on the device; as for every entry point, that first call
+ *   must not be inside a stream capture (MOEACT_EUNSUPPORTED).
  *   All calls share the array and it keeps the last call's contents; nothing
  *   in it needs to start at zero (every partial is written before it is
  *   read).  Calls that overlap on the GPU (other streams, other host threads)
@@ -356,8 +359,32 @@ moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream)
  * sigmoid table's copy) -- a defensive bound that ends the kernel instead of
  * letting it hang -- or found its shared-memory sigmoid table outside the
  * 16-bit address range its lookups use (bit 3); never expected in normal
- * operation.  Synchronous.  No counterpart on the pages. */
+ * operation.  Every wait gives up after one second of GPU time (the global
+ * timer), and the kernel then waits (bounded again) for its copies in flight
+ * and returns, its outputs incomplete.  Bit 4 is set only by
+ * moeact_wait_selftest.  Synchronous.  No counterpart on the pages. */
+#define MOEACT_DEVERR_FWD_WAIT 0x1u
+#define MOEACT_DEVERR_BWD_WAIT 0x2u
+#define MOEACT_DEVERR_TABLE_WAIT 0x4u
+#define MOEACT_DEVERR_TABLE_ADDR 0x8u
+#define MOEACT_DEVERR_WAIT_SELFTEST 0x10u
 moeact_status moeact_device_error(uint32_t* flags);
+
+/* ---------------------------------------------------------------------
+ * moeact_wait_selftest -- checks the bounded wait of the fused kernels on the
+ * GPU without any fault: one thread sets up an mbarrier that completes on
+ * one arrival, arrives on it only when `arrive` is 1 (with 0 nothing ever
+ * arrives), and waits for it through the same bounded-wait routine the fused
+ * kernels use, with a limit of `limit_us` microseconds (1 .. 2000000, else
+ * MOEACT_ERANGE) instead of their one second.  A wait that gives up sets
+ * MOEACT_DEVERR_WAIT_SELFTEST in the device error word, as a fused kernel
+ * sets its bit.  result: device memory, 2 x uint64, 8-byte aligned
+ * (MOEACT_EALIGN): result[0] = 1 if the wait saw the barrier complete, 0 if
+ * it gave up; result[1] = nanoseconds waited.  Asynchronous on `stream`.
+ * No counterpart on the pages (failure detection of this library).
+ * ------------------------------------------------------------------- */
+moeact_status moeact_wait_selftest(int arrive, uint32_t limit_us, uint64_t* result,
+                                   void* stream);
 
 /* ---------------------------------------------------------------------
  * Test hook: sigma for every bf16 bit pattern (65536 fp32 values written to

@@ -18,6 +18,10 @@
 #include "variants.cuh"
 
 namespace moeact {
+static_assert(kErrFwdWait == MOEACT_DEVERR_FWD_WAIT && kErrBwdWait == MOEACT_DEVERR_BWD_WAIT &&
+                  kErrTableWait == MOEACT_DEVERR_TABLE_WAIT &&
+                  kErrTableAddr == MOEACT_DEVERR_TABLE_ADDR,
+              "device error bits differ from include/moeact.h");
 namespace {
 
 thread_local char t_err[512] = "";
@@ -55,6 +59,20 @@ __device__ uint32_t g_err_word;
 uint32_t* g_err_ptr[kMaxDevices];
 float* g_sig_ptr[kMaxDevices];   // g_sigma_table on each device
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Scratch of the allocation-free backward (scaled_swiglu_mxfp8_bwd_noalloc).
+// Some callers cannot hand the library a workspace: code that runs where a
+// device allocation is not acceptable at the point of the call (cudaMalloc
+// may synchronise the device and its latency is unbounded), or a host
+// framework that owns all device memory through its own allocator and offers
+// the kernel layer no way to request scratch.  For them the dscale partial
+// sums live in a fixed array compiled into this library (every GPU that loads
+// the library holds it until the process exits).  In host code the array's
+// name is only a host-side stand-in, so its device address is taken once per
+// device, with that device current, by cudaGetSymbolAddress in init_device.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices];
 
 moeact_status init_device(int dev) {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -115,6 +133,8 @@ moeact_status init_device(int dev) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
   e = cudaGetSymbolAddress(reinterpret_cast<void**>(&g_sig_ptr[dev]), g_sigma_table);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+  e = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
 
   cudaStream_t st;
   e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
@@ -229,7 +249,8 @@ moeact_status check_groups(const int64_t* ro, const int64_t* cb, int32_t E, int3
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Backward workspace: the dscale partials, one fp32 per (64-column tile, row).
+// Backward workspace: the dscale partials, one fp32 per (128-column tile
+// (kTileCols), row).
 size_t ws_bytes_needed(int64_t M, int64_t N) {
   return (size_t)ceil_div(N, kTileCols) * (size_t)M * 4;
 }
@@ -810,6 +831,25 @@ moeact_status moeact_device_error(uint32_t* flags) {
   return MOEACT_OK;
 }
 
+moeact_status moeact_wait_selftest(int arrive, uint32_t limit_us, uint64_t* result,
+                                  void* stream) {
+  t_err[0] = 0;
+  if (!result) return fail(MOEACT_EINVAL, "result is required");
+  if (!aligned(result, 8)) return fail(MOEACT_EALIGN, "result must be 8-byte aligned");
+  if (arrive != 0 && arrive != 1) return fail(MOEACT_EINVAL, "arrive must be 0 or 1");
+  if (limit_us < 1 || limit_us > 2000000u)
+    return fail(MOEACT_ERANGE, "limit_us must be in [1, 2000000] (got %u)", limit_us);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int dev;
+  moeact_status st = ensure_ready(cs, &dev);
+  if (st) return st;
+  wait_probe_kernel<<<1, 32, 0, cs>>>((uint64_t)limit_us * 1000u, arrive, g_err_ptr[dev],
+                                      MOEACT_DEVERR_WAIT_SELFTEST, result);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait self-test launch");
+  return MOEACT_OK;
+}
+
 moeact_status moeact_sigmoid_dump(float* out, void* stream) {
   t_err[0] = 0;
   if (!out) return fail(MOEACT_EINVAL, "out is required");
@@ -827,57 +867,29 @@ moeact_status moeact_sigmoid_dump(float* out, void* stream) {
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
-// Backward without any allocation.  Some callers cannot hand the library a
-// workspace: code that runs where a device allocation is not acceptable at the
-// point of the call (cudaMalloc may synchronise the device and its latency is
-// unbounded), or a host framework that owns all device memory through its own
-// allocator and offers the kernel layer no way to request scratch.  For them
-// the dscale partial sums live in a fixed array compiled into this library
-// (every GPU that loads the library holds it until the process exits).
-namespace moeact {
-namespace {
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-// Device address of the array, per device.  In host code the array's name is
-// only a host-side stand-in, so the address is taken once per device, with
-// that device current, by cudaGetSymbolAddress.
-void* g_noalloc_ptr[kMaxDevices];
-std::mutex g_noalloc_mu;
-
-moeact_status noalloc_scratch(int dev, void** out) {
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
-  return MOEACT_OK;
-}
-}  // namespace
-}  // namespace moeact
-
+// Backward without any allocation (see g_noalloc_scratch above): the dense
+// SwiGLU backward with the dscale partials in the built-in array.
 extern "C" moeact_status scaled_swiglu_mxfp8_bwd_noalloc(
     const void* dy, int64_t lddy, const void* x, int64_t ldx, const float* s, int64_t M,
     int64_t N, int dirs, void* dx, float* dscale, moeact_mx_out out, void* stream) {
   t_err[0] = 0;
+  // the shape checks first, so that a bad shape gets the error any entry
+  // point gives it; then the scratch bound, in a form that cannot wrap
+  moeact_status st = check_shape(x, ldx, s, M, N, kSwiGLU);
+  if (st) return st;
   void* ws = nullptr;
   size_t ws_bytes = 0;
-  if (dscale != nullptr && M > 0 && N > 0) {
-    const size_t need = ws_bytes_needed(M, N);
-    if (need > kNoAllocScratchBytes)
+  if (dscale != nullptr && M > 0) {
+    const int64_t tiles = ceil_div(N, kTileCols);
+    if (M > (int64_t)(kNoAllocScratchBytes / 4) / tiles)
       return fail(MOEACT_ERANGE,
-                  "dscale for M=%lld, N=%lld needs %zu bytes of scratch; the built-in scratch "
+                  "dscale for M=%lld, N=%lld needs %lld bytes of scratch; the built-in scratch "
                   "holds %zu (ceil(N/128) * M <= 4194304); use scaled_swiglu_mxfp8_bwd with a "
                   "workspace",
-                  (long long)M, (long long)N, need, kNoAllocScratchBytes);
-    int dev = 0;
-    const cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices) return fail(MOEACT_EUNSUPPORTED, "device index %d", dev);
-    const moeact_status st = noalloc_scratch(dev, &ws);
-    if (st != MOEACT_OK) return st;
+                  (long long)M, (long long)N, (long long)(tiles * M * 4), kNoAllocScratchBytes);
+    int dev;
+    if ((st = ensure_ready(static_cast<cudaStream_t>(stream), &dev))) return st;
+    ws = g_noalloc_ptr[dev];
     ws_bytes = kNoAllocScratchBytes;
   }
   return scaled_swiglu_mxfp8_bwd(dy, lddy, x, ldx, s, M, N, dirs, 0, dx, dscale, out, ws,

@@ -197,13 +197,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for a phase of `bar` with an iteration limit (each try_wait may itself
-// suspend for a short, hardware-chosen time); false on timeout.
-constexpr uint32_t kSpinLimit = 1u << 22;
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for a phase of `bar` for at most `limit_ns` nanoseconds of wall time
+// (the global timer is read every 64 polls; each try_wait may itself suspend
+// for a short, hardware-chosen time); false on timeout.  A copy of a few KiB
+// lands in microseconds, so the kernels' limit, one second, is only ever
+// reached by a copy that will never complete.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // 1-D bulk copy (this CTA only) of `bytes` (a multiple of 16, both addresses

@@ -170,4 +170,27 @@ __global__ void __launch_bounds__(256) dscale_reduce_kernel(const float* __restr
   dscale[row] = acc;
 }
 
+// ---------------------------------------------------------------- wait check
+// Exercises the bounded wait the fused kernels use on their copies: thread 0
+// initialises an mbarrier that completes on one arrival, arrives on it only
+// when `arrive` is set, and waits for it with mbar_wait_for(limit_ns).  A
+// wait that gives up sets `code` in the device error word, as a fused kernel
+// does.  out[0] = 1 if the wait saw the phase complete, 0 if it gave up;
+// out[1] = the nanoseconds it waited.  Nothing else is touched.
+__global__ void wait_probe_kernel(uint64_t limit_ns, int arrive, uint32_t* err, uint32_t code,
+                                  uint64_t* out) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  mbar_init_fence();
+  if (arrive)
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&bar)) : "memory");
+  const uint64_t t0 = global_ns();
+  const bool done = mbar_wait_for(&bar, 0u, limit_ns);
+  const uint64_t t1 = global_ns();
+  if (!done) atomicOr(err, code);
+  out[0] = done ? 1u : 0u;
+  out[1] = t1 - t0;
+}
+
 }  // namespace moeact

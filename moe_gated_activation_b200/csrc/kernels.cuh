@@ -344,6 +344,13 @@ __device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
   if (half == 1) r.cur.next();
 }
 
+// Bits of the device error word (the same values as MOEACT_DEVERR_* in
+// include/moeact.h, checked there by capi.cu).
+constexpr uint32_t kErrFwdWait = 0x1u;     // a forward gave up waiting for its copies
+constexpr uint32_t kErrBwdWait = 0x2u;     // a backward gave up waiting for its copies
+constexpr uint32_t kErrTableWait = 0x4u;   // the sigmoid table's copy never landed
+constexpr uint32_t kErrTableAddr = 0x8u;   // the table lies outside 16-bit addresses
+
 __device__ __forceinline__ void report_timeout(const Params& p, uint32_t code) {
   atomicOr(p.err, code);
 }
@@ -355,7 +362,7 @@ __device__ __forceinline__ void report_timeout(const Params& p, uint32_t code) {
 template <bool FRONT>
 __device__ __forceinline__ bool sig_table_addressable(const Params& p, const Smem& m) {
   if (!FRONT || smem_addr(m.sig) + kSigBytes <= 0x10000u) return true;
-  if (threadIdx.x == 0) report_timeout(p, 8u);
+  if (threadIdx.x == 0) report_timeout(p, kErrTableAddr);
   return false;
 }
 
@@ -751,7 +758,7 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
   ring_prime<C::kOps, C::kSlots, GROUPED, (DIRS & kIlv) != 0>(p, m, ring, &tm_x, nullptr, K, lane);
   if (C::kSig && !mbar_wait(sig_bar, 0u)) {
     if (lane == 0) {
-      report_timeout(p, 4u);
+      report_timeout(p, kErrTableWait);
       ring_drain(ring, 0);
     }
     return;
@@ -790,7 +797,7 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
     sv = svn;
     if (!ok) {
       if (lane == 0) {
-        report_timeout(p, 1u);
+        report_timeout(p, kErrFwdWait);
         ring_drain(ring, 2 * j);
       }
       return;
@@ -1335,7 +1342,7 @@ __global__ void __launch_bounds__(Cfg<ACT, true>::kThreads, 1)
   ring_prime<C::kOps, C::kSlots, GROUPED>(p, m, ring, &tm_x, &tm_dy, K, lane);
   if (C::kSig && !mbar_wait(sig_bar, 0u)) {
     if (lane == 0) {
-      report_timeout(p, 4u);
+      report_timeout(p, kErrTableWait);
       ring_drain(ring, 0);
     }
     return;
@@ -1379,7 +1386,7 @@ __global__ void __launch_bounds__(Cfg<ACT, true>::kThreads, 1)
     sv = svn;
     if (!ok) {
       if (lane == 0) {
-        report_timeout(p, 2u);
+        report_timeout(p, kErrBwdWait);
         ring_drain(ring, 2 * j);
       }
       return;

@@ -40,3 +40,21 @@ def cuda_device():
     cap = torch.cuda.get_device_capability(0)
     assert cap == (10, 0), f"GPU tests target sm_100a (B200); found capability {cap}"
     return torch.device("cuda", 0)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def device_error_word_stays_clear():
+    """After the whole session: if the library ran kernels on a GPU, none of
+    them may have given up a bounded wait (moeact_device_error reads 0).  The
+    wait self-test sets and reads its own bit, so it leaves the word clear."""
+    yield
+    import ctypes
+    import torch
+    if not (torch.cuda.is_available() and torch.cuda.is_initialized()):
+        return
+    from moe_gated_activation_b200 import _capi
+    if _capi._lib is None:
+        return
+    v = ctypes.c_uint32(0)
+    _capi.call("moeact_device_error", ctypes.byref(v))
+    assert v.value == 0, f"device error word {v.value:#x}: a kernel gave up a bounded wait"

@@ -1,17 +1,54 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports
 every function include/moeact.h declares, and rejects invalid arguments on the
 host before touching CUDA (pytorch/ao PR #4743, Numerics and tests: every
-launcher error path is exercised)."""
+launcher error path is exercised).
+
+These calls are meant to fail on the host.  Their pointers point into this
+module's own host buffer, and they only ever run in a process that sees no
+GPU: where one is visible, the module runs itself again in a child process
+with CUDA_VISIBLE_DEVICES empty, so that a regressed host check can never
+launch a kernel on them."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
+import numpy as np
 import pytest
 
 from moe_gated_activation_b200 import _capi
 from moe_gated_activation_b200 import build as mbuild
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+_CHILD = os.environ.get("MOEACT_HOST_CHECKS_CHILD") == "1"
+
+
+def _gpu_visible():
+    import torch
+    return torch.cuda.is_available()
+
+
+GPU_VISIBLE = (not _CHILD) and _gpu_visible()
+
+
+@pytest.fixture(autouse=True)
+def _only_without_a_gpu(request):
+    if GPU_VISIBLE and request.node.originalname != "test_host_checks_run_without_a_gpu":
+        pytest.skip("runs in a child process with no GPU visible "
+                    "(test_host_checks_run_without_a_gpu)")
+
+
+def test_host_checks_run_without_a_gpu():
+    """With a GPU visible, this module's checks run again in a child process
+    that sees none (and must pass there)."""
+    if not GPU_VISIBLE:
+        return
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", MOEACT_HOST_CHECKS_CHILD="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                        os.path.abspath(__file__)], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
 @pytest.fixture(scope="module")
@@ -49,7 +86,11 @@ def test_status_strings(lib):
     assert lib.moeact_status_string(99) == b"unknown status"
 
 
-A16 = 1 << 20          # a fake, 16-byte-aligned device address (never dereferenced)
+# This module's own host memory (1 MiB); A16 is a 16-byte-aligned address in
+# it, and A16 + k (k < 64) stays inside it.  No call here gets as far as using
+# a pointer.
+_BUF = np.zeros(1 << 20, dtype=np.uint8)
+A16 = (_BUF.ctypes.data + 15) & ~15
 MX_ROW = _capi.MxOut(A16, A16, None, None)
 MX_BOTH = _capi.MxOut(A16, A16, A16, A16)
 

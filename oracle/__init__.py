@@ -490,3 +490,47 @@ def interleaved_bwd(dy_bits, x_bits, s, N, dirs, G, act="swiglu", row_offs=None,
     out["dscale"] = r["dscale"]
     return out
 
+
+
+# ---------------------------------------------------------------- activation -> FC2 GEMM
+# TE PR #3238, Greptile summary and sequence diagram: the grouped activation
+# hands its quantized grouped tensor straight to the grouped linear that
+# follows it (ForwardScaledActivationGroupedLinear).  Here that linear is the
+# expert's FC2: out[i, h] = sum_k A[i, k] * W_e[h, k] for a row i of expert e,
+# where A is the rowwise (1 x 32 along k) MXFP8 of the scaled SwiGLU output
+# -- the forward above, rowwise only (rowwise blocks never depend on the
+# grouping) -- and W_e [H, N] is the expert's weight, itself MXFP8 with 1 x 32
+# blocks along k.  Both are taken at their exact dequantized values
+# (code value x 2^(scale - 127)); the product is summed in binary64 by a
+# library matmul, the one step a library routine performs.
+def e4m3_values() -> np.ndarray:
+    """The value of every E4M3 code (binary64, exact), NaN for 0x7F / 0xFF."""
+    lib = _load()
+    return np.array([lib.orc_e4m3_decode(c) for c in range(256)], np.float64)
+
+
+def mxfp8_dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Exact values of rowwise MXFP8 data: codes uint8 [..., W], E8M0 scales
+    uint8 [..., W/32] (255 is NaN)."""
+    codes = np.asarray(codes, np.uint8)
+    scales = np.asarray(scales, np.uint8)
+    v = e4m3_values()[codes]
+    mult = np.where(scales == 255, np.nan, np.ldexp(1.0, scales.astype(np.int64) - 127))
+    return v * np.repeat(mult, 32, axis=-1)
+
+
+def grouped_fc2(x_bits, s, N, row_offs, w_codes, w_scales, staged=False) -> np.ndarray:
+    """out [M, H] (binary64) of the activation -> MXFP8 -> FC2 path: rows
+    [row_offs[e], row_offs[e+1]) use expert e's weight (w_codes uint8
+    [E, H, N] E4M3, w_scales uint8 [E, H, N/32] E8M0)."""
+    a = act_fwd(x_bits, s, N, ROWWISE, SWIGLU, staged)
+    a_val = mxfp8_dequantize_rows(a["row_codes"], a["row_scales"])
+    ro = _c(row_offs, np.int64)
+    E, H = w_codes.shape[0], w_codes.shape[1]
+    out = np.zeros((a_val.shape[0], H), np.float64)
+    for e in range(E):
+        r0, r1 = int(ro[e]), int(ro[e + 1])
+        if r1 > r0:
+            w_val = mxfp8_dequantize_rows(w_codes[e], w_scales[e])
+            out[r0:r1] = a_val[r0:r1] @ w_val.T
+    return out

@@ -133,10 +133,20 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
+FC2_SOURCES = ("fc2.cuh", "kern_fc2.cu")
+
+
+def kernel_source_hash(kernel="act"):
+    """Hash of the sources a kernel's profile depends on: the fused activation
+    kernels ("act": every csrc file but the fused FC2's own) or the fused FC2
+    ("fc2": its own files and the shared device helpers)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "moe_gated_activation_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        if kernel == "act" and name in FC2_SOURCES:
+            continue
+        if kernel == "fc2" and name not in FC2_SOURCES + ("device_common.cuh", "kernels.cuh"):
+            continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -149,7 +159,7 @@ def ncu_traffic(workload, kernel, dirs_name):
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
-    cur = kernel_source_hash()
+    cur = kernel_source_hash("fc2" if kernel == "fc2_kernel" else "act")
     with open(p) as f:
         for line in f:
             line = line.split("#", 1)[0].split()
@@ -565,6 +575,136 @@ def run_e2e(mg, wl, inp, dev, dirs, S, args, world):
             "ms_per_step": round(ms / steps, 4), "pipeline": pipe}
 
 
+# ------------------------------------------------------------------ activation -> FC2
+def measured_bf16_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:  # noqa: BLE001
+        return 1590.0, "fallback"
+
+
+def run_fc2(args):
+    """The activation -> MXFP8 -> expert FC2 GEMM fused on the tensor cores
+    (grouped_scaled_swiglu_mxfp8_fc2) on the Qwen3-MoE-like workload c3
+    (65536 routed rows over 128 experts, N = 768) into an FC2 of width
+    --fc2-width (the model's hidden size, 2048), with a seeded MXFP8 weight.
+    One step = one launch (its own CUDA graph, event nodes at its ends) after
+    an L2 flush.  Reports TFLOP/s against the fp8 dense peak (twice the
+    measured bf16 GEMM peak: the tensor cores' fp8 rate is twice their bf16
+    rate) and the HBM bytes of the launch against the copy peak; `saved_bytes`
+    is the traffic of the quantized activation an unfused path would write
+    and read back (codes + rowwise scales, twice)."""
+    import moe_gated_activation_b200 as mg
+    from moe_gated_activation_b200.workloads import WORKLOADS, fc2_weights, make_inputs
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    mg.init()
+    wl = WORKLOADS["c3"]
+    inp = make_inputs(wl, device=dev, with_dy=False)
+    x, s, m = inp["x"], inp["s"], inp["m_splits"]
+    M, N, H, E = wl.M, wl.N, args.fc2_width, int(m.numel())
+    wc, ws = fc2_weights(E, H, N, 11, device=dev)
+    ro, _, st = mg.splits_to_offsets(m.to(dev), M)
+    out = torch.empty(M, H, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        mg.grouped_scaled_swiglu_mxfp8_fc2(x, s, ro, wc, ws, status=st, out=out)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())}")
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            ev[0].record(side)
+            call()
+            ev[1].record(side)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+
+    def timed(n):
+        t = []
+        for i in range(n):
+            flush.fill_(float(i & 7))
+            flush.amax()
+            g.replay()
+            torch.cuda.synchronize()
+            t.append(ev[0].elapsed_time(ev[1]))
+        return t
+
+    timed(args.warmup)
+    sampler = ClockSampler(dev)
+    with sampler:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        sampler.active = True
+        times = timed(args.steps)
+        sampler.active = False
+        if world > 1:
+            torch.distributed.barrier()
+    err = device_error_word()
+    if err != 0 or int(st.item()) != 0:
+        raise SystemExit(f"device error word {err:#x}, status {int(st.item())}")
+    total_ms = max_over_ranks(sum(times), world, dev)
+    ms = total_ms / args.steps
+    flops = 2.0 * M * N * H
+    nonempty = int((m > 0).sum())
+    hbm_bytes = 2 * M * 2 * N + 4 * M + nonempty * H * (N + N // 32) + 2 * M * H
+    saved = 2 * (M * N + M * N // 32)
+    bf16, kind = measured_bf16_tflops()
+    fp8_peak = 2.0 * bf16
+    hbm_peak, hbm_kind = measured_peak()
+    tflops = world * args.steps * flops / (total_ms * 1e-3) / 1e12
+    gbs = hbm_bytes / (ms * 1e-3) / 1e9
+    bound = "tensor" if flops / (fp8_peak * 1e12) >= hbm_bytes / (hbm_peak * 1e9) else "hbm"
+    outd = {
+        "metric": "fused act+MXFP8+FC2 grouped GEMM TFLOP/s (tcgen05, block-scaled E4M3)",
+        "value": round(tflops, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 (bf16 out)",
+        "data": "synthetic (seeded torch generators; c3 activation input, uniform MXFP8 weight)",
+        "config": {"workload": f"c3 -> FC2: {wl.title}, FC2 width {H}", "M": M, "N": N, "H": H,
+                   "groups": E, "kernel": "grouped_scaled_swiglu_mxfp8_fc2",
+                   "l2": "flushed before every launch (256 MiB written then read)",
+                   "launch": "one CUDA graph per launch (event nodes at its ends)"},
+        "roofline": {"bound": bound, "kernel": "fc2_kernel",
+                     "achieved": round(tflops, 1), "peak": round(fp8_peak, 1),
+                     "peak_kind": f"2 x {kind} bf16 GEMM peak", "unit": "TFLOP/s",
+                     "frac": round(tflops / fp8_peak, 4),
+                     "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "peak_kind": hbm_kind,
+                             "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+                             "algorithmic_bytes": hbm_bytes},
+                     "traffic": ncu_traffic("c3", "fc2_kernel", f"H{H}"),
+                     "time_stat": "mean"},
+        "saved_bytes": saved,
+        "us_median": round(1e3 * statistics.median(times), 2),
+        "us_min": round(1e3 * min(times), 2),
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(),
+    }
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(outd))
+
+
 # ------------------------------------------------------------------ oracle timing
 def host_cores():
     try:
@@ -739,11 +879,18 @@ def main():
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of CUDA graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--fc2", action="store_true",
+                    help="time the activation -> MXFP8 -> FC2 GEMM fused on the tensor cores "
+                         "(workload c3) instead of the activation path")
+    ap.add_argument("--fc2-width", type=int, default=2048,
+                    help="FC2 output width (the model's hidden size) for --fc2")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.fc2:
+        run_fc2(args)
     else:
         run_ours(args)
 

@@ -362,13 +362,57 @@ moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream)
  * operation.  Every wait gives up after one second of GPU time (the global
  * timer), and the kernel then waits (bounded again) for its copies in flight
  * and returns, its outputs incomplete.  Bit 4 is set only by
- * moeact_wait_selftest.  Synchronous.  No counterpart on the pages. */
+ * moeact_wait_selftest; bit 5 by the fused FC2 kernel
+ * (grouped_scaled_swiglu_mxfp8_fc2).  Synchronous.  No counterpart on the pages. */
 #define MOEACT_DEVERR_FWD_WAIT 0x1u
 #define MOEACT_DEVERR_BWD_WAIT 0x2u
 #define MOEACT_DEVERR_TABLE_WAIT 0x4u
 #define MOEACT_DEVERR_TABLE_ADDR 0x8u
 #define MOEACT_DEVERR_WAIT_SELFTEST 0x10u
+#define MOEACT_DEVERR_FC2_WAIT 0x20u
 moeact_status moeact_device_error(uint32_t* flags);
+
+/* ---------------------------------------------------------------------
+ * grouped_scaled_swiglu_mxfp8_fc2 -- the scaled SwiGLU + rowwise MXFP8 of
+ * each expert's rows fused with that expert's FC2 GEMM on the tensor cores
+ * [TE: the grouped scaled activation's quantized grouped tensor feeds the
+ * grouped linear that follows it, ForwardScaledActivationGroupedLinear
+ * (Greptile summary; sequence diagram)]:
+ *   out[i, h] = sum_k A[i, k] * W_e[h, k]   for every row i of expert e,
+ * where A is the rowwise MXFP8 (1 x 32 blocks along k) of y = SwiGLU(x) * s,
+ * bit for bit what grouped_scaled_swiglu_mxfp8_fwd writes with dirs =
+ * MOEACT_ROWWISE (staged rounding as there), and W_e is the expert's MXFP8
+ * weight.  The products of the dequantized operands are summed in fp32 by
+ * the tensor cores (tcgen05.mma, order not specified) and the sum is rounded
+ * to bf16 (nearest even).  A itself is never written to memory.
+ *   x, ldx, s, M, N, staged_rounding: as grouped_scaled_swiglu_mxfp8_fwd
+ *     ([gate | up] halves only); N a multiple of 128 (else MOEACT_EINVAL),
+ *     at most 768 (the quantized 128-row block stays in shared memory; else
+ *     MOEACT_EUNSUPPORTED).
+ *   row_offs [E + 1], num_groups = E, status: as the grouped forward
+ *     (offsets from splits_to_offsets; every split size allowed: rows past
+ *     an expert's end in its last 128-row block are neither read as its own
+ *     nor written); offsets that are not those of valid splits set *status = 3
+ *     and write nothing.
+ *   w_codes: E4M3 [E, H, N], row-major: expert e's weight, row h = output
+ *     column h, its N k-values contiguous; 16-byte aligned.
+ *   w_scales: E8M0 [E, H, N/32], row-major (1 x 32 blocks along k), 16-byte
+ *     aligned.
+ *   H: output width, a positive multiple of 128, E * H < 2^31.
+ *   out: bf16 [M, ldo] (caller-owned, 16-byte aligned), ldo >= H and a
+ *     multiple of 8; columns [0, H) of every row are written.
+ *   noop_flag: nullable device int32; non-zero at execution time makes the
+ *     call write nothing (CUDA-graph replay, as moeact_mx_out.noop_flag).
+ * Allocates nothing; asynchronous on `stream`.  Bounded waits report
+ * MOEACT_DEVERR_FC2_WAIT through moeact_device_error.
+ * ------------------------------------------------------------------- */
+moeact_status grouped_scaled_swiglu_mxfp8_fc2(const void* x, int64_t ldx, const float* s,
+                                              int64_t M, int64_t N, int staged_rounding,
+                                              const int64_t* row_offs, int32_t num_groups,
+                                              int32_t* status, const void* w_codes,
+                                              const void* w_scales, int64_t H, void* out,
+                                              int64_t ldo, const int32_t* noop_flag,
+                                              void* stream);
 
 /* ---------------------------------------------------------------------
  * moeact_wait_selftest -- checks the bounded wait of the fused kernels on the

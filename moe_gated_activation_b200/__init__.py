@@ -15,6 +15,7 @@ from .ops import (  # noqa: F401
     grouped_scaled_clamped_swiglu_mxfp8_fwd,
     grouped_scaled_srelu_mxfp8_bwd,
     grouped_scaled_srelu_mxfp8_fwd,
+    grouped_scaled_swiglu_mxfp8_fc2,
     grouped_scaled_swiglu_mxfp8_bwd,
     grouped_scaled_swiglu_mxfp8_fwd,
     clamped_sigmoid_table,

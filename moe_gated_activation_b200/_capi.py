@@ -19,7 +19,7 @@ ROWWISE, COLWISE = 1, 2
 DEV_OK, DEV_NEGATIVE_SPLIT, DEV_SPLIT_SUM, DEV_BAD_OFFSETS, DEV_UNALIGNED_GROUPS = range(5)
 SCALES_ROWMAJOR, SCALES_GEMM = 0, 1
 DEVERR_FWD_WAIT, DEVERR_BWD_WAIT, DEVERR_TABLE_WAIT, DEVERR_TABLE_ADDR = 0x1, 0x2, 0x4, 0x8
-DEVERR_WAIT_SELFTEST = 0x10
+DEVERR_WAIT_SELFTEST, DEVERR_FC2_WAIT = 0x10, 0x20
 MAX_GROUPS = 2040
 
 
@@ -74,6 +74,8 @@ _SIGS = {
     "moeact_clamped_sigmoid_dump": ([F, P, P], I),
     "moeact_device_error": ([P], I),
     "moeact_wait_selftest": ([I, ctypes.c_uint32, P, P], I),
+    "grouped_scaled_swiglu_mxfp8_fc2": ([P, I64, P, I64, I64, I, P, I32, P, P, P, I64, P, I64, P,
+                                         P], I),
     "scaled_swiglu_mxfp8_bwd_noalloc": ([P, I64, P, I64, P, I64, I64, I, P, P, MxOut, P], I),
 }
 

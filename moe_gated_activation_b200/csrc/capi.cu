@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/moeact.h"
+#include "fc2.cuh"
 #include "host_kernels.cuh"
 #include "variants.cuh"
 
@@ -129,6 +130,8 @@ moeact_status init_device(int dev) {
   e = cudaFuncSetAttribute(sigma_table_dump, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSigBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  e = fc2_prepare();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (fused FC2)");
   e = cudaGetSymbolAddress(reinterpret_cast<void**>(&g_err_ptr[dev]), g_err_word);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
   e = cudaGetSymbolAddress(reinterpret_cast<void**>(&g_sig_ptr[dev]), g_sigma_table);
@@ -309,6 +312,22 @@ moeact_status make_map_ilv(CUtensorMap* map, const void* base, int64_t N, int64_
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOEACT_OK;
+}
+
+// Tensor map of an E4M3 weight [rows, K] (K contiguous bytes per row), read
+// in boxes of 128 bytes of K x 128 rows with 128-byte swizzling: the layout
+// the tensor cores read K-major operands in.
+moeact_status make_map_w(CUtensorMap* map, const void* base, int64_t K, int64_t rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MOEACT_OK;
@@ -828,6 +847,59 @@ moeact_status moeact_device_error(uint32_t* flags) {
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero));
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   *flags = v;
+  return MOEACT_OK;
+}
+
+moeact_status grouped_scaled_swiglu_mxfp8_fc2(const void* x, int64_t ldx, const float* s,
+                                              int64_t M, int64_t N, int staged_rounding,
+                                              const int64_t* row_offs, int32_t num_groups,
+                                              int32_t* status, const void* w_codes,
+                                              const void* w_scales, int64_t H, void* out,
+                                              int64_t ldo, const int32_t* noop_flag,
+                                              void* stream) {
+  t_err[0] = 0;
+  moeact_status st = check_shape(x, ldx, s, M, N, kSwiGLU);
+  if (st) return st;
+  if (N % 128 != 0) return fail(MOEACT_EINVAL, "N must be a multiple of 128 (got %lld)", (long long)N);
+  if (N > kFc2MaxN)
+    return fail(MOEACT_EUNSUPPORTED, "N above %d: the quantized 128-row block must fit in shared memory", kFc2MaxN);
+  if (staged_rounding != 0 && staged_rounding != 1) return fail(MOEACT_EINVAL, "staged_rounding must be 0 or 1");
+  if (!row_offs || !status) return fail(MOEACT_EINVAL, "row_offs and status are required");
+  if (num_groups < 1 || num_groups > MOEACT_MAX_GROUPS) return fail(MOEACT_EINVAL, "num_groups must be in [1, %d]", MOEACT_MAX_GROUPS);
+  if (!aligned(row_offs, 8) || !aligned(status, 4)) return fail(MOEACT_EALIGN, "row_offs must be 8-byte aligned, status 4-byte aligned");
+  if (!w_codes || !w_scales || !out) return fail(MOEACT_EINVAL, "w_codes, w_scales and out are required");
+  if (!aligned(w_codes, 16) || !aligned(w_scales, 16) || !aligned(out, 16))
+    return fail(MOEACT_EALIGN, "w_codes, w_scales and out must be 16-byte aligned");
+  if (H <= 0 || H % 128 != 0) return fail(MOEACT_EINVAL, "H must be a positive multiple of 128 (got %lld)", (long long)H);
+  if (H * (int64_t)num_groups > INT32_MAX) return fail(MOEACT_ERANGE, "num_groups * H above 2^31 - 1");
+  if (ldo < H) return fail(MOEACT_EINVAL, "ldo (%lld) smaller than H", (long long)ldo);
+  if (ldo % 8 != 0) return fail(MOEACT_EALIGN, "ldo must be a multiple of 8 elements");
+  if (ldo > (((int64_t)1) << 40) || M * ldo > (((int64_t)1) << 61)) return fail(MOEACT_ERANGE, "out extent too large");
+  if (noop_flag && !aligned(noop_flag, 4)) return fail(MOEACT_EALIGN, "noop_flag must be 4-byte aligned");
+  if (M == 0) return MOEACT_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int dev;
+  if ((st = ensure_ready(cs, &dev))) return st;
+  CUtensorMap tx, tw;
+  if ((st = make_map(&tx, x, 2 * N, M, ldx))) return st;
+  if ((st = make_map_w(&tw, w_codes, N, H * num_groups))) return st;
+  Fc2Params p{};
+  p.s = s;
+  p.M = M;
+  p.N = (int)N;
+  p.H = (int)H;
+  p.row_offs = row_offs;
+  p.E = num_groups;
+  p.status = status;
+  p.w_scales = static_cast<const uint8_t*>(w_scales);
+  p.out = static_cast<uint16_t*>(out);
+  p.ldo = ldo;
+  p.sig_src = g_sig_ptr[dev];
+  p.noop = noop_flag;
+  p.err = g_err_ptr[dev];
+  const int64_t grid = ceil_div(M, 128) + num_groups;
+  const cudaError_t e = fc2_launch(p, tx, tw, staged_rounding, (unsigned)grid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "fused FC2 launch");
   return MOEACT_OK;
 }
 

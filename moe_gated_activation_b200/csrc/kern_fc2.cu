@@ -1,0 +1,575 @@
+// The scaled SwiGLU + rowwise MXFP8 of an expert's rows fused with that
+// expert's FC2 GEMM on the fifth-generation tensor cores (sm_100a).
+//
+// TransformerEngine PR #3238 (Greptile summary, sequence diagram): the
+// grouped scaled activation emits quantized grouped storage that the grouped
+// linear after it consumes (ForwardScaledActivationGroupedLinear).  Here both
+// run in one kernel and the quantized activation stays on chip:
+//
+//   out[i, h] = sum_k A[i, k] * W_e[h, k]     (row i of expert e)
+//
+// A = rowwise MXFP8 (1 x 32 blocks along k, E8M0 RCEIL scales, E4M3 codes)
+// of y = SwiGLU(x) * s, exactly as the stand-alone forward computes it;
+// W_e = the expert's weight, MXFP8 with 1 x 32 blocks along k; the products
+// of the block-scaled operands are summed by the tensor cores in fp32 and the
+// result rounded to bf16.
+//
+// One CTA per (expert, 128-row block); 10 warps:
+//   warps 0-7  prologue: stream the block's gate / up rows in by TMA (one
+//              16-row half-tile slot per warp), compute y and its rowwise
+//              MXFP8, write the codes into shared memory in the tensor
+//              cores' K-major 128-byte-swizzled layout and the scales into
+//              tensor memory; then, per 128-column output tile, write the
+//              weight's scales into tensor memory and drain the accumulator
+//              (tcgen05.ld) into bf16 rows of `out`;
+//   warp 8     TMA producer of the weight tiles (128 rows x 128 bytes of k,
+//              swizzled), a 7-stage ring that reuses the prologue's staging
+//              and sigmoid-table memory;
+//   warp 9     allocates tensor memory and issues the MMAs (one thread):
+//              tcgen05.mma.kind::mxf8f6f4.block_scale, M = N = 128, K = 32,
+//              two accumulators in tensor memory so that one tile's drain
+//              overlaps the next tile's MMAs.
+// Every wait is bounded (one second); on a timeout the kernel records
+// MOEACT_DEVERR_FC2_WAIT, lets its copies and MMAs in flight finish (bounded
+// again), frees its tensor memory and returns.
+#include "fc2.cuh"
+#include "kernels.cuh"
+
+namespace moeact {
+namespace {
+
+constexpr int kAtom = 16384;              // 128 rows x 128 bytes of k (one swizzle atom column)
+constexpr int kStages = 7;                // weight ring
+constexpr int kStageBytes = 16384;        // 128 weight rows x 128 bytes of k
+constexpr int kXSlotBytes = 2 * kOpHalfBytes;   // gate + up of 16 rows x 128 columns
+constexpr int kXBytes = 8 * kXSlotBytes;  // the prologue's slots (8 warps)
+// The staging region: the weight ring, or (prologue) the X slots and the
+// sigmoid table after them.
+constexpr int kRBytes = ((kXBytes + kSigBytes > kStages * kStageBytes ? kXBytes + kSigBytes
+                                                                       : kStages * kStageBytes) +
+                         1023) / 1024 * 1024;
+constexpr int kMiscBytes = 2048;
+constexpr int kSfaCol = 256;              // tensor-memory columns: accumulators [0, 256),
+constexpr int kSfbCol = 288;              // A scales [256, 288), W scales [288, 352)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kErrFc2Wait = 0x20u;
+
+// misc ints
+constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscE = 2, kMiscBlk = 3, kMiscTotal = 4,
+              kMiscScan = 16;
+
+// ------------------------------------------------------------ tcgen05 wrappers
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_addr(dst)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrives on `bar` once every tcgen05 operation this thread issued before has
+// completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_addr(bar)) : "memory");
+}
+// D (+)= A x B^T with E8M0 block scales: A [128 x 32] and B [128 x 32] E4M3
+// from shared-memory descriptors, scales from tensor memory.
+__device__ __forceinline__ void tc_mma_mx(uint32_t d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p; }"
+      ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Four 32-bit words into four consecutive columns of the warp's 32 lanes
+// (thread t: lane t).
+__device__ __forceinline__ void tc_st4(uint32_t taddr, uint32_t v0, uint32_t v1, uint32_t v2,
+                                       uint32_t v3) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+               ::"r"(taddr), "r"(v0), "r"(v1), "r"(v2), "r"(v3) : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// 32 consecutive columns of the warp's 32 lanes (thread t: lane t).
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+        "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+        "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile in the 128-byte
+// swizzled layout: rows of 128 bytes, 8-row groups 1024 bytes apart (the
+// stride byte offset), 16-byte chunks of row r stored at chunk ^ (r mod 8);
+// descriptor version 1 (sm_100).  `saddr` may sit 32, 64 or 96 bytes into a
+// 1024-byte-aligned atom (the K steps of one atom).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 x E4M3,
+// both K-major, N = 128 (bits 17-22: N / 8), E8M0 scales (bit 23), M = 128
+// (bits 24-28: M / 16); the scale byte of each 32-bit tensor-memory word that
+// this K step uses is `sf` for both operands (bits 4-5 and 29-30).
+__device__ __forceinline__ uint32_t mx_idesc(uint32_t sf) {
+  return (16u << 17) | (1u << 23) | (8u << 24) | (sf << 4) | (sf << 29);
+}
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+  return p + ((1024u - (smem_addr(p) & 1023u)) & 1023u);
+}
+
+struct Fc2Smem {
+  unsigned char* A;       // [N/128 atoms][128 rows][128 bytes], swizzled
+  unsigned char* R;       // staging: weight ring / X slots + sigmoid table
+  const float* sig;
+  uint64_t* xbar;         // [8]
+  uint64_t* sig_bar;
+  uint64_t* pro_done;     // count 8: the block's A codes and scales are complete
+  uint64_t* b_full;       // [7]
+  uint64_t* b_empty;      // [7]
+  uint64_t* sfb_full;     // [2] count 8: the weight scales of a tile are in tensor memory
+  uint64_t* d_full;       // [2] an accumulator holds a finished tile
+  uint64_t* d_empty;      // [2] count 8: an accumulator has been drained
+  uint64_t* mma_done;
+  int* misc;
+};
+
+__device__ __forceinline__ bool aborted(const Fc2Smem& m) {
+  return *reinterpret_cast<volatile int*>(m.misc + kMiscAbort) != 0;
+}
+// The same verdict in every lane of the warp (the tcgen05 loads and stores
+// that follow are warp-collective).
+__device__ __forceinline__ bool warp_aborted(const Fc2Smem& m) {
+  return __any_sync(kFull, aborted(m));
+}
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  return __all_sync(kFull, mbar_wait(bar, parity));
+}
+__device__ __forceinline__ void set_abort(const Fc2Params& p, const Fc2Smem& m) {
+  *reinterpret_cast<volatile int*>(m.misc + kMiscAbort) = 1;
+  atomicOr(p.err, kErrFc2Wait);
+}
+
+// ------------------------------------------------------------ prologue
+// One 16-row half of a warp-tile (32 rows of the block's quarter q x the 128
+// columns of atom a): y = SwiGLU(g, u) * s, its rowwise E8M0 scales (returned
+// packed as in fwd_tile: lane l holds blocks l >> 3 of rows 2 (l & 7) + {0,1})
+// and its E4M3 codes, stored into the atom at the swizzled positions.
+template <bool STAGED>
+__device__ __forceinline__ uint32_t fc2_half(const Fc2Smem& m, const unsigned char* slot,
+                                             int lane, int q, int a, int h, int nvq, float sv) {
+  float Y[16][4];
+  const unsigned char* sm = slot + 8 * lane;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint2 G = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
+    const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
+    const float sr = __shfl_sync(kFull, sv, 16 * h + i);
+    const float2 s2 = make_float2(sr, sr);
+    float2 sg01, sg23;
+    sigma_pair(m.sig, G.x, sg01.x, sg01.y);
+    sigma_pair(m.sig, G.y, sg23.x, sg23.y);
+    const float2 si01 = mul2(bf16x2_to_f2(G.x), sg01), si23 = mul2(bf16x2_to_f2(G.y), sg23);
+    const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
+    float2 h01, h23;
+    if (STAGED) {
+      const float2 a01 = bf16x2_to_f2(pack_bf16x2(si01.x, si01.y));
+      const float2 a23 = bf16x2_to_f2(pack_bf16x2(si23.x, si23.y));
+      const float2 p01 = mul2(a01, u01), p23 = mul2(a23, u23);
+      h01 = bf16x2_to_f2(pack_bf16x2(p01.x, p01.y));
+      h23 = bf16x2_to_f2(pack_bf16x2(p23.x, p23.y));
+    } else {
+      h01 = mul2(si01, u01);
+      h23 = mul2(si23, u23);
+    }
+    const float2 y01 = mul2(h01, s2), y23 = mul2(h23, s2);
+    const bool live = 16 * h + i < nvq;   // rows past the expert's end stay zero
+    Y[i][0] = live ? y01.x : 0.0f;
+    Y[i][1] = live ? y01.y : 0.0f;
+    Y[i][2] = live ? y23.x : 0.0f;
+    Y[i][3] = live ? y23.y : 0.0f;
+  }
+  __syncwarp();
+  uint32_t Am[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    Am[i] = __float_as_uint(max_nan(max3_nan(fabsf(Y[i][0]), fabsf(Y[i][1]), fabsf(Y[i][2])),
+                                    fabsf(Y[i][3])));
+  bfly_max_u32<8>(Am, lane, 4);
+  bfly_max_u32<4>(Am, lane, 2);
+  bfly_max_u32<2>(Am, lane, 1);
+  const uint32_t b0 = e8m0_from_amax(Am[0]), b1 = e8m0_from_amax(Am[1]);
+  const uint32_t m0 = scale_multiplier(b0), m1 = scale_multiplier(b1);
+  unsigned char* atom = m.A + a * kAtom;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t mm = __shfl_sync(kFull, (i & 1) ? m1 : m0, (lane & 24) | (i >> 1));
+    const uint32_t code = e4m3x2_2(make_float2(Y[i][0], Y[i][1]), mm, mm) |
+                          (e4m3x2_2(make_float2(Y[i][2], Y[i][3]), mm, mm) << 16);
+    const int row = 32 * q + 16 * h + i;
+    *reinterpret_cast<uint32_t*>(atom + row * 128 + ((((lane >> 2) ^ (row & 7))) << 4) +
+                                 ((lane & 3) << 2)) = code;
+  }
+  return b0 | (b1 << 8);
+}
+
+// The weight scales of output tile n (its 128 rows of W_e, all of k) into
+// tensor-memory buffer n & 1, in the layout the block-scaled MMA reads the
+// scales of its N operand: for each group of four k-blocks, four columns;
+// lane l of every 32-lane quarter, column c holds the word (four E8M0 bytes,
+// one per k-block) of tile row 32 c + l -- the same 32 x 4 words repeated in
+// all four quarters, each quarter written by its own warps (this warp: its
+// half of the groups).
+__device__ __forceinline__ void fc2_write_sfb(const Fc2Params& p, const Fc2Smem& m, int e, int n,
+                                              int q, int half_sel, int lane, uint32_t tbase) {
+  const int KA = p.N >> 7, KB = p.N >> 5;
+  const int b = n & 1;
+  const uint8_t* srow = p.w_scales + ((int64_t)e * p.H + 128 * n + lane) * KB;
+  const int64_t step = 32 * (int64_t)KB;   // 32 rows further
+  const uint32_t t = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(kSfbCol + 32 * b);
+  for (int g = half_sel; g < KA; g += 2) {
+    const uint8_t* c = srow + 4 * g;
+    tc_st4(t + 4 * g, __ldg(reinterpret_cast<const uint32_t*>(c)),
+           __ldg(reinterpret_cast<const uint32_t*>(c + step)),
+           __ldg(reinterpret_cast<const uint32_t*>(c + 2 * step)),
+           __ldg(reinterpret_cast<const uint32_t*>(c + 3 * step)));
+  }
+  tc_wait_st();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(m.sfb_full + b);
+}
+
+template <bool STAGED>
+__device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2Smem& m, int e,
+                         int64_t row0, int mrows, uint32_t tbase) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, half_sel = warp >> 2;
+  const int KA = p.N >> 7;
+  const int nvq = max(0, min(32, mrows - 32 * q));   // rows of this quarter in the expert
+  const int n_atoms = KA > half_sel ? (KA - half_sel + 1) / 2 : 0;
+  const int Kw = 2 * n_atoms;                          // half-tiles of this warp
+  unsigned char* slot = m.R + warp * kXSlotBytes;
+  uint64_t* xb = m.xbar + warp;
+  auto issue = [&](int j) {
+    const int a = half_sel + 2 * (j >> 1);
+    const int y = (int)row0 + 32 * q + 16 * (j & 1);
+    mbar_expect_tx(xb, kXSlotBytes);
+    tma_load_2d(slot, tm_x, 128 * a, y, xb);
+    tma_load_2d(slot + kOpHalfBytes, tm_x, p.N + 128 * a, y, xb);
+  };
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(m.sig_bar, 2 * kSigHalfBytes);
+    bulk_load(const_cast<float*>(m.sig), p.sig_src, kSigHalfBytes, m.sig_bar);
+    bulk_load(const_cast<float*>(m.sig) + kSigNegOffset, p.sig_src + kSigNegOffset,
+              kSigHalfBytes, m.sig_bar);
+  }
+  if (lane == 0 && Kw > 0) issue(0);
+  const float sv = lane < nvq ? __ldg(p.s + row0 + 32 * q + lane) : 0.0f;
+  bool ok = warp_wait(m.sig_bar, 0u);
+  int waited = 0;   // half-tiles whose copy this warp has seen land
+  uint32_t bh0 = 0;
+  for (int j = 0; ok && j < Kw; ++j) {
+    if (!warp_wait(xb, (uint32_t)j & 1u)) { ok = false; break; }
+    waited = j + 1;
+    const int a = half_sel + 2 * (j >> 1), h = j & 1;
+    const uint32_t bh = fc2_half<STAGED>(m, slot, lane, q, a, h, nvq, sv);
+    // fc2_half has read the slot (its values are in use): refill it
+    if (lane == 0 && j + 1 < Kw) issue(j + 1);
+    if (h == 0) {
+      bh0 = bh;
+    } else {
+      // lane l: the four block scales of row 32 q + l for atom a.  The MMA
+      // reads the scale of its M-operand row 32 q + l from lane 32 q + l,
+      // column q of the group (the layout of fc2_write_sfb, of which each
+      // quarter needs only its own column); the word goes to all four.
+      const uint32_t v = gather_row_scales(bh0, bh, lane, 0, 1);
+      tc_st4(tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(kSfaCol + 4 * a), v, v, v, v);
+    }
+  }
+  if (!ok) {
+    set_abort(p, m);
+    // copies this warp issued that never landed: wait for them (bounded)
+    if (lane == 0) {
+      if (waited < Kw) mbar_wait(xb, (uint32_t)waited & 1u);
+      mbar_wait(m.sig_bar, 0u);
+    }
+  }
+  tc_wait_st();
+  fence_proxy_async_smem();   // the codes written above are read by the tensor cores
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(m.pro_done);
+
+  // ---- output tiles: weight scales two tiles ahead, then drain each tile
+  const int T = p.H >> 7;
+  for (int n = 0; n < T && n < 2; ++n) fc2_write_sfb(p, m, e, n, q, half_sel, lane, tbase);
+  for (int n = 0; n < T; ++n) {
+    if (warp_aborted(m)) break;
+    const int b = n & 1;
+    if (!warp_wait(m.d_full + b, (uint32_t)(n >> 1) & 1u)) { set_abort(p, m); break; }
+    tc_fence_after();
+    uint32_t v[64];
+    const uint32_t t = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * b + 64 * half_sel);
+    tc_ld32(t, v);
+    tc_ld32(t + 32, v + 32);
+    tc_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(m.d_empty + b);
+    const int row = 32 * q + lane;
+    if (row < mrows) {
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (row0 + row) * p.ldo + 128 * n + 64 * half_sel);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+        w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+        w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+        w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+        dst[c] = w;
+      }
+    }
+    if (n + 2 < T) fc2_write_sfb(p, m, e, n + 2, q, half_sel, lane, tbase);
+  }
+}
+
+// Warp 8, one thread: the weight tiles of every output tile, in k order.
+__device__ void fc2_producer(const CUtensorMap* tm_w, const Fc2Params& p, const Fc2Smem& m,
+                             int e) {
+  const int KA = p.N >> 7, T = p.H >> 7;
+  int issued = 0;
+  if (!mbar_wait(m.pro_done, 0u)) set_abort(p, m);
+  for (int g = 0; g < T * KA && !aborted(m); ++g) {
+    const int n = g / KA, ks = g - n * KA, slot = g % kStages;
+    if (g >= kStages && !mbar_wait(m.b_empty + slot, (uint32_t)(g / kStages - 1) & 1u)) {
+      set_abort(p, m);
+      break;
+    }
+    mbar_expect_tx(m.b_full + slot, kStageBytes);
+    tma_load_2d(m.R + slot * kStageBytes, tm_w, 128 * ks, e * p.H + 128 * n, m.b_full + slot);
+    issued = g + 1;
+  }
+  // every copy issued has landed before the CTA can exit (bounded)
+  for (int g = max(0, issued - kStages); g < issued; ++g)
+    mbar_wait(m.b_full + g % kStages, (uint32_t)(g / kStages) & 1u);
+}
+
+// Warp 9, one thread: the MMAs of every output tile.
+__device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
+  const int KA = p.N >> 7, T = p.H >> 7;
+  bool ok = mbar_wait(m.pro_done, 0u) && !aborted(m);
+  if (!ok) set_abort(p, m);
+  tc_fence_after();
+  const uint32_t a_base = smem_addr(m.A), r_base = smem_addr(m.R);
+  for (int n = 0; ok && n < T; ++n) {
+    const int b = n & 1;
+    if (!mbar_wait(m.sfb_full + b, (uint32_t)(n >> 1) & 1u) ||
+        (n >= 2 && !mbar_wait(m.d_empty + b, (uint32_t)((n >> 1) - 1) & 1u))) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    for (int ks = 0; ks < KA; ++ks) {
+      const int g = n * KA + ks, slot = g % kStages;
+      if (aborted(m) || !mbar_wait(m.b_full + slot, (uint32_t)(g / kStages) & 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t ad = umma_desc_sw128(a_base + ks * kAtom + 32 * j);
+        const uint64_t bd = umma_desc_sw128(r_base + slot * kStageBytes + 32 * j);
+        tc_mma_mx(tbase + 128 * b, ad, bd, mx_idesc((uint32_t)j), tbase + kSfaCol + 4 * ks,
+                  tbase + kSfbCol + 32 * b + 4 * ks, (ks | j) != 0 ? 1u : 0u);
+      }
+      tc_commit(m.b_empty + slot);   // the stage is free once these MMAs are done
+    }
+    if (!ok) break;
+    tc_commit(m.d_full + b);
+  }
+  if (!ok) set_abort(p, m);
+  // every MMA issued has completed before tensor memory is freed (bounded)
+  tc_commit(m.mma_done);
+  mbar_wait(m.mma_done, 0u);
+}
+
+template <bool STAGED>
+__global__ void __launch_bounds__(kFc2Threads, 1)
+    fc2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+               const Fc2Params p) {
+  if (p.noop != nullptr && *p.noop != 0) return;
+  extern __shared__ __align__(1024) unsigned char fc2_smem[];
+  unsigned char* base = align1024(fc2_smem);
+  Fc2Smem m;
+  const int KA = p.N >> 7;
+  m.A = base;
+  m.R = base + KA * kAtom;
+  m.sig = reinterpret_cast<const float*>(m.R + kXBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(m.R + kRBytes);
+  m.xbar = bars;
+  m.sig_bar = bars + 8;
+  m.pro_done = bars + 9;
+  m.b_full = bars + 10;
+  m.b_empty = bars + 10 + kStages;
+  m.sfb_full = bars + 10 + 2 * kStages;
+  m.d_full = m.sfb_full + 2;
+  m.d_empty = m.sfb_full + 4;
+  m.mma_done = m.sfb_full + 6;
+  m.misc = reinterpret_cast<int*>(bars + 32);
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  // ---- this CTA's (expert, 128-row block); the offsets are validated first
+  const int E = p.E;
+  const int C = (E + kFc2Threads - 1) / kFc2Threads;
+  const int e_lo = min(E, tid * C), e_hi = min(E, e_lo + C);
+  int local = 0, bad = 0;
+  for (int e = e_lo; e < e_hi; ++e) {
+    const int64_t r0 = p.row_offs[e], r1 = p.row_offs[e + 1];
+    if (r1 < r0 || r0 < 0 || r1 > p.M) bad = 1;
+    else local += (int)((r1 - r0 + 127) >> 7);
+  }
+  if (tid == 0 && (p.row_offs[0] != 0 || p.row_offs[E] != p.M)) bad = 1;
+  m.misc[kMiscScan + tid] = local;
+  const int any_bad = __syncthreads_or(bad);
+  if (blockIdx.x == 0 && tid == 0) *p.status = any_bad ? 3 : 0;
+  if (any_bad) return;
+  if (tid == 0) {
+    int acc = 0;
+    for (int t = 0; t < kFc2Threads; ++t) {
+      const int v = m.misc[kMiscScan + t];
+      m.misc[kMiscScan + t] = acc;
+      acc += v;
+    }
+    m.misc[kMiscTotal] = acc;
+  }
+  __syncthreads();
+  const int u = blockIdx.x;
+  if (u >= m.misc[kMiscTotal]) return;
+  {
+    int acc = m.misc[kMiscScan + tid];
+    if (u >= acc && u < acc + local) {
+      for (int e = e_lo; e < e_hi; ++e) {
+        const int nb = (int)((p.row_offs[e + 1] - p.row_offs[e] + 127) >> 7);
+        if (u < acc + nb) {
+          m.misc[kMiscE] = e;
+          m.misc[kMiscBlk] = u - acc;
+          break;
+        }
+        acc += nb;
+      }
+    }
+  }
+  __syncthreads();
+  const int e = m.misc[kMiscE];
+  const int64_t row0 = p.row_offs[e] + 128 * (int64_t)m.misc[kMiscBlk];
+  const int mrows = (int)min((int64_t)128, p.row_offs[e + 1] - row0);
+
+  // ---- barriers and tensor memory
+  if (tid == 0) {
+    for (int i = 0; i < 8; ++i) mbar_init(m.xbar + i, 1);
+    mbar_init(m.sig_bar, 1);
+    mbar_init(m.pro_done, 8);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(m.b_full + i, 1);
+      mbar_init(m.b_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(m.sfb_full + i, 8);
+      mbar_init(m.d_full + i, 1);
+      mbar_init(m.d_empty + i, 8);
+    }
+    mbar_init(m.mma_done, 1);
+    m.misc[kMiscAbort] = 0;
+    mbar_init_fence();
+  }
+  if (warp == 9) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(m.misc + kMiscTmem), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(m.misc + kMiscTmem);
+
+  if (warp < 8) {
+    fc2_math<STAGED>(&tm_x, p, m, e, row0, mrows, tbase);
+  } else if (warp == 8) {
+    if ((tid & 31) == 0) fc2_producer(&tm_w, p, m, e);
+    __syncwarp();
+  } else {
+    if ((tid & 31) == 0) fc2_mma(p, m, tbase);
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int fc2_smem_bytes(int N) { return 1024 + (N / 128) * kAtom + kRBytes + kMiscBytes; }
+
+cudaError_t fc2_prepare() {
+  const int bytes = fc2_smem_bytes(kFc2MaxN);
+  cudaError_t e = cudaFuncSetAttribute(fc2_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fc2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes);
+  return e;
+}
+
+cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
+                       int staged, unsigned grid, cudaStream_t stream) {
+  const int bytes = fc2_smem_bytes(p.N);
+  if (staged)
+    fc2_kernel<true><<<grid, kFc2Threads, bytes, stream>>>(tm_x, tm_w, p);
+  else
+    fc2_kernel<false><<<grid, kFc2Threads, bytes, stream>>>(tm_x, tm_w, p);
+  return cudaGetLastError();
+}
+
+static_assert(kMiscScan * 4 + kFc2Threads * 4 + 32 * 8 <= kMiscBytes, "misc region too small");
+static_assert(kXBytes + kSigBytes <= kRBytes && kStages * kStageBytes <= kRBytes,
+              "staging region too small");
+static_assert(kSfbCol + 64 <= (int)kTmemCols && kSfaCol + 32 <= kSfbCol,
+              "tensor-memory columns overlap");
+
+}  // namespace moeact

@@ -292,22 +292,11 @@ struct Ring {
   int k_issue;       // next half-tile to issue
 };
 
-// FWD_ILV: a forward whose input interleaves gate and up in blocks (kIlv).
-template <int OPS, int SLOTS, bool GROUPED, bool FWD_ILV = false>
-__device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
-                                           Ring<OPS, SLOTS>& r, const void* tm_x,
-                                           const void* tm_dy) {
-  const int k = r.k_issue;
-  const int half = k & 1;
-  if (half == 0) {
-    int nrows;
-    slab_rows<GROUPED>(p, m, r.cur.slab, r.row0, nrows);
-  }
-  const int slot = k % SLOTS;
-  unsigned char* dst = r.slots + slot * OPS * kOpHalfBytes;
-  uint64_t* bar = r.bars + slot;
-  const int x = r.cur.tile * kTileCols, y = (int)r.row0 + half * kHalfRows;
-  mbar_expect_tx(bar, OPS * kOpHalfBytes);
+// Issues the boxes of one half-tile at column x, row y into shared memory
+// (dst, completing on bar).
+template <int OPS, bool FWD_ILV>
+__device__ __forceinline__ void ring_boxes(const Params& p, unsigned char* dst, uint64_t* bar,
+                                           const void* tm_x, const void* tm_dy, int x, int y) {
   if (OPS == 3 || (OPS == 2 && tm_dy != nullptr)) {
     // backward: dY, then x (gate), then up (SwiGLU).  A SwiGLU input has a 3-D
     // map whose middle coordinate picks gate (0) or up (1), so that columns
@@ -340,6 +329,25 @@ __device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
     tma_load_2d(dst, tm_x, x, y, bar);
     if (OPS == 2) tma_load_2d(dst + kOpHalfBytes, tm_x, x + p.N, y, bar);
   }
+}
+
+// FWD_ILV: a forward whose input interleaves gate and up in blocks (kIlv).
+template <int OPS, int SLOTS, bool GROUPED, bool FWD_ILV = false>
+__device__ __forceinline__ void ring_issue(const Params& p, const Smem& m,
+                                           Ring<OPS, SLOTS>& r, const void* tm_x,
+                                           const void* tm_dy) {
+  const int k = r.k_issue;
+  const int half = k & 1;
+  if (half == 0) {
+    int nrows;
+    slab_rows<GROUPED>(p, m, r.cur.slab, r.row0, nrows);
+  }
+  const int slot = k % SLOTS;
+  unsigned char* dst = r.slots + slot * OPS * kOpHalfBytes;
+  uint64_t* bar = r.bars + slot;
+  const int x = r.cur.tile * kTileCols, y = (int)r.row0 + half * kHalfRows;
+  mbar_expect_tx(bar, OPS * kOpHalfBytes);
+  ring_boxes<OPS, FWD_ILV>(p, dst, bar, tm_x, tm_dy, x, y);
   r.k_issue = k + 1;
   if (half == 1) r.cur.next();
 }

@@ -457,3 +457,52 @@ def sigmoid_table(device="cuda"):
     out = torch.empty(65536, dtype=torch.float32, device=device)
     _capi.call("moeact_sigmoid_dump", _ptr(out), _stream(out.device))
     return out
+
+
+# ------------------------------------------------------------------ activation -> FC2
+def grouped_scaled_swiglu_mxfp8_fc2(x, s, row_offs, w_codes, w_scales, *, status=None,
+                                    staged_rounding=False, out=None, noop_flag=None):
+    """The scaled SwiGLU + rowwise MXFP8 of each expert's rows fused with the
+    expert's FC2 GEMM on the tensor cores (TE PR #3238: the quantized grouped
+    activation feeds the grouped linear after it).
+
+    x bf16 [M, 2N] ([gate | up]), s fp32 [M], row_offs int64 [E + 1] (from
+    splits_to_offsets); w_codes E4M3 [E, H, N] (uint8 or float8_e4m3fn, row h
+    of expert e = output column h), w_scales uint8 E8M0 [E, H, N/32].
+    Returns (out bf16 [M, H], status); `out=` takes a caller-owned bf16
+    [M, >= H] tensor with unit column stride."""
+    N = x.shape[1] // 2
+    _check_rows(x, "x", torch.bfloat16, 2 * N)
+    M = x.shape[0]
+    _check_s(s, M, x.device)
+    dev = x.device
+    if w_codes.dtype == torch.float8_e4m3fn:
+        w_codes = w_codes.view(torch.uint8)
+    if w_codes.dtype != torch.uint8 or w_codes.dim() != 3 or w_codes.shape[2] != N or \
+            not w_codes.is_contiguous() or w_codes.device != dev:
+        raise ValueError(f"w_codes must be a contiguous uint8 / float8_e4m3fn [E, H, {N}] tensor "
+                         f"on {dev}")
+    E, H = w_codes.shape[0], w_codes.shape[1]
+    if w_scales.dtype != torch.uint8 or tuple(w_scales.shape) != (E, H, N // 32) or \
+            not w_scales.is_contiguous() or w_scales.device != dev:
+        raise ValueError(f"w_scales must be a contiguous uint8 [{E}, {H}, {N // 32}] tensor on {dev}")
+    if row_offs.dtype != torch.int64 or tuple(row_offs.shape) != (E + 1,) or not row_offs.is_cuda:
+        raise ValueError(f"row_offs must be an int64 CUDA tensor of {E + 1} offsets")
+    if status is None:
+        status = torch.empty(1, dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    elif out.dtype != torch.bfloat16 or out.dim() != 2 or out.shape[0] != M or \
+            out.shape[1] < H or out.stride(1) != 1 or out.device != dev:
+        raise ValueError(f"out must be a bf16 [{M}, >= {H}] tensor with unit column stride on {dev}")
+    if noop_flag is not None and (noop_flag.dtype != torch.int32 or not noop_flag.is_cuda):
+        raise ValueError("noop_flag must be an int32 CUDA tensor")
+    if M == 0:
+        status.zero_()
+        return out, status
+    ldx = x.stride(0) if M > 1 else max(x.stride(0), x.shape[1])
+    ldo = out.stride(0) if M > 1 else max(out.stride(0), H)
+    _capi.call("grouped_scaled_swiglu_mxfp8_fc2", _ptr(x), ldx, _ptr(s), M, N,
+               int(bool(staged_rounding)), _ptr(row_offs), E, _ptr(status), _ptr(w_codes),
+               _ptr(w_scales), H, _ptr(out), ldo, _ptr(noop_flag), _stream(dev))
+    return out, status

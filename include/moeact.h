@@ -396,8 +396,12 @@ moeact_status moeact_device_error(uint32_t* flags);
  *     and write nothing.
  *   w_codes: E4M3 [E, H, N], row-major: expert e's weight, row h = output
  *     column h, its N k-values contiguous; 16-byte aligned.
- *   w_scales: E8M0 [E, H, N/32], row-major (1 x 32 blocks along k), 16-byte
- *     aligned.
+ *   w_scales: E8M0 scales of the weight (1 x 32 blocks along k), per expert
+ *     the [H, N/32] matrix in the GEMM-ready tiled layout of
+ *     MOEACT_SCALES_GEMM (tiles of 128 rows x 4 scale columns, 512 bytes,
+ *     in row-major tile order; element (r, c) of a tile at byte
+ *     (r mod 32) * 16 + (r / 32) * 4 + c), experts one after another:
+ *     E * H * N/32 bytes, 16-byte aligned.
  *   H: output width, a positive multiple of 128, E * H < 2^31.
  *   out: bf16 [M, ldo] (caller-owned, 16-byte aligned), ldo >= H and a
  *     multiple of 8; columns [0, H) of every row are written.

@@ -39,24 +39,27 @@ namespace moeact {
 namespace {
 
 constexpr int kAtom = 16384;              // 128 rows x 128 bytes of k (one swizzle atom column)
-constexpr int kStages = 7;                // weight ring
+constexpr int kEpiWarpBytes = 4096;       // the epilogue's per-warp staging: 32 rows x 128 B
+constexpr int kEpiBytes = 8 * kEpiWarpBytes;
 constexpr int kStageBytes = 16384;        // 128 weight rows x 128 bytes of k
 constexpr int kXSlotBytes = 2 * kOpHalfBytes;   // gate + up of 16 rows x 128 columns
 constexpr int kXBytes = 8 * kXSlotBytes;  // the prologue's slots (8 warps)
-// The staging region: the weight ring, or (prologue) the X slots and the
-// sigmoid table after them.
-constexpr int kRBytes = ((kXBytes + kSigBytes > kStages * kStageBytes ? kXBytes + kSigBytes
-                                                                       : kStages * kStageBytes) +
-                         1023) / 1024 * 1024;
+// The staging region: (prologue) the X slots and the sigmoid table after
+// them; (GEMM) the weight ring and the epilogue's staging, as many ring stages
+// as fit.
+constexpr int kRBytes = (kXBytes + kSigBytes + 1023) / 1024 * 1024;
+constexpr int kStages = (kRBytes - kEpiBytes) / kStageBytes;   // weight ring
 constexpr int kMiscBytes = 2048;
+constexpr int kSfSlotBytes = 512 * (kFc2MaxN / 128);   // a tile's weight scales (tiled layout)
+constexpr int kSfSlots = 4;                               // loaded three tiles ahead
+constexpr int kSfBytes = (kSfSlots * kSfSlotBytes + 1023) / 1024 * 1024;
 constexpr int kSfaCol = 256;              // tensor-memory columns: accumulators [0, 256),
 constexpr int kSfbCol = 288;              // A scales [256, 288), W scales [288, 352)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kErrFc2Wait = 0x20u;
 
 // misc ints
-constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscE = 2, kMiscBlk = 3, kMiscTotal = 4,
-              kMiscScan = 16;
+constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscE = 2, kMiscBlk = 3, kMiscScan = 16;
 
 // ------------------------------------------------------------ tcgen05 wrappers
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
@@ -120,8 +123,19 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t* v) {
 __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Copies a 32-row x 16-byte matrix from shared memory into columns
+// [taddr, taddr + 4) of lanes 0-31 of every 32-lane quarter (each row to its
+// lane, bytes 4c .. 4c + 3 to column c).
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
@@ -135,6 +149,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Shared-memory descriptor of a source of tcgen05.cp: 16-byte rows, no
+// swizzling, 8-row groups 128 bytes apart (rows contiguous).
+__device__ __forceinline__ uint64_t cp_desc_rows16(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
 // Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 x E4M3,
@@ -151,6 +172,7 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
 
 struct Fc2Smem {
   unsigned char* A;       // [N/128 atoms][128 rows][128 bytes], swizzled
+  unsigned char* sf;      // [2 tiles][N/128 groups][512 bytes]: weight scales, tiled
   unsigned char* R;       // staging: weight ring / X slots + sigmoid table
   const float* sig;
   uint64_t* xbar;         // [8]
@@ -158,7 +180,8 @@ struct Fc2Smem {
   uint64_t* pro_done;     // count 8: the block's A codes and scales are complete
   uint64_t* b_full;       // [7]
   uint64_t* b_empty;      // [7]
-  uint64_t* sfb_full;     // [2] count 8: the weight scales of a tile are in tensor memory
+  uint64_t* sf_full;      // [3] a tile's weight scales have landed in shared memory
+  uint64_t* sf_empty;     // [3] ... and have been copied to tensor memory and used
   uint64_t* d_full;       // [2] an accumulator holds a finished tile
   uint64_t* d_empty;      // [2] count 8: an accumulator has been drained
   uint64_t* mma_done;
@@ -244,33 +267,6 @@ __device__ __forceinline__ uint32_t fc2_half(const Fc2Smem& m, const unsigned ch
   return b0 | (b1 << 8);
 }
 
-// The weight scales of output tile n (its 128 rows of W_e, all of k) into
-// tensor-memory buffer n & 1, in the layout the block-scaled MMA reads the
-// scales of its N operand: for each group of four k-blocks, four columns;
-// lane l of every 32-lane quarter, column c holds the word (four E8M0 bytes,
-// one per k-block) of tile row 32 c + l -- the same 32 x 4 words repeated in
-// all four quarters, each quarter written by its own warps (this warp: its
-// half of the groups).
-__device__ __forceinline__ void fc2_write_sfb(const Fc2Params& p, const Fc2Smem& m, int e, int n,
-                                              int q, int half_sel, int lane, uint32_t tbase) {
-  const int KA = p.N >> 7, KB = p.N >> 5;
-  const int b = n & 1;
-  const uint8_t* srow = p.w_scales + ((int64_t)e * p.H + 128 * n + lane) * KB;
-  const int64_t step = 32 * (int64_t)KB;   // 32 rows further
-  const uint32_t t = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(kSfbCol + 32 * b);
-  for (int g = half_sel; g < KA; g += 2) {
-    const uint8_t* c = srow + 4 * g;
-    tc_st4(t + 4 * g, __ldg(reinterpret_cast<const uint32_t*>(c)),
-           __ldg(reinterpret_cast<const uint32_t*>(c + step)),
-           __ldg(reinterpret_cast<const uint32_t*>(c + 2 * step)),
-           __ldg(reinterpret_cast<const uint32_t*>(c + 3 * step)));
-  }
-  tc_wait_st();
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(m.sfb_full + b);
-}
-
 template <bool STAGED>
 __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2Smem& m, int e,
                          int64_t row0, int mrows, uint32_t tbase) {
@@ -312,8 +308,9 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
     } else {
       // lane l: the four block scales of row 32 q + l for atom a.  The MMA
       // reads the scale of its M-operand row 32 q + l from lane 32 q + l,
-      // column q of the group (the layout of fc2_write_sfb, of which each
-      // quarter needs only its own column); the word goes to all four.
+      // column q of the group (the layout the weight scales are copied in by
+      // fc2_mma, of which each quarter needs only its own column); the word
+      // goes to all four.
       const uint32_t v = gather_row_scales(bh0, bh, lane, 0, 1);
       tc_st4(tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(kSfaCol + 4 * a), v, v, v, v);
     }
@@ -332,9 +329,8 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
   __syncwarp();
   if (lane == 0) mbar_arrive(m.pro_done);
 
-  // ---- output tiles: weight scales two tiles ahead, then drain each tile
+  // ---- output tiles: drain each accumulator into bf16 rows
   const int T = p.H >> 7;
-  for (int n = 0; n < T && n < 2; ++n) fc2_write_sfb(p, m, e, n, q, half_sel, lane, tbase);
   for (int n = 0; n < T; ++n) {
     if (warp_aborted(m)) break;
     const int b = n & 1;
@@ -348,28 +344,65 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(m.d_empty + b);
-    const int row = 32 * q + lane;
-    if (row < mrows) {
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (row0 + row) * p.ldo + 128 * n + 64 * half_sel);
+    // through this warp's staging in shared memory (16-byte chunk c of row t
+    // at chunk c ^ (a function of t), so that 8 consecutive threads or rows
+    // touch 8 different bank groups), then several lanes per row: each store
+    // instruction writes whole row segments
+    unsigned char* stg = m.R + kStages * kStageBytes + warp * kEpiWarpBytes;
+    constexpr int kChunks = kEpiWarpBytes / 32 / 16;      // 16-byte chunks of a staged row
+    constexpr int kPasses = 8 / kChunks;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+    for (int ps = 0; ps < kPasses; ++ps) {
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        const uint32_t* vv = v + 8 * (ps * kChunks + c);
         uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-        w.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-        w.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-        w.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-        dst[c] = w;
+        w.x = pack_bf16x2(__uint_as_float(vv[0]), __uint_as_float(vv[1]));
+        w.y = pack_bf16x2(__uint_as_float(vv[2]), __uint_as_float(vv[3]));
+        w.z = pack_bf16x2(__uint_as_float(vv[4]), __uint_as_float(vv[5]));
+        w.w = pack_bf16x2(__uint_as_float(vv[6]), __uint_as_float(vv[7]));
+        const int sw = kChunks == 8 ? (lane & 7) : ((lane >> 1) & 3);
+        *reinterpret_cast<uint4*>(stg + lane * (16 * kChunks) + ((c ^ sw) << 4)) = w;
       }
+      __syncwarp();
+      const int cc = lane % kChunks;
+#pragma unroll
+      for (int k = 0; k < kChunks; ++k) {
+        const int r = (32 / kChunks) * k + lane / kChunks;
+        const int sw = kChunks == 8 ? (r & 7) : ((r >> 1) & 3);
+        const uint4 w = *reinterpret_cast<const uint4*>(stg + r * (16 * kChunks) + ((cc ^ sw) << 4));
+        if (32 * q + r < mrows)
+          *reinterpret_cast<uint4*>(p.out + (row0 + 32 * q + r) * p.ldo + 128 * n +
+                                    64 * half_sel + 8 * (ps * kChunks + cc)) = w;
+      }
+      __syncwarp();
     }
-    if (n + 2 < T) fc2_write_sfb(p, m, e, n + 2, q, half_sel, lane, tbase);
   }
 }
 
-// Warp 8, one thread: the weight tiles of every output tile, in k order.
+// Warp 8, one thread: the weight tiles of every output tile, in k order,
+// and each output tile's weight scales (N/128 tiles of 512 bytes, contiguous
+// in the tiled layout) kSfSlots - 1 output tiles ahead: the scales of tile
+// n + 3 go out after the last weight tile of tile n, when the slot they reuse
+// (tile n - 1's) is already free, and have two tiles of MMAs to land.
 __device__ void fc2_producer(const CUtensorMap* tm_w, const Fc2Params& p, const Fc2Smem& m,
                              int e) {
   const int KA = p.N >> 7, T = p.H >> 7;
-  int issued = 0;
+  int issued = 0, sf_issued = 0;
+  auto issue_sf = [&](int n) {   // false on a timeout
+    const int ss = n % kSfSlots;
+    if (n >= kSfSlots &&
+        !mbar_wait(m.sf_empty + ss, (uint32_t)(n / kSfSlots - 1) & 1u))
+      return false;
+    mbar_expect_tx(m.sf_full + ss, 512 * KA);
+    bulk_load(m.sf + ss * kSfSlotBytes, p.w_scales + ((int64_t)e * T + n) * KA * 512, 512 * KA,
+              m.sf_full + ss);
+    sf_issued = n + 1;
+    return true;
+  };
+  // the first scales do not wait for the prologue (their slots are not
+  // shared with it); the weight tiles reuse the prologue's staging memory
+  for (int n = 0; n < T && n < kSfSlots - 1; ++n) issue_sf(n);
   if (!mbar_wait(m.pro_done, 0u)) set_abort(p, m);
   for (int g = 0; g < T * KA && !aborted(m); ++g) {
     const int n = g / KA, ks = g - n * KA, slot = g % kStages;
@@ -380,10 +413,16 @@ __device__ void fc2_producer(const CUtensorMap* tm_w, const Fc2Params& p, const 
     mbar_expect_tx(m.b_full + slot, kStageBytes);
     tma_load_2d(m.R + slot * kStageBytes, tm_w, 128 * ks, e * p.H + 128 * n, m.b_full + slot);
     issued = g + 1;
+    if (ks == KA - 1 && n + kSfSlots - 1 < T && !issue_sf(n + kSfSlots - 1)) {
+      set_abort(p, m);
+      break;
+    }
   }
   // every copy issued has landed before the CTA can exit (bounded)
   for (int g = max(0, issued - kStages); g < issued; ++g)
     mbar_wait(m.b_full + g % kStages, (uint32_t)(g / kStages) & 1u);
+  for (int n = max(0, sf_issued - kSfSlots); n < sf_issued; ++n)
+    mbar_wait(m.sf_full + n % kSfSlots, (uint32_t)(n / kSfSlots) & 1u);
 }
 
 // Warp 9, one thread: the MMAs of every output tile.
@@ -392,15 +431,22 @@ __device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
   bool ok = mbar_wait(m.pro_done, 0u) && !aborted(m);
   if (!ok) set_abort(p, m);
   tc_fence_after();
-  const uint32_t a_base = smem_addr(m.A), r_base = smem_addr(m.R);
+  const uint32_t a_base = smem_addr(m.A), r_base = smem_addr(m.R), sf_base = smem_addr(m.sf);
   for (int n = 0; ok && n < T; ++n) {
     const int b = n & 1;
-    if (!mbar_wait(m.sfb_full + b, (uint32_t)(n >> 1) & 1u) ||
+    // the accumulator and the weight-scale columns of buffer b are free once
+    // tile n - 2 has been drained (its MMAs, and so their reads, are done)
+    if (!mbar_wait(m.sf_full + n % kSfSlots, (uint32_t)(n / kSfSlots) & 1u) ||
         (n >= 2 && !mbar_wait(m.d_empty + b, (uint32_t)((n >> 1) - 1) & 1u))) {
       ok = false;
       break;
     }
     tc_fence_after();
+    // the tile's weight scales: smem -> tensor memory, ordered before the
+    // MMAs below (both issued by this thread)
+    for (int g = 0; g < KA; ++g)
+      tc_cp_32x128b_warpx4(tbase + kSfbCol + 32 * b + 4 * g,
+                           cp_desc_rows16(sf_base + (n % kSfSlots) * kSfSlotBytes + 512 * g));
     for (int ks = 0; ks < KA; ++ks) {
       const int g = n * KA + ks, slot = g % kStages;
       if (aborted(m) || !mbar_wait(m.b_full + slot, (uint32_t)(g / kStages) & 1u)) {
@@ -419,6 +465,7 @@ __device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
     }
     if (!ok) break;
     tc_commit(m.d_full + b);
+    tc_commit(m.sf_empty + n % kSfSlots);   // the smem scales of this tile are no longer needed
   }
   if (!ok) set_abort(p, m);
   // every MMA issued has completed before tensor memory is freed (bounded)
@@ -436,7 +483,8 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
   Fc2Smem m;
   const int KA = p.N >> 7;
   m.A = base;
-  m.R = base + KA * kAtom;
+  m.sf = base + KA * kAtom;
+  m.R = m.sf + kSfBytes;
   m.sig = reinterpret_cast<const float*>(m.R + kXBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(m.R + kRBytes);
   m.xbar = bars;
@@ -444,11 +492,12 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
   m.pro_done = bars + 9;
   m.b_full = bars + 10;
   m.b_empty = bars + 10 + kStages;
-  m.sfb_full = bars + 10 + 2 * kStages;
-  m.d_full = m.sfb_full + 2;
-  m.d_empty = m.sfb_full + 4;
-  m.mma_done = m.sfb_full + 6;
-  m.misc = reinterpret_cast<int*>(bars + 32);
+  m.sf_full = bars + 10 + 2 * kStages;
+  m.sf_empty = m.sf_full + kSfSlots;
+  m.d_full = m.sf_empty + kSfSlots;
+  m.d_empty = m.d_full + 2;
+  m.mma_done = m.d_empty + 2;
+  m.misc = reinterpret_cast<int*>(bars + 40);
   const int tid = threadIdx.x, warp = tid >> 5;
 
   // ---- this CTA's (expert, 128-row block); the offsets are validated first
@@ -462,24 +511,29 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
     else local += (int)((r1 - r0 + 127) >> 7);
   }
   if (tid == 0 && (p.row_offs[0] != 0 || p.row_offs[E] != p.M)) bad = 1;
-  m.misc[kMiscScan + tid] = local;
+  // exclusive prefix of the per-thread block counts: a shuffle scan inside
+  // each warp, then the 10 warp totals
+  const int lane0 = tid & 31;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(kFull, incl, off);
+    if (lane0 >= off) incl += v;
+  }
+  if (lane0 == 31) m.misc[kMiscScan + warp] = incl;
   const int any_bad = __syncthreads_or(bad);
   if (blockIdx.x == 0 && tid == 0) *p.status = any_bad ? 3 : 0;
   if (any_bad) return;
-  if (tid == 0) {
-    int acc = 0;
-    for (int t = 0; t < kFc2Threads; ++t) {
-      const int v = m.misc[kMiscScan + t];
-      m.misc[kMiscScan + t] = acc;
-      acc += v;
-    }
-    m.misc[kMiscTotal] = acc;
+  int wbase = 0, total = 0;
+  for (int w = 0; w < kFc2Threads / 32; ++w) {
+    const int v = m.misc[kMiscScan + w];
+    if (w < warp) wbase += v;
+    total += v;
   }
-  __syncthreads();
   const int u = blockIdx.x;
-  if (u >= m.misc[kMiscTotal]) return;
+  if (u >= total) return;
   {
-    int acc = m.misc[kMiscScan + tid];
+    int acc = wbase + incl - local;
     if (u >= acc && u < acc + local) {
       for (int e = e_lo; e < e_hi; ++e) {
         const int nb = (int)((p.row_offs[e + 1] - p.row_offs[e] + 127) >> 7);
@@ -506,8 +560,11 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
       mbar_init(m.b_full + i, 1);
       mbar_init(m.b_empty + i, 1);
     }
+    for (int i = 0; i < kSfSlots; ++i) {
+      mbar_init(m.sf_full + i, 1);
+      mbar_init(m.sf_empty + i, 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(m.sfb_full + i, 8);
       mbar_init(m.d_full + i, 1);
       mbar_init(m.d_empty + i, 8);
     }
@@ -544,7 +601,7 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
 
 }  // namespace
 
-int fc2_smem_bytes(int N) { return 1024 + (N / 128) * kAtom + kRBytes + kMiscBytes; }
+int fc2_smem_bytes(int N) { return 1024 + (N / 128) * kAtom + kSfBytes + kRBytes + kMiscBytes; }
 
 cudaError_t fc2_prepare() {
   const int bytes = fc2_smem_bytes(kFc2MaxN);
@@ -566,9 +623,13 @@ cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, const CUtens
   return cudaGetLastError();
 }
 
-static_assert(kMiscScan * 4 + kFc2Threads * 4 + 32 * 8 <= kMiscBytes, "misc region too small");
-static_assert(kXBytes + kSigBytes <= kRBytes && kStages * kStageBytes <= kRBytes,
-              "staging region too small");
+static_assert(kMiscScan * 4 + (kFc2Threads / 32) * 4 + 40 * 8 <= kMiscBytes,
+              "misc region too small");
+static_assert(10 + 2 * kStages + 2 * kSfSlots + 5 <= 40, "barrier region too small");
+static_assert(kSfBytes % 1024 == 0, "the staging region must stay 1024-byte aligned");
+static_assert(kXBytes + kSigBytes <= kRBytes, "staging region too small");
+static_assert(kStages * kStageBytes + kEpiBytes <= kRBytes && kStages >= 4,
+              "epilogue staging does not fit");
 static_assert(kSfbCol + 64 <= (int)kTmemCols && kSfaCol + 32 <= kSfbCol,
               "tensor-memory columns overlap");
 

@@ -63,12 +63,20 @@ def _check(got, ref, bound, what):
     return float((err / np.maximum(lim, 1e-300)).max())
 
 
+def _tiled(ws):
+    """Row-major weight scales [E, H, N/32] -> the kernel's GEMM-ready tiled
+    layout per expert (the oracle's pinned layout function)."""
+    ws = np.asarray(ws)
+    return torch.from_numpy(np.stack([oracle.scales_gemm_layout(w).reshape(w.shape)
+                                      for w in ws]))
+
+
 def _run(case, N, splits, wc, ws, dev, staged=False):
     m = torch.tensor(splits, dtype=torch.int64)
     M = int(m.sum())
     ro, cb, st = mg.splits_to_offsets(m.to(dev), M)
     x, s = case["x"].to(dev), case["s"].to(dev)
-    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(x, s, ro, wc.to(dev), ws.to(dev),
+    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(x, s, ro, wc.to(dev), _tiled(ws).to(dev),
                                                   staged_rounding=staged)
     torch.cuda.synchronize()
     assert int(st.item()) == 0 and int(st2.item()) == 0
@@ -129,6 +137,7 @@ def test_fc2_writes_nothing_for_bad_offsets_or_a_set_noop_flag(cuda_device):
     N, H, M = 128, 128, 256
     case = random_case(M, N, 41)
     wc, ws = fc2_weights(2, H, N, 8)
+    ws = _tiled(ws)
     dev = cuda_device
     x, s = case["x"].to(dev), case["s"].to(dev)
     bad = torch.tensor([0, 200, 100], dtype=torch.int64, device=dev)   # ends past M
@@ -161,7 +170,8 @@ def test_fc2_at_the_qwen3_moe_workload_sampled_rows(cuda_device):
     E = int(m.numel())
     wc, ws = fc2_weights(E, H, N, 11, device=dev)
     ro, cb, st = mg.splits_to_offsets(m.to(dev), M)
-    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(inp["x"], inp["s"], ro, wc, ws)
+    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(inp["x"], inp["s"], ro, wc,
+                                                  _tiled(ws.cpu()).to(dev))
     torch.cuda.synchronize()
     assert int(st.item()) == 0 and int(st2.item()) == 0
     ro_h = ro.cpu().numpy()

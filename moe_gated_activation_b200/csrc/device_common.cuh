@@ -189,14 +189,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
-               "selp.u32 %0, 1, 0, p; }"
-               : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
-  return ok != 0;
-}
-
 // Nanoseconds of the GPU's global timer.
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
@@ -204,18 +196,35 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Tests whether the phase of `bar` with the given parity has completed; a
+// thread whose phase has not completed is suspended until it does or
+// `hint_ns` nanoseconds pass (it takes no issue slots from the warps that are
+// working meanwhile).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; "
+               "selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns) : "memory");
+  return ok != 0;
+}
+
 // Waits for a phase of `bar` for at most `limit_ns` nanoseconds of wall time
-// (the global timer is read every 64 polls; each try_wait may itself suspend
-// for a short, hardware-chosen time); false on timeout.  A copy of a few KiB
-// lands in microseconds, so the kernels' limit, one second, is only ever
-// reached by a copy that will never complete.
+// (the global timer is read every 4 polls); false on timeout.  Each poll
+// may suspend the thread for up to 100 us -- it resumes as soon as the phase
+// completes -- so that a warp waiting for its data takes no issue slots from
+// the warps that compute (measured 1-2% faster on the Qwen3-MoE-shaped
+// workload, neutral on the largest).  A copy of a few KiB lands in
+// microseconds, so the kernels' limit, one second, is only ever reached by a
+// copy that will never complete.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint32_t kWaitHintNs = 100000;
 __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    for (int i = 0; i < 4; ++i)
+      if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
     if (global_ns() - t0 > limit_ns) return false;
   }
 }

@@ -319,13 +319,15 @@ moeact_status scaled_swiglu_mxfp8_bwd_noalloc(const void* dy, int64_t lddy, cons
  * interleaved by glu_interleave, W = 2N in the backward; no staged
  * rounding).  alpha must lie in
  * [0.8125, 2] and limit be > 0 (+Inf allowed), else MOEACT_EINVAL.  The
- * first call with a given alpha on a device builds that alpha's sigmoid table
- * (device memory, kept until exit; synchronises the device once; at most 8
- * distinct alphas per device, else MOEACT_ERANGE); it must not be inside a
- * stream capture (MOEACT_EUNSUPPORTED) -- call moeact_init_clamped(alpha)
- * first.  With alpha = 1 and limit = +Inf it is SwiGLU with up + 1 for up.
+ * first call with a given (alpha, limit) on a device builds that pair's
+ * sigmoid table, sigma(RN(alpha * min(g, limit))) for every bf16 gate g
+ * (device memory, kept until exit; synchronises the device once; at most 32
+ * distinct pairs per device, else MOEACT_ERANGE); it must not be inside a
+ * stream capture (MOEACT_EUNSUPPORTED) -- call moeact_init_clamped(alpha,
+ * limit) first.  With alpha = 1 and limit = +Inf it is SwiGLU with up + 1
+ * for up.
  * ------------------------------------------------------------------- */
-moeact_status moeact_init_clamped(float alpha);
+moeact_status moeact_init_clamped(float alpha, float limit);
 moeact_status scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
                                               int64_t M, int64_t N, int dirs, float alpha,
                                               float limit, int32_t glu_interleave,
@@ -350,9 +352,10 @@ moeact_status grouped_scaled_clamped_swiglu_mxfp8_bwd(
     const int64_t* row_offs, const int64_t* colblk_offs, int32_t num_groups, int32_t* status,
     void* dx, float* dscale, moeact_mx_out out, void* workspace, size_t workspace_bytes,
     void* stream);
-/* Test hook: the table of sigma(RN(alpha * g)) over all 65536 bf16 g, fp32
- * [65536] (as moeact_sigmoid_dump). */
-moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream);
+/* Test hook: the table of sigma(RN(alpha * min(g, limit))) over all 65536
+ * bf16 g, fp32 [65536] (as moeact_sigmoid_dump; limit = +Inf: the unclamped
+ * sigma(RN(alpha * g))). */
+moeact_status moeact_clamped_sigmoid_dump(float alpha, float limit, float* out, void* stream);
 
 /* Reads and clears this device's error word: non-zero if a kernel gave up
  * waiting for its own input copies (bit 0 forward, bit 1 backward, bit 2 the

@@ -63,7 +63,7 @@ _SIGS = {
     "grouped_scaled_srelu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, P, P, I32, P, P, P,
                                         MxOut, P, SZ, P], I),
     "moeact_sigmoid_dump": ([P, P], I),
-    "moeact_init_clamped": ([F], I),
+    "moeact_init_clamped": ([F, F], I),
     "scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, I32, MxOut, P], I),
     "grouped_scaled_clamped_swiglu_mxfp8_fwd": ([P, I64, P, I64, I64, I, F, F, I32, P, P, I32, P,
                                                  MxOut, P], I),
@@ -71,7 +71,7 @@ _SIGS = {
                                          P, SZ, P], I),
     "grouped_scaled_clamped_swiglu_mxfp8_bwd": ([P, I64, P, I64, P, I64, I64, I, F, F, I32, P, P,
                                                  I32, P, P, P, MxOut, P, SZ, P], I),
-    "moeact_clamped_sigmoid_dump": ([F, P, P], I),
+    "moeact_clamped_sigmoid_dump": ([F, F, P, P], I),
     "moeact_device_error": ([P], I),
     "moeact_wait_selftest": ([I, ctypes.c_uint32, P, P], I),
     "grouped_scaled_swiglu_mxfp8_fc2": ([P, I64, P, I64, I64, I, P, I32, P, P, P, I64, P, I64, P,

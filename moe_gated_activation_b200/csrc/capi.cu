@@ -150,8 +150,8 @@ moeact_status init_device(int dev) {
     int* d_unc = nullptr;
     e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d_unc), g_sigma_uncertain);
     if (e == cudaSuccess) {
-      sigma_table_init<<<(kSigEntriesPadded + 255) / 256, 256, 0, st>>>(g_sig_ptr[dev], 1.0f,
-                                                                          d_unc);
+      sigma_table_init<<<(kSigEntriesPadded + 255) / 256, 256, 0, st>>>(
+          g_sig_ptr[dev], 1.0f, INFINITY, 1.0f, d_unc);
       e = cudaGetLastError();
     }
   }
@@ -357,9 +357,10 @@ int group_smem(bool sig, bool grouped, int E) { return (grouped && !sig) ? group
 // sufficient: for |g| < 2^-25, sigma(RN(alpha g)) rounds to 1/2 when alpha <=
 // 2, and for |g| >= 128 it is 0 or 1 when alpha >= 13/16.
 constexpr float kClampAlphaMin = 0.8125f, kClampAlphaMax = 2.0f;
-constexpr int kMaxAlphaTables = 8;
+constexpr int kMaxAlphaTables = 32;
 struct AlphaTable {
   uint32_t alpha_bits;
+  uint32_t limit_bits;
   float* tab;
 };
 AlphaTable g_alpha_tab[kMaxDevices][kMaxAlphaTables];
@@ -372,24 +373,36 @@ moeact_status check_clamp_args(float alpha, float limit) {
   return MOEACT_OK;
 }
 
-// The device table of sigma(RN(alpha * g)) for `alpha`, built on first use.
-moeact_status alpha_table(int dev, float alpha, cudaStream_t call_stream, const float** out) {
-  uint32_t bits;
+bool sigmoid_f32_host(float z, float* out);
+
+// The device table of a ClampedSwiGLU call, built on first use: sigma(RN(alpha
+// * g)) for every bf16 gate g <= limit and sigma(RN(alpha * limit)) for every
+// gate above it (limit = +Inf: the unclamped table), so that the kernels take
+// a clamped gate's sigmoid from the table like any other.
+moeact_status alpha_table(int dev, float alpha, float limit, cudaStream_t call_stream,
+                          const float** out) {
+  uint32_t bits, lbits;
   std::memcpy(&bits, &alpha, 4);
+  std::memcpy(&lbits, &limit, 4);
   std::lock_guard<std::mutex> lk(g_mu);
   for (int i = 0; i < g_n_alpha[dev]; ++i)
-    if (g_alpha_tab[dev][i].alpha_bits == bits) {
+    if (g_alpha_tab[dev][i].alpha_bits == bits && g_alpha_tab[dev][i].limit_bits == lbits) {
       *out = g_alpha_tab[dev][i].tab;
       return MOEACT_OK;
     }
   if (g_n_alpha[dev] == kMaxAlphaTables)
-    return fail(MOEACT_ERANGE, "more than %d distinct alpha values on one device", kMaxAlphaTables);
+    return fail(MOEACT_ERANGE, "more than %d distinct (alpha, limit) pairs on one device",
+                kMaxAlphaTables);
+  float sig_limit = 1.0f;   // sigma(RN(alpha * limit)), fp32
+  if (!sigmoid_f32_host(alpha * limit, &sig_limit))
+    return fail(MOEACT_EUNSUPPORTED, "sigma(alpha * limit) could not be certified");
   cudaStreamCaptureStatus capt = cudaStreamCaptureStatusNone;
   if (call_stream && cudaStreamIsCapturing(call_stream, &capt) == cudaSuccess &&
       capt != cudaStreamCaptureStatusNone)
     return fail(MOEACT_EUNSUPPORTED,
-                "first use of alpha %g inside a stream capture; call moeact_init_clamped() first",
-                (double)alpha);
+                "first use of alpha %g, limit %g inside a stream capture; call "
+                "moeact_init_clamped() first",
+                (double)alpha, (double)limit);
   float* tab = nullptr;
   int* d_unc = nullptr;
   cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&tab), kSigBytes);
@@ -400,7 +413,8 @@ moeact_status alpha_table(int dev, float alpha, cudaStream_t call_stream, const 
   if (e == cudaSuccess) e = cudaMemsetAsync(tab, 0, kSigBytes, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(d_unc, 0, sizeof(int), st);
   if (e == cudaSuccess) {
-    sigma_table_init<<<(kSigEntriesPadded + 255) / 256, 256, 0, st>>>(tab, alpha, d_unc);
+    sigma_table_init<<<(kSigEntriesPadded + 255) / 256, 256, 0, st>>>(tab, alpha, limit,
+                                                                        sig_limit, d_unc);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaMemcpyAsync(&unc, d_unc, sizeof(int), cudaMemcpyDeviceToHost, st);
@@ -413,7 +427,7 @@ moeact_status alpha_table(int dev, float alpha, cudaStream_t call_stream, const 
     return fail(MOEACT_ECUDA, "sigmoid table for alpha %g: %d entries could not be certified",
                 (double)alpha, unc);
   }
-  g_alpha_tab[dev][g_n_alpha[dev]++] = {bits, tab};
+  g_alpha_tab[dev][g_n_alpha[dev]++] = {bits, lbits, tab};
   *out = tab;
   return MOEACT_OK;
 }
@@ -473,14 +487,13 @@ moeact_status act_params(const ActArgs& a, int dev, cudaStream_t cs, Params& p) 
   p.sig_src = g_sig_ptr[dev];
   p.clamp_L = a.limit;
   p.clamp_alpha = a.alpha;
-  p.clamp_sigL = 1.0f;
+  // the largest bf16 not above L (L > 0: its fp32 bits truncated), both halves
+  uint32_t lb;
+  std::memcpy(&lb, &a.limit, 4);
+  lb >>= 16;
+  p.clamp_Lb2 = lb | (lb << 16);
   if (a.act != kClamped) return MOEACT_OK;
-  moeact_status st = alpha_table(dev, a.alpha, cs, &p.sig_src);
-  if (st) return st;
-  const float z = a.alpha * a.limit;   // RN(alpha * L), fp32
-  if (!sigmoid_f32_host(z, &p.clamp_sigL))
-    return fail(MOEACT_EUNSUPPORTED, "sigma(alpha * limit) could not be certified");
-  return MOEACT_OK;
+  return alpha_table(dev, a.alpha, a.limit, cs, &p.sig_src);
 }
 
 moeact_status fwd_common(const ActArgs& a, const void* x, int64_t ldx, const float* s,
@@ -764,14 +777,14 @@ moeact_status grouped_scaled_srelu_mxfp8_bwd(const void* dy, int64_t lddy, const
 }
 
 // ---------------------------------------------------------------- ClampedSwiGLU
-moeact_status moeact_init_clamped(float alpha) {
+moeact_status moeact_init_clamped(float alpha, float limit) {
   t_err[0] = 0;
-  moeact_status st = check_clamp_args(alpha, 1.0f);
+  moeact_status st = check_clamp_args(alpha, limit);
   if (st) return st;
   int dev;
   if ((st = ensure_ready(nullptr, &dev))) return st;
   const float* tab;
-  return alpha_table(dev, alpha, nullptr, &tab);
+  return alpha_table(dev, alpha, limit, nullptr, &tab);
 }
 
 moeact_status scaled_clamped_swiglu_mxfp8_fwd(const void* x, int64_t ldx, const float* s,
@@ -816,17 +829,17 @@ moeact_status grouped_scaled_clamped_swiglu_mxfp8_bwd(
                     workspace_bytes, stream, true);
 }
 
-moeact_status moeact_clamped_sigmoid_dump(float alpha, float* out, void* stream) {
+moeact_status moeact_clamped_sigmoid_dump(float alpha, float limit, float* out, void* stream) {
   t_err[0] = 0;
   if (!out) return fail(MOEACT_EINVAL, "out is required");
   if (!aligned(out, 4)) return fail(MOEACT_EALIGN, "out must be 4-byte aligned");
-  moeact_status st = check_clamp_args(alpha, 1.0f);
+  moeact_status st = check_clamp_args(alpha, limit);
   if (st) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int dev;
   if ((st = ensure_ready(cs, &dev))) return st;
   const float* tab;
-  if ((st = alpha_table(dev, alpha, cs, &tab))) return st;
+  if ((st = alpha_table(dev, alpha, limit, cs, &tab))) return st;
   sigma_table_dump<<<128, 256, kSigBytes, cs>>>(tab, out);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sigmoid dump launch");

@@ -94,6 +94,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Per 16-bit lane of two packed bf16 pairs: 0xFFFF where a > b, else 0 (an
+// ordered comparison: false when either value is NaN).
+__device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.gt.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // relu that keeps NaN (NaN in -> NaN out); negative and zero inputs give +0.
 __device__ __forceinline__ float relu_keep_nan(float v) {
   return v > 0.0f ? v : (v != v ? v : 0.0f);
@@ -147,6 +155,14 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
       "mov.b64 rc, {%6, %7}; fma.rn.f32x2 rd, ra, rb, rc; mov.b64 {%0, %1}, rd; }"
       : "=f"(r.x), "=f"(r.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("{ .reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; "
+      "add.rn.f32x2 rd, ra, rb; mov.b64 {%0, %1}, rd; }"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return r;
 }
 

@@ -26,12 +26,25 @@ __device__ __align__(16) float g_sigma_table[kSigBytes / 4];
 // binary64 value lies within 2^-48 (relative) of a rounding boundary are
 // counted as uncertain (none are expected for alpha = 1: the closest true
 // value stays 2^-37 away; the caller refuses a table with any).
-__global__ void sigma_table_init(float* tab, float alpha, int* uncertain) {
+//
+// A ClampedSwiGLU table also takes the clamp of the gate at `limit`: every
+// entry of a gate above it holds sig_limit = sigma(RN(alpha * limit))
+// (certified by the caller).  The entries that stand for a range of gates
+// stay right for every gate of their range: sigma is 1/2 on both sides of a
+// limit below 2^-25 (the first entry, |g| <= 2^-25), and gates of 128 and
+// above (the last entry) either all lie above the limit or, for a limit of
+// 128 or more and alpha >= 13/16, have sigma 1 on both sides of it.
+__global__ void sigma_table_init(float* tab, float alpha, float limit, float sig_limit,
+                                 int* uncertain) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= kSigEntries) return;
   const uint32_t neg = i >= (int)kSigPerSign ? 1u : 0u;
   const uint32_t mag = (uint32_t)i - neg * kSigPerSign + kSigLo;
   const float g = __uint_as_float(((neg << 15) | mag) << 16);
+  if (g > limit) {
+    tab[sig_slot(i)] = sig_limit;
+    return;
+  }
   const float z = __fmul_rn(alpha, g);
   if (fabsf(z) < 0x1p-9f) {
     const double hi = 0.5 + 0.25 * (double)z;

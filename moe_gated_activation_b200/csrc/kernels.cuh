@@ -81,11 +81,14 @@ struct Params {
   int n_tiles;
   int gemm_scales;    // scales in the GEMM-ready tiled layout (see gemm_row_scales_off)
   const float* sig_src;   // the sigmoid table to stage (device memory, shared-memory layout)
-  // ClampedSwiGLU: gate and up limit L, slope alpha (folded into sig_src),
-  // and sigma(RN(alpha * L)), the sigmoid of a clamped gate
+  // ClampedSwiGLU: gate and up limit L and slope alpha.  Both are folded
+  // into sig_src, which holds sigma(RN(alpha * g)) for g <= L and
+  // sigma(RN(alpha * L)) for every gate above L.  clamp_Lb2: the largest
+  // bf16 not above L, in both halves (a bf16 value is above L exactly when it
+  // is above that).
   float clamp_L;
   float clamp_alpha;
-  float clamp_sigL;
+  uint32_t clamp_Lb2;
   const int32_t* noop;   // nullable: a non-zero flag makes the call write nothing
   // Gated layouts of x and dX (width 2N): ilv == 0 is [gate | up] halves;
   // ilv = G > 0 is G gate columns, then the G matching up columns, repeated.
@@ -522,51 +525,47 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
   return r;
 }
 
-// A pair of gates (fp32, with their sigmoids from the table) clamped at L: a
-// gate above L becomes L and takes sigma(RN(alpha * L)); NaN passes through.
-__device__ __forceinline__ void clamp_gates(float2& g, float2& sg, const Params& p) {
-  sg.x = g.x > p.clamp_L ? p.clamp_sigL : sg.x;
-  sg.y = g.y > p.clamp_L ? p.clamp_sigL : sg.y;
-  g.x = min_nan(g.x, p.clamp_L);
-  g.y = min_nan(g.y, p.clamp_L);
+// A pair of gates clamped at L (NaN passes through).  Their sigmoids need no
+// clamp: the table of a ClampedSwiGLU call holds sigma(RN(alpha * L)) for
+// every gate above L.
+__device__ __forceinline__ float2 clamp_gate_pair(float2 g, float L) {
+  return make_float2(min_nan(g.x, L), min_nan(g.y, L));
 }
 
 // clamp(u, -L, L) + 1 for a pair of ups (NaN passes through).
 __device__ __forceinline__ float2 clamped_up_plus_one(float2 u, float L) {
-  return make_float2(__fadd_rn(max_nan(min_nan(u.x, L), -L), 1.0f),
-                     __fadd_rn(max_nan(min_nan(u.y, L), -L), 1.0f));
+  return add2(make_float2(max_nan(min_nan(u.x, L), -L), max_nan(min_nan(u.y, L), -L)),
+              make_float2(1.0f, 1.0f));
 }
 
 // Backward of ClampedSwiGLU for the four columns of a lane in one row (p =
-// dY * s): the SwiGLU form with slope alpha, dsilu = fma(RN(alpha * silu),
-// 1 - sig, sig); a clamped gate or up gets a zero gradient.
+// dY * s), as packed bf16 pairs: the SwiGLU form with slope alpha, dsilu =
+// fma(RN(alpha * silu), 1 - sig, sig).  A gate above L or an up outside
+// [-L, L] gets a +0 gradient: its half of the packed pair is cleared, so that
+// a NaN or Inf in dY does not reach it.  The comparisons take the bf16 inputs
+// as they are (NaN compares false).
 __device__ __forceinline__ void clamped_bwd_math(const Params& p, const float* sig, uint2 G,
-                                                 uint2 U, float2 p01, float2 p23, float2& dg01,
-                                                 float2& dg23, float2& du01, float2& du23,
+                                                 uint2 U, float2 p01, float2 p23, uint32_t& dg0,
+                                                 uint32_t& dg1, uint32_t& du0, uint32_t& du1,
                                                  float2& h01, float2& h23) {
   const float L = p.clamp_L;
-  const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
   float2 sg01, sg23;
   sigma_pair(sig, G.x, sg01.x, sg01.y);
   sigma_pair(sig, G.y, sg23.x, sg23.y);
-  float2 g01 = bf16x2_to_f2(G.x), g23 = bf16x2_to_f2(G.y);
-  clamp_gates(g01, sg01, p);
-  clamp_gates(g23, sg23, p);
-  const float2 si01 = mul2(g01, sg01), si23 = mul2(g23, sg23);
-  const float2 v01 = clamped_up_plus_one(u01, L), v23 = clamped_up_plus_one(u23, L);
+  const float2 si01 = mul2(clamp_gate_pair(bf16x2_to_f2(G.x), L), sg01);
+  const float2 si23 = mul2(clamp_gate_pair(bf16x2_to_f2(G.y), L), sg23);
+  const float2 v01 = clamped_up_plus_one(bf16x2_to_f2(U.x), L);
+  const float2 v23 = clamped_up_plus_one(bf16x2_to_f2(U.y), L);
   const float2 one = make_float2(1.0f, 1.0f), a2 = make_float2(p.clamp_alpha, p.clamp_alpha);
   const float2 ds01 = fma2(mul2(a2, si01), sub2(one, sg01), sg01);
   const float2 ds23 = fma2(mul2(a2, si23), sub2(one, sg23), sg23);
   const float2 dga = mul2(mul2(p01, v01), ds01), dgb = mul2(mul2(p23, v23), ds23);
   const float2 dua = mul2(p01, si01), dub = mul2(p23, si23);
-  const auto cu = [L](float u) { return fabsf(u) > L; };
-  // the gate comparisons are made here, from the input bits, rather than
-  // kept from the clamp (fewer values live across the math)
-  const auto cg = [L](float g) { return g > L; };
-  dg01 = make_float2(cg(bf16_lo_p(G.x)) ? 0.0f : dga.x, cg(bf16_hi_p(G.x)) ? 0.0f : dga.y);
-  dg23 = make_float2(cg(bf16_lo_p(G.y)) ? 0.0f : dgb.x, cg(bf16_hi_p(G.y)) ? 0.0f : dgb.y);
-  du01 = make_float2(cu(u01.x) ? 0.0f : dua.x, cu(u01.y) ? 0.0f : dua.y);
-  du23 = make_float2(cu(u23.x) ? 0.0f : dub.x, cu(u23.y) ? 0.0f : dub.y);
+  const uint32_t Lb2 = p.clamp_Lb2;
+  dg0 = pack_bf16x2(dga.x, dga.y) & ~bf16x2_gt_mask(G.x, Lb2);
+  dg1 = pack_bf16x2(dgb.x, dgb.y) & ~bf16x2_gt_mask(G.y, Lb2);
+  du0 = pack_bf16x2(dua.x, dua.y) & ~bf16x2_gt_mask(U.x & 0x7FFF7FFFu, Lb2);
+  du1 = pack_bf16x2(dub.x, dub.y) & ~bf16x2_gt_mask(U.y & 0x7FFF7FFFu, Lb2);
   h01 = mul2(si01, v01);
   h23 = mul2(si23, v23);
 }
@@ -607,10 +606,8 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
         float2 sg01, sg23;
         sigma_pair(m.sig, G.x, sg01.x, sg01.y);
         sigma_pair(m.sig, G.y, sg23.x, sg23.y);
-        float2 g01 = bf16x2_to_f2(G.x), g23 = bf16x2_to_f2(G.y);
-        clamp_gates(g01, sg01, p);
-        clamp_gates(g23, sg23, p);
-        const float2 si01 = mul2(g01, sg01), si23 = mul2(g23, sg23);
+        const float2 si01 = mul2(clamp_gate_pair(bf16x2_to_f2(G.x), p.clamp_L), sg01);
+        const float2 si23 = mul2(clamp_gate_pair(bf16x2_to_f2(G.y), p.clamp_L), sg23);
         h01 = mul2(si01, clamped_up_plus_one(bf16x2_to_f2(U.x), p.clamp_L));
         h23 = mul2(si23, clamped_up_plus_one(bf16x2_to_f2(U.y), p.clamp_L));
       } else if (ACT == kSwiGLU) {
@@ -825,12 +822,7 @@ __device__ __forceinline__ void bwd_row(const Params& p, const float* sig, uint2
   const float2 p01 = mul2(d01, s2), p23 = mul2(d23, s2);
   float2 h01, h23;
   if (ACT == kClamped) {
-    float2 dga, dgb, dua, dub;
-    clamped_bwd_math(p, sig, G, U, p01, p23, dga, dgb, dua, dub, h01, h23);
-    dg0 = pack_bf16x2(dga.x, dga.y);
-    dg1 = pack_bf16x2(dgb.x, dgb.y);
-    du0 = pack_bf16x2(dua.x, dua.y);
-    du1 = pack_bf16x2(dub.x, dub.y);
+    clamped_bwd_math(p, sig, G, U, p01, p23, dg0, dg1, du0, du1, h01, h23);
   } else if (ACT == kSwiGLU) {
     const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
     float2 sg01, sg23;
@@ -906,9 +898,10 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
       const float2 d01 = bf16x2_to_f2(D.x), d23 = bf16x2_to_f2(D.y);
       const float2 p01 = mul2(d01, s2), p23 = mul2(d23, s2);
       float2 dg01, dg23, du01, du23, h01, h23;
+      uint32_t qg0, qg1, qu0, qu1;   // the packed bf16 gradients
       if (ACT == kClamped) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
-        clamped_bwd_math(p, m.sig, G, U, p01, p23, dg01, dg23, du01, du23, h01, h23);
+        clamped_bwd_math(p, m.sig, G, U, p01, p23, qg0, qg1, qu0, qu1, h01, h23);
       } else if (ACT == kSwiGLU) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
         const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
@@ -935,11 +928,17 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
         h01 = mul2(make_float2(r0, r1), make_float2(r0, r1));
         h23 = mul2(make_float2(r2, r3), make_float2(r2, r3));
       }
+      if (ACT != kClamped) {
+        qg0 = pack_bf16x2(dg01.x, dg01.y);
+        qg1 = pack_bf16x2(dg23.x, dg23.y);
+        qu0 = pack_bf16x2(du01.x, du01.y);
+        qu1 = pack_bf16x2(du23.x, du23.y);
+      }
       const bool live = FULL || r < nrows;
-      DG[r][0] = live ? pack_bf16x2(dg01.x, dg01.y) : 0u;
-      DG[r][1] = live ? pack_bf16x2(dg23.x, dg23.y) : 0u;
-      DU[r][0] = (live && ACT != kSReLU) ? pack_bf16x2(du01.x, du01.y) : 0u;
-      DU[r][1] = (live && ACT != kSReLU) ? pack_bf16x2(du23.x, du23.y) : 0u;
+      DG[r][0] = live ? qg0 : 0u;
+      DG[r][1] = live ? qg1 : 0u;
+      DU[r][0] = (live && ACT != kSReLU) ? qu0 : 0u;
+      DU[r][1] = (live && ACT != kSReLU) ? qu1 : 0u;
       P[i] = live ? __fmaf_rn(d23.y, h23.y, __fmaf_rn(d23.x, h23.x,
                               __fmaf_rn(d01.y, h01.y, __fmul_rn(d01.x, h01.x))))
                   : 0.0f;

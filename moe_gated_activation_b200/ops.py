@@ -433,16 +433,18 @@ def grouped_scaled_clamped_swiglu_mxfp8_bwd(dy, x, s, row_offs, colblk_offs, *,
                 glu_interleave=glu_interleave), status
 
 
-def init_clamped(alpha=CLAMPED_ALPHA):
-    """Build the sigmoid table of a ClampedSwiGLU slope on the current device
-    (the first call with that alpha would; this one may precede a capture)."""
-    _capi.call("moeact_init_clamped", alpha)
+def init_clamped(alpha=CLAMPED_ALPHA, limit=CLAMPED_LIMIT):
+    """Build the sigmoid table of a ClampedSwiGLU (slope, limit) on the current
+    device (the first call with that pair would; this one may precede a
+    capture)."""
+    _capi.call("moeact_init_clamped", alpha, limit)
 
 
-def clamped_sigmoid_table(alpha=CLAMPED_ALPHA, device="cuda"):
-    """fp32 sigma(RN(alpha * g)) for all 65536 bf16 g, as the kernels compute it."""
+def clamped_sigmoid_table(alpha=CLAMPED_ALPHA, limit=float("inf"), device="cuda"):
+    """fp32 sigma(RN(alpha * min(g, limit))) for all 65536 bf16 g, as the
+    kernels look it up."""
     out = torch.empty(65536, dtype=torch.float32, device=device)
-    _capi.call("moeact_clamped_sigmoid_dump", alpha, _ptr(out), _stream(out.device))
+    _capi.call("moeact_clamped_sigmoid_dump", alpha, limit, _ptr(out), _stream(out.device))
     return out
 
 

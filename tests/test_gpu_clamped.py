@@ -15,7 +15,9 @@ from parity import assert_bf16_close, assert_dscale, bf16_u16, compare_mx
 pytestmark = pytest.mark.gpu
 
 INF = float("inf")
-PARAMS = [(1.702, 7.0), (1.0, 2.5), (2.0, 0.75), (0.8125, INF)]
+# 3.3 is not a bf16 value: a bf16 gate or up lies above it exactly when it
+# lies above 3.296875, the bf16 below it
+PARAMS = [(1.702, 7.0), (1.0, 2.5), (2.0, 0.75), (0.8125, INF), (1.0, 3.3)]
 SHAPES = [(32, 32), (96, 224), (100, 192), (257, 320)]
 
 
@@ -41,11 +43,28 @@ def _dscale_bound(dyb, xb, s, N, alpha, L):
 @pytest.mark.parametrize("alpha", [1.702, 1.0, 0.8125, 2.0])
 def test_sigmoid_table_of_a_slope_on_all_bf16(cuda_device, alpha):
     a = _f32(alpha)
-    got = mg.clamped_sigmoid_table(a, cuda_device).cpu().numpy()
+    got = mg.clamped_sigmoid_table(a, device=cuda_device).cpu().numpy()
     ref = oracle.clamped_sigmoid_table(a)
     bits = np.arange(65536, dtype=np.uint32)
     is_nan = ((bits & 0x7F80) == 0x7F80) & ((bits & 0x7F) != 0)
     same = got.view(np.uint32) == ref.view(np.uint32)
+    assert same[~is_nan].all(), np.nonzero(~same & ~is_nan)[0][:10]
+
+
+@pytest.mark.parametrize("alpha,L", [(1.702, 7.0), (2.0, 0.75), (0.8125, 0.015625)])
+def test_sigmoid_table_with_the_gate_clamp_on_all_bf16(cuda_device, alpha, L):
+    """The table a call with a finite limit looks up: sigma(RN(alpha * min(g,
+    L))), i.e. the oracle's unclamped entry of the gate, or of L (a bf16
+    value here) for every gate above L."""
+    a = _f32(alpha)
+    got = mg.clamped_sigmoid_table(a, L, device=cuda_device).cpu().numpy()
+    ref = oracle.clamped_sigmoid_table(a)
+    bits = np.arange(65536, dtype=np.uint32)
+    g = (bits << 16).view(np.float32)
+    lbits = int(np.array([L], np.float32).view(np.uint32)[0] >> 16)
+    want = np.where(g > L, ref[lbits], ref)
+    is_nan = np.isnan(g)
+    same = got.view(np.uint32) == want.view(np.uint32)
     assert same[~is_nan].all(), np.nonzero(~same & ~is_nan)[0][:10]
 
 
@@ -89,6 +108,11 @@ def test_special_values(cuda_device):
     s = s.clone()
     s[12] = 0.0
     s[13] = -0.5
+    # non-finite dY where the gate (row 0) or the up (rows 1, 2) is clamped:
+    # the clamped input's gradient is +0 all the same
+    dy = dy.float()
+    dy[0, 3], dy[0, 4], dy[1, 5], dy[2, 6] = float("nan"), float("inf"), float("nan"), -float("inf")
+    dy = dy.to(torch.bfloat16)
     xb, sn, dyb = bf16_bits(x), s.numpy(), bf16_bits(dy)
     xg, sg, dyg = x.to(cuda_device), s.to(cuda_device), dy.to(cuda_device)
     got = mg.scaled_clamped_swiglu_mxfp8_fwd(xg, sg, alpha=a, limit=l)

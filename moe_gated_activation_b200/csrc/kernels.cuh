@@ -108,8 +108,8 @@ template <int ACT, bool BWD>
 struct Cfg {
   static constexpr bool kSig = ACT != kSReLU;   // gated: sigmoid table, gate + up
   // the table first in shared memory, looked up by 16-bit addresses
-  // (sigma_pair_s): the SwiGLU forward, where it measured faster
-  static constexpr bool kSigFront = !BWD && ACT == kSwiGLU;
+  // (sigma_pair_s): the gated forwards, where it measured faster
+  static constexpr bool kSigFront = !BWD && (ACT == kSwiGLU || ACT == kClamped);
   static constexpr int kOps = BWD ? (kSig ? 3 : 2) : (kSig ? 2 : 1);
   static constexpr int kWarps = BWD ? (kSig ? 7 : 8) : 8;
   static constexpr int kSlots = (!BWD && !kSig) ? 3 : 2;
@@ -126,12 +126,11 @@ constexpr int kGapRo = 6144;
 __host__ __device__ constexpr int group_bytes(int E) { return 2 * ((E + 1 + 3) / 4) * 16; }
 
 // Shared memory of a CTA: 128 B of alignment slack, then the sigmoid table
-// (padded to 1 KiB) and the ring (Cfg::kSigFront: the SwiGLU forward), or the
-// ring and the table (the other gated kernels), or the ring and the group
-// offsets (SReLU); then the mbarriers.  A table in front has shared-memory
-// addresses that fit in 16 bits (see sigma_pair_s); the backward and the
-// ClampedSwiGLU forward measured slower with that order, and look their
-// table up through its pointer.
+// (padded to 1 KiB) and the ring (Cfg::kSigFront: the gated forwards), or the
+// ring and the table (the gated backwards), or the ring and the group offsets
+// (SReLU); then the mbarriers.  A table in front has shared-memory addresses
+// that fit in 16 bits (see sigma_pair_s); the backwards measured slower with
+// that order, and look their table up through its pointer.
 constexpr int kSigRegion = (kSigBytes + 1023) / 1024 * 1024;
 template <int ACT, bool BWD>
 __host__ __device__ constexpr int smem_bytes(bool grouped, int E) {
@@ -604,8 +603,8 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
       if (ACT == kClamped) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
         float2 sg01, sg23;
-        sigma_pair(m.sig, G.x, sg01.x, sg01.y);
-        sigma_pair(m.sig, G.y, sg23.x, sg23.y);
+        sigma_pair_s(m.sig_key, G.x, sg01.x, sg01.y);
+        sigma_pair_s(m.sig_key, G.y, sg23.x, sg23.y);
         const float2 si01 = mul2(clamp_gate_pair(bf16x2_to_f2(G.x), p.clamp_L), sg01);
         const float2 si23 = mul2(clamp_gate_pair(bf16x2_to_f2(G.y), p.clamp_L), sg23);
         h01 = mul2(si01, clamped_up_plus_one(bf16x2_to_f2(U.x), p.clamp_L));

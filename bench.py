@@ -612,8 +612,9 @@ def run_fc2(args):
     inp = make_inputs(wl, device=dev, with_dy=False)
     x, s, m = inp["x"], inp["s"], inp["m_splits"]
     M, N, H, E = wl.M, wl.N, args.fc2_width, int(m.numel())
-    # uniform random scale bytes: the same law in any layout, so they serve
-    # as the tiled weight scales the kernel reads without a conversion
+    # uniform random code and scale bytes: the same law in any layout, so
+    # they serve as the tiled weight codes and scales the kernel reads
+    # without a conversion
     wc, ws = fc2_weights(E, H, N, 11, device=dev)
     ro, _, st = mg.splits_to_offsets(m.to(dev), M)
     out = torch.empty(M, H, dtype=torch.bfloat16, device=dev)

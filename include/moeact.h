@@ -397,8 +397,14 @@ moeact_status moeact_device_error(uint32_t* flags);
  *     an expert's end in its last 128-row block are neither read as its own
  *     nor written); offsets that are not those of valid splits set *status = 3
  *     and write nothing.
- *   w_codes: E4M3 [E, H, N], row-major: expert e's weight, row h = output
- *     column h, its N k-values contiguous; 16-byte aligned.
+ *   w_codes: E4M3 codes of the weights, expert e's [H, N] matrix (row h =
+ *     output column h, N k-values) in the tensor cores' K-major operand
+ *     layout: tiles of 128 rows x 128 k (16 KiB), row blocks in order and,
+ *     within a row block, k blocks in order; in a tile, row r's 128 bytes at
+ *     offset 128 r, its 16-byte chunk c (k values 16c .. 16c + 15) at chunk
+ *     position c ^ (r mod 8) (the 128-byte swizzle); experts one after
+ *     another: E * H * N bytes, 16-byte aligned.  (A weight is tiled once;
+ *     each tile then arrives in one contiguous bulk copy.)
  *   w_scales: E8M0 scales of the weight (1 x 32 blocks along k), per expert
  *     the [H, N/32] matrix in the GEMM-ready tiled layout of
  *     MOEACT_SCALES_GEMM (tiles of 128 rows x 4 scale columns, 512 bytes,

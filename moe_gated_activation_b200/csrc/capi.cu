@@ -317,22 +317,6 @@ moeact_status make_map_ilv(CUtensorMap* map, const void* base, int64_t N, int64_
   return MOEACT_OK;
 }
 
-// Tensor map of an E4M3 weight [rows, K] (K contiguous bytes per row), read
-// in boxes of 128 bytes of K x 128 rows with 128-byte swizzling: the layout
-// the tensor cores read K-major operands in.
-moeact_status make_map_w(CUtensorMap* map, const void* base, int64_t K, int64_t rows) {
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)K};
-  const cuuint32_t box[2] = {128, 128};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
-                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(MOEACT_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-  return MOEACT_OK;
-}
-
 // The backward's map of x: SReLU [rows][N]; gated [rows][2][N] or, with an
 // interleave G, [rows][N/G][2][G].
 moeact_status make_x_map(CUtensorMap* map, int act, const void* x, int64_t N, int ilv,
@@ -893,9 +877,8 @@ moeact_status grouped_scaled_swiglu_mxfp8_fc2(const void* x, int64_t ldx, const 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int dev;
   if ((st = ensure_ready(cs, &dev))) return st;
-  CUtensorMap tx, tw;
+  CUtensorMap tx;
   if ((st = make_map(&tx, x, 2 * N, M, ldx))) return st;
-  if ((st = make_map_w(&tw, w_codes, N, H * num_groups))) return st;
   Fc2Params p{};
   p.s = s;
   p.M = M;
@@ -904,6 +887,7 @@ moeact_status grouped_scaled_swiglu_mxfp8_fc2(const void* x, int64_t ldx, const 
   p.row_offs = row_offs;
   p.E = num_groups;
   p.status = status;
+  p.w_codes = static_cast<const uint8_t*>(w_codes);
   p.w_scales = static_cast<const uint8_t*>(w_scales);
   p.out = static_cast<uint16_t*>(out);
   p.ldo = ldo;
@@ -911,7 +895,7 @@ moeact_status grouped_scaled_swiglu_mxfp8_fc2(const void* x, int64_t ldx, const 
   p.noop = noop_flag;
   p.err = g_err_ptr[dev];
   const int64_t grid = ceil_div(M, 128) + num_groups;
-  const cudaError_t e = fc2_launch(p, tx, tw, staged_rounding, (unsigned)grid, cs);
+  const cudaError_t e = fc2_launch(p, tx, staged_rounding, (unsigned)grid, cs);
   if (e != cudaSuccess) return cuda_fail(e, "fused FC2 launch");
   return MOEACT_OK;
 }

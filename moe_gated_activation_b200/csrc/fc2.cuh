@@ -27,7 +27,8 @@ struct Fc2Params {
   const int64_t* row_offs;    // [E + 1]
   int E;
   int32_t* status;
-  const uint8_t* w_scales;    // E8M0 [E, H, N/32], row-major
+  const uint8_t* w_codes;     // E4M3, per expert H/128 x N/128 operand tiles of 16 KiB
+  const uint8_t* w_scales;    // E8M0, per expert the [H, N/32] matrix in 128 x 4 tiles
   uint16_t* out;              // bf16 [M, ldo]
   int64_t ldo;
   const float* sig_src;       // the sigmoid table (device memory, shared-memory layout)
@@ -44,9 +45,8 @@ int fc2_smem_bytes(int N);
 cudaError_t fc2_prepare();
 // Launches the fused kernel: one CTA per possible 128-row block of an expert
 // (`grid` = ceil(M/128) + E covers every split); tm_x is the bf16 [M, 2N]
-// input in 128 x 16 boxes, tm_w the E4M3 weight [E*H, N] in 128 x 128
-// boxes with 128-byte swizzling.
-cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
-                       int staged, unsigned grid, cudaStream_t stream);
+// input in 128 x 16 boxes.
+cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, int staged, unsigned grid,
+                       cudaStream_t stream);
 
 }  // namespace moeact

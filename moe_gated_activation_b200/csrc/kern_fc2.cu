@@ -19,12 +19,15 @@
 //              16-row half-tile slot per warp), compute y and its rowwise
 //              MXFP8, write the codes into shared memory in the tensor
 //              cores' K-major 128-byte-swizzled layout and the scales into
-//              tensor memory; then, per 128-column output tile, write the
-//              weight's scales into tensor memory and drain the accumulator
-//              (tcgen05.ld) into bf16 rows of `out`;
-//   warp 8     TMA producer of the weight tiles (128 rows x 128 bytes of k,
-//              swizzled), a 7-stage ring that reuses the prologue's staging
-//              and sigmoid-table memory;
+//              tensor memory; then, per 128-column output tile, drain the
+//              accumulator (tcgen05.ld) into bf16 rows of `out`, warps 0-3
+//              writing the weight scales of the tile two ahead into the
+//              drained buffer's scale columns (tcgen05.st: a tcgen05.cp would
+//              cost the tensor pipe time, measured 6% of the kernel);
+//   warp 8     producer of the weight tiles (128 rows x 128 bytes of k,
+//              stored pre-swizzled in the tensor cores' operand layout, so
+//              each is one contiguous 16 KiB bulk copy), a 5-stage ring that
+//              reuses the prologue's staging and sigmoid-table memory;
 //   warp 9     allocates tensor memory and issues the MMAs (one thread):
 //              tcgen05.mma.kind::mxf8f6f4.block_scale, M = N = 128, K = 32,
 //              two accumulators in tensor memory so that one tile's drain
@@ -123,12 +126,25 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t* v) {
 __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-// Copies a 32-row x 16-byte matrix from shared memory into columns
-// [taddr, taddr + 4) of lanes 0-31 of every 32-lane quarter (each row to its
-// lane, bytes 4c .. 4c + 3 to column c).
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
+// Non-suspending test of a phase, and a spin on it bounded by the global
+// timer: the single threads that feed the tensor cores (weight producer, MMA
+// issuer) spin rather than suspend, as their wake-up latency is on the
+// critical path (measured 2% faster than suspending waits).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; "
+               "selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -145,13 +161,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Shared-memory descriptor of a source of tcgen05.cp: 16-byte rows, no
-// swizzling, 8-row groups 128 bytes apart (rows contiguous).
-__device__ __forceinline__ uint64_t cp_desc_rows16(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
-         ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
 // Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 x E4M3,
@@ -177,7 +186,7 @@ struct Fc2Smem {
   uint64_t* b_full;       // [7]
   uint64_t* b_empty;      // [7]
   uint64_t* sf_full;      // [3] a tile's weight scales have landed in shared memory
-  uint64_t* sf_empty;     // [3] ... and have been copied to tensor memory and used
+  uint64_t* sf_empty;     // [3] ... and have been copied to tensor memory (count 4)
   uint64_t* d_full;       // [2] an accumulator holds a finished tile
   uint64_t* d_empty;      // [2] count 8: an accumulator has been drained
   uint64_t* mma_done;
@@ -263,6 +272,29 @@ __device__ __forceinline__ uint32_t fc2_half(const Fc2Smem& m, const unsigned ch
   return b0 | (b1 << 8);
 }
 
+// Warps 0-3 (warp q: lanes 32 q .. 32 q + 31): output tile t's weight scales
+// from its shared-memory slot (N/128 groups of 512 bytes, row 32 c + l's four
+// k-block scales at byte 16 l + 4 c) into the scale columns of accumulator
+// buffer t & 1: lane l, column 4 g + c of every quarter holds row 32 c + l's
+// word (the layout the MMA reads), written with tcgen05.st so that the
+// tensor pipe spends no time on it.  The slot is released afterwards.
+// Returns false on a timeout.
+__device__ __forceinline__ bool fc2_put_w_scales(const Fc2Params& p, const Fc2Smem& m, int t,
+                                                 int q, int lane, uint32_t tbase) {
+  const int KA = p.N >> 7;
+  if (!warp_wait(m.sf_full + t % kSfSlots, (uint32_t)(t / kSfSlots) & 1u)) return false;
+  const unsigned char* src = m.sf + (t % kSfSlots) * kSfSlotBytes + 16 * lane;
+  const uint32_t dst = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(kSfbCol + 32 * (t & 1));
+  for (int g = 0; g < KA; ++g) {
+    const uint4 w = *reinterpret_cast<const uint4*>(src + 512 * g);
+    tc_st4(dst + 4 * g, w.x, w.y, w.z, w.w);
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(m.sf_empty + t % kSfSlots);
+  tc_wait_st();
+  return true;
+}
+
 template <bool STAGED>
 __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2Smem& m, int e,
                          int64_t row0, int mrows, uint32_t tbase) {
@@ -319,6 +351,14 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
       mbar_wait(m.sig_bar, 0u);
     }
   }
+  const int T = p.H >> 7;
+  // the weight scales of the first two output tiles
+  if (ok && half_sel == 0)
+    for (int t = 0; t < 2 && t < T; ++t)
+      if (!fc2_put_w_scales(p, m, t, q, lane, tbase)) {
+        set_abort(p, m);
+        break;
+      }
   tc_wait_st();
   fence_proxy_async_smem();   // the codes written above are read by the tensor cores
   tc_fence_before();
@@ -326,7 +366,6 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
   if (lane == 0) mbar_arrive(m.pro_done);
 
   // ---- output tiles: drain each accumulator into bf16 rows
-  const int T = p.H >> 7;
   for (int n = 0; n < T; ++n) {
     if (warp_aborted(m)) break;
     const int b = n & 1;
@@ -337,6 +376,12 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
     tc_ld32(t, v);
     tc_ld32(t + 32, v + 32);
     tc_wait_ld();
+    // buffer b's scale columns are free (tile n's MMAs are done): tile n + 2's
+    // go there before the buffer is released
+    if (half_sel == 0 && n + 2 < T && !fc2_put_w_scales(p, m, n + 2, q, lane, tbase)) {
+      set_abort(p, m);
+      break;
+    }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(m.d_empty + b);
@@ -376,13 +421,14 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
   }
 }
 
-// Warp 8, one thread: the weight tiles of every output tile, in k order,
-// and each output tile's weight scales (N/128 tiles of 512 bytes, contiguous
-// in the tiled layout) kSfSlots - 1 output tiles ahead: the scales of tile
-// n + 3 go out after the last weight tile of tile n, when the slot they reuse
-// (tile n - 1's) is already free, and have two tiles of MMAs to land.
-__device__ void fc2_producer(const CUtensorMap* tm_w, const Fc2Params& p, const Fc2Smem& m,
-                             int e) {
+// Warp 8, one thread: the weight tiles of every output tile, in k order
+// (each a contiguous 16 KiB of the tiled weight: one bulk copy, which
+// streams into an SM faster than a 2-D tensor copy of the same tile), and
+// each output tile's weight scales (N/128 tiles of 512 bytes, contiguous in
+// the tiled layout) kSfSlots - 1 output tiles ahead: the scales of tile n + 3
+// go out after the last weight tile of tile n, when the slot they reuse (tile
+// n - 1's) is already free, and have two tiles of MMAs to land.
+__device__ void fc2_producer(const Fc2Params& p, const Fc2Smem& m, int e) {
   const int KA = p.N >> 7, T = p.H >> 7;
   int issued = 0, sf_issued = 0;
   auto issue_sf = [&](int n) {   // false on a timeout
@@ -402,12 +448,14 @@ __device__ void fc2_producer(const CUtensorMap* tm_w, const Fc2Params& p, const 
   if (!mbar_wait(m.pro_done, 0u)) set_abort(p, m);
   for (int g = 0; g < T * KA && !aborted(m); ++g) {
     const int n = g / KA, ks = g - n * KA, slot = g % kStages;
-    if (g >= kStages && !mbar_wait(m.b_empty + slot, (uint32_t)(g / kStages - 1) & 1u)) {
+    if (g >= kStages && !mbar_spin(m.b_empty + slot, (uint32_t)(g / kStages - 1) & 1u)) {
       set_abort(p, m);
       break;
     }
     mbar_expect_tx(m.b_full + slot, kStageBytes);
-    tma_load_2d(m.R + slot * kStageBytes, tm_w, 128 * ks, e * p.H + 128 * n, m.b_full + slot);
+    bulk_load(m.R + slot * kStageBytes,
+              p.w_codes + (((int64_t)e * T + n) * KA + ks) * (int64_t)kStageBytes, kStageBytes,
+              m.b_full + slot);
     issued = g + 1;
     if (ks == KA - 1 && n + kSfSlots - 1 < T && !issue_sf(n + kSfSlots - 1)) {
       set_abort(p, m);
@@ -427,25 +475,19 @@ __device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
   bool ok = mbar_wait(m.pro_done, 0u) && !aborted(m);
   if (!ok) set_abort(p, m);
   tc_fence_after();
-  const uint32_t a_base = smem_addr(m.A), r_base = smem_addr(m.R), sf_base = smem_addr(m.sf);
+  const uint32_t a_base = smem_addr(m.A), r_base = smem_addr(m.R);
   for (int n = 0; ok && n < T; ++n) {
     const int b = n & 1;
-    // the accumulator and the weight-scale columns of buffer b are free once
-    // tile n - 2 has been drained (its MMAs, and so their reads, are done)
-    if (!mbar_wait(m.sf_full + n % kSfSlots, (uint32_t)(n / kSfSlots) & 1u) ||
-        (n >= 2 && !mbar_wait(m.d_empty + b, (uint32_t)((n >> 1) - 1) & 1u))) {
+    // accumulator b is free, and holds tile n's weight scales, once tile
+    // n - 2 has been drained (tiles 0 and 1: once the prologue is done)
+    if (n >= 2 && !mbar_spin(m.d_empty + b, (uint32_t)((n >> 1) - 1) & 1u)) {
       ok = false;
       break;
     }
     tc_fence_after();
-    // the tile's weight scales: smem -> tensor memory, ordered before the
-    // MMAs below (both issued by this thread)
-    for (int g = 0; g < KA; ++g)
-      tc_cp_32x128b_warpx4(tbase + kSfbCol + 32 * b + 4 * g,
-                           cp_desc_rows16(sf_base + (n % kSfSlots) * kSfSlotBytes + 512 * g));
     for (int ks = 0; ks < KA; ++ks) {
       const int g = n * KA + ks, slot = g % kStages;
-      if (aborted(m) || !mbar_wait(m.b_full + slot, (uint32_t)(g / kStages) & 1u)) {
+      if (aborted(m) || !mbar_spin(m.b_full + slot, (uint32_t)(g / kStages) & 1u)) {
         ok = false;
         break;
       }
@@ -461,7 +503,6 @@ __device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
     }
     if (!ok) break;
     tc_commit(m.d_full + b);
-    tc_commit(m.sf_empty + n % kSfSlots);   // the smem scales of this tile are no longer needed
   }
   if (!ok) set_abort(p, m);
   // every MMA issued has completed before tensor memory is freed (bounded)
@@ -471,8 +512,7 @@ __device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
 
 template <bool STAGED>
 __global__ void __launch_bounds__(kFc2Threads, 1)
-    fc2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-               const Fc2Params p) {
+    fc2_kernel(const __grid_constant__ CUtensorMap tm_x, const Fc2Params p) {
   if (p.noop != nullptr && *p.noop != 0) return;
   extern __shared__ __align__(1024) unsigned char fc2_smem[];
   unsigned char* base = align1024(fc2_smem);
@@ -558,7 +598,7 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
     }
     for (int i = 0; i < kSfSlots; ++i) {
       mbar_init(m.sf_full + i, 1);
-      mbar_init(m.sf_empty + i, 1);
+      mbar_init(m.sf_empty + i, 4);   // warps 0-3 have copied the slot to tensor memory
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(m.d_full + i, 1);
@@ -580,7 +620,7 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
   if (warp < 8) {
     fc2_math<STAGED>(&tm_x, p, m, e, row0, mrows, tbase);
   } else if (warp == 8) {
-    if ((tid & 31) == 0) fc2_producer(&tm_w, p, m, e);
+    if ((tid & 31) == 0) fc2_producer(p, m, e);
     __syncwarp();
   } else {
     if ((tid & 31) == 0) fc2_mma(p, m, tbase);
@@ -609,13 +649,13 @@ cudaError_t fc2_prepare() {
   return e;
 }
 
-cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, const CUtensorMap& tm_w,
-                       int staged, unsigned grid, cudaStream_t stream) {
+cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, int staged, unsigned grid,
+                       cudaStream_t stream) {
   const int bytes = fc2_smem_bytes(p.N);
   if (staged)
-    fc2_kernel<true><<<grid, kFc2Threads, bytes, stream>>>(tm_x, tm_w, p);
+    fc2_kernel<true><<<grid, kFc2Threads, bytes, stream>>>(tm_x, p);
   else
-    fc2_kernel<false><<<grid, kFc2Threads, bytes, stream>>>(tm_x, tm_w, p);
+    fc2_kernel<false><<<grid, kFc2Threads, bytes, stream>>>(tm_x, p);
   return cudaGetLastError();
 }
 

@@ -469,10 +469,13 @@ def grouped_scaled_swiglu_mxfp8_fc2(x, s, row_offs, w_codes, w_scales, *, status
     activation feeds the grouped linear after it).
 
     x bf16 [M, 2N] ([gate | up]), s fp32 [M], row_offs int64 [E + 1] (from
-    splits_to_offsets); w_codes E4M3 [E, H, N] (uint8 or float8_e4m3fn, row h
-    of expert e = output column h), w_scales uint8 E8M0 [E, H, N/32] whose
-    bytes hold each expert's [H, N/32] scale matrix in the GEMM-ready tiled
-    layout (128 x 4 tiles of 512 bytes, as gemm_scales=True writes).
+    splits_to_offsets); w_codes E4M3 [E, H, N] (uint8 or float8_e4m3fn) whose
+    bytes hold each expert's [H, N] code matrix (row h = output column h) in
+    the tensor cores' tiled operand layout (128 x 128 tiles of 16 KiB, rows
+    128-byte swizzled; see include/moeact.h), w_scales uint8 E8M0
+    [E, H, N/32] whose bytes hold each expert's [H, N/32] scale matrix in the
+    GEMM-ready tiled layout (128 x 4 tiles of 512 bytes, as gemm_scales=True
+    writes).
     Returns (out bf16 [M, H], status); `out=` takes a caller-owned bf16
     [M, >= H] tensor with unit column stride."""
     N = x.shape[1] // 2

@@ -176,8 +176,10 @@ def fc2_weights(E, H, N, seed, device="cpu", scale_lo=118, scale_hi=124):
     """A seeded MXFP8 FC2 weight for the fused activation -> FC2 path: E4M3
     codes uint8 [E, H, N] drawn uniformly over the finite codes (0x7F and
     0xFF, the NaNs, excluded) and E8M0 scales uint8 [E, H, N/32] uniform in
-    [scale_lo, scale_hi].  (The FC2 width of the Qwen3-MoE configuration is
-    its hidden size, 2048.)"""
+    [scale_lo, scale_hi].  Both are i.i.d. uniform, so the same bytes serve
+    as the tiled operand and scale layouts the fused kernel reads (a
+    permutation of i.i.d. bytes has their law).  (The FC2 width of the
+    Qwen3-MoE configuration is its hidden size, 2048.)"""
     g = _gen(device, seed)
     c = torch.randint(0, 254, (E, H, N), generator=g, device=device, dtype=torch.int32)
     c = c + (c >= 0x7F).to(torch.int32)          # 0..126 -> 0x00..0x7E, 127..253 -> 0x80..0xFE

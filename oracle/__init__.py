@@ -302,6 +302,25 @@ def scales_gemm_layout(S: np.ndarray) -> np.ndarray:
     return out
 
 
+def codes_gemm_layout(W: np.ndarray) -> np.ndarray:
+    """E4M3 codes [R, K] (R, K multiples of 128) -> the tensor cores' K-major
+    operand tiles (flat uint8, R * K bytes): 128-row blocks in order, within a
+    row block 128-byte k blocks in order, each a 16 KiB tile holding row r's
+    128 bytes at offset 128 r with its 16-byte chunk c at chunk position
+    c ^ (r mod 8) (the 128-byte swizzle).  A permutation of the bytes (any
+    dtype is permuted alike, so an index matrix gives the permutation)."""
+    W = np.ascontiguousarray(W)
+    R, K = W.shape
+    if R % 128 or K % 128:
+        raise ValueError("codes_gemm_layout needs rows and columns in multiples of 128")
+    src = W.reshape(R // 128, 128, K // 128, 8, 16)      # [row block, r, k block, chunk, byte]
+    tiles = np.empty((R // 128, K // 128, 128, 8, 16), W.dtype)
+    for r in range(128):
+        for c in range(8):
+            tiles[:, :, r, c ^ (r % 8), :] = src[:, r, :, c, :]
+    return tiles.reshape(-1)
+
+
 def col_scales_gemm_layout(cs: np.ndarray, W: int, row_offs, colblk_offs) -> np.ndarray:
     """Row-major colwise scales [S, W] of a grouped tensor -> per expert, the
     transposed [W, m_e/32] matrix in the GEMM layout, experts in order."""

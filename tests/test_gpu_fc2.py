@@ -71,13 +71,28 @@ def _tiled(ws):
                                       for w in ws]))
 
 
+_PERM = {}
+
+
+def _tiled_codes(wc):
+    """Row-major weight codes [E, H, N] (torch, any device) -> the kernel's
+    tiled operand layout per expert: the oracle's pinned layout function,
+    applied as the permutation it gives an index matrix."""
+    E, H, N = wc.shape
+    if (H, N) not in _PERM:
+        _PERM[(H, N)] = torch.from_numpy(
+            oracle.codes_gemm_layout(np.arange(H * N, dtype=np.int64).reshape(H, N)))
+    perm = _PERM[(H, N)].to(wc.device)
+    return wc.reshape(E, H * N)[:, perm].reshape(E, H, N).contiguous()
+
+
 def _run(case, N, splits, wc, ws, dev, staged=False):
     m = torch.tensor(splits, dtype=torch.int64)
     M = int(m.sum())
     ro, cb, st = mg.splits_to_offsets(m.to(dev), M)
     x, s = case["x"].to(dev), case["s"].to(dev)
-    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(x, s, ro, wc.to(dev), _tiled(ws).to(dev),
-                                                  staged_rounding=staged)
+    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(x, s, ro, _tiled_codes(wc).to(dev),
+                                                  _tiled(ws).to(dev), staged_rounding=staged)
     torch.cuda.synchronize()
     assert int(st.item()) == 0 and int(st2.item()) == 0
     _, oro, _ = oracle.splits_to_offsets(m.numpy(), M)
@@ -137,7 +152,7 @@ def test_fc2_writes_nothing_for_bad_offsets_or_a_set_noop_flag(cuda_device):
     N, H, M = 128, 128, 256
     case = random_case(M, N, 41)
     wc, ws = fc2_weights(2, H, N, 8)
-    ws = _tiled(ws)
+    wc, ws = _tiled_codes(wc), _tiled(ws)
     dev = cuda_device
     x, s = case["x"].to(dev), case["s"].to(dev)
     bad = torch.tensor([0, 200, 100], dtype=torch.int64, device=dev)   # ends past M
@@ -170,7 +185,7 @@ def test_fc2_at_the_qwen3_moe_workload_sampled_rows(cuda_device):
     E = int(m.numel())
     wc, ws = fc2_weights(E, H, N, 11, device=dev)
     ro, cb, st = mg.splits_to_offsets(m.to(dev), M)
-    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(inp["x"], inp["s"], ro, wc,
+    out, st2 = mg.grouped_scaled_swiglu_mxfp8_fc2(inp["x"], inp["s"], ro, _tiled_codes(wc),
                                                   _tiled(ws.cpu()).to(dev))
     torch.cuda.synchronize()
     assert int(st.item()) == 0 and int(st2.item()) == 0

@@ -183,10 +183,10 @@ struct Fc2Smem {
   uint64_t* xbar;         // [8]
   uint64_t* sig_bar;
   uint64_t* pro_done;     // count 8: the block's A codes and scales are complete
-  uint64_t* b_full;       // [7]
-  uint64_t* b_empty;      // [7]
-  uint64_t* sf_full;      // [3] a tile's weight scales have landed in shared memory
-  uint64_t* sf_empty;     // [3] ... and have been copied to tensor memory (count 4)
+  uint64_t* b_full;       // [kStages] a weight stage has landed
+  uint64_t* b_empty;      // [kStages] ... and its MMAs are done
+  uint64_t* sf_full;      // [kSfSlots] a tile's weight scales have landed in shared memory
+  uint64_t* sf_empty;     // [kSfSlots] ... and have been copied to tensor memory (count 4)
   uint64_t* d_full;       // [2] an accumulator holds a finished tile
   uint64_t* d_empty;      // [2] count 8: an accumulator has been drained
   uint64_t* mma_done;

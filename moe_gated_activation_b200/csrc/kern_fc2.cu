@@ -421,93 +421,130 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
   }
 }
 
-// Warp 8, one thread: the weight tiles of every output tile, in k order
-// (each a contiguous 16 KiB of the tiled weight: one bulk copy, which
-// streams into an SM faster than a 2-D tensor copy of the same tile), and
-// each output tile's weight scales (N/128 tiles of 512 bytes, contiguous in
-// the tiled layout) kSfSlots - 1 output tiles ahead: the scales of tile n + 3
-// go out after the last weight tile of tile n, when the slot they reuse (tile
-// n - 1's) is already free, and have two tiles of MMAs to land.
+// One lane of a converged warp (elect.sync), the same lane every call.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile("{ .reg .pred p; elect.sync _|p, 0xffffffff; selp.u32 %0, 1, 0, p; }" : "=r"(r));
+  return r != 0;
+}
+
+// Warp 8, converged, one elected lane issuing (as the MMA warp, for the same
+// reason): the weight tiles of every output tile, in k order (each a
+// contiguous 16 KiB of the tiled weight: one bulk copy, which streams into an
+// SM faster than a 2-D tensor copy of the same tile), and each output tile's
+// weight scales (N/128 tiles of 512 bytes, contiguous in the tiled layout)
+// kSfSlots - 1 output tiles ahead: the scales of tile n + 3 go out after the
+// last weight tile of tile n, when the slot they reuse (tile n - 1's) is
+// already free, and have two tiles of MMAs to land.
 __device__ void fc2_producer(const Fc2Params& p, const Fc2Smem& m, int e) {
   const int KA = p.N >> 7, T = p.H >> 7;
+  const bool leader = elect_one();
   int issued = 0, sf_issued = 0;
   auto issue_sf = [&](int n) {   // false on a timeout
     const int ss = n % kSfSlots;
     if (n >= kSfSlots &&
-        !mbar_wait(m.sf_empty + ss, (uint32_t)(n / kSfSlots - 1) & 1u))
+        !__all_sync(kFull, mbar_spin(m.sf_empty + ss, (uint32_t)(n / kSfSlots - 1) & 1u)))
       return false;
-    mbar_expect_tx(m.sf_full + ss, 512 * KA);
-    bulk_load(m.sf + ss * kSfSlotBytes, p.w_scales + ((int64_t)e * T + n) * KA * 512, 512 * KA,
-              m.sf_full + ss);
+    if (leader) {
+      mbar_expect_tx(m.sf_full + ss, 512 * KA);
+      bulk_load(m.sf + ss * kSfSlotBytes, p.w_scales + ((int64_t)e * T + n) * KA * 512,
+                512 * KA, m.sf_full + ss);
+    }
+    __syncwarp();
     sf_issued = n + 1;
     return true;
   };
   // the first scales do not wait for the prologue (their slots are not
   // shared with it); the weight tiles reuse the prologue's staging memory
   for (int n = 0; n < T && n < kSfSlots - 1; ++n) issue_sf(n);
-  if (!mbar_wait(m.pro_done, 0u)) set_abort(p, m);
-  for (int g = 0; g < T * KA && !aborted(m); ++g) {
+  if (!__all_sync(kFull, mbar_wait(m.pro_done, 0u)) && leader) set_abort(p, m);
+  const uint8_t* wsrc = p.w_codes + (int64_t)e * T * KA * kStageBytes;
+  for (int g = 0; g < T * KA && !warp_aborted(m); ++g) {
     const int n = g / KA, ks = g - n * KA, slot = g % kStages;
-    if (g >= kStages && !mbar_spin(m.b_empty + slot, (uint32_t)(g / kStages - 1) & 1u)) {
-      set_abort(p, m);
+    if (g >= kStages &&
+        !__all_sync(kFull, mbar_spin(m.b_empty + slot, (uint32_t)(g / kStages - 1) & 1u))) {
+      if (leader) set_abort(p, m);
       break;
     }
-    mbar_expect_tx(m.b_full + slot, kStageBytes);
-    bulk_load(m.R + slot * kStageBytes,
-              p.w_codes + (((int64_t)e * T + n) * KA + ks) * (int64_t)kStageBytes, kStageBytes,
-              m.b_full + slot);
+    if (leader) {
+      mbar_expect_tx(m.b_full + slot, kStageBytes);
+      bulk_load(m.R + slot * kStageBytes, wsrc + (int64_t)g * kStageBytes, kStageBytes,
+                m.b_full + slot);
+    }
+    __syncwarp();
     issued = g + 1;
     if (ks == KA - 1 && n + kSfSlots - 1 < T && !issue_sf(n + kSfSlots - 1)) {
-      set_abort(p, m);
+      if (leader) set_abort(p, m);
       break;
     }
   }
   // every copy issued has landed before the CTA can exit (bounded)
-  for (int g = max(0, issued - kStages); g < issued; ++g)
-    mbar_wait(m.b_full + g % kStages, (uint32_t)(g / kStages) & 1u);
-  for (int n = max(0, sf_issued - kSfSlots); n < sf_issued; ++n)
-    mbar_wait(m.sf_full + n % kSfSlots, (uint32_t)(n / kSfSlots) & 1u);
+  if (leader) {
+    for (int g = max(0, issued - kStages); g < issued; ++g)
+      mbar_wait(m.b_full + g % kStages, (uint32_t)(g / kStages) & 1u);
+    for (int n = max(0, sf_issued - kSfSlots); n < sf_issued; ++n)
+      mbar_wait(m.sf_full + n % kSfSlots, (uint32_t)(n / kSfSlots) & 1u);
+  }
+  __syncwarp();
 }
 
-// Warp 9, one thread: the MMAs of every output tile.
+// Warp 9, the whole warp converged, one elected lane issuing: the MMAs of
+// every output tile.  The loop runs on all 32 lanes so that its operands
+// (descriptors, tensor-memory addresses) are warp-uniform values the
+// tcgen05 instructions take directly; issued from a single-thread branch
+// they were rebuilt before every MMA, and the issue, not the tensor pipe,
+// set the rate.  A K step of 32 bytes advances a descriptor's start-address
+// field by 2 (16-byte units; shared-memory addresses stay below 2^18, so
+// the field never carries).
 __device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
   const int KA = p.N >> 7, T = p.H >> 7;
-  bool ok = mbar_wait(m.pro_done, 0u) && !aborted(m);
-  if (!ok) set_abort(p, m);
+  const bool leader = elect_one();
+  bool ok = __all_sync(kFull, mbar_wait(m.pro_done, 0u)) && !warp_aborted(m);
+  if (!ok && leader) set_abort(p, m);
   tc_fence_after();
-  const uint32_t a_base = smem_addr(m.A), r_base = smem_addr(m.R);
+  const uint64_t a_desc0 = umma_desc_sw128(smem_addr(m.A));
+  const uint64_t b_desc0 = umma_desc_sw128(smem_addr(m.R));
   for (int n = 0; ok && n < T; ++n) {
     const int b = n & 1;
     // accumulator b is free, and holds tile n's weight scales, once tile
     // n - 2 has been drained (tiles 0 and 1: once the prologue is done)
-    if (n >= 2 && !mbar_spin(m.d_empty + b, (uint32_t)((n >> 1) - 1) & 1u)) {
+    if (n >= 2 && !__all_sync(kFull, mbar_spin(m.d_empty + b, (uint32_t)((n >> 1) - 1) & 1u))) {
       ok = false;
       break;
     }
     tc_fence_after();
+    const uint32_t d = tbase + 128 * b;
     for (int ks = 0; ks < KA; ++ks) {
       const int g = n * KA + ks, slot = g % kStages;
-      if (aborted(m) || !mbar_spin(m.b_full + slot, (uint32_t)(g / kStages) & 1u)) {
+      if (warp_aborted(m) ||
+          !__all_sync(kFull, mbar_spin(m.b_full + slot, (uint32_t)(g / kStages) & 1u))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const uint64_t ad = a_desc0 + (uint64_t)((ks * kAtom) >> 4);
+      const uint64_t bd = b_desc0 + (uint64_t)((slot * kStageBytes) >> 4);
+      const uint32_t sfa = tbase + kSfaCol + 4 * ks, sfb = tbase + kSfbCol + 32 * b + 4 * ks;
+      if (leader) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint64_t ad = umma_desc_sw128(a_base + ks * kAtom + 32 * j);
-        const uint64_t bd = umma_desc_sw128(r_base + slot * kStageBytes + 32 * j);
-        tc_mma_mx(tbase + 128 * b, ad, bd, mx_idesc((uint32_t)j), tbase + kSfaCol + 4 * ks,
-                  tbase + kSfbCol + 32 * b + 4 * ks, (ks | j) != 0 ? 1u : 0u);
+        for (int j = 0; j < 4; ++j)
+          tc_mma_mx(d, ad + 2 * j, bd + 2 * j, mx_idesc((uint32_t)j), sfa, sfb,
+                    (ks | j) != 0 ? 1u : 0u);
+        tc_commit(m.b_empty + slot);   // the stage is free once these MMAs are done
       }
-      tc_commit(m.b_empty + slot);   // the stage is free once these MMAs are done
+      __syncwarp();
     }
     if (!ok) break;
-    tc_commit(m.d_full + b);
+    if (leader) tc_commit(m.d_full + b);
+    __syncwarp();
   }
-  if (!ok) set_abort(p, m);
+  if (!ok && leader) set_abort(p, m);
   // every MMA issued has completed before tensor memory is freed (bounded)
-  tc_commit(m.mma_done);
-  mbar_wait(m.mma_done, 0u);
+  if (leader) {
+    tc_commit(m.mma_done);
+    mbar_wait(m.mma_done, 0u);
+  }
+  __syncwarp();
 }
 
 template <bool STAGED>
@@ -620,11 +657,9 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
   if (warp < 8) {
     fc2_math<STAGED>(&tm_x, p, m, e, row0, mrows, tbase);
   } else if (warp == 8) {
-    if ((tid & 31) == 0) fc2_producer(p, m, e);
-    __syncwarp();
+    fc2_producer(p, m, e);
   } else {
-    if ((tid & 31) == 0) fc2_mma(p, m, tbase);
-    __syncwarp();
+    fc2_mma(p, m, tbase);
   }
 
   tc_fence_before();

@@ -336,9 +336,9 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
     } else {
       // lane l: the four block scales of row 32 q + l for atom a.  The MMA
       // reads the scale of its M-operand row 32 q + l from lane 32 q + l,
-      // column q of the group (the layout the weight scales are copied in by
-      // fc2_mma, of which each quarter needs only its own column); the word
-      // goes to all four.
+      // column q of the group (the layout fc2_put_w_scales writes the
+      // weight's scales in, of which each quarter needs only its own
+      // column); the word goes to all four.
       const uint32_t v = gather_row_scales(bh0, bh, lane, 0, 1);
       tc_st4(tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(kSfaCol + 4 * a), v, v, v, v);
     }

@@ -135,6 +135,8 @@ def test_each_expert_uses_its_own_weight_and_rows(cuda_device):
     (384, 256, [37, 300, 0, 91], False),          # ragged: partial 128-row blocks
     (768, 512, [256, 128, 0, 384], False),         # the Qwen3-MoE width
     (768, 256, [200, 56], True),                   # staged rounding
+    (128, 128, [1], False),                        # a single row
+    (256, 128, [0, 1, 0, 129], False),             # one-row and 129-row experts
 ])
 def test_fc2_matches_the_oracle(cuda_device, N, H, splits, staged):
     M = sum(splits)

@@ -476,6 +476,11 @@ moeact_status act_params(const ActArgs& a, int dev, cudaStream_t cs, Params& p) 
   std::memcpy(&lb, &a.limit, 4);
   lb >>= 16;
   p.clamp_Lb2 = lb | (lb << 16);
+  {
+    uint32_t lbits;
+    std::memcpy(&lbits, &a.limit, 4);
+    p.clamp_bf16 = (lbits & 0xFFFFu) == 0u;   // L is itself a bf16 value
+  }
   if (a.act != kClamped) return MOEACT_OK;
   return alpha_table(dev, a.alpha, a.limit, cs, &p.sig_src);
 }

@@ -102,6 +102,25 @@ __device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
   return r;
 }
 
+// Per 16-bit lane: 0xFFFF where a != b (ordered: false when either is NaN).
+__device__ __forceinline__ uint32_t bf16x2_ne_mask(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.ne.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// NaN-propagating minimum / maximum of two packed bf16 pairs (exact).
+__device__ __forceinline__ uint32_t bf16x2_min_nan(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_max_nan(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // relu that keeps NaN (NaN in -> NaN out); negative and zero inputs give +0.
 __device__ __forceinline__ float relu_keep_nan(float v) {
   return v > 0.0f ? v : (v != v ? v : 0.0f);

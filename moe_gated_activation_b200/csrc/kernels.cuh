@@ -89,6 +89,7 @@ struct Params {
   float clamp_L;
   float clamp_alpha;
   uint32_t clamp_Lb2;
+  int clamp_bf16;     // L is itself a bf16 value (then clamp_Lb2 is L, both halves)
   const int32_t* noop;   // nullable: a non-zero flag makes the call write nothing
   // Gated layouts of x and dX (width 2N): ilv == 0 is [gate | up] halves;
   // ilv = G > 0 is G gate columns, then the G matching up columns, repeated.
@@ -543,28 +544,50 @@ __device__ __forceinline__ float2 clamped_up_plus_one(float2 u, float L) {
 // [-L, L] gets a +0 gradient: its half of the packed pair is cleared, so that
 // a NaN or Inf in dY does not reach it.  The comparisons take the bf16 inputs
 // as they are (NaN compares false).
+// LB: L is a bf16 value, so both clamps are exact packed bf16 min / max on
+// the inputs (one instruction per pair instead of one or two per value) and
+// an up is clamped exactly when its clamp differs from it.
+template <bool LB>
 __device__ __forceinline__ void clamped_bwd_math(const Params& p, const float* sig, uint2 G,
                                                  uint2 U, float2 p01, float2 p23, uint32_t& dg0,
                                                  uint32_t& dg1, uint32_t& du0, uint32_t& du1,
                                                  float2& h01, float2& h23) {
   const float L = p.clamp_L;
+  const uint32_t Lb2 = p.clamp_Lb2;
   float2 sg01, sg23;
   sigma_pair(sig, G.x, sg01.x, sg01.y);
   sigma_pair(sig, G.y, sg23.x, sg23.y);
-  const float2 si01 = mul2(clamp_gate_pair(bf16x2_to_f2(G.x), L), sg01);
-  const float2 si23 = mul2(clamp_gate_pair(bf16x2_to_f2(G.y), L), sg23);
-  const float2 v01 = clamped_up_plus_one(bf16x2_to_f2(U.x), L);
-  const float2 v23 = clamped_up_plus_one(bf16x2_to_f2(U.y), L);
+  float2 si01, si23, v01, v23;
+  uint2 UC = make_uint2(0u, 0u);
+  if (LB) {
+    const uint32_t nL2 = Lb2 ^ 0x80008000u;
+    UC = make_uint2(bf16x2_min_nan(bf16x2_max_nan(U.x, nL2), Lb2),
+                    bf16x2_min_nan(bf16x2_max_nan(U.y, nL2), Lb2));
+    si01 = mul2(bf16x2_to_f2(bf16x2_min_nan(G.x, Lb2)), sg01);
+    si23 = mul2(bf16x2_to_f2(bf16x2_min_nan(G.y, Lb2)), sg23);
+    const float2 one = make_float2(1.0f, 1.0f);
+    v01 = add2(bf16x2_to_f2(UC.x), one);
+    v23 = add2(bf16x2_to_f2(UC.y), one);
+  } else {
+    si01 = mul2(clamp_gate_pair(bf16x2_to_f2(G.x), L), sg01);
+    si23 = mul2(clamp_gate_pair(bf16x2_to_f2(G.y), L), sg23);
+    v01 = clamped_up_plus_one(bf16x2_to_f2(U.x), L);
+    v23 = clamped_up_plus_one(bf16x2_to_f2(U.y), L);
+  }
   const float2 one = make_float2(1.0f, 1.0f), a2 = make_float2(p.clamp_alpha, p.clamp_alpha);
   const float2 ds01 = fma2(mul2(a2, si01), sub2(one, sg01), sg01);
   const float2 ds23 = fma2(mul2(a2, si23), sub2(one, sg23), sg23);
   const float2 dga = mul2(mul2(p01, v01), ds01), dgb = mul2(mul2(p23, v23), ds23);
   const float2 dua = mul2(p01, si01), dub = mul2(p23, si23);
-  const uint32_t Lb2 = p.clamp_Lb2;
   dg0 = pack_bf16x2(dga.x, dga.y) & ~bf16x2_gt_mask(G.x, Lb2);
   dg1 = pack_bf16x2(dgb.x, dgb.y) & ~bf16x2_gt_mask(G.y, Lb2);
-  du0 = pack_bf16x2(dua.x, dua.y) & ~bf16x2_gt_mask(U.x & 0x7FFF7FFFu, Lb2);
-  du1 = pack_bf16x2(dub.x, dub.y) & ~bf16x2_gt_mask(U.y & 0x7FFF7FFFu, Lb2);
+  if (LB) {
+    du0 = pack_bf16x2(dua.x, dua.y) & ~bf16x2_ne_mask(UC.x, U.x);
+    du1 = pack_bf16x2(dub.x, dub.y) & ~bf16x2_ne_mask(UC.y, U.y);
+  } else {
+    du0 = pack_bf16x2(dua.x, dua.y) & ~bf16x2_gt_mask(U.x & 0x7FFF7FFFu, Lb2);
+    du1 = pack_bf16x2(dub.x, dub.y) & ~bf16x2_gt_mask(U.y & 0x7FFF7FFFu, Lb2);
+  }
   h01 = mul2(si01, v01);
   h23 = mul2(si23, v23);
 }
@@ -574,7 +597,7 @@ __device__ __forceinline__ void clamped_bwd_math(const Params& p, const float* s
 // 8 lanes.  Rowwise work runs per 16-row half: after the 3-step butterfly
 // (off = 4, 2, 1) lane l holds the amax of rows 16h + 2(l & 7) + {0, 1} of
 // block l >> 3.
-template <int ACT, int DIRS, bool STAGED, bool GROUPED, bool FULL, int OPS, int SLOTS>
+template <int ACT, int DIRS, bool STAGED, bool GROUPED, bool FULL, bool LB, int OPS, int SLOTS>
 __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OPS, SLOTS>& ring,
                                          int k0, int K, int64_t slab, int tile, int64_t row0,
                                          int nrows, float sv, int lane, const void* tm_x,
@@ -605,10 +628,20 @@ __device__ __forceinline__ void fwd_tile(const Params& p, const Smem& m, Ring<OP
         float2 sg01, sg23;
         sigma_pair_s(m.sig_key, G.x, sg01.x, sg01.y);
         sigma_pair_s(m.sig_key, G.y, sg23.x, sg23.y);
-        const float2 si01 = mul2(clamp_gate_pair(bf16x2_to_f2(G.x), p.clamp_L), sg01);
-        const float2 si23 = mul2(clamp_gate_pair(bf16x2_to_f2(G.y), p.clamp_L), sg23);
-        h01 = mul2(si01, clamped_up_plus_one(bf16x2_to_f2(U.x), p.clamp_L));
-        h23 = mul2(si23, clamped_up_plus_one(bf16x2_to_f2(U.y), p.clamp_L));
+        if (LB) {
+          // L is a bf16 value: both clamps as packed bf16 min / max (exact)
+          const uint32_t L2 = p.clamp_Lb2, nL2 = L2 ^ 0x80008000u;
+          const float2 one = make_float2(1.0f, 1.0f);
+          const float2 si01 = mul2(bf16x2_to_f2(bf16x2_min_nan(G.x, L2)), sg01);
+          const float2 si23 = mul2(bf16x2_to_f2(bf16x2_min_nan(G.y, L2)), sg23);
+          h01 = mul2(si01, add2(bf16x2_to_f2(bf16x2_min_nan(bf16x2_max_nan(U.x, nL2), L2)), one));
+          h23 = mul2(si23, add2(bf16x2_to_f2(bf16x2_min_nan(bf16x2_max_nan(U.y, nL2), L2)), one));
+        } else {
+          const float2 si01 = mul2(clamp_gate_pair(bf16x2_to_f2(G.x), p.clamp_L), sg01);
+          const float2 si23 = mul2(clamp_gate_pair(bf16x2_to_f2(G.y), p.clamp_L), sg23);
+          h01 = mul2(si01, clamped_up_plus_one(bf16x2_to_f2(U.x), p.clamp_L));
+          h23 = mul2(si23, clamped_up_plus_one(bf16x2_to_f2(U.y), p.clamp_L));
+        }
       } else if (ACT == kSwiGLU) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
         float2 sg01, sg23;
@@ -789,12 +822,22 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
       svn = lane < nrowsn ? __ldg(p.s + row0n + lane) : 0.0f;
     }
     const bool full = nrows == 32 && (cur.tile + 1) * kTileCols <= p.N;
-    if (full)
-      fwd_tile<ACT, DIRS, STAGED, GROUPED, true>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
-                                                 nrows, sv, lane, &tm_x, ok);
-    else
-      fwd_tile<ACT, DIRS, STAGED, GROUPED, false>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
-                                                  nrows, sv, lane, &tm_x, ok);
+    // (ClampedSwiGLU with a bf16 limit: the packed-clamp form of the tile)
+    if (ACT == kClamped && p.clamp_bf16) {
+      if (full)
+        fwd_tile<ACT, DIRS, STAGED, GROUPED, true, ACT == kClamped>(
+            p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, sv, lane, &tm_x, ok);
+      else
+        fwd_tile<ACT, DIRS, STAGED, GROUPED, false, ACT == kClamped>(
+            p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, sv, lane, &tm_x, ok);
+    } else if (full) {
+      fwd_tile<ACT, DIRS, STAGED, GROUPED, true, false>(p, m, ring, 2 * j, K, cur.slab, cur.tile,
+                                                        row0, nrows, sv, lane, &tm_x, ok);
+    } else {
+      fwd_tile<ACT, DIRS, STAGED, GROUPED, false, false>(p, m, ring, 2 * j, K, cur.slab,
+                                                         cur.tile, row0, nrows, sv, lane, &tm_x,
+                                                         ok);
+    }
     cur = nx;
     row0 = row0n;
     nrows = nrowsn;
@@ -812,7 +855,7 @@ __global__ void __launch_bounds__(Cfg<ACT, false>::kThreads, 1)
 // ------------------------------------------------------------- backward row
 // The backward of one row's four columns (a lane's share): packed bf16
 // dgate/dup pairs and the row's dscale partial sum_c dY*h.
-template <int ACT>
+template <int ACT, bool LB>
 __device__ __forceinline__ void bwd_row(const Params& p, const float* sig, uint2 D, uint2 G,
                                         uint2 U, float sr, uint32_t& dg0, uint32_t& dg1,
                                         uint32_t& du0, uint32_t& du1, float& part) {
@@ -821,7 +864,7 @@ __device__ __forceinline__ void bwd_row(const Params& p, const float* sig, uint2
   const float2 p01 = mul2(d01, s2), p23 = mul2(d23, s2);
   float2 h01, h23;
   if (ACT == kClamped) {
-    clamped_bwd_math(p, sig, G, U, p01, p23, dg0, dg1, du0, du1, h01, h23);
+    clamped_bwd_math<LB>(p, sig, G, U, p01, p23, dg0, dg1, du0, du1, h01, h23);
   } else if (ACT == kSwiGLU) {
     const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
     float2 sg01, sg23;
@@ -900,7 +943,7 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
       uint32_t qg0, qg1, qu0, qu1;   // the packed bf16 gradients
       if (ACT == kClamped) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
-        clamped_bwd_math(p, m.sig, G, U, p01, p23, qg0, qg1, qu0, qu1, h01, h23);
+        clamped_bwd_math<false>(p, m.sig, G, U, p01, p23, qg0, qg1, qu0, qu1, h01, h23);
       } else if (ACT == kSwiGLU) {
         const uint2 U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
         const float2 u01 = bf16x2_to_f2(U.x), u23 = bf16x2_to_f2(U.y);
@@ -1078,7 +1121,7 @@ __device__ __forceinline__ void bwd_tile(const Params& p, const Smem& m, Ring<OP
 // the half (stored), the half's dscale partial (ph, rows 2(l&15) + {0,1}),
 // its rowwise scales (bh, this lane's reduced E8M0 bytes) and codes, and folds
 // the colwise maxima into acg / acu.  Returns false if the slot never landed.
-template <int ACT, int DIRS, bool GROUPED, bool FULL, int OPS, int SLOTS>
+template <int ACT, int DIRS, bool GROUPED, bool FULL, bool LB, int OPS, int SLOTS>
 __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
                                             Ring<OPS, SLOTS>& ring, int k0, int h, int K,
                                             int nrows, float sv, int lane, bool colok, int Wq,
@@ -1104,7 +1147,7 @@ __device__ __forceinline__ bool bwd_half_rr(const Params& p, const Smem& m,
     if (ACT != kSReLU) U = *reinterpret_cast<const uint2*>(sm + 2 * kOpHalfBytes + i * kRowBytes);
     const float sr = __shfl_sync(kFull, sv, r);
     float part;
-    bwd_row<ACT>(p, m.sig, D, G, U, sr, DG[i][0], DG[i][1], DU[i][0], DU[i][1], part);
+    bwd_row<ACT, LB>(p, m.sig, D, G, U, sr, DG[i][0], DG[i][1], DU[i][0], DU[i][1], part);
     const bool live = FULL || i < nrh;
     // rows past the slab's end: past M they read as zero (and give zeros); in
     // a grouped call they are the next group's rows, which must not count
@@ -1235,7 +1278,7 @@ __device__ __forceinline__ void bwd_colwise_rr(int U, int nrows, bool colok, int
   }
 }
 
-template <int ACT, int DIRS, bool GROUPED, bool FULL, int OPS, int SLOTS>
+template <int ACT, int DIRS, bool GROUPED, bool FULL, bool LB, int OPS, int SLOTS>
 __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
                                             Ring<OPS, SLOTS>& ring, int k0, int K, int64_t slab,
                                             int tile, int64_t row0, int nrows, float sv, int lane,
@@ -1258,7 +1301,7 @@ __device__ __forceinline__ void bwd_tile_rr(const Params& p, const Smem& m,
   for (int h = 0; h < 2; ++h) {
     float v;
     uint32_t b;
-    if (!bwd_half_rr<ACT, DIRS, GROUPED, FULL>(p, m, ring, k0, h, K, nrows, sv, lane, colok, Wq,
+    if (!bwd_half_rr<ACT, DIRS, GROUPED, FULL, LB>(p, m, ring, k0, h, K, nrows, sv, lane, colok, Wq,
                                                rqb, dxb, tm_x, tm_dy, v, b, acg, acu)) {
       ok_flag = false;
       return;
@@ -1376,12 +1419,21 @@ __global__ void __launch_bounds__(Cfg<ACT, true>::kThreads, 1)
     }
     const bool full = nrows == 32 && (cur.tile + 1) * kTileCols <= p.N;
     if (REREAD) {
-      if (full)
-        bwd_tile_rr<ACT, DIRS, GROUPED, true>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
-                                              nrows, sv, lane, &tm_x, &tm_dy, ok);
-      else
-        bwd_tile_rr<ACT, DIRS, GROUPED, false>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0,
-                                               nrows, sv, lane, &tm_x, &tm_dy, ok);
+      // (ClampedSwiGLU with a bf16 limit: the packed-clamp form of the tile)
+      if (ACT == kClamped && p.clamp_bf16) {
+        if (full)
+          bwd_tile_rr<ACT, DIRS, GROUPED, true, ACT == kClamped>(
+              p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, sv, lane, &tm_x, &tm_dy, ok);
+        else
+          bwd_tile_rr<ACT, DIRS, GROUPED, false, ACT == kClamped>(
+              p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, sv, lane, &tm_x, &tm_dy, ok);
+      } else if (full) {
+        bwd_tile_rr<ACT, DIRS, GROUPED, true, false>(p, m, ring, 2 * j, K, cur.slab, cur.tile,
+                                                     row0, nrows, sv, lane, &tm_x, &tm_dy, ok);
+      } else {
+        bwd_tile_rr<ACT, DIRS, GROUPED, false, false>(p, m, ring, 2 * j, K, cur.slab, cur.tile,
+                                                      row0, nrows, sv, lane, &tm_x, &tm_dy, ok);
+      }
     } else {
       bwd_tile<ACT, DIRS, GROUPED>(p, m, ring, 2 * j, K, cur.slab, cur.tile, row0, nrows, full,
                                    sv, lane, &tm_x, &tm_dy, ok);

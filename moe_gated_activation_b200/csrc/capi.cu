@@ -263,10 +263,10 @@ size_t ws_bytes_needed(int64_t M, int64_t N) {
 // elements, read in boxes of 128 columns x 16 rows; out-of-range elements read
 // as zero.  Encoded on the host for every call (no allocation).
 moeact_status make_map(CUtensorMap* map, const void* base, int64_t width, int64_t rows,
-                       int64_t ld) {
+                       int64_t ld, int box_rows = kHalfRows) {
   const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  const cuuint32_t box[2] = {(cuuint32_t)kTileCols, (cuuint32_t)kHalfRows};
+  const cuuint32_t box[2] = {(cuuint32_t)kTileCols, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -883,7 +883,7 @@ moeact_status grouped_scaled_swiglu_mxfp8_fc2(const void* x, int64_t ldx, const 
   int dev;
   if ((st = ensure_ready(cs, &dev))) return st;
   CUtensorMap tx;
-  if ((st = make_map(&tx, x, 2 * N, M, ldx))) return st;
+  if ((st = make_map(&tx, x, 2 * N, M, ldx, kFc2XBoxRows))) return st;
   Fc2Params p{};
   p.s = s;
   p.M = M;
@@ -899,7 +899,8 @@ moeact_status grouped_scaled_swiglu_mxfp8_fc2(const void* x, int64_t ldx, const 
   p.sig_src = g_sig_ptr[dev];
   p.noop = noop_flag;
   p.err = g_err_ptr[dev];
-  const int64_t grid = ceil_div(M, 128) + num_groups;
+  p.n_sms = g_sms[dev];
+  const int64_t grid = ceil_div(M, 128) + num_groups + g_sms[dev];
   const cudaError_t e = fc2_launch(p, tx, staged_rounding, (unsigned)grid, cs);
   if (e != cudaSuccess) return cuda_fail(e, "fused FC2 launch");
   return MOEACT_OK;

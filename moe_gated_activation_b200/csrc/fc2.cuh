@@ -34,18 +34,21 @@ struct Fc2Params {
   const float* sig_src;       // the sigmoid table (device memory, shared-memory layout)
   const int32_t* noop;        // nullable
   uint32_t* err;              // device error word
+  int n_sms;                  // SMs of the device (the last wave's blocks are split to fill them)
 };
 
 constexpr int kFc2MaxN = 768;
 constexpr int kFc2Threads = 320;   // 8 math warps, a TMA warp, an MMA warp
+constexpr int kFc2XBoxRows = 8;    // rows of X per tensor-map box (a prologue sub-slot)
 
 // Dynamic shared memory of a launch with activation width N.
 int fc2_smem_bytes(int N);
 // Sets the kernels' shared-memory limit (once per device).
 cudaError_t fc2_prepare();
-// Launches the fused kernel: one CTA per possible 128-row block of an expert
-// (`grid` = ceil(M/128) + E covers every split); tm_x is the bf16 [M, 2N]
-// input in 128 x 16 boxes.
+// Launches the fused kernel: one CTA per 128-row block of an expert, or per
+// part of one when the last wave of blocks is split over several CTAs
+// (`grid` = ceil(M/128) + E + n_sms covers every split and every tail); tm_x
+// is the bf16 [M, 2N] input in 128 x kFc2XBoxRows boxes.
 cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, int staged, unsigned grid,
                        cudaStream_t stream);
 

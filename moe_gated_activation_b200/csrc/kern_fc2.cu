@@ -14,9 +14,12 @@
 // of the block-scaled operands are summed by the tensor cores in fp32 and the
 // result rounded to bf16.
 //
-// One CTA per (expert, 128-row block); 10 warps:
+// One CTA per (expert, 128-row block), or per range of its output tiles for
+// the blocks of a last, partial wave (split so that the wave fills the SMs);
+// 10 warps:
 //   warps 0-7  prologue: stream the block's gate / up rows in by TMA (one
-//              16-row half-tile slot per warp), compute y and its rowwise
+//              16-row half-tile slot per warp, as two 8-row sub-slots each
+//              refilled as soon as it is read), compute y and its rowwise
 //              MXFP8, write the codes into shared memory in the tensor
 //              cores' K-major 128-byte-swizzled layout and the scales into
 //              tensor memory; then, per 128-column output tile, drain the
@@ -47,6 +50,11 @@ constexpr int kEpiBytes = 8 * kEpiWarpBytes;
 constexpr int kStageBytes = 16384;        // 128 weight rows x 128 bytes of k
 constexpr int kXSlotBytes = 2 * kOpHalfBytes;   // gate + up of 16 rows x 128 columns
 constexpr int kXBytes = 8 * kXSlotBytes;  // the prologue's slots (8 warps)
+// A warp's slot as two sub-slots of kFc2XBoxRows rows (gate rows, then up
+// rows), each refilled as soon as its rows are read.
+constexpr int kXSub = 16 / kFc2XBoxRows;
+constexpr int kXSubBytes = kXSlotBytes / kXSub;
+constexpr int kXSubOpBytes = kXSubBytes / 2;
 // The staging region: (prologue) the X slots and the sigmoid table after
 // them; (GEMM) the weight ring and the epilogue's staging, as many ring stages
 // as fit.
@@ -60,6 +68,9 @@ constexpr int kSfaCol = 256;              // tensor-memory columns: accumulators
 constexpr int kSfbCol = 288;              // A scales [256, 288), W scales [288, 352)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kErrFc2Wait = 0x20u;
+
+constexpr int kXBars = 8 * kXSub;         // the prologue's sub-slot barriers
+constexpr int kBarSlots = 64;             // mbarriers at the start of the misc region
 
 // misc ints
 constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscE = 2, kMiscBlk = 3, kMiscScan = 16;
@@ -180,7 +191,7 @@ struct Fc2Smem {
   unsigned char* sf;      // [2 tiles][N/128 groups][512 bytes]: weight scales, tiled
   unsigned char* R;       // staging: weight ring / X slots + sigmoid table
   const float* sig;
-  uint64_t* xbar;         // [8]
+  uint64_t* xbar;         // [8 * kXSub]: the prologue sub-slots, kXSub per warp
   uint64_t* sig_bar;
   uint64_t* pro_done;     // count 8: the block's A codes and scales are complete
   uint64_t* b_full;       // [kStages] a weight stage has landed
@@ -214,15 +225,25 @@ __device__ __forceinline__ void set_abort(const Fc2Params& p, const Fc2Smem& m) 
 // columns of atom a): y = SwiGLU(g, u) * s, its rowwise E8M0 scales (returned
 // packed as in fwd_tile: lane l holds blocks l >> 3 of rows 2 (l & 7) + {0,1})
 // and its E4M3 codes, stored into the atom at the swizzled positions.
-template <bool STAGED>
+// The half's rows arrive in kXSub sub-slots: `wait(sub)` before a sub-slot's
+// first row (false on a timeout: `ok` is cleared and nothing is written),
+// `refill(sub)` once every lane has read its last row.
+template <bool STAGED, typename Wait, typename Refill>
 __device__ __forceinline__ uint32_t fc2_half(const Fc2Smem& m, const unsigned char* slot,
-                                             int lane, int q, int a, int h, int nvq, float sv) {
+                                             int lane, int q, int a, int h, int nvq, float sv,
+                                             Wait&& wait, Refill&& refill, bool& ok) {
   float Y[16][4];
   const unsigned char* sm = slot + 8 * lane;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint2 G = *reinterpret_cast<const uint2*>(sm + i * kRowBytes);
-    const uint2 U = *reinterpret_cast<const uint2*>(sm + kOpHalfBytes + i * kRowBytes);
+    const int sub = i / kFc2XBoxRows, ri = i % kFc2XBoxRows;
+    if (ri == 0 && !wait(sub)) {
+      ok = false;
+      return 0;
+    }
+    const uint2 G = *reinterpret_cast<const uint2*>(sm + sub * kXSubBytes + ri * kRowBytes);
+    const uint2 U =
+        *reinterpret_cast<const uint2*>(sm + sub * kXSubBytes + kXSubOpBytes + ri * kRowBytes);
     const float sr = __shfl_sync(kFull, sv, 16 * h + i);
     const float2 s2 = make_float2(sr, sr);
     float2 sg01, sg23;
@@ -247,8 +268,12 @@ __device__ __forceinline__ uint32_t fc2_half(const Fc2Smem& m, const unsigned ch
     Y[i][1] = live ? y01.y : 0.0f;
     Y[i][2] = live ? y23.x : 0.0f;
     Y[i][3] = live ? y23.y : 0.0f;
+    if (ri == kFc2XBoxRows - 1) {
+      // every lane has read the sub-slot: its next copy overlaps the rest
+      __syncwarp();
+      refill(sub);
+    }
   }
-  __syncwarp();
   uint32_t Am[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i)
@@ -297,7 +322,7 @@ __device__ __forceinline__ bool fc2_put_w_scales(const Fc2Params& p, const Fc2Sm
 
 template <bool STAGED>
 __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2Smem& m, int e,
-                         int64_t row0, int mrows, uint32_t tbase) {
+                         int64_t row0, int mrows, uint32_t tbase, int t0, int T) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, half_sel = warp >> 2;
   const int KA = p.N >> 7;
@@ -305,13 +330,18 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
   const int n_atoms = KA > half_sel ? (KA - half_sel + 1) / 2 : 0;
   const int Kw = 2 * n_atoms;                          // half-tiles of this warp
   unsigned char* slot = m.R + warp * kXSlotBytes;
-  uint64_t* xb = m.xbar + warp;
-  auto issue = [&](int j) {
+  uint64_t* xb = m.xbar + kXSub * warp;
+  // unit u: sub-slot u % kXSub of half-tile u / kXSub; sub-slot b's barrier
+  // completes once per unit, parity (u / kXSub) & 1
+  const int U = kXSub * Kw;
+  auto issue = [&](int u) {
+    const int j = u / kXSub, b = u % kXSub;
     const int a = half_sel + 2 * (j >> 1);
-    const int y = (int)row0 + 32 * q + 16 * (j & 1);
-    mbar_expect_tx(xb, kXSlotBytes);
-    tma_load_2d(slot, tm_x, 128 * a, y, xb);
-    tma_load_2d(slot + kOpHalfBytes, tm_x, p.N + 128 * a, y, xb);
+    const int y = (int)row0 + 32 * q + 16 * (j & 1) + kFc2XBoxRows * b;
+    unsigned char* dst = slot + b * kXSubBytes;
+    mbar_expect_tx(xb + b, kXSubBytes);
+    tma_load_2d(dst, tm_x, 128 * a, y, xb + b);
+    tma_load_2d(dst + kXSubOpBytes, tm_x, p.N + 128 * a, y, xb + b);
   };
   if (threadIdx.x == 0) {
     mbar_expect_tx(m.sig_bar, 2 * kSigHalfBytes);
@@ -319,18 +349,28 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
     bulk_load(const_cast<float*>(m.sig) + kSigNegOffset, p.sig_src + kSigNegOffset,
               kSigHalfBytes, m.sig_bar);
   }
-  if (lane == 0 && Kw > 0) issue(0);
+  if (lane == 0)
+    for (int u = 0; u < kXSub && u < U; ++u) issue(u);
   const float sv = lane < nvq ? __ldg(p.s + row0 + 32 * q + lane) : 0.0f;
   bool ok = warp_wait(m.sig_bar, 0u);
-  int waited = 0;   // half-tiles whose copy this warp has seen land
+  int waited = 0;   // units whose copy this warp has seen land
   uint32_t bh0 = 0;
   for (int j = 0; ok && j < Kw; ++j) {
-    if (!warp_wait(xb, (uint32_t)j & 1u)) { ok = false; break; }
-    waited = j + 1;
     const int a = half_sel + 2 * (j >> 1), h = j & 1;
-    const uint32_t bh = fc2_half<STAGED>(m, slot, lane, q, a, h, nvq, sv);
-    // fc2_half has read the slot (its values are in use): refill it
-    if (lane == 0 && j + 1 < Kw) issue(j + 1);
+    const uint32_t bh = fc2_half<STAGED>(
+        m, slot, lane, q, a, h, nvq, sv,
+        [&](int b) {
+          const int u = kXSub * j + b;
+          if (!warp_wait(xb + b, (uint32_t)(u / kXSub) & 1u)) return false;
+          waited = u + 1;
+          return true;
+        },
+        [&](int b) {
+          const int u = kXSub * (j + 1) + b;
+          if (lane == 0 && u < U) issue(u);
+        },
+        ok);
+    if (!ok) break;
     if (h == 0) {
       bh0 = bh;
     } else {
@@ -347,11 +387,11 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
     set_abort(p, m);
     // copies this warp issued that never landed: wait for them (bounded)
     if (lane == 0) {
-      if (waited < Kw) mbar_wait(xb, (uint32_t)waited & 1u);
+      for (int u = waited; u < U && u < waited + kXSub; ++u)
+        mbar_wait(xb + u % kXSub, (uint32_t)(u / kXSub) & 1u);
       mbar_wait(m.sig_bar, 0u);
     }
   }
-  const int T = p.H >> 7;
   // the weight scales of the first two output tiles
   if (ok && half_sel == 0)
     for (int t = 0; t < 2 && t < T; ++t)
@@ -413,7 +453,7 @@ __device__ void fc2_math(const CUtensorMap* tm_x, const Fc2Params& p, const Fc2S
         const int sw = kChunks == 8 ? (r & 7) : ((r >> 1) & 3);
         const uint4 w = *reinterpret_cast<const uint4*>(stg + r * (16 * kChunks) + ((cc ^ sw) << 4));
         if (32 * q + r < mrows)
-          *reinterpret_cast<uint4*>(p.out + (row0 + 32 * q + r) * p.ldo + 128 * n +
+          *reinterpret_cast<uint4*>(p.out + (row0 + 32 * q + r) * p.ldo + 128 * (t0 + n) +
                                     64 * half_sel + 8 * (ps * kChunks + cc)) = w;
       }
       __syncwarp();
@@ -436,8 +476,9 @@ __device__ __forceinline__ bool elect_one() {
 // kSfSlots - 1 output tiles ahead: the scales of tile n + 3 go out after the
 // last weight tile of tile n, when the slot they reuse (tile n - 1's) is
 // already free, and have two tiles of MMAs to land.
-__device__ void fc2_producer(const Fc2Params& p, const Fc2Smem& m, int e) {
-  const int KA = p.N >> 7, T = p.H >> 7;
+__device__ void fc2_producer(const Fc2Params& p, const Fc2Smem& m, int e, int t0, int T) {
+  const int KA = p.N >> 7;
+  const int64_t tile0 = (int64_t)e * (p.H >> 7) + t0;   // the expert's tile t0 in the tiled layout
   const bool leader = elect_one();
   int issued = 0, sf_issued = 0;
   auto issue_sf = [&](int n) {   // false on a timeout
@@ -447,8 +488,8 @@ __device__ void fc2_producer(const Fc2Params& p, const Fc2Smem& m, int e) {
       return false;
     if (leader) {
       mbar_expect_tx(m.sf_full + ss, 512 * KA);
-      bulk_load(m.sf + ss * kSfSlotBytes, p.w_scales + ((int64_t)e * T + n) * KA * 512,
-                512 * KA, m.sf_full + ss);
+      bulk_load(m.sf + ss * kSfSlotBytes, p.w_scales + (tile0 + n) * KA * 512, 512 * KA,
+                m.sf_full + ss);
     }
     __syncwarp();
     sf_issued = n + 1;
@@ -458,7 +499,7 @@ __device__ void fc2_producer(const Fc2Params& p, const Fc2Smem& m, int e) {
   // shared with it); the weight tiles reuse the prologue's staging memory
   for (int n = 0; n < T && n < kSfSlots - 1; ++n) issue_sf(n);
   if (!__all_sync(kFull, mbar_wait(m.pro_done, 0u)) && leader) set_abort(p, m);
-  const uint8_t* wsrc = p.w_codes + (int64_t)e * T * KA * kStageBytes;
+  const uint8_t* wsrc = p.w_codes + tile0 * KA * kStageBytes;
   for (int g = 0; g < T * KA && !warp_aborted(m); ++g) {
     const int n = g / KA, ks = g - n * KA, slot = g % kStages;
     if (g >= kStages &&
@@ -496,8 +537,8 @@ __device__ void fc2_producer(const Fc2Params& p, const Fc2Smem& m, int e) {
 // set the rate.  A K step of 32 bytes advances a descriptor's start-address
 // field by 2 (16-byte units; shared-memory addresses stay below 2^18, so
 // the field never carries).
-__device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase) {
-  const int KA = p.N >> 7, T = p.H >> 7;
+__device__ void fc2_mma(const Fc2Params& p, const Fc2Smem& m, uint32_t tbase, int T) {
+  const int KA = p.N >> 7;
   const bool leader = elect_one();
   bool ok = __all_sync(kFull, mbar_wait(m.pro_done, 0u)) && !warp_aborted(m);
   if (!ok && leader) set_abort(p, m);
@@ -561,16 +602,16 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
   m.sig = reinterpret_cast<const float*>(m.R + kXBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(m.R + kRBytes);
   m.xbar = bars;
-  m.sig_bar = bars + 8;
-  m.pro_done = bars + 9;
-  m.b_full = bars + 10;
-  m.b_empty = bars + 10 + kStages;
-  m.sf_full = bars + 10 + 2 * kStages;
+  m.sig_bar = bars + kXBars;
+  m.pro_done = bars + kXBars + 1;
+  m.b_full = bars + kXBars + 2;
+  m.b_empty = m.b_full + kStages;
+  m.sf_full = m.b_empty + kStages;
   m.sf_empty = m.sf_full + kSfSlots;
   m.d_full = m.sf_empty + kSfSlots;
   m.d_empty = m.d_full + 2;
   m.mma_done = m.d_empty + 2;
-  m.misc = reinterpret_cast<int*>(bars + 40);
+  m.misc = reinterpret_cast<int*>(bars + kBarSlots);
   const int tid = threadIdx.x, warp = tid >> 5;
 
   // ---- this CTA's (expert, 128-row block); the offsets are validated first
@@ -603,8 +644,23 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
     if (w < warp) wbase += v;
     total += v;
   }
-  const int u = blockIdx.x;
-  if (u >= total) return;
+  // this CTA's block and output tiles [t0, t0 + tn): blocks of the whole
+  // waves take every tile; when the last wave holds r < n_sms blocks, each of
+  // its blocks is split over k = min(n_sms / r, T) CTAs by output tiles (each
+  // part repeats the block's prologue), so that the wave fills the SMs
+  const int T = p.H >> 7;
+  const int r_tail = total % p.n_sms;
+  const int k_split = r_tail > 0 ? min(p.n_sms / r_tail, T) : 1;
+  const int n_whole = total - (k_split > 1 ? r_tail : 0);
+  int u = blockIdx.x, t0 = 0, tn = T;
+  if (u >= n_whole) {
+    const int v = u - n_whole;
+    if (k_split == 1 || v >= r_tail * k_split) return;
+    const int part = v % k_split;
+    u = n_whole + v / k_split;
+    t0 = part * T / k_split;
+    tn = (part + 1) * T / k_split - t0;
+  }
   {
     int acc = wbase + incl - local;
     if (u >= acc && u < acc + local) {
@@ -626,7 +682,7 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
 
   // ---- barriers and tensor memory
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(m.xbar + i, 1);
+    for (int i = 0; i < kXBars; ++i) mbar_init(m.xbar + i, 1);
     mbar_init(m.sig_bar, 1);
     mbar_init(m.pro_done, 8);
     for (int i = 0; i < kStages; ++i) {
@@ -655,11 +711,11 @@ __global__ void __launch_bounds__(kFc2Threads, 1)
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(m.misc + kMiscTmem);
 
   if (warp < 8) {
-    fc2_math<STAGED>(&tm_x, p, m, e, row0, mrows, tbase);
+    fc2_math<STAGED>(&tm_x, p, m, e, row0, mrows, tbase, t0, tn);
   } else if (warp == 8) {
-    fc2_producer(p, m, e);
+    fc2_producer(p, m, e, t0, tn);
   } else {
-    fc2_mma(p, m, tbase);
+    fc2_mma(p, m, tbase, tn);
   }
 
   tc_fence_before();
@@ -694,9 +750,11 @@ cudaError_t fc2_launch(const Fc2Params& p, const CUtensorMap& tm_x, int staged, 
   return cudaGetLastError();
 }
 
-static_assert(kMiscScan * 4 + (kFc2Threads / 32) * 4 + 40 * 8 <= kMiscBytes,
+static_assert(kMiscScan * 4 + (kFc2Threads / 32) * 4 + kBarSlots * 8 <= kMiscBytes,
               "misc region too small");
-static_assert(10 + 2 * kStages + 2 * kSfSlots + 5 <= 40, "barrier region too small");
+static_assert(kXBars + 2 + 2 * kStages + 2 * kSfSlots + 5 <= kBarSlots,
+              "barrier region too small");
+static_assert(16 % kFc2XBoxRows == 0 && kXSubBytes % 128 == 0, "sub-slot geometry");
 static_assert(kSfBytes % 1024 == 0, "the staging region must stay 1024-byte aligned");
 static_assert(kXBytes + kSigBytes <= kRBytes, "staging region too small");
 static_assert(kStages * kStageBytes + kEpiBytes <= kRBytes && kStages >= 4,

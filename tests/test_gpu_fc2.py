@@ -137,6 +137,11 @@ def test_each_expert_uses_its_own_weight_and_rows(cuda_device):
     (768, 256, [200, 56], True),                   # staged rounding
     (128, 128, [1], False),                        # a single row
     (256, 128, [0, 1, 0, 129], False),             # one-row and 129-row experts
+    # fewer blocks than SMs: each block's output tiles split over several CTAs,
+    # unevenly here (5 tiles in parts of 1, 2, 2 when 38 blocks meet 148 SMs)
+    (256, 640, [1200, 0, 3536], False),
+    # more blocks than SMs: whole blocks, then a split last wave
+    (128, 256, [20403, 77], False),
 ])
 def test_fc2_matches_the_oracle(cuda_device, N, H, splits, staged):
     M = sum(splits)

@@ -116,6 +116,29 @@ def test_identity_weight_returns_the_dequantized_activation(cuda_device):
     assert np.array_equal(out.float().cpu().numpy().astype(np.float64), ref)
 
 
+def test_identity_weight_with_gates_at_the_ends_of_the_sigmoid_table(cuda_device):
+    """Gates where sigma saturates, at the largest tabulated magnitude (127.5)
+    and past it (clamped to it: the same fp32 sigma, 1 or +0), and where it
+    rounds to 1/2; every output equals the dequantized activation exactly."""
+    N, M = 256, 256
+    case = random_case(M, N, 33, std=2.0)
+    x = case["x"]
+    special = torch.tensor([127.5, 128.0, 129.0, 1000.0, 30000.0, 17.25, 17.5, 88.0, 103.5,
+                            104.0, 2.0 ** -25, 2.0 ** -24, 1e-8, 0.0, 126.0, 127.0])
+    special = torch.cat([special, -special]).to(torch.bfloat16)
+    g = torch.Generator().manual_seed(34)
+    pos = torch.randperm(M * N, generator=g)[: M * N // 8]
+    gate = x[:, :N].reshape(-1).clone()
+    gate[pos] = special[torch.randint(0, special.numel(), (pos.numel(),), generator=g)]
+    x[:, :N] = gate.reshape(M, N)
+    wc, ws = _identity(1, N)
+    out, oro = _run(case, N, [M], wc, ws, cuda_device)
+    ref = oracle.grouped_fc2(bf16_bits(case["x"]), case["s"].numpy(), N, oro, wc.numpy(),
+                             ws.numpy())
+    assert np.isfinite(ref).all()
+    assert np.array_equal(out.float().cpu().numpy().astype(np.float64), ref)
+
+
 def test_each_expert_uses_its_own_weight_and_rows(cuda_device):
     # ragged and empty experts; expert e's weight is 2^(e - 2) times the identity
     N = 384

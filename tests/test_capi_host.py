@@ -216,3 +216,42 @@ def test_glu_interleave_arguments(lib, ilv, N, status):
                                                   MX_ROW, None)
     assert clamped == status
 
+
+
+def fc2(lib, x=A16, ldx=512, s=A16, M=64, N=256, staged=0, ro=A16, E=4, st=A16, wc=A16,
+        ws=A16, H=256, out=A16, ldo=256, noop=None):
+    return lib.grouped_scaled_swiglu_mxfp8_fc2(x, ldx, s, M, N, staged, ro, E, st, wc, ws, H, out,
+                                               ldo, noop, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), _capi.EINVAL),
+    (dict(N=96, ldx=192), _capi.EINVAL),          # N not a multiple of 128
+    (dict(N=896, ldx=1792), _capi.EUNSUPPORTED),  # the 128-row block must fit on chip
+    (dict(staged=2), _capi.EINVAL),
+    (dict(ro=None), _capi.EINVAL),
+    (dict(st=None), _capi.EINVAL),
+    (dict(E=0), _capi.EINVAL),
+    (dict(E=_capi.MAX_GROUPS + 1), _capi.EINVAL),
+    (dict(ro=A16 + 4), _capi.EALIGN),
+    (dict(st=A16 + 2), _capi.EALIGN),
+    (dict(wc=None), _capi.EINVAL),
+    (dict(ws=None), _capi.EINVAL),
+    (dict(out=None), _capi.EINVAL),
+    (dict(wc=A16 + 8), _capi.EALIGN),
+    (dict(out=A16 + 8), _capi.EALIGN),
+    (dict(H=0), _capi.EINVAL),
+    (dict(H=192, ldo=192), _capi.EINVAL),         # H not a multiple of 128
+    (dict(ldo=128), _capi.EINVAL),                # narrower than H
+    (dict(ldo=260), _capi.EALIGN),                # not a multiple of 8 elements
+    (dict(noop=A16 + 2), _capi.EALIGN),
+    (dict(ldx=256), _capi.EINVAL),                # narrower than 2N
+    (dict(H=1 << 21, E=1024, ldo=1 << 21), _capi.ERANGE),   # E * H above 2^31 - 1
+])
+def test_fc2_argument_errors(lib, kw, status):
+    assert fc2(lib, **kw) == status
+    assert lib.moeact_last_error()
+
+
+def test_fc2_empty_input_is_ok_without_launch(lib):
+    assert fc2(lib, M=0) == _capi.OK

@@ -165,6 +165,9 @@ def test_each_expert_uses_its_own_weight_and_rows(cuda_device):
     (256, 640, [1200, 0, 3536], False),
     # more blocks than SMs: whole blocks, then a split last wave
     (128, 256, [20403, 77], False),
+    # a wide FC2 (32 output tiles) over three blocks: 148 / 3 = 49 parts
+    # capped at one tile each
+    (256, 4096, [300, 84], False),
 ])
 def test_fc2_matches_the_oracle(cuda_device, N, H, splits, staged):
     M = sum(splits)
@@ -176,6 +179,33 @@ def test_fc2_matches_the_oracle(cuda_device, N, H, splits, staged):
     ref = oracle.grouped_fc2(xb, s, N, oro, wc.numpy(), ws.numpy(), staged=staged)
     bound = _bound(xb, s, N, oro, wc.numpy(), ws.numpy(), staged)
     _check(out, ref, bound, f"N={N} H={H} splits={splits}")
+
+
+def test_fc2_reads_a_strided_input_and_writes_into_a_wider_output(cuda_device):
+    """X as a column slice of a wider tensor (row stride 2N + 64) and `out` as
+    the first H columns of a wider buffer: the same bits as the contiguous
+    call, the extra output columns untouched, the input unchanged."""
+    dev = cuda_device
+    N, H, splits = 256, 384, [200, 0, 184]
+    M, E = sum(splits), len(splits)
+    case = random_case(M, N, 43, std=1.5)
+    wc, ws = fc2_weights(E, H, N, 44)
+    wc, ws = _tiled_codes(wc).to(dev), _tiled(ws).to(dev)
+    ro, _, st = mg.splits_to_offsets(torch.tensor(splits, dtype=torch.int64, device=dev), M)
+    x, s = case["x"].to(dev), case["s"].to(dev)
+    ref, st0 = mg.grouped_scaled_swiglu_mxfp8_fc2(x, s, ro, wc, ws)
+    wide = torch.zeros(M, 2 * N + 64, dtype=torch.bfloat16, device=dev)
+    wide[:, 32:32 + 2 * N] = x
+    xv = wide[:, 32:32 + 2 * N]
+    before = wide.clone()
+    big = torch.full((M, H + 64), 7.0, dtype=torch.bfloat16, device=dev)
+    out, st1 = mg.grouped_scaled_swiglu_mxfp8_fc2(xv, s, ro, wc, ws, out=big[:, :H])
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and int(st0.item()) == 0 and int(st1.item()) == 0
+    assert xv.stride(0) == 2 * N + 64 and out.stride(0) == H + 64
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    assert bool((big[:, H:] == 7.0).all())
+    assert torch.equal(wide.view(torch.int16), before.view(torch.int16))
 
 
 def test_fc2_writes_nothing_for_bad_offsets_or_a_set_noop_flag(cuda_device):

@@ -411,9 +411,15 @@ moeact_status moeact_device_error(uint32_t* flags);
  *     in row-major tile order; element (r, c) of a tile at byte
  *     (r mod 32) * 16 + (r / 32) * 4 + c), experts one after another:
  *     E * H * N/32 bytes, 16-byte aligned.
- *   H: output width, a positive multiple of 128, E * H < 2^31.
- *   out: bf16 [M, ldo] (caller-owned, 16-byte aligned), ldo >= H and a
- *     multiple of 8; columns [0, H) of every row are written.
+ *   H: output width, a positive multiple of 128 (else MOEACT_EINVAL),
+ *     E * H < 2^31 (else MOEACT_ERANGE).
+ *   out: bf16 [M, ldo] (caller-owned, 16-byte aligned), ldo >= H (else
+ *     MOEACT_EINVAL) and a multiple of 8 (else MOEACT_EALIGN); columns
+ *     [0, H) of every row are written, the rest of each row is not touched.
+ *   Null x, s, row_offs, status, w_codes, w_scales or out: MOEACT_EINVAL;
+ *   row_offs not 8-byte, status or noop_flag not 4-byte, w_codes, w_scales or
+ *   out not 16-byte aligned: MOEACT_EALIGN.  M == 0: MOEACT_OK, nothing
+ *   launched.
  *   noop_flag: nullable device int32; non-zero at execution time makes the
  *     call write nothing (CUDA-graph replay, as moeact_mx_out.noop_flag).
  * Allocates nothing; asynchronous on `stream`.  Bounded waits report

@@ -168,6 +168,8 @@ def test_each_expert_uses_its_own_weight_and_rows(cuda_device):
     # a wide FC2 (32 output tiles) over three blocks: 148 / 3 = 49 parts
     # capped at one tile each
     (256, 4096, [300, 84], False),
+    # many small experts (one partial block each, empty ones among them)
+    (128, 256, [(7 * e) % 5 for e in range(300)], False),
 ])
 def test_fc2_matches_the_oracle(cuda_device, N, H, splits, staged):
     M = sum(splits)
